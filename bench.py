@@ -1,0 +1,534 @@
+"""Benchmark of the ternary linear layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|fused|sweep]
+                    [--impl ours|reference]
+
+One JSON line on rank 0.  A *step* is one pass of the whole hot path over one
+batch of synthetic input: quantise + pack the fp32 latent weights (absmean
+gamma, 2-bit codes), quantise the activations per token, run the ternary
+contraction with the fused rescale (and, for the fused workload, the
+RMSNorm + FWHT prologue).
+
+Default workload ("decode"): K = N = 4096, per-row gamma, W ~ N(0, 0.02),
+activations ~ N(0, 1) with 0.1 % outliers x20, token batches M = 1 and M = 8.
+A ring of L = 64 distinct layers keeps every working set above L2: per step the
+64 fp32 weights (4 GiB) are re-packed (the packed ring is 256 MiB), both
+batches are quantised, and each batch runs through the GEMV of all 64 layers.
+Metric: algorithmic HBM bytes of the step / step time (GB/s).
+
+Timing: CUDA graphs for each segment (pack, activation quantisation, GEMV
+M=1, GEMV M=8), CUDA events between segments on the launching stream, barrier
++ synchronize around the timed steps, max over ranks.  Per-kernel average
+launch time = segment time / launches in the segment.
+
+--impl reference times the CPU oracle (the plain C reference) on a bounded
+sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ternary GEMM TOPS (M>=512) & packed-weight HBM GB/s (M<=16), % of roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_HBM = 6650.0
+FALLBACK_BF16 = 1590.0
+INT8_OVER_BF16 = 2.0  # nominal dense int8 (4.5 POPS) / bf16 (2.25 PFLOP/s)
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm": FALLBACK_HBM, "bf16": FALLBACK_BF16, "bf16_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ternary_bit_linear_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None if the
+    kernels changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        if t.get("source_hash") != kernel_source_hash():
+            return None
+        return t["kernels"].get(kernel)
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        med = float(np.median(self.samples)) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+class Workload:
+    """Builds device buffers and the per-segment launch lists of one step."""
+
+    def __init__(self, name, tq, S, torch, dev, layers):
+        self.name, self.tq, self.torch, self.dev = name, tq, torch, dev
+        f32, u8, i8, i32 = torch.float32, torch.uint8, torch.int8, torch.int32
+        self.segments = []  # (label, kernel_name, launches, algorithmic bytes or ops, [fns])
+        if name == "decode":
+            N = K = 4096
+            self.N, self.K, self.Ms, self.L = N, K, [1, 8], layers
+            self.per_row = True
+            W = torch.from_numpy(S.decode_weights(N, K, seed=0))
+            self.W = [W.to(dev) for _ in range(self.L)]  # distinct buffers, same values
+            self.X = {M: torch.from_numpy(S.decode_acts(M, K, seed=0)) for M in self.Ms}
+        elif name == "prefill":
+            M, N, K = 2048, 11008, 4096
+            self.N, self.K, self.Ms, self.L = N, K, [M], 1
+            self.per_row = False
+            W, X = S.prefill(M, N, K, seed=0)
+            self.W = [torch.from_numpy(W).to(dev)]
+            self.X = {M: torch.from_numpy(X)}
+        elif name == "fused":
+            M, N, K = 512, 5632, 2048
+            self.N, self.K, self.Ms, self.L = N, K, [M], 1
+            self.per_row = False
+            W, X = S.fused(M, N, K, seed=0)
+            self.W = [torch.from_numpy(W).to(dev)]
+            self.X = {M: torch.from_numpy(X)}
+        elif name == "sweep":
+            N = K = 8192
+            self.N, self.K, self.Ms, self.L = N, K, [1, 4, 16, 64, 512, 4096], 1
+            self.per_row = True
+            self.W = [torch.from_numpy(S.sweep_weights(N, K, seed=0)).to(dev)]
+            self.X = {M: torch.from_numpy(S.sweep_acts(M, K, seed=0)) for M in self.Ms}
+        else:
+            raise SystemExit(f"unknown workload {name}")
+        N, K, L = self.N, self.K, self.L
+        self.flags = tq.GAMMA_PER_ROW if self.per_row else 0
+        self.packed = [torch.empty((N, K // 4), dtype=u8, device=dev) for _ in range(L)]
+        self.gamma = [torch.empty((N if self.per_row else 1,), dtype=f32, device=dev) for _ in range(L)]
+        nws = tq.pack_workspace_bytes(N, K, self.flags)
+        self.pack_ws = torch.empty((max(nws, 16),), dtype=u8, device=dev)
+        self.Xd = {M: x.to(dev) for M, x in self.X.items()}
+        self.xq = {M: torch.empty((M, K), dtype=i8, device=dev) for M in self.Ms}
+        self.sx = {M: torch.empty((M,), dtype=f32, device=dev) for M in self.Ms}
+        self.rs = {M: torch.empty((M,), dtype=i32, device=dev) for M in self.Ms}
+        self.y = {M: [torch.empty((M, N), dtype=f32, device=dev) for _ in range(L)] for M in self.Ms}
+        if name == "fused":
+            fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM
+            self.fused_flags = fl
+            self.fused_ws = torch.empty((tq.fused_workspace_bytes(self.Ms[0], K, fl),), dtype=u8, device=dev)
+
+        # --- segments of one step ---
+        pack_bytes = 4 * N * K + N * K // 4 + 4 * (N if self.per_row else 1)
+        pack_launches = 1 if self.per_row else 3
+        self.segments.append(("pack", "pack", L, L * pack_bytes, L * pack_launches,
+                              [lambda l=l: tq.quantize_ternary_pack_(self.W[l], self.flags, self.packed[l],
+                                                                      self.gamma[l], self.pack_ws)
+                               for l in range(L)]))
+        if name == "fused":
+            M = self.Ms[0]
+            ops = 2 * M * N * K
+            self.segments.append(("fused M=%d" % M, "fused", 1, ops, 2, [
+                lambda: tq.bitlinear_fused_(self.Xd[M], self.packed[0], self.gamma[0], self.fused_flags,
+                                            self.y[M][0], self.fused_ws)]))
+            return
+        act_bytes = sum(4 * M * K + M * K + 8 * M for M in self.Ms)
+        self.segments.append(("act", "act_quant", len(self.Ms), act_bytes, len(self.Ms), [
+            lambda M=M: tq.quantize_act_int8_(self.Xd[M], 0, 0.05, 40.0, self.xq[M], self.sx[M], self.rs[M])
+            for M in self.Ms]))
+        for M in self.Ms:
+            gemv = M <= 16
+            work = (N * K // 4 + 4 * N * (1 if self.per_row else 0) + M * K + 8 * M + 4 * M * N) if gemv \
+                else 2 * M * N * K
+            self.segments.append(("gemv M=%d" % M if gemv else "gemm M=%d" % M,
+                                  "gemv" if gemv else "gemm", L, L * work, L, [
+                lambda l=l, M=M: tq.ternary_gemm_(self.xq[M], self.sx[M], self.rs[M], self.packed[l],
+                                                  self.gamma[l], self.flags, self.y[M][l])
+                for l in range(L)]))
+
+    def step_bytes(self):
+        return sum(s[3] for s in self.segments if s[1] in ("pack", "act_quant", "gemv"))
+
+    def step_ops(self):
+        return sum(s[3] for s in self.segments if s[1] in ("gemm", "fused"))
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import ternary_bit_linear_b200 as tq
+    from ternary_bit_linear_b200 import build as tqbuild
+    from ternary_bit_linear_b200 import synthetic as S
+
+    if rank == 0 or not os.path.exists(tqbuild.LIB):
+        tqbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    tq.load()
+    wl = Workload(args.workload, tq, S, torch, dev, args.layers)
+    stream = torch.cuda.Stream(device=dev)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for seg in wl.segments:  # eager warm-up of every launch, then capture
+            for fn in seg[5]:
+                fn()
+        torch.cuda.synchronize()
+        for seg in wl.segments:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for fn in seg[5]:
+                    fn()
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    def step():
+        for g in graphs:
+            g.replay()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    assert tq.device_status(stream) == 0
+
+    nseg = len(graphs)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nseg + 1)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        with torch.cuda.stream(stream):
+            for k in range(args.steps):
+                evs[k][0].record(stream)
+                for i, g in enumerate(graphs):
+                    g.replay()
+                    evs[k][i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    seg_ms = np.zeros(nseg)
+    for k in range(args.steps):
+        for i in range(nseg):
+            seg_ms[i] += evs[k][i].elapsed_time(evs[k][i + 1])
+    total_ms = float(seg_ms.sum())
+    total_ms = allreduce_max(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    assert tq.device_status(stream) == 0
+
+    # --- end to end through the public API with host buffers ---
+    e2e = run_e2e(args, wl, tq, torch, stream, graphs, world)
+
+    pk = peaks()
+    kernels = {}
+    for (label, kname, launches, work, nlaunch, _), ms in zip(wl.segments, seg_ms):
+        per_launch_ms = ms / args.steps / launches
+        if kname in ("gemm", "fused"):
+            ach = work / launches / (per_launch_ms * 1e-3) / 1e12
+            peak = pk["bf16"] * INT8_OVER_BF16
+            kernels[label] = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
+                              "unit": "TOPS", "frac": round(ach / peak, 4),
+                              "us_per_launch": round(per_launch_ms * 1e3, 3)}
+        else:
+            ach = work / launches / (per_launch_ms * 1e-3) / 1e9
+            kernels[label] = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"],
+                              "unit": "GB/s", "frac": round(ach / pk["hbm"], 4),
+                              "us_per_launch": round(per_launch_ms * 1e3, 3)}
+    dom = max(zip(wl.segments, seg_ms), key=lambda t: t[1])[0]
+    dk = kernels[dom[0]]
+    roofline = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
+                "unit": "GB/s" if dk["unit"] == "GB/s" else "TOPS", "frac": dk["frac"],
+                "traffic": traffic_for(dom[1] + ":" + args.workload), "kernel": dom[0],
+                "peak_source": pk["source"] + (" hbm_gbs (copy, burst)" if dk["bound"] == "hbm"
+                                               else " bf16_tflops x2 (nominal int8/bf16 ratio)")}
+    if wl.name in ("decode",):
+        value = wl.step_bytes() * world / (ms_per_step * 1e-3) / 1e9
+        unit = "GB/s"
+    else:
+        value = wl.step_ops() * world / (ms_per_step * 1e-3) / 1e12
+        unit = "TOPS"
+    launches = sum(s[4] for s in wl.segments) * args.steps
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+    clocks = sampler.summary()
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic", "config": wl_config(wl, world),
+        "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
+        "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    del graphs
+
+
+def wl_config(wl, world):
+    c = {"workload": {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers" % wl.L,
+                      "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma",
+                      "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512",
+                      "sweep": "M sweep over K=N=8192, per-row gamma"}[wl.name],
+         "M": wl.Ms, "N": wl.N, "K": wl.K, "layers": wl.L,
+         "gamma": "per-row" if wl.per_row else "per-tensor",
+         "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
+             wl.L * wl.N * wl.K * 4 >> 20, wl.L * wl.N * wl.K // 4 >> 20),
+         "parallelism": "replicas x%d" % world if world > 1 else "single GPU"}
+    return c
+
+
+def run_e2e(args, wl, tq, torch, stream, graphs, world):
+    """Same step through the public calls with pinned host inputs copied in and
+    the step's outputs copied back inside the timed region."""
+    host_x = {M: x.pin_memory() for M, x in wl.X.items()}
+    outs = [y for M in wl.Ms for y in wl.y[M]]
+    host_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in outs]
+    h2d = sum(x.numel() * 4 for x in host_x.values())
+    d2h = sum(y.numel() * 4 for y in outs)
+    steps = max(3, min(args.steps, 50))
+
+    def one():
+        for M in wl.Ms:
+            wl.Xd[M].copy_(host_x[M], non_blocking=True)
+        for g in graphs:
+            g.replay()
+        for y, hy in zip(outs, host_y):
+            hy.copy_(y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            one()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    ms = allreduce_max(t0.elapsed_time(t1), world) / steps
+    if wl.name == "decode":
+        v, u = wl.step_bytes() * world / (ms * 1e-3) / 1e9, "GB/s"
+    else:
+        v, u = wl.step_ops() * world / (ms * 1e-3) / 1e12, "TOPS"
+    return {"value": round(v, 2), "unit": u, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms, 4), "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline / reference arm
+# ---------------------------------------------------------------------------
+def oracle_sample(workload):
+    """One bounded unit of the workload on the oracle: returns (fn, work, what)."""
+    import oracle
+    from ternary_bit_linear_b200 import synthetic as S
+
+    if workload == "decode":
+        N = K = 4096
+        W = S.decode_weights(N, K, seed=0)
+        Xs = {M: S.decode_acts(M, K, seed=0) for M in (1, 8)}
+
+        def fn():
+            packed, gamma = oracle.quantize_pack(W, per_row=True)
+            for M, X in Xs.items():
+                xq, sx, _ = oracle.act_quant(X)
+                oracle.dequant(oracle.matmul_addsub(xq, packed), gamma, sx, True)
+        work = (4 * N * K + N * K // 4 + 4 * N) + sum(
+            4 * M * K + M * K + 8 * M + N * K // 4 + 4 * N + M * K + 8 * M + 4 * M * N for M in (1, 8))
+        return fn, work, "one full layer of the step (pack 4096x4096 per-row, act-quant + GEMV for M=1 and M=8)", "GB/s"
+    if workload in ("prefill", "fused", "sweep"):
+        if workload == "prefill":
+            M, N, K, per_row = 2048, 11008, 4096, False
+            W, X = S.prefill(M, N, K, seed=0)
+        elif workload == "fused":
+            M, N, K, per_row = 512, 5632, 2048, False
+            W, X = S.fused(M, N, K, seed=0)
+        else:
+            M, N, K, per_row = 4096, 8192, 8192, True
+            W, X = S.sweep_weights(N, K, seed=0), S.sweep_acts(64, K, seed=0)
+        rows = 8
+        Xs = X[:rows]
+        packed, gamma = oracle.quantize_pack(W, per_row=per_row)
+
+        def fn():
+            if workload == "fused":
+                oracle.bitlinear(Xs, packed, gamma, per_row)
+            else:
+                xq, sx, _ = oracle.act_quant(Xs)
+                oracle.dequant(oracle.matmul_addsub(xq, packed), gamma, sx, per_row)
+        return fn, 2 * rows * N * K, "%d tokens of the contraction (weights pre-packed)" % rows, "TOPS"
+    raise SystemExit(workload)
+
+
+def cpu_baseline(workload, budget_s=15.0):
+    fn, work, what, unit = oracle_sample(workload)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or el / n * (n + 1) > 2 * budget_s:
+            break
+    scale = 1e9 if unit == "GB/s" else 1e12
+    return {"value": round(work * n / el / scale, 6), "unit": unit, "cores": 1, "kind": "oracle",
+            "sample": "%s, x%d, %.1f s, single-threaded C" % (what, n, el), "host_cores": os.cpu_count()}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    fn, work, what, unit = oracle_sample(args.workload)
+    for _ in range(args.warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    el = time.perf_counter() - t0
+    scale = 1e9 if unit == "GB/s" else 1e12
+    v = work * args.steps / el / scale
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic", "config": {"workload": args.workload, "sample": what},
+        "cpu_baseline": {"value": round(v, 6), "unit": unit, "cores": 1, "kind": "oracle",
+                         "sample": what + " per step"},
+        "e2e": {"value": round(v, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def allreduce_max(v, world):
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fused", "sweep"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

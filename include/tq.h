@@ -1,0 +1,199 @@
+/*
+ * tq.h -- C ABI of libtq, a B200 (sm_100a) implementation of the ternary
+ * (BitNet b1.58 style) linear layer.
+ *
+ *   weights:     gamma = mean|w| (per tensor, or per output row),
+ *                q = clamp(round(w / gamma), -1, 1), packed 2 bits per value,
+ *                four per byte, LSB first, -1 = 0b00, 0 = 0b01, +1 = 0b10.
+ *   activations: per token, eta = max|x| (>= 1e-6), x_q = clamp(round(x * 127/eta),
+ *                -127, 127), s_x = eta / 127.
+ *   output:      y[m][n] = (sum_k x_q[m][k] * q[n][k]) * gamma_n * s_x[m].
+ *   optional prologue: RMSNorm, then a blockwise 512-point fast Walsh-Hadamard
+ *                rotation, before the activation quantisation.
+ *
+ * Sources (page title, section):
+ *   Foundry, docs/quantization.md: "Ternary Format / Encoding" (bit codes and
+ *     byte layout), "Ternary Quantization (BitNet b1.58) / How It Works"
+ *     (absmean gamma, round and clamp, add/subtract matmul scaled by gamma).
+ *   Hetman-2b, src/quantization.py: section 1 (FWHT B=512), section 2
+ *     (AbsmeanWeightQuantizer, SymmetricActivationQuantizer), section 4
+ *     (SubLayerRMSNorm), section 5 (BitLinear.forward and export_packed_weights),
+ *     section 7 (simulate_hardware_bitnet_gemv).
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers on the current CUDA device, owned
+ *     by the caller; the library allocates nothing on these paths.  Work is
+ *     enqueued on `stream` (NULL = legacy default stream) and the call returns
+ *     without waiting for it.
+ *   - Layouts are row-major and dense: W / x are [rows][K] with K contiguous;
+ *     packed weights are [N][K/4] bytes; y is [M][N].
+ *   - Every pointer must be 16-byte aligned (TQ_ERR_ALIGN otherwise).
+ *   - Shape rules: 1 <= M, N; 64 <= K <= 65536 and K % 64 == 0 (the packed row
+ *     of K/4 bytes is then a whole number of 16-byte vectors); K % 512 == 0
+ *     when the FWHT is requested.  Violations return TQ_ERR_SHAPE.
+ *   - Arguments are checked before anything is enqueued: a call that returns an
+ *     error has launched nothing and written nothing.  Launch failures return
+ *     TQ_ERR_CUDA.  Waits inside kernels are bounded; a wait that gives up
+ *     records TQ_ERR_TIMEOUT in a per-device status word read (and cleared) by
+ *     tq_get_device_status().
+ *   - Inputs and outputs must not overlap, except where an entry point says so.
+ *   - Non-finite inputs give unspecified (but memory-safe) results unless
+ *     TQ_FLAG_SANITIZE_NONFINITE is set.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *tq_stream_t;
+
+typedef enum tq_status {
+    TQ_OK = 0,
+    TQ_ERR_NULL = 1,    /* a required pointer is NULL                        */
+    TQ_ERR_SHAPE = 2,   /* a size is out of range or breaks a divisibility rule */
+    TQ_ERR_ALIGN = 3,   /* a pointer is not 16-byte aligned                   */
+    TQ_ERR_ARG = 4,     /* unknown flag, overlap, or workspace too small      */
+    TQ_ERR_CUDA = 5,    /* a CUDA runtime call or a kernel launch failed      */
+    TQ_ERR_DEVICE = 6,  /* the current device is not compute capability 10.0  */
+    TQ_ERR_TIMEOUT = 7  /* a bounded wait inside a kernel gave up             */
+} tq_status;
+
+/* flags */
+#define TQ_GAMMA_PER_ROW (1u << 0)           /* one gamma per output row (else one per tensor) */
+#define TQ_FLAG_FWHT (1u << 1)               /* blockwise FWHT-512 before act. quantisation    */
+#define TQ_FLAG_RMSNORM (1u << 2)            /* RMSNorm before the FWHT                        */
+#define TQ_FLAG_ETA_CLAMP (1u << 3)          /* clamp eta to [eta_min, eta_max]                */
+#define TQ_FLAG_SANITIZE_NONFINITE (1u << 4) /* quench NaN / +-Inf inputs first                */
+
+/*
+ * Absmean ternarisation and 2-bit packing of an fp32 weight matrix.
+ * Foundry docs/quantization.md, "How It Works" steps 1-3 and "Ternary Format /
+ * Encoding"; Hetman-2b section 5 BitLinear.export_packed_weights; the per-row
+ * variant is Foundry's per-channel granularity (fq_quantize_ternary_per_channel).
+ *
+ *   w       [N][K] fp32, read only.
+ *   flags   TQ_GAMMA_PER_ROW and/or TQ_FLAG_SANITIZE_NONFINITE (nan -> 0,
+ *           +-inf -> +-1 before anything else, Hetman-2b section 2).
+ *   packed  [N][K/4] bytes, written: byte j of row n holds codes 4j..4j+3 in bits
+ *           (0,1) (2,3) (4,5) (6,7); 0b11 is never produced.
+ *   gamma   [N] (per row) or [1] (per tensor) fp32, written: the fp32 nearest to
+ *           the exact mean of |w| (ties to even), then max(., 1e-6).
+ *   workspace / workspace_bytes: device scratch of at least
+ *           tq_pack_workspace_bytes(N, K, flags) bytes (0 for per-row gamma, where
+ *           workspace may be NULL).  Contents on entry are ignored.
+ * Codes: q = +1 iff the fp32 quotient w / gamma rounds (half to even) above 0.5,
+ * -1 iff below -0.5, else 0.
+ */
+TQ_API tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigned flags,
+                                   uint8_t *packed, float *gamma, void *workspace,
+                                   size_t workspace_bytes, tq_stream_t stream);
+
+/* Scratch bytes tq_quantize_ternary_pack needs for these arguments. */
+TQ_API size_t tq_pack_workspace_bytes(int64_t N, int64_t K, unsigned flags);
+
+/*
+ * Per-token symmetric int8 quantisation.
+ * Hetman-2b section 2 SymmetricActivationQuantizer.forward (reduction over the
+ * last dimension); s_x = eta / 127 is the scale the output is multiplied by.
+ *
+ *   x       [M][K] fp32, read only.
+ *   flags   TQ_FLAG_ETA_CLAMP (eta clamped to [eta_min, eta_max] after the 1e-6
+ *           floor), TQ_FLAG_SANITIZE_NONFINITE (nan -> 0, +-inf -> +-eta_max).
+ *   xq      [M][K] int8, written, values in [-127, 127].
+ *   s_x     [M] fp32, written.
+ *   rowsum  [M] int32, written: sum_k xq[m][k].  tq_ternary_gemm needs it.
+ */
+TQ_API tq_status tq_quantize_act_int8(const float *x, int64_t M, int64_t K, unsigned flags,
+                               float eta_min, float eta_max, int8_t *xq, float *s_x,
+                               int32_t *rowsum, tq_stream_t stream);
+
+/*
+ * Blockwise fast Walsh-Hadamard transform over 512-element blocks of each row,
+ * fp32: stages h = 1, 2, ..., 256 of (a + b, a - b), then, if normalize != 0,
+ * a multiply by the fp32 value of 1/sqrt(512).  Hetman-2b section 1
+ * (fast_walsh_hadamard_transform_512, blockwise_fwht_forward).
+ *
+ *   x  [rows][K] fp32 (K % 512 == 0), read;  y [rows][K] fp32, written.
+ *   y == x (in place) is allowed; any other overlap is not.
+ * Results are bit-identical to that stage order.
+ */
+TQ_API tq_status tq_fwht512(const float *x, float *y, int64_t rows, int64_t K, int normalize,
+                     tq_stream_t stream);
+
+/*
+ * Ternary x int8 contraction with the fp32 rescale fused in its epilogue.
+ * Hetman-2b section 5 steps 5-6 and section 7; Foundry "Native Matmul Kernel".
+ *
+ *   xq, s_x, rowsum  quantised activations as written by tq_quantize_act_int8
+ *                    ([M][K] int8, [M] fp32, [M] int32).
+ *   packed, gamma    as written by tq_quantize_ternary_pack ([N][K/4], [N] or [1]).
+ *   flags            TQ_GAMMA_PER_ROW selects gamma[N] (else gamma[0]).
+ *   y                [M][N] fp32, written: y = fp32(acc) * (gamma_n * s_x[m]).
+ *   acc              [M][N] int32 or NULL: if given, the exact integer sums
+ *                    acc[m][n] = sum_k xq[m][k] * q[n][k] are written too.
+ * M <= 16 runs an HBM-bound GEMV; larger M runs a tcgen05 int8 tensor-core GEMM.
+ */
+TQ_API tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                          const uint8_t *packed, const float *gamma, unsigned flags,
+                          int64_t M, int64_t N, int64_t K, float *y, int32_t *acc,
+                          tq_stream_t stream);
+
+/*
+ * Whole layer on pre-packed weights: [quench] -> [RMSNorm] -> [FWHT-512] ->
+ * per-token int8 -> contraction -> rescale.  Hetman-2b section 5
+ * BitLinear.forward steps 0-6.
+ *
+ *   x           [M][K] fp32, read.
+ *   rms_gain    [K] fp32 or NULL (unit gain); used with TQ_FLAG_RMSNORM.
+ *   rms_eps     RMSNorm epsilon (1e-6 in the pages).
+ *   eta_min/max used with TQ_FLAG_ETA_CLAMP (0.05 / 40 in the pages).
+ *   flags       any of the TQ_* flags above.
+ *   packed, gamma, M, N, K as for tq_ternary_gemm.
+ *   y           [M][N] fp32, written.
+ *   xq_out      [M][K] int8 or NULL; s_x_out [M] fp32 or NULL: if given, the
+ *               quantised activations are left there.
+ *   workspace   at least tq_fused_workspace_bytes(M, K, flags) bytes of device
+ *               scratch (x_q, s_x, rowsum live there when xq_out / s_x_out are
+ *               NULL).  Contents on entry are ignored.
+ * RMSNorm sums squares in fp64; the FWHT and the quantiser are bit-identical to
+ * the fp32 definitions.
+ */
+TQ_API tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_eps,
+                             float eta_min, float eta_max, unsigned flags,
+                             const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
+                             int64_t K, float *y, int8_t *xq_out, float *s_x_out,
+                             void *workspace, size_t workspace_bytes, tq_stream_t stream);
+
+/* Scratch bytes tq_bitlinear_fused needs for these arguments. */
+TQ_API size_t tq_fused_workspace_bytes(int64_t M, int64_t K, unsigned flags);
+
+/*
+ * Waits for `stream`, then returns and clears the current device's status word:
+ * TQ_OK, or TQ_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the
+ * last call.  TQ_ERR_CUDA if the synchronisation itself failed.
+ */
+TQ_API tq_status tq_get_device_status(tq_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+TQ_API const char *tq_status_string(tq_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+TQ_API int tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

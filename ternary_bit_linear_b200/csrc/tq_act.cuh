@@ -1,0 +1,372 @@
+// tq_act.cuh -- per-token int8 quantisation, RMSNorm and the blockwise
+// FWHT-512 (standalone, and fused as the prologue of the whole layer).
+//
+// Hetman-2b, src/quantization.py:
+//   section 1  fast_walsh_hadamard_transform_512 / blockwise_fwht_forward:
+//              stages h = 1, 2, ..., 256 of (a + b, a - b) in fp32, then a
+//              multiply by fp32(1/sqrt(512)).  The kernels below perform
+//              exactly these fp32 operations on the same operands, so their
+//              results are bit-identical to that stage order.
+//   section 2  SymmetricActivationQuantizer.forward: eta = max|x| (>= 1e-6,
+//              optionally clamped), scale = 127/eta, x_q = clamp(round(x*scale)).
+//   section 4  SubLayerRMSNorm.forward: x * rsqrt(mean(x^2) + eps) * g.
+//   section 5  BitLinear.forward step 0: quench nan -> 0, +-inf -> +-eta_max.
+//
+// Layout of a 512-block inside one warp: lane l holds the 16 elements
+//   i = 128*j + 4*l + e   (j, e in 0..3)
+// loaded as four coalesced float4 (one per j).  Stages h = 1, 2 pair elements
+// inside a float4 (bit 0/1 of i = e), h = 4..64 pair lanes (bits 2..6 = lane
+// bits 0..4, exchanged with shfl.xor), h = 128, 256 pair float4s (j bits).
+#pragma once
+
+#include "tq_common.cuh"
+
+namespace tq {
+
+constexpr int kActThreads = 256;
+
+struct ActParams {
+    int sanitize;    // quench non-finite inputs (nan -> 0, +-inf -> +-eta_max)
+    int clamp_eta;   // clamp eta to [eta_min, eta_max]
+    float eta_min, eta_max;
+    int rmsnorm;     // (fused prologue only)
+    float rms_eps;
+    const float *rms_gain;  // [K] or nullptr
+};
+
+__device__ __forceinline__ float quench(float x, float eta_max) {
+    if (x != x) return 0.0f;
+    if (isinf(x)) return x > 0.0f ? eta_max : -eta_max;
+    return x;
+}
+
+// round half to even, clamp to [-127, 127]; NaN -> 0
+__device__ __forceinline__ int quant_code(float x, float scale) {
+    const float t = rintf(__fmul_rn(x, scale));
+    if (t != t) return 0;
+    return (int)fminf(fmaxf(t, -127.0f), 127.0f);
+}
+
+__device__ __forceinline__ float eta_of(float amax, const ActParams &p) {
+    float eta = amax > 1e-6f ? amax : 1e-6f;
+    if (p.clamp_eta) eta = fminf(fmaxf(eta, p.eta_min), p.eta_max);
+    return eta;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// Block-wide reductions in a fixed order; result valid in every thread.
+// `red` needs 32 slots.
+template <int NT>
+__device__ __forceinline__ float block_max(float v, float *red) {
+    v = warp_max(v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = lane < NT / 32 ? red[lane] : 0.0f;
+    t = warp_max(t);
+    __syncthreads();
+    return t;
+}
+template <int NT>
+__device__ __forceinline__ int block_sum_i(int v, int *red) {
+    v = warp_sum_i(v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    int t = lane < NT / 32 ? red[lane] : 0;
+    t = warp_sum_i(t);
+    __syncthreads();
+    return t;
+}
+template <int NT>
+__device__ __forceinline__ double block_sum_d(double v, double *red) {
+    v = warp_sum_d(v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = lane < NT / 32 ? red[lane] : 0.0;
+    t = warp_sum_d(t);
+    __syncthreads();
+    return t;
+}
+
+__device__ __forceinline__ uint32_t pack_codes4(int a, int b, int c, int d) {
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+           ((uint32_t)(d & 0xff) << 24);
+}
+
+// x * r * g in fp64, rounded once (RMSNorm output of one element).
+__device__ __forceinline__ float rms_apply(float x, double r, const float *gain, int k) {
+    const double g = gain ? (double)__ldg(gain + k) : 1.0;
+    return __double2float_rn(__dmul_rn(__dmul_rn((double)x, r), g));
+}
+
+// ---------------------------------------------------------------------------
+// Per-token quantisation (optionally after RMSNorm), one CTA per token.
+// VEC > 0: the row lives in registers (K <= 1024*VEC); VEC == 0: streamed.
+// ---------------------------------------------------------------------------
+template <int VEC>
+__global__ void __launch_bounds__(kActThreads)
+    act_quant_kernel(const float *__restrict__ x, int K, ActParams p, int8_t *__restrict__ xq,
+                     float *__restrict__ s_x, int32_t *__restrict__ rowsum) {
+    __shared__ float redf[32];
+    __shared__ int redi[32];
+    __shared__ double redd[32];
+    const int64_t m = blockIdx.x;
+    const int nv = K >> 2, tid = threadIdx.x;
+    const float4 *src = reinterpret_cast<const float4 *>(x + m * (int64_t)K);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(xq + m * (int64_t)K);
+
+    auto load = [&](int idx) {
+        float4 v = __ldg(src + idx);
+        if (p.sanitize)
+            v = make_float4(quench(v.x, p.eta_max), quench(v.y, p.eta_max), quench(v.z, p.eta_max),
+                            quench(v.w, p.eta_max));
+        return v;
+    };
+
+    float4 v[VEC > 0 ? VEC : 1];
+    double r = 1.0;
+    if (VEC > 0) {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            const int idx = tid + i * kActThreads;
+            v[i] = idx < nv ? load(idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    if (p.rmsnorm) {
+        double ss = 0.0;
+        if (VEC > 0) {
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) {
+                ss = __fma_rn((double)v[i].x, (double)v[i].x, ss);
+                ss = __fma_rn((double)v[i].y, (double)v[i].y, ss);
+                ss = __fma_rn((double)v[i].z, (double)v[i].z, ss);
+                ss = __fma_rn((double)v[i].w, (double)v[i].w, ss);
+            }
+        } else {
+            for (int idx = tid; idx < nv; idx += kActThreads) {
+                const float4 t = load(idx);
+                ss = __fma_rn((double)t.x, (double)t.x, ss);
+                ss = __fma_rn((double)t.y, (double)t.y, ss);
+                ss = __fma_rn((double)t.z, (double)t.z, ss);
+                ss = __fma_rn((double)t.w, (double)t.w, ss);
+            }
+        }
+        ss = block_sum_d<kActThreads>(ss, redd);
+        r = __drcp_rn(__dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
+        if (VEC > 0) {
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) {
+                const int k = 4 * (tid + i * kActThreads);
+                v[i] = make_float4(rms_apply(v[i].x, r, p.rms_gain, k),
+                                   rms_apply(v[i].y, r, p.rms_gain, k + 1),
+                                   rms_apply(v[i].z, r, p.rms_gain, k + 2),
+                                   rms_apply(v[i].w, r, p.rms_gain, k + 3));
+            }
+        }
+    }
+    auto normed = [&](int idx) {
+        float4 t = load(idx);
+        if (p.rmsnorm) {
+            const int k = 4 * idx;
+            t = make_float4(rms_apply(t.x, r, p.rms_gain, k), rms_apply(t.y, r, p.rms_gain, k + 1),
+                            rms_apply(t.z, r, p.rms_gain, k + 2),
+                            rms_apply(t.w, r, p.rms_gain, k + 3));
+        }
+        return t;
+    };
+
+    float amax = 0.0f;
+    if (VEC > 0) {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i)
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)),
+                                     fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+    } else {
+        for (int idx = tid; idx < nv; idx += kActThreads) {
+            const float4 t = normed(idx);
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+        }
+    }
+    amax = block_max<kActThreads>(amax, redf);
+    const float eta = eta_of(amax, p);
+    const float scale = __fdiv_rn(127.0f, eta);
+
+    int sum = 0;
+    auto emit = [&](int idx, float4 t) {
+        const int a = quant_code(t.x, scale), b = quant_code(t.y, scale),
+                  c = quant_code(t.z, scale), d = quant_code(t.w, scale);
+        dst[idx] = pack_codes4(a, b, c, d);
+        sum += a + b + c + d;
+    };
+    if (VEC > 0) {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            const int idx = tid + i * kActThreads;
+            if (idx < nv) emit(idx, v[i]);
+        }
+    } else {
+        for (int idx = tid; idx < nv; idx += kActThreads) emit(idx, normed(idx));
+    }
+    sum = block_sum_i<kActThreads>(sum, redi);
+    if (tid == 0) {
+        s_x[m] = __fdiv_rn(eta, 127.0f);
+        if (rowsum) rowsum[m] = sum;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// FWHT-512 of the 16 values a warp lane holds (layout in the file header).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void butterfly(float &a, float &b) {
+    const float s = __fadd_rn(a, b), d = __fsub_rn(a, b);
+    a = s;
+    b = d;
+}
+
+__device__ __forceinline__ void fwht512_regs(float (&f)[16], bool normalize) {
+    const int lane = threadIdx.x & 31;
+    // h = 1 (e bit 0), h = 2 (e bit 1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        butterfly(f[4 * j + 0], f[4 * j + 1]);
+        butterfly(f[4 * j + 2], f[4 * j + 3]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        butterfly(f[4 * j + 0], f[4 * j + 2]);
+        butterfly(f[4 * j + 1], f[4 * j + 3]);
+    }
+    // h = 4 .. 64: partner lane = lane ^ s; the lane with the bit clear holds a
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1) {
+        const bool upper = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, f[i], s);
+            f[i] = upper ? __fsub_rn(o, f[i]) : __fadd_rn(f[i], o);
+        }
+    }
+    // h = 128 (j bit 0), h = 256 (j bit 1)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        butterfly(f[0 + e], f[4 + e]);
+        butterfly(f[8 + e], f[12 + e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        butterfly(f[0 + e], f[8 + e]);
+        butterfly(f[4 + e], f[12 + e]);
+    }
+    if (normalize) {
+        const float c = __int_as_float(0x3D3504F3);  // fp32(1/sqrt(512))
+#pragma unroll
+        for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], c);
+    }
+}
+
+// Standalone transform: one warp per 512-block, 8 warps per CTA.
+__global__ void __launch_bounds__(256)
+    fwht512_kernel(const float *x, float *y, int64_t nblocks, int normalize) {
+    const int64_t blk = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (blk >= nblocks) return;
+    const int lane = threadIdx.x & 31;
+    const float4 *src = reinterpret_cast<const float4 *>(x + blk * 512);
+    float4 *dst = reinterpret_cast<float4 *>(y + blk * 512);
+    float f[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 v = src[j * 32 + lane];
+        f[4 * j + 0] = v.x;
+        f[4 * j + 1] = v.y;
+        f[4 * j + 2] = v.z;
+        f[4 * j + 3] = v.w;
+    }
+    fwht512_regs(f, normalize != 0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        dst[j * 32 + lane] = make_float4(f[4 * j + 0], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+}
+
+// ---------------------------------------------------------------------------
+// Fused prologue of the whole layer: [quench] -> [RMSNorm] -> FWHT-512 ->
+// per-token int8.  One CTA per token, one warp per 512-block (K = 512 * NW).
+// ---------------------------------------------------------------------------
+template <int NW>
+__global__ void __launch_bounds__(NW * 32)
+    prologue_fwht_kernel(const float *__restrict__ x, ActParams p, int8_t *__restrict__ xq,
+                         float *__restrict__ s_x, int32_t *__restrict__ rowsum) {
+    __shared__ float redf[32];
+    __shared__ int redi[32];
+    __shared__ double redd[32];
+    constexpr int K = 512 * NW;
+    const int64_t m = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float *row = x + m * (int64_t)K + warp * 512;
+    float f[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float4 v = __ldg(reinterpret_cast<const float4 *>(row) + j * 32 + lane);
+        if (p.sanitize)
+            v = make_float4(quench(v.x, p.eta_max), quench(v.y, p.eta_max), quench(v.z, p.eta_max),
+                            quench(v.w, p.eta_max));
+        f[4 * j + 0] = v.x;
+        f[4 * j + 1] = v.y;
+        f[4 * j + 2] = v.z;
+        f[4 * j + 3] = v.w;
+    }
+    if (p.rmsnorm) {
+        double ss = 0.0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ss = __fma_rn((double)f[i], (double)f[i], ss);
+        ss = block_sum_d<NW * 32>(ss, redd);
+        const double r =
+            __drcp_rn(__dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = warp * 512 + j * 128 + lane * 4 + e;
+                f[4 * j + e] = rms_apply(f[4 * j + e], r, p.rms_gain, k);
+            }
+    }
+    fwht512_regs(f, true);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = block_max<NW * 32>(amax, redf);
+    const float eta = eta_of(amax, p);
+    const float scale = __fdiv_rn(127.0f, eta);
+    int sum = 0;
+    uint32_t *dst = reinterpret_cast<uint32_t *>(xq + m * (int64_t)K + warp * 512);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int a = quant_code(f[4 * j + 0], scale), b = quant_code(f[4 * j + 1], scale),
+                  c = quant_code(f[4 * j + 2], scale), d = quant_code(f[4 * j + 3], scale);
+        dst[j * 32 + lane] = pack_codes4(a, b, c, d);
+        sum += a + b + c + d;
+    }
+    sum = block_sum_i<NW * 32>(sum, redi);
+    if (threadIdx.x == 0) {
+        s_x[m] = __fdiv_rn(eta, 127.0f);
+        rowsum[m] = sum;
+    }
+}
+
+}  // namespace tq

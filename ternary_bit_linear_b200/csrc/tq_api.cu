@@ -1,0 +1,444 @@
+// tq_api.cu -- the C ABI of libtq (declared in include/tq.h).
+//
+// Host side only: argument checks (before anything is enqueued), tensor-map
+// encoding for the TMA copies, launch configuration and dispatch.  All
+// arithmetic of the method runs in the kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "tq.h"
+#include "tq_act.cuh"
+#include "tq_common.cuh"
+#include "tq_gemm.cuh"
+#include "tq_gemv.cuh"
+#include "tq_pack.cuh"
+
+namespace {
+
+using namespace tq;
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxK = 65536;
+
+inline cudaStream_t cs(tq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+struct DeviceInfo {
+    int checked = 0;  // 0 unknown, 1 ok, -1 wrong arch
+    int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Current device must be compute capability 10.0 (sm_100a code only).
+tq_status check_device(int *sms_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return TQ_ERR_DEVICE;
+    DeviceInfo &d = g_dev[dev];
+    if (d.checked == 0) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (d.checked == 0) {
+            int maj = 0, min = 0, sms = 0;
+            if (cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&min, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return TQ_ERR_CUDA;
+            d.sms = sms;
+            d.checked = (maj == 10 && min == 0) ? 1 : -1;
+        }
+    }
+    if (d.checked < 0) return TQ_ERR_DEVICE;
+    if (sms_out) *sms_out = d.sms;
+    return TQ_OK;
+}
+
+inline tq_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+inline tq_status check_k(int64_t K) {
+    if (K < 64 || K > kMaxK || (K % 64) != 0) return TQ_ERR_SHAPE;
+    return TQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime, no -lcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load();
+    if (!f) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        f = reinterpret_cast<EncodeTiledFn>(p);
+        fn.store(f);
+    }
+    return f;
+}
+
+// 2-D uint8 tensor [rows][cols] (row stride = cols bytes), box [box_rows][box_cols].
+bool make_tmap_u8(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                  uint32_t box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Launch helpers
+// ---------------------------------------------------------------------------
+template <int BT>
+tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                      const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
+                      int64_t K, float *y, int32_t *acc, cudaStream_t st) {
+    using L = GemmLayout<BT>;
+    static std::atomic<int> attr_done[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev].load()) {
+        if (cudaFuncSetAttribute(gemm_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::kDynamic) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        attr_done[dev].store(1);
+    }
+    CUtensorMap tx, tw;
+    if (!make_tmap_u8(&tx, xq, (uint64_t)K, (uint64_t)M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_u8(&tw, packed, (uint64_t)(K / 4), (uint64_t)N, kTileK / 4, kTileN,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+        return TQ_ERR_CUDA;
+    dim3 grid((unsigned)((N + kTileN - 1) / kTileN), (unsigned)((M + BT - 1) / BT));
+    gemm_kernel<BT><<<grid, kGemmThreads, L::kDynamic, st>>>(tx, tw, s_x, rowsum, gamma, per_row,
+                                                              (int)M, (int)N, (int)K, y, acc);
+    return launch_status();
+}
+
+template <int NB, int MAXSTEP>
+tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                      const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
+                      int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
+    const int64_t nstrips = (N + 15) / 16;
+    static std::atomic<int> occ[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int per_sm = occ[dev].load();
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_kernel<NB, MAXSTEP>,
+                                                          kGemvWarps * 32, 0) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        if (per_sm < 1) per_sm = 1;
+        occ[dev].store(per_sm);
+    }
+    const int64_t grid = nstrips < (int64_t)per_sm * sms ? nstrips : (int64_t)per_sm * sms;
+    gemv_kernel<NB, MAXSTEP><<<(unsigned)grid, kGemvWarps * 32, 0, st>>>(
+        xq, s_x, rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc);
+    return launch_status();
+}
+
+template <int NW>
+void launch_prologue(const float *x, const ActParams &p, int64_t M, int8_t *xq, float *sx,
+                     int32_t *rs, cudaStream_t st) {
+    prologue_fwht_kernel<NW><<<(unsigned)M, NW * 32, 0, st>>>(x, p, xq, sx, rs);
+}
+
+typedef void (*PrologueFn)(const float *, const ActParams &, int64_t, int8_t *, float *, int32_t *,
+                           cudaStream_t);
+
+template <int... NWs>
+struct PrologueTable {
+    static constexpr PrologueFn fns[sizeof...(NWs)] = {&launch_prologue<NWs>...};
+};
+template <int... NWs>
+constexpr PrologueFn PrologueTable<NWs...>::fns[sizeof...(NWs)];
+using Prologues = PrologueTable<1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16, 17, 18, 19,
+                                20, 21, 22, 23, 24, 25, 26, 27, 28, 29, 30, 31, 32>;
+constexpr int64_t kMaxFwhtFusedK = 512 * 32;
+
+void launch_act(const float *x, const ActParams &p, int64_t M, int64_t K, int8_t *xq, float *sx,
+                int32_t *rs, cudaStream_t st) {
+    const int nv = (int)(K / 4);
+    const unsigned grid = (unsigned)M;
+    if (nv <= 256)
+        act_quant_kernel<1><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+    else if (nv <= 512)
+        act_quant_kernel<2><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+    else if (nv <= 1024)
+        act_quant_kernel<4><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+    else if (nv <= 2048)
+        act_quant_kernel<8><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+    else
+        act_quant_kernel<0><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+}
+
+size_t pack_parts(int64_t nv) {
+    const int64_t chunk_min = 4096;  // float4 per CTA, at least
+    int64_t chunk = (nv + 1183) / 1184;
+    if (chunk < chunk_min) chunk = chunk_min;
+    return (size_t)((nv + chunk - 1) / chunk);
+}
+
+tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                        const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
+                        int64_t N, int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
+    const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
+    if (M <= 16 && K <= kGemvMaxK) {
+        const int steps = (int)((K / 4 + 64 * kGemvWarps - 1) / (64 * kGemvWarps));
+        if (M <= 8) {
+            if (steps <= 1) return launch_gemv<1, 1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+            if (steps <= 2) return launch_gemv<1, 2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+            return launch_gemv<1, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+        }
+        if (steps <= 1) return launch_gemv<2, 1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+        if (steps <= 2) return launch_gemv<2, 2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+        return launch_gemv<2, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+    }
+    if (M <= 64) return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
+    if (M <= 128) return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
+    return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq_version(void) { return 100; }
+
+const char *tq_status_string(tq_status s) {
+    switch (s) {
+        case TQ_OK: return "ok";
+        case TQ_ERR_NULL: return "a required pointer is NULL";
+        case TQ_ERR_SHAPE: return "a size is out of range or breaks a divisibility rule";
+        case TQ_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case TQ_ERR_ARG: return "unknown flag, overlapping buffers, or workspace too small";
+        case TQ_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+        case TQ_ERR_DEVICE: return "the current device is not compute capability 10.0 (sm_100a)";
+        case TQ_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up";
+    }
+    return "unknown status";
+}
+
+size_t tq_pack_workspace_bytes(int64_t N, int64_t K, unsigned flags) {
+    if (flags & TQ_GAMMA_PER_ROW) return 0;
+    if (N <= 0 || K <= 0) return 0;
+    return pack_parts(N * K / 4) * sizeof(DD) + 16;
+}
+
+tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigned flags,
+                                   uint8_t *packed, float *gamma, void *workspace,
+                                   size_t workspace_bytes, tq_stream_t stream) {
+    if (!w || !packed || !gamma) return TQ_ERR_NULL;
+    if (N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE)) return TQ_ERR_ARG;
+    if (!aligned16(w) || !aligned16(packed) || !aligned16(gamma)) return TQ_ERR_ALIGN;
+    const bool per_row = flags & TQ_GAMMA_PER_ROW;
+    const size_t wbytes = (size_t)(N * K) * 4, pbytes = (size_t)(N * K / 4),
+                 gbytes = (per_row ? (size_t)N : 1) * 4;
+    if (overlap(w, wbytes, packed, pbytes) || overlap(w, wbytes, gamma, gbytes) ||
+        overlap(packed, pbytes, gamma, gbytes))
+        return TQ_ERR_ARG;
+    const size_t need = tq_pack_workspace_bytes(N, K, flags);
+    if (need) {
+        if (!workspace) return TQ_ERR_NULL;
+        if (!aligned16(workspace)) return TQ_ERR_ALIGN;
+        if (workspace_bytes < need) return TQ_ERR_ARG;
+        if (overlap(workspace, need, w, wbytes) || overlap(workspace, need, packed, pbytes) ||
+            overlap(workspace, need, gamma, gbytes))
+            return TQ_ERR_ARG;
+    }
+    if (tq_status e = check_device(nullptr)) return e;
+    const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
+    cudaStream_t st = cs(stream);
+    const int nv = (int)(K / 4);
+    auto rows = [&](const float *t, int reverse) {
+        const unsigned grid = (unsigned)N;
+        if (nv <= 256)
+            pack_rows_kernel<1><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+        else if (nv <= 512)
+            pack_rows_kernel<2><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+        else if (nv <= 1024)
+            pack_rows_kernel<4><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+        else if (nv <= 2048)
+            pack_rows_kernel<8><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+        else
+            pack_rows_kernel<0><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+    };
+    if (per_row) {
+        rows(nullptr, 0);
+        return launch_status();
+    }
+    const int64_t total_v = N * K / 4;
+    const size_t nparts = pack_parts(total_v);
+    const int64_t chunk = (total_v + (int64_t)nparts - 1) / (int64_t)nparts;
+    DD *partial = reinterpret_cast<DD *>(workspace);
+    float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + nparts * sizeof(DD));
+    absum_partial_kernel<<<(unsigned)nparts, kPackThreads, 0, st>>>(w, total_v, chunk, sanitize, partial);
+    absum_finalize_kernel<<<1, kPackThreads, 0, st>>>(partial, (int)nparts, (double)N * (double)K, gamma, thresh);
+    rows(thresh, 1);
+    return launch_status();
+}
+
+tq_status tq_quantize_act_int8(const float *x, int64_t M, int64_t K, unsigned flags, float eta_min,
+                               float eta_max, int8_t *xq, float *s_x, int32_t *rowsum,
+                               tq_stream_t stream) {
+    if (!x || !xq || !s_x || !rowsum) return TQ_ERR_NULL;
+    if (M < 1 || M > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (flags & ~(TQ_FLAG_ETA_CLAMP | TQ_FLAG_SANITIZE_NONFINITE)) return TQ_ERR_ARG;
+    if ((flags & TQ_FLAG_ETA_CLAMP) && !(eta_min > 0.0f && eta_min <= eta_max)) return TQ_ERR_ARG;
+    if ((flags & TQ_FLAG_SANITIZE_NONFINITE) && !(eta_max > 0.0f && eta_max < 3.0e38f)) return TQ_ERR_ARG;
+    if (!aligned16(x) || !aligned16(xq) || !aligned16(s_x) || !aligned16(rowsum)) return TQ_ERR_ALIGN;
+    const size_t xb = (size_t)(M * K) * 4, qb = (size_t)(M * K), mb = (size_t)M * 4;
+    if (overlap(x, xb, xq, qb) || overlap(x, xb, s_x, mb) || overlap(x, xb, rowsum, mb) ||
+        overlap(xq, qb, s_x, mb) || overlap(xq, qb, rowsum, mb) || overlap(s_x, mb, rowsum, mb))
+        return TQ_ERR_ARG;
+    if (tq_status e = check_device(nullptr)) return e;
+    ActParams p{};
+    p.sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
+    p.clamp_eta = (flags & TQ_FLAG_ETA_CLAMP) ? 1 : 0;
+    p.eta_min = eta_min;
+    p.eta_max = eta_max;
+    launch_act(x, p, M, K, xq, s_x, rowsum, cs(stream));
+    return launch_status();
+}
+
+tq_status tq_fwht512(const float *x, float *y, int64_t rows, int64_t K, int normalize,
+                     tq_stream_t stream) {
+    if (!x || !y) return TQ_ERR_NULL;
+    if (rows < 1 || K < 512 || K % 512 != 0 || K > kMaxK) return TQ_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(y)) return TQ_ERR_ALIGN;
+    const size_t b = (size_t)(rows * K) * 4;
+    if (x != y && overlap(x, b, y, b)) return TQ_ERR_ARG;
+    if (tq_status e = check_device(nullptr)) return e;
+    const int64_t nblocks = rows * (K / 512);
+    fwht512_kernel<<<(unsigned)((nblocks + 7) / 8), 256, 0, cs(stream)>>>(x, y, nblocks, normalize);
+    return launch_status();
+}
+
+tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                          const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
+                          int64_t N, int64_t K, float *y, int32_t *acc, tq_stream_t stream) {
+    if (!xq || !s_x || !rowsum || !packed || !gamma || !y) return TQ_ERR_NULL;
+    if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (flags & ~TQ_GAMMA_PER_ROW) return TQ_ERR_ARG;
+    if (!aligned16(xq) || !aligned16(s_x) || !aligned16(rowsum) || !aligned16(packed) ||
+        !aligned16(gamma) || !aligned16(y) || (acc && !aligned16(acc)))
+        return TQ_ERR_ALIGN;
+    const size_t yb = (size_t)(M * N) * 4;
+    const size_t gb = ((flags & TQ_GAMMA_PER_ROW) ? (size_t)N : 1) * 4;
+    const void *ins[5] = {xq, s_x, rowsum, packed, gamma};
+    const size_t inb[5] = {(size_t)(M * K), (size_t)M * 4, (size_t)M * 4, (size_t)(N * K / 4), gb};
+    for (int i = 0; i < 5; ++i)
+        if (overlap(ins[i], inb[i], y, yb) || (acc && overlap(ins[i], inb[i], acc, yb))) return TQ_ERR_ARG;
+    if (acc && overlap(acc, yb, y, yb)) return TQ_ERR_ARG;
+    int sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    return gemm_dispatch(xq, s_x, rowsum, packed, gamma, flags, M, N, K, y, acc, sms, cs(stream));
+}
+
+size_t tq_fused_workspace_bytes(int64_t M, int64_t K, unsigned flags) {
+    (void)flags;
+    if (M <= 0 || K <= 0) return 0;
+    const size_t xq = ((size_t)(M * K) + 255) & ~(size_t)255;
+    const size_t v = (((size_t)M * 4) + 255) & ~(size_t)255;
+    return xq + 2 * v;
+}
+
+tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_eps, float eta_min,
+                             float eta_max, unsigned flags, const uint8_t *packed,
+                             const float *gamma, int64_t M, int64_t N, int64_t K, float *y,
+                             int8_t *xq_out, float *s_x_out, void *workspace,
+                             size_t workspace_bytes, tq_stream_t stream) {
+    if (!x || !packed || !gamma || !y || !workspace) return TQ_ERR_NULL;
+    if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    const unsigned known = TQ_GAMMA_PER_ROW | TQ_FLAG_FWHT | TQ_FLAG_RMSNORM | TQ_FLAG_ETA_CLAMP |
+                           TQ_FLAG_SANITIZE_NONFINITE;
+    if (flags & ~known) return TQ_ERR_ARG;
+    if ((flags & TQ_FLAG_FWHT) && (K % 512 != 0 || K > kMaxFwhtFusedK)) return TQ_ERR_SHAPE;
+    if ((flags & TQ_FLAG_ETA_CLAMP) && !(eta_min > 0.0f && eta_min <= eta_max)) return TQ_ERR_ARG;
+    if ((flags & TQ_FLAG_SANITIZE_NONFINITE) && !(eta_max > 0.0f && eta_max < 3.0e38f)) return TQ_ERR_ARG;
+    if ((flags & TQ_FLAG_RMSNORM) && !(rms_eps >= 0.0f)) return TQ_ERR_ARG;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(gamma) || !aligned16(y) ||
+        !aligned16(workspace) || (rms_gain && !aligned16(rms_gain)) || (xq_out && !aligned16(xq_out)) ||
+        (s_x_out && !aligned16(s_x_out)))
+        return TQ_ERR_ALIGN;
+    const size_t need = tq_fused_workspace_bytes(M, K, flags);
+    if (workspace_bytes < need) return TQ_ERR_ARG;
+    const size_t xb = (size_t)(M * K) * 4, yb = (size_t)(M * N) * 4, qb = (size_t)(M * K),
+                 pb = (size_t)(N * K / 4), gb = ((flags & TQ_GAMMA_PER_ROW) ? (size_t)N : 1) * 4;
+    const void *outs[4] = {y, workspace, xq_out, s_x_out};
+    const size_t outb[4] = {yb, need, qb, (size_t)M * 4};
+    const void *ins[4] = {x, packed, gamma, rms_gain};
+    const size_t inb[4] = {xb, pb, gb, (size_t)K * 4};
+    for (int o = 0; o < 4; ++o) {
+        if (!outs[o]) continue;
+        for (int i = 0; i < 4; ++i)
+            if (ins[i] && overlap(outs[o], outb[o], ins[i], inb[i])) return TQ_ERR_ARG;
+        for (int o2 = o + 1; o2 < 4; ++o2)
+            if (outs[o2] && overlap(outs[o], outb[o], outs[o2], outb[o2])) return TQ_ERR_ARG;
+    }
+    int sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    cudaStream_t st = cs(stream);
+
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    const size_t xq_sz = ((size_t)(M * K) + 255) & ~(size_t)255;
+    const size_t v_sz = (((size_t)M * 4) + 255) & ~(size_t)255;
+    int8_t *xq = xq_out ? xq_out : reinterpret_cast<int8_t *>(ws);
+    float *sx = s_x_out ? s_x_out : reinterpret_cast<float *>(ws + xq_sz);
+    int32_t *rs = reinterpret_cast<int32_t *>(ws + xq_sz + v_sz);
+
+    ActParams p{};
+    p.sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
+    p.clamp_eta = (flags & TQ_FLAG_ETA_CLAMP) ? 1 : 0;
+    p.eta_min = eta_min;
+    p.eta_max = eta_max;
+    p.rmsnorm = (flags & TQ_FLAG_RMSNORM) ? 1 : 0;
+    p.rms_eps = rms_eps;
+    p.rms_gain = rms_gain;
+    if (flags & TQ_FLAG_FWHT)
+        Prologues::fns[K / 512 - 1](x, p, M, xq, sx, rs, st);
+    else
+        launch_act(x, p, M, K, xq, sx, rs, st);
+    if (tq_status e = launch_status()) return e;
+    return gemm_dispatch(xq, sx, rs, packed, gamma, flags & TQ_GAMMA_PER_ROW, M, N, K, y, nullptr,
+                         sms, st);
+}
+
+tq_status tq_get_device_status(tq_stream_t stream) {
+    if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return TQ_ERR_CUDA;
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, tq::g_status, sizeof v) != cudaSuccess) return TQ_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(tq::g_status, &zero, sizeof zero) != cudaSuccess) return TQ_ERR_CUDA;
+    return (v & tq::kStatusTimeout) ? TQ_ERR_TIMEOUT : TQ_OK;
+}
+
+}  // extern "C"

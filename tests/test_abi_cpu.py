@@ -1,0 +1,106 @@
+"""CPU-side checks of the C ABI: the library builds, loads and exports every
+entry point include/tq.h declares, and argument validation rejects bad calls
+with the documented status before touching the device (fake, never
+dereferenced pointers; no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ternary_bit_linear_b200 as tq
+from ternary_bit_linear_b200 import build as tqbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "tq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tqbuild.build()
+    return tq.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"TQ_API\s+[\w\s\*]+?\b(tq_\w+)\s*\(", src)
+
+
+def test_header_declares_the_five_calls_and_helpers():
+    names = set(declared_functions())
+    for n in ["tq_quantize_ternary_pack", "tq_quantize_act_int8", "tq_fwht512",
+              "tq_ternary_gemm", "tq_bitlinear_fused"]:
+        assert n in names
+    assert names == set(tq.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert lib.tq_version() == 100
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert lib.tq_status_string(code)
+    assert b"unknown" in lib.tq_status_string(99)
+
+
+def test_workspace_sizes(lib):
+    assert lib.tq_pack_workspace_bytes(4096, 4096, tq.GAMMA_PER_ROW) == 0
+    n = lib.tq_pack_workspace_bytes(11008, 4096, 0)
+    assert n >= 16 + 16 and n < 1 << 20
+    assert lib.tq_fused_workspace_bytes(512, 2048, tq.FLAG_FWHT) >= 512 * 2048 + 2 * 512 * 4
+
+
+FAKE = 0x10000000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def P(off=0):
+    return ctypes.c_void_p(FAKE + off)
+
+
+def test_pack_validation(lib):
+    f = lib.tq_quantize_ternary_pack
+    assert f(None, 4, 64, 1, P(), P(1 << 20), None, 0, None) == 1            # NULL
+    assert f(P(), 4, 60, 1, P(1 << 20), P(2 << 20), None, 0, None) == 2      # K % 64
+    assert f(P(), 0, 64, 1, P(1 << 20), P(2 << 20), None, 0, None) == 2      # N = 0
+    assert f(P(4), 4, 64, 1, P(1 << 20), P(2 << 20), None, 0, None) == 3     # misaligned
+    assert f(P(), 4, 64, 1 << 7, P(1 << 20), P(2 << 20), None, 0, None) == 4  # unknown flag
+    assert f(P(), 4, 64, 1, P(16), P(2 << 20), None, 0, None) == 4           # overlap w/packed
+    assert f(P(), 4, 64, 0, P(1 << 20), P(2 << 20), None, 0, None) == 1      # needs workspace
+    assert f(P(), 4, 64, 0, P(1 << 20), P(2 << 20), P(3 << 20), 8, None) == 4  # too small
+
+
+def test_act_and_fwht_validation(lib):
+    f = lib.tq_quantize_act_int8
+    assert f(P(), 2, 64, 0, 0.05, 40.0, P(1 << 20), P(2 << 20), None, None) == 1
+    assert f(P(), 2, 96, 0, 0.05, 40.0, P(1 << 20), P(2 << 20), P(3 << 20), None) == 2
+    assert f(P(), 2, 64, tq.FLAG_ETA_CLAMP, 0.0, 40.0, P(1 << 20), P(2 << 20), P(3 << 20), None) == 4
+    assert f(P(), 2, 64, 0, 0.05, 40.0, P(112), P(2 << 20), P(3 << 20), None) == 4  # overlap
+    g = lib.tq_fwht512
+    assert g(P(), P(1 << 20), 2, 1000, 1, None) == 2
+    assert g(P(), P(16), 2, 512, 1, None) == 4  # partial overlap (in place is allowed)
+
+
+def test_gemm_and_fused_validation(lib):
+    f = lib.tq_ternary_gemm
+    args = [P(), P(1 << 20), P(2 << 20), P(3 << 20), P(4 << 20), 0, 8, 8, 64, P(5 << 20), None, None]
+    bad = list(args)
+    bad[5] = 4
+    assert f(*bad) == 4
+    bad = list(args)
+    bad[8] = 32
+    assert f(*bad) == 2
+    bad = list(args)
+    bad[9] = P(16)  # y overlaps x_q
+    assert f(*bad) == 4
+    bad = list(args)
+    bad[2] = None
+    assert f(*bad) == 1
+    h = lib.tq_bitlinear_fused
+    fused = [P(), None, 1e-6, 0.05, 40.0, tq.FLAG_FWHT, P(1 << 20), P(2 << 20), 4, 8, 640,
+             P(3 << 20), None, None, P(4 << 20), 1 << 20, None]
+    assert h(*fused) == 2  # FWHT needs K % 512 == 0
+    fused[10] = 512
+    fused[15] = 16
+    assert h(*fused) == 4  # workspace too small

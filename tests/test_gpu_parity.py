@@ -1,0 +1,361 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bars (from the method's contract):
+  * packed bytes, gamma, int8 codes, s_x, rowsum, int32 accumulators and the
+    FWHT output: bit-exact;
+  * fp32 outputs y: max relative error 1e-5;
+  * after the fused RMSNorm + FWHT prologue: int8 codes within 1 LSB on at most
+    1e-4 of the elements (the RMSNorm sum of squares is reduced in a different
+    order than the oracle's).
+Oracle-side inputs (packed weights, x_q) are produced by the oracle and fed to
+the GPU kernels that consume them; nothing produced by the GPU is fed to the
+oracle.
+"""
+import functools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from ternary_bit_linear_b200 import synthetic as S
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+REL = 1e-5
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def assert_y_close(y, y_ref):
+    y, y_ref = np.asarray(y, np.float64), np.asarray(y_ref, np.float64)
+    zero = y_ref == 0
+    assert np.all(y[zero] == 0), "y must be exactly 0 where acc == 0"
+    rel = np.abs(y[~zero] - y_ref[~zero]) / np.abs(y_ref[~zero])
+    assert rel.size == 0 or rel.max() <= REL, f"max rel err {rel.max():.3e}"
+
+
+@functools.lru_cache(maxsize=None)
+def cached(name, *args):
+    return getattr(S, name)(*args)
+
+
+# ---------------------------------------------------------------------------
+# quantise + pack
+# ---------------------------------------------------------------------------
+
+PACK_SHAPES = [(1, 64), (3, 192), (17, 512), (129, 4160), (64, 8192), (5, 8256), (2, 65536)]
+
+
+@pytest.mark.parametrize("N,K", PACK_SHAPES)
+@pytest.mark.parametrize("per_row", [True, False])
+def test_pack_matches_oracle(cuda_lib, N, K, per_row):
+    W = S.normal((N, K), 0.02, 7, 100 + N)
+    if N > 2:
+        W[1] = S.laplace((K,), 0.05, 7, 200 + N)
+        W[2] = 0.0  # all-zero row: gamma -> 1e-6, all codes 0
+    packed, gamma = cuda_lib.quantize_ternary_pack(dev(W), per_row=per_row)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row)
+    assert np.array_equal(host(gamma), g_ref)
+    assert np.array_equal(host(packed), p_ref)
+
+
+def test_pack_sanitize_nonfinite(cuda_lib):
+    W = S.normal((8, 512), 0.02, 3, 31)
+    W[0, 0], W[1, 7], W[2, 9], W[5, 511] = np.nan, np.inf, -np.inf, np.nan
+    for per_row in (True, False):
+        packed, gamma = cuda_lib.quantize_ternary_pack(dev(W), per_row=per_row, sanitize=True)
+        p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row, sanitize=True)
+        assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
+
+
+def test_pack_exact_ties():
+    import ternary_bit_linear_b200 as tq
+
+    u23 = np.float32(2.0 ** -23)
+    rows = []
+    base = np.tile(np.array([1.0, -1.0], np.float32), 30)
+    # gamma = 1 exactly: ties at 0.5 and 1.5, then just above 0.5 (paired so the mean stays 1)
+    rows.append(np.concatenate([[0.5, -0.5, 1.5, -1.5], base]))
+    rows.append(np.concatenate([[0.5 + u23, -(0.5 + u23), 1.5 - u23, -(1.5 - u23)], base]))
+    # gamma = 0.75 exactly: tie at 0.375, just above at 0.375 + 2^-23
+    base75 = np.tile(np.array([0.75, -0.75], np.float32), 30)
+    rows.append(np.concatenate([[0.375, -0.375, 1.125, -1.125], base75]))
+    rows.append(np.concatenate([[0.375 + u23, -(0.375 + u23), 1.125 - u23, -(1.125 - u23)], base75]))
+    W = np.array(rows, np.float32)
+    packed, gamma = tq.quantize_ternary_pack(dev(W), per_row=True)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=True)
+    assert g_ref.tolist() == [1.0, 1.0, 0.75, 0.75]
+    q_ref, _ = oracle.unpack(p_ref, 64)
+    assert q_ref[:, :4].tolist() == [[0, 0, 1, -1], [1, -1, 1, -1], [0, 0, 1, -1], [1, -1, 1, -1]]
+    assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
+
+
+def test_pack_dense_threshold_sweep(cuda_lib):
+    # Row r: one probe value w_r followed by 63 entries of +-1.  Its gamma is
+    # (|w_r| + 63) / 64, and w_r / gamma crosses 0.5 at w_r = 63/127.  4096
+    # consecutive fp32 probes around that point (and their negatives) exercise
+    # the exact rounding boundary of the code decision.
+    centre = np.float32(63.0 / 127.0)
+    bits = centre.view(np.int32) + np.arange(-2048, 2048, dtype=np.int32)
+    probes = bits.view(np.float32)
+    probes = np.concatenate([probes, -probes])
+    filler = np.tile(np.array([1.0, -1.0], np.float32), 32)[:63]
+    W = np.concatenate([probes[:, None], np.tile(filler, (probes.size, 1))], axis=1).astype(np.float32)
+    packed, gamma = cuda_lib.quantize_ternary_pack(dev(W), per_row=True)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=True)
+    q_ref, _ = oracle.unpack(p_ref, 64)
+    assert 0 < (q_ref[:, 0] != 0).sum() < probes.size  # the sweep straddles the boundary
+    assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
+
+
+@pytest.mark.parametrize("which", ["decode", "prefill", "fused", "sweep"])
+def test_pack_full_size(cuda_lib, which):
+    if which == "decode":
+        W, per_row = cached("decode_weights", 4096, 4096), True
+    elif which == "prefill":
+        W, per_row = cached("prefill", 2048, 11008, 4096)[0], False
+    elif which == "fused":
+        W, per_row = cached("fused", 512, 5632, 2048)[0], False
+    else:
+        W, per_row = cached("sweep_weights", 8192, 8192), True
+    packed, gamma = cuda_lib.quantize_ternary_pack(dev(W), per_row=per_row)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row)
+    assert np.array_equal(host(gamma), g_ref)
+    assert np.array_equal(host(packed), p_ref)
+
+
+# ---------------------------------------------------------------------------
+# activation quantisation and FWHT
+# ---------------------------------------------------------------------------
+
+ACT_SHAPES = [(1, 64), (3, 192), (4, 512), (8, 4096), (17, 4160), (2, 8192), (5, 8256), (3, 65536)]
+
+
+@pytest.mark.parametrize("M,K", ACT_SHAPES)
+@pytest.mark.parametrize("clamp", [False, True])
+def test_act_quant_matches_oracle(cuda_lib, M, K, clamp):
+    X = S.decode_acts(M, K, seed=11)
+    if M > 2:
+        X[1] = 0.0  # zero token
+        X[2] *= np.float32(1e-4)  # tiny token (eta clamp lower bound when clamping)
+    xq, sx, rs = cuda_lib.quantize_act_int8(dev(X), clamp_eta=clamp)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X, clamp_eta=clamp)
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(sx), sx_ref)
+    assert np.array_equal(host(rs), rs_ref)
+
+
+def test_act_quant_golden_ties_and_sanitize(cuda_lib):
+    x = np.zeros((2, 64), np.float32)
+    x[0, :8] = [1.0, 0.5, -0.5, 0.25, 0.125, -1.0, 0.0, 0.75]
+    x[1] = S.normal((64,), 1.0, 1, 5)
+    x[1, 3], x[1, 9], x[1, 10] = np.nan, np.inf, -np.inf
+    xq, sx, rs = cuda_lib.quantize_act_int8(dev(x), sanitize=True, eta_max=40.0)
+    xs = oracle.sanitize_acts(x, 40.0)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(xs)
+    assert xq_ref[0, :8].tolist() == [127, 64, -64, 32, 16, -127, 0, 95]
+    assert np.array_equal(host(xq), xq_ref) and np.array_equal(host(sx), sx_ref)
+    assert np.array_equal(host(rs), rs_ref)
+
+
+def test_act_quant_prefill_full_size(cuda_lib):
+    X = cached("prefill", 2048, 11008, 4096)[1]
+    xq, sx, rs = cuda_lib.quantize_act_int8(dev(X))
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    assert np.array_equal(host(xq), xq_ref) and np.array_equal(host(sx), sx_ref)
+    assert np.array_equal(host(rs), rs_ref)
+
+
+@pytest.mark.parametrize("rows,K", [(1, 512), (8, 1536), (33, 2048), (4, 8192), (3, 65536)])
+@pytest.mark.parametrize("normalize", [True, False])
+def test_fwht_bit_exact(cuda_lib, rows, K, normalize):
+    X = S.student_t3((rows, K), 2, 40 + rows)
+    y = cuda_lib.fwht512(dev(X), normalize=normalize)
+    assert np.array_equal(host(y), oracle.fwht512(X, normalize=normalize))
+
+
+def test_fwht_in_place_and_spike(cuda_lib):
+    x = np.zeros((1, 512), np.float32)
+    x[0, 256] = 100.0
+    t = dev(x)
+    cuda_lib.fwht512_(t, t, True)
+    y = host(t)
+    assert np.array_equal(y, oracle.fwht512(x))
+    assert abs(np.abs(y).max() - 100.0 / math.sqrt(512.0)) < 1e-4
+
+
+# ---------------------------------------------------------------------------
+# contraction (GEMV for M <= 16, tcgen05 GEMM above)
+# ---------------------------------------------------------------------------
+
+def run_gemm(tq, W, X, per_row):
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    y, acc = tq.ternary_gemm(dev(xq_ref), dev(sx_ref), dev(rs_ref), dev(p_ref), dev(g_ref),
+                             per_row=per_row, with_acc=True)
+    return host(y), host(acc), (p_ref, g_ref, xq_ref, sx_ref)
+
+
+GEMM_CASES = [
+    # GEMV (M <= 16)
+    (1, 1, 64), (1, 17, 192), (2, 128, 512), (3, 129, 1088), (5, 200, 4096), (8, 384, 4160),
+    (9, 64, 8192), (15, 33, 2048), (16, 256, 4096), (16, 31, 8192), (1, 4096, 4096),
+    # tcgen05 GEMM
+    (17, 128, 512), (33, 130, 640), (64, 256, 1024), (65, 129, 4096), (100, 17, 192),
+    (128, 384, 2048), (129, 128, 64), (255, 200, 1088), (256, 256, 4096), (300, 384, 1536),
+    (513, 257, 512), (12, 128, 8256), (1000, 1, 128),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+@pytest.mark.parametrize("per_row", [True, False])
+def test_gemm_matches_oracle(cuda_lib, M, N, K, per_row):
+    W = S.normal((N, K), 0.02, 5, 1000 + N)
+    X = S.decode_acts(M, K, seed=6)
+    y, acc, (p_ref, g_ref, xq_ref, sx_ref) = run_gemm(cuda_lib, W, X, per_row)
+    acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
+    assert np.array_equal(acc, acc_ref)
+    assert_y_close(y, oracle.dequant(acc_ref, g_ref, sx_ref, per_row))
+
+
+def test_gemm_extreme_codes(cuda_lib):
+    # all +1 / all -1 / all 0 weight rows and +-127 activations: |acc| = 127*K
+    K, N, M = 4096, 130, 40
+    W = np.zeros((N, K), np.float32)
+    W[0::3] = 1.0
+    W[1::3] = -1.0
+    X = np.where(S.normal((M, K), 1.0, 1, 9) > 0, 1.0, -1.0).astype(np.float32)
+    X[0] = 1.0
+    for m_sub in (M, 4):  # tcgen05 GEMM and GEMV
+        y, acc, (p_ref, g_ref, xq_ref, sx_ref) = run_gemm(cuda_lib, W, X[:m_sub], True)
+        acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
+        assert acc_ref[0, 0] == 127 * K
+        assert np.array_equal(acc, acc_ref)
+        assert_y_close(y, oracle.dequant(acc_ref, g_ref, sx_ref, True))
+
+
+def sampled_gemm_check(tq, W, X, per_row, sample):
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    y, acc = tq.ternary_gemm(dev(xq_ref), dev(sx_ref), dev(rs_ref), dev(p_ref), dev(g_ref),
+                             per_row=per_row, with_acc=True)
+    y, acc = host(y), host(acc)
+    acc_ref = oracle.matmul_addsub(xq_ref[sample], p_ref)
+    assert np.array_equal(acc[sample], acc_ref)
+    assert_y_close(y[sample], oracle.dequant(acc_ref, g_ref, sx_ref[sample], per_row))
+    # every row (sampled or not) obeys the rescale identity exactly in fp32 terms
+    g = g_ref if per_row else np.full(W.shape[0], g_ref[0], np.float32)
+    y_from_acc = acc.astype(np.float32) * (g[None, :] * sx_ref[:, None])
+    assert np.array_equal(y, y_from_acc.astype(np.float32))
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_decode_full_size(cuda_lib, M):
+    W = cached("decode_weights", 4096, 4096)
+    X = S.decode_acts(M, 4096, seed=0)
+    sampled_gemm_check(cuda_lib, W, X, True, np.arange(M))
+
+
+def test_prefill_full_size_sampled(cuda_lib):
+    W, X = cached("prefill", 2048, 11008, 4096)
+    sampled_gemm_check(cuda_lib, W, X, False, np.arange(0, 2048, 97))
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 64, 512, 4096])
+def test_sweep_full_size_sampled(cuda_lib, M):
+    W = cached("sweep_weights", 8192, 8192)
+    X = S.sweep_acts(M, 8192, seed=0)
+    sample = np.arange(M) if M <= 16 else np.unique(np.r_[0, np.arange(3, M, max(1, M // 12)), M - 1])
+    sampled_gemm_check(cuda_lib, W, X, True, sample)
+
+
+# ---------------------------------------------------------------------------
+# fused layer
+# ---------------------------------------------------------------------------
+
+def check_fused(tq, X, W, per_row, sample=None, **kw):
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row)
+    okw = dict(kw)
+    for k in ("return_xq",):
+        okw.pop(k, None)
+    rmsnorm = okw.pop("rmsnorm", True)
+    fwht = okw.pop("fwht", True)
+    gain = okw.get("rms_gain")
+    y, xq, sx = tq.bitlinear_fused(dev(X), dev(p_ref), dev(g_ref), per_row=per_row,
+                                   rmsnorm=rmsnorm, fwht=fwht, return_xq=True,
+                                   **{k: (dev(v) if k == "rms_gain" and v is not None else v)
+                                      for k, v in okw.items()})
+    y, xq, sx = host(y), host(xq), host(sx)
+    rows = np.arange(X.shape[0]) if sample is None else sample
+    y_ref, xq_ref, sx_ref, acc_ref = oracle.bitlinear(X[rows], p_ref, g_ref, per_row,
+                                                      use_rmsnorm=rmsnorm, use_fwht=fwht, **okw)
+    d = np.abs(xq[rows].astype(np.int32) - xq_ref.astype(np.int32))
+    assert d.max() <= 1
+    assert (d != 0).sum() <= 1e-4 * d.size
+    rel_sx = np.abs(sx[rows] - sx_ref) / sx_ref
+    assert rel_sx.max() <= REL
+    flips = (d != 0).sum(axis=1)
+    if flips.sum() == 0 and np.array_equal(sx[rows], sx_ref):
+        assert_y_close(y[rows], y_ref)
+    else:  # a flipped code moves acc by at most 1 per flip
+        g = g_ref if per_row else np.full(W.shape[0], g_ref[0], np.float32)
+        bound = flips[:, None] * g[None, :] * sx_ref[:, None] * (1 + 1e-5) + REL * np.abs(y_ref) \
+            + np.abs(y_ref) * rel_sx[:, None]
+        assert np.all(np.abs(y[rows] - y_ref) <= bound)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 64, 512), (3, 300, 1536), (16, 128, 2048), (17, 200, 1024),
+                                   (200, 130, 512), (40, 64, 8192)])
+def test_fused_matches_oracle(cuda_lib, M, N, K):
+    W = S.normal((N, K), 0.02, 9, N)
+    X = S.student_t3((M, K), 9, 7)
+    check_fused(cuda_lib, X, W, False)
+
+
+@pytest.mark.parametrize("variant", ["no_rms", "no_fwht", "plain", "gain", "clamp", "sanitize",
+                                     "per_row"])
+def test_fused_variants(cuda_lib, variant):
+    M, N, K = 20, 96, 1024
+    W = S.normal((N, K), 0.02, 10, 1)
+    X = S.student_t3((M, K), 10, 2)
+    kw = {}
+    per_row = False
+    if variant == "no_rms":
+        kw["rmsnorm"] = False
+    elif variant == "no_fwht":
+        kw["fwht"] = False
+    elif variant == "plain":
+        kw.update(rmsnorm=False, fwht=False)
+        K2 = 640
+        W, X = W[:, :K2].copy(), X[:, :K2].copy()
+    elif variant == "gain":
+        kw["rms_gain"] = S.normal((K,), 1.0, 10, 3)
+    elif variant == "clamp":
+        kw["clamp_eta"] = True
+        X[3] *= np.float32(1e-3)
+        X[4] *= np.float32(500.0)
+    elif variant == "sanitize":
+        kw["sanitize"] = True
+        X[0, 1], X[2, 5], X[7, 1023] = np.nan, np.inf, -np.inf
+    elif variant == "per_row":
+        per_row = True
+    check_fused(cuda_lib, X, W, per_row, **kw)
+
+
+def test_fused_full_size(cuda_lib):
+    W, X = cached("fused", 512, 5632, 2048)
+    check_fused(cuda_lib, X, W, False, sample=np.arange(0, 512, 37))
+
+
+def test_device_status_clean(cuda_lib):
+    assert cuda_lib.device_status() == 0
