@@ -338,17 +338,31 @@ def run_ours(args, rank, world, local_rank):
     del graphs
 
 
+WORKLOAD_SHAPES = {  # name -> (Ms, N, K, layers, per_row)
+    "decode": ([1, 8], 4096, 4096, 64, True),
+    "prefill": ([2048], 11008, 4096, 1, False),
+    "fused": ([512], 5632, 2048, 1, False),
+    "sweep": ([1, 4, 16, 64, 512, 4096], 8192, 8192, 1, True),
+}
+
+
+def config_for(name, layers, world):
+    Ms, N, K, L, per_row = WORKLOAD_SHAPES[name]
+    if name == "decode":
+        L = layers
+    desc = {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers" % L,
+            "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma",
+            "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512",
+            "sweep": "M sweep over K=N=8192, per-row gamma"}[name]
+    return {"workload": desc, "M": Ms, "N": N, "K": K, "layers": L,
+            "gamma": "per-row" if per_row else "per-tensor",
+            "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
+                L * N * K * 4 >> 20, L * N * K // 4 >> 20),
+            "parallelism": "replicas x%d" % world if world > 1 else "single GPU"}
+
+
 def wl_config(wl, world):
-    c = {"workload": {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers" % wl.L,
-                      "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma",
-                      "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512",
-                      "sweep": "M sweep over K=N=8192, per-row gamma"}[wl.name],
-         "M": wl.Ms, "N": wl.N, "K": wl.K, "layers": wl.L,
-         "gamma": "per-row" if wl.per_row else "per-tensor",
-         "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
-             wl.L * wl.N * wl.K * 4 >> 20, wl.L * wl.N * wl.K // 4 >> 20),
-         "parallelism": "replicas x%d" % world if world > 1 else "single GPU"}
-    return c
+    return config_for(wl.name, wl.L, world)
 
 
 def run_e2e(args, wl, tq, torch, stream, graphs, world):
@@ -468,7 +482,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic", "config": {"workload": args.workload, "sample": what},
+        "data": "synthetic", "config": dict(config_for(args.workload, args.layers, world), sample=what),
         "cpu_baseline": {"value": round(v, 6), "unit": unit, "cores": 1, "kind": "oracle",
                          "sample": what + " per step"},
         "e2e": {"value": round(v, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

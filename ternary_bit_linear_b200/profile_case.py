@@ -1,0 +1,63 @@
+"""Run one kernel of the hot path a few times on a chosen shape -- the small,
+self-contained command that ncu captures are taken on.
+
+    python -m ternary_bit_linear_b200.profile_case --kernel gemv --M 8 --N 4096 --K 4096 --reps 3
+
+Inputs are random device tensors of the workloads' distributions (values do
+not affect timing); every call goes through the C ABI.  Exits non-zero if a
+call fails or the device status word reports a timeout.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+import ternary_bit_linear_b200 as tq
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", required=True,
+                    choices=["pack_row", "pack_tensor", "act", "fwht", "gemv", "gemm", "fused"])
+    ap.add_argument("--M", type=int, default=8)
+    ap.add_argument("--N", type=int, default=4096)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args()
+    tq.load()
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    M, N, K = a.M, a.N, a.K
+    W = torch.randn((N, K), generator=g, device=dev) * 0.02
+    X = torch.randn((M, K), generator=g, device=dev)
+    per_row = a.kernel != "pack_tensor"
+    packed, gamma = tq.quantize_ternary_pack(W, per_row=per_row)
+    xq, sx, rs = tq.quantize_act_int8(X)
+    y = torch.empty((M, N), device=dev)
+    flags = tq.GAMMA_PER_ROW if per_row else 0
+    ws = torch.empty((max(16, tq.fused_workspace_bytes(M, K, tq.FLAG_FWHT | tq.FLAG_RMSNORM)),),
+                     dtype=torch.uint8, device=dev)
+    pws = torch.empty((max(16, tq.pack_workspace_bytes(N, K, flags)),), dtype=torch.uint8, device=dev)
+    Xr = torch.empty_like(X)
+    torch.cuda.synchronize()
+    for _ in range(a.reps):
+        if a.kernel in ("pack_row", "pack_tensor"):
+            tq.quantize_ternary_pack_(W, flags, packed, gamma, pws)
+        elif a.kernel == "act":
+            tq.quantize_act_int8_(X, 0, 0.05, 40.0, xq, sx, rs)
+        elif a.kernel == "fwht":
+            tq.fwht512_(X, Xr)
+        elif a.kernel in ("gemv", "gemm"):
+            tq.ternary_gemm_(xq, sx, rs, packed, gamma, flags, y)
+        else:
+            tq.bitlinear_fused_(X, packed, gamma, tq.FLAG_FWHT | tq.FLAG_RMSNORM, y, ws)
+    torch.cuda.synchronize()
+    st = tq.device_status()
+    if st != 0:
+        raise SystemExit(f"device status {st}")
+    print(f"{a.kernel} M={M} N={N} K={K} reps={a.reps} ok")
+
+
+if __name__ == "__main__":
+    main()
