@@ -104,6 +104,30 @@ TQ_API tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, 
 TQ_API size_t tq_pack_workspace_bytes(int64_t N, int64_t K, unsigned flags);
 
 /*
+ * Same result as tq_quantize_ternary_pack, for callers that cannot allocate
+ * device memory (a runtime whose allocator owns all of HBM and refuses new
+ * reservations, a host that only receives device pointers, or a path where a
+ * cudaMalloc and the synchronisation it may cause are not allowed).  It takes
+ * no workspace: the per-tensor partial sums live in a fixed ~32 KB array inside
+ * the library, held on every GPU that loads it until the process exits.  The
+ * pages have no counterpart of this entry point; it only moves scratch memory.
+ *
+ *   w, N, K, flags, packed, gamma, stream: as for tq_quantize_ternary_pack.
+ *   Limit: with per-tensor gamma, N * K <= 134,217,728 weights (2048 partial
+ *   sums of 65,536 weights); larger calls return TQ_ERR_SHAPE and launch
+ *   nothing.  Per-row gamma uses no scratch and has no extra limit.
+ *   Sharing: every call uses the same array, so calls whose work overlaps on the
+ *   GPU (e.g. on two streams at once) race; serialise them.  Each call writes
+ *   the scratch before reading it, so nothing needs clearing between calls.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before capturing work into a CUDA graph.
+ */
+TQ_API tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N, int64_t K,
+                                                  unsigned flags, uint8_t *packed, float *gamma,
+                                                  tq_stream_t stream);
+
+/*
  * Per-token symmetric int8 quantisation.
  * Hetman-2b section 2 SymmetricActivationQuantizer.forward (reduction over the
  * last dimension); s_x = eta / 127 is the scale the output is multiplied by.

@@ -32,6 +32,7 @@ _P, _I64, _U, _F, _I, _SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint, cty
 SIGNATURES = {
     "tq_quantize_ternary_pack": (_I, [_P, _I64, _I64, _U, _P, _P, _P, _SZ, _P]),
     "tq_pack_workspace_bytes": (_SZ, [_I64, _I64, _U]),
+    "tq_quantize_ternary_pack_noalloc": (_I, [_P, _I64, _I64, _U, _P, _P, _P]),
     "tq_quantize_act_int8": (_I, [_P, _I64, _I64, _U, _F, _F, _P, _P, _P, _P]),
     "tq_fwht512": (_I, [_P, _P, _I64, _I64, _I, _P]),
     "tq_ternary_gemm": (_I, [_P, _P, _P, _P, _P, _U, _I64, _I64, _I64, _P, _P, _P]),

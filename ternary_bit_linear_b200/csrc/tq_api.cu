@@ -442,3 +442,113 @@ tq_status tq_get_device_status(tq_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free variant of tq_quantize_ternary_pack.
+//
+// Per-tensor gamma needs scratch for the partial sums of |w|; the regular entry
+// point takes it from the caller.  Some callers cannot provide it: a runtime
+// whose allocator has reserved all device memory up front and forbids new
+// reservations, a host that only holds device pointers handed to it by someone
+// else and has no allocator of its own, or code on a path where a cudaMalloc
+// (which may synchronise the device) is not allowed.  This variant keeps that
+// scratch in a fixed array compiled into the library instead.
+//
+// Limits and sharing rules:
+//   * the array holds kNoAllocSlots partial sums of kNoAllocChunk float4 each,
+//     so per-tensor gamma is limited to N*K <= kNoAllocMaxElems weights
+//     (134,217,728, e.g. 8192 x 16384); larger calls return TQ_ERR_SHAPE
+//     before launching anything.  Per-row gamma needs no scratch and has no
+//     extra limit.
+//   * every GPU that loads the library holds the array (about 32 KB) until the
+//     process exits.
+//   * all calls share the one array: calls whose work overlaps on the GPU (for
+//     example on two streams at once) race and give wrong results.  Each call
+//     writes every slot it reads before reading it, so nothing needs clearing
+//     and leftovers from a previous call are harmless.
+//   * the device address of the array is looked up (cudaGetSymbolAddress) on
+//     the first call made on each device, with that device current; make that
+//     first call before capturing work into a CUDA graph.
+// ===========================================================================
+namespace {
+
+constexpr int kNoAllocSlots = 2048;
+constexpr int64_t kNoAllocChunk = 16384;  // float4 per partial sum (65,536 weights)
+constexpr int64_t kNoAllocMaxElems = (int64_t)kNoAllocSlots * kNoAllocChunk * 4;
+constexpr size_t kNoAllocThreshOff = (size_t)kNoAllocSlots * sizeof(tq::DD);
+constexpr size_t kNoAllocBytes = kNoAllocThreshOff + 256;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+void *g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (looked up once).
+tq_status noalloc_scratch_addr(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return TQ_ERR_DEVICE;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return TQ_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return TQ_OK;
+}
+
+void launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
+                      float *gamma, const float *t, int reverse, cudaStream_t st) {
+    const int nv = (int)(K / 4);
+    const unsigned grid = (unsigned)N;
+    if (nv <= 256)
+        pack_rows_kernel<1><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+    else if (nv <= 512)
+        pack_rows_kernel<2><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+    else if (nv <= 1024)
+        pack_rows_kernel<4><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+    else if (nv <= 2048)
+        pack_rows_kernel<8><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+    else
+        pack_rows_kernel<0><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
+}
+
+}  // namespace
+
+extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N, int64_t K,
+                                                     unsigned flags, uint8_t *packed,
+                                                     float *gamma, tq_stream_t stream) {
+    if (!w || !packed || !gamma) return TQ_ERR_NULL;
+    if (N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE)) return TQ_ERR_ARG;
+    const bool per_row = flags & TQ_GAMMA_PER_ROW;
+    if (!per_row && N * K > kNoAllocMaxElems) return TQ_ERR_SHAPE;
+    if (!aligned16(w) || !aligned16(packed) || !aligned16(gamma)) return TQ_ERR_ALIGN;
+    const size_t wbytes = (size_t)(N * K) * 4, pbytes = (size_t)(N * K / 4),
+                 gbytes = (per_row ? (size_t)N : 1) * 4;
+    if (overlap(w, wbytes, packed, pbytes) || overlap(w, wbytes, gamma, gbytes) ||
+        overlap(packed, pbytes, gamma, gbytes))
+        return TQ_ERR_ARG;
+    if (tq_status e = check_device(nullptr)) return e;
+    const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
+    cudaStream_t st = cs(stream);
+    if (per_row) {
+        launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, st);
+        return launch_status();
+    }
+    void *scratch = nullptr;
+    if (tq_status e = noalloc_scratch_addr(&scratch)) return e;
+    const int64_t total_v = N * K / 4;
+    const int64_t nparts = (total_v + kNoAllocChunk - 1) / kNoAllocChunk;  // <= kNoAllocSlots
+    DD *partial = reinterpret_cast<DD *>(scratch);
+    float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kNoAllocThreshOff);
+    absum_partial_kernel<<<(unsigned)nparts, kPackThreads, 0, st>>>(w, total_v, kNoAllocChunk,
+                                                                     sanitize, partial);
+    absum_finalize_kernel<<<1, kPackThreads, 0, st>>>(partial, (int)nparts,
+                                                      (double)N * (double)K, gamma, thresh);
+    launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, st);
+    return launch_status();
+}
