@@ -156,23 +156,26 @@ class Workload:
             self.X = {M: torch.from_numpy(S.decode_acts(M, K, seed=0)) for M in self.Ms}
         elif name == "prefill":
             M, N, K = 2048, 11008, 4096
-            self.N, self.K, self.Ms, self.L = N, K, [M], 1
+            self.N, self.K, self.Ms, self.L = N, K, [M], layers
             self.per_row = False
             W, X = S.prefill(M, N, K, seed=0)
-            self.W = [torch.from_numpy(W).to(dev)]
+            W = torch.from_numpy(W)
+            self.W = [W.to(dev) for _ in range(self.L)]
             self.X = {M: torch.from_numpy(X)}
         elif name == "fused":
             M, N, K = 512, 5632, 2048
-            self.N, self.K, self.Ms, self.L = N, K, [M], 1
+            self.N, self.K, self.Ms, self.L = N, K, [M], layers
             self.per_row = False
             W, X = S.fused(M, N, K, seed=0)
-            self.W = [torch.from_numpy(W).to(dev)]
+            W = torch.from_numpy(W)
+            self.W = [W.to(dev) for _ in range(self.L)]
             self.X = {M: torch.from_numpy(X)}
         elif name == "sweep":
             N = K = 8192
-            self.N, self.K, self.Ms, self.L = N, K, [1, 4, 16, 64, 512, 4096], 1
+            self.N, self.K, self.Ms, self.L = N, K, [1, 4, 16, 64, 512, 4096], layers
             self.per_row = True
-            self.W = [torch.from_numpy(S.sweep_weights(N, K, seed=0)).to(dev)]
+            W = torch.from_numpy(S.sweep_weights(N, K, seed=0))
+            self.W = [W.to(dev) for _ in range(self.L)]
             self.X = {M: torch.from_numpy(S.sweep_acts(M, K, seed=0)) for M in self.Ms}
         else:
             raise SystemExit(f"unknown workload {name}")
@@ -189,7 +192,7 @@ class Workload:
         self.y = {M: [torch.empty((M, N), dtype=f32, device=dev) for _ in range(L)] for M in self.Ms}
         if name == "fused":
             fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM
-            self.fused_flags = fl
+            self.fused_flags = fl | tq.FLAG_WEIGHTS_STATIC
             self.fused_ws = torch.empty((tq.fused_workspace_bytes(self.Ms[0], K, fl),), dtype=u8, device=dev)
 
         # --- segments of one step ---
@@ -202,9 +205,10 @@ class Workload:
         if name == "fused":
             M = self.Ms[0]
             ops = 2 * M * N * K
-            self.segments.append(("fused M=%d" % M, "fused", 1, ops, 2, [
-                lambda: tq.bitlinear_fused_(self.Xd[M], self.packed[0], self.gamma[0], self.fused_flags,
-                                            self.y[M][0], self.fused_ws)]))
+            self.segments.append(("fused M=%d" % M, "fused", L, L * ops, 2 * L, [
+                lambda l=l: tq.bitlinear_fused_(self.Xd[M], self.packed[l], self.gamma[l],
+                                                self.fused_flags, self.y[M][l], self.fused_ws)
+                for l in range(L)]))
             return
         act_bytes = sum(4 * M * K + M * K + 8 * M for M in self.Ms)
         self.segments.append(("act", "act_quant", len(self.Ms), act_bytes, len(self.Ms), [
@@ -217,7 +221,8 @@ class Workload:
             self.segments.append(("gemv M=%d" % M if gemv else "gemm M=%d" % M,
                                   "gemv" if gemv else "gemm", L, L * work, L, [
                 lambda l=l, M=M: tq.ternary_gemm_(self.xq[M], self.sx[M], self.rs[M], self.packed[l],
-                                                  self.gamma[l], self.flags, self.y[M][l])
+                                                  self.gamma[l], self.flags | tq.FLAG_WEIGHTS_STATIC,
+                                                  self.y[M][l])
                 for l in range(L)]))
 
     def step_bytes(self):
@@ -239,7 +244,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     tq.load()
-    wl = Workload(args.workload, tq, S, torch, dev, args.layers)
+    wl = Workload(args.workload, tq, S, torch, dev, args.layers or WORKLOAD_SHAPES[args.workload][3])
     stream = torch.cuda.Stream(device=dev)
     graphs = []
     with torch.cuda.stream(stream):
@@ -338,22 +343,21 @@ def run_ours(args, rank, world, local_rank):
     del graphs
 
 
-WORKLOAD_SHAPES = {  # name -> (Ms, N, K, layers, per_row)
+WORKLOAD_SHAPES = {  # name -> (Ms, N, K, default ring of layers, per_row)
     "decode": ([1, 8], 4096, 4096, 64, True),
-    "prefill": ([2048], 11008, 4096, 1, False),
-    "fused": ([512], 5632, 2048, 1, False),
-    "sweep": ([1, 4, 16, 64, 512, 4096], 8192, 8192, 1, True),
+    "prefill": ([2048], 11008, 4096, 4, False),
+    "fused": ([512], 5632, 2048, 8, False),
+    "sweep": ([1, 4, 16, 64, 512, 4096], 8192, 8192, 8, True),
 }
 
 
 def config_for(name, layers, world):
     Ms, N, K, L, per_row = WORKLOAD_SHAPES[name]
-    if name == "decode":
-        L = layers
+    L = layers or L
     desc = {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers" % L,
-            "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma",
-            "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512",
-            "sweep": "M sweep over K=N=8192, per-row gamma"}[name]
+            "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma, ring of %d layers" % L,
+            "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512, ring of %d layers" % L,
+            "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L}[name]
     return {"workload": desc, "M": Ms, "N": N, "K": K, "layers": L,
             "gamma": "per-row" if per_row else "per-tensor",
             "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
@@ -515,7 +519,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fused", "sweep"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--layers", type=int, default=0, help="ring of distinct layers (0: workload default)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

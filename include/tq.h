@@ -76,6 +76,18 @@ typedef enum tq_status {
 #define TQ_FLAG_RMSNORM (1u << 2)            /* RMSNorm before the FWHT                        */
 #define TQ_FLAG_ETA_CLAMP (1u << 3)          /* clamp eta to [eta_min, eta_max]                */
 #define TQ_FLAG_SANITIZE_NONFINITE (1u << 4) /* quench NaN / +-Inf inputs first                */
+#define TQ_FLAG_WEIGHTS_STATIC (1u << 5)     /* see "Launch overlap" below                      */
+
+/*
+ * Launch overlap.  Every kernel is launched with programmatic dependent launch:
+ * it may be scheduled while the previous kernel on the stream is still
+ * finishing, and waits for that kernel's results before reading or writing
+ * any buffer.  With TQ_FLAG_WEIGHTS_STATIC (tq_ternary_gemm,
+ * tq_bitlinear_fused) the caller promises that the packed weights and gamma
+ * were not written by the immediately preceding work on the stream (true for
+ * the layers of a model during inference); the small-M GEMV then starts
+ * streaming weights before that wait.  Without the flag nothing is read early.
+ */
 
 /*
  * Absmean ternarisation and 2-bit packing of an fp32 weight matrix.
@@ -163,7 +175,8 @@ TQ_API tq_status tq_fwht512(const float *x, float *y, int64_t rows, int64_t K, i
  *   xq, s_x, rowsum  quantised activations as written by tq_quantize_act_int8
  *                    ([M][K] int8, [M] fp32, [M] int32).
  *   packed, gamma    as written by tq_quantize_ternary_pack ([N][K/4], [N] or [1]).
- *   flags            TQ_GAMMA_PER_ROW selects gamma[N] (else gamma[0]).
+ *   flags            TQ_GAMMA_PER_ROW selects gamma[N] (else gamma[0]);
+ *                    TQ_FLAG_WEIGHTS_STATIC as described under "Launch overlap".
  *   y                [M][N] fp32, written: y = fp32(acc) * (gamma_n * s_x[m]).
  *   acc              [M][N] int32 or NULL: if given, the exact integer sums
  *                    acc[m][n] = sum_k xq[m][k] * q[n][k] are written too.

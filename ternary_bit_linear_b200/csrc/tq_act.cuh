@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kActThreads)
     __shared__ float redf[32];
     __shared__ int redi[32];
     __shared__ double redd[32];
+    pdl_wait();
+    pdl_trigger();
     const int64_t m = blockIdx.x;
     const int nv = K >> 2, tid = threadIdx.x;
     const float4 *src = reinterpret_cast<const float4 *>(x + m * (int64_t)K);
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kActThreads)
             }
         }
         ss = block_sum_d<kActThreads>(ss, redd);
-        r = __drcp_rn(__dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
+        r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
         if (VEC > 0) {
 #pragma unroll
             for (int i = 0; i < VEC; ++i) {
@@ -284,6 +286,8 @@ __device__ __forceinline__ void fwht512_regs(float (&f)[16], bool normalize) {
 // Standalone transform: one warp per 512-block, 8 warps per CTA.
 __global__ void __launch_bounds__(256)
     fwht512_kernel(const float *x, float *y, int64_t nblocks, int normalize) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t blk = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (blk >= nblocks) return;
     const int lane = threadIdx.x & 31;
@@ -316,6 +320,8 @@ __global__ void __launch_bounds__(NW * 32)
     __shared__ int redi[32];
     __shared__ double redd[32];
     constexpr int K = 512 * NW;
+    pdl_wait();
+    pdl_trigger();
     const int64_t m = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float *row = x + m * (int64_t)K + warp * 512;
@@ -337,7 +343,7 @@ __global__ void __launch_bounds__(NW * 32)
         for (int i = 0; i < 16; ++i) ss = __fma_rn((double)f[i], (double)f[i], ss);
         ss = block_sum_d<NW * 32>(ss, redd);
         const double r =
-            __drcp_rn(__dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
+            __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll

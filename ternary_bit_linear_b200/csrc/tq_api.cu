@@ -68,6 +68,27 @@ inline tq_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
+// Every kernel is launched with programmatic dependent launch allowed; each
+// kernel waits (griddepcontrol.wait) before touching memory an earlier kernel
+// may have produced, so the attribute only lets launches overlap.
+template <typename... KArgs, typename... Args>
+tq_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess
+               ? TQ_OK
+               : TQ_ERR_CUDA;
+}
+
 inline tq_status check_k(int64_t K) {
     if (K < 64 || K > kMaxK || (K % 64) != 0) return TQ_ERR_SHAPE;
     return TQ_OK;
@@ -117,7 +138,7 @@ bool make_tmap_u8(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows
 template <int BT>
 tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
-                      int64_t K, float *y, int32_t *acc, cudaStream_t st) {
+                      int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
     using L = GemmLayout<BT>;
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
@@ -128,43 +149,64 @@ tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
     }
-    CUtensorMap tx, tw;
-    if (!make_tmap_u8(&tx, xq, (uint64_t)K, (uint64_t)M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_u8(&tw, packed, (uint64_t)(K / 4), (uint64_t)N, kTileK / 4, kTileN,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    CUtensorMap tx;
+    if (!make_tmap_u8(&tx, xq, (uint64_t)K, (uint64_t)M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B))
         return TQ_ERR_CUDA;
-    dim3 grid((unsigned)((N + kTileN - 1) / kTileN), (unsigned)((M + BT - 1) / BT));
-    gemm_kernel<BT><<<grid, kGemmThreads, L::kDynamic, st>>>(tx, tw, s_x, rowsum, gamma, per_row,
-                                                              (int)M, (int)N, (int)K, y, acc);
-    return launch_status();
+    const int64_t tiles = ((M + BT - 1) / BT) * ((N + kTileN - 1) / kTileN);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
+    return launch_pdl(gemm_kernel<BT>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, packed,
+                      s_x, rowsum, gamma, per_row, (int)M, (int)N, (int)K, y, acc);
 }
 
-template <int NB, int MAXSTEP>
+// Grid: at most half of the CTAs that fit on the device, so that the next
+// kernel's CTAs can be resident (and prefetching its weights under
+// programmatic dependent launch) while this one finishes; one strip per CTA
+// when that is enough, else a persistent ring of two stages.
+template <int NB, int MAXSTEP, int W>
 tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
-                      int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
-    const int64_t nstrips = (N + 15) / 16;
-    static std::atomic<int> occ[kMaxDevices];
+                      int64_t K, float *y, int32_t *acc, int static_w, int sms, cudaStream_t st) {
+    static std::atomic<int> occ1[kMaxDevices], occ2[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
-    int per_sm = occ[dev].load();
-    if (per_sm == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_kernel<NB, MAXSTEP>,
-                                                          kGemvWarps * 32, 0) != cudaSuccess)
+    const int sb = gemv_stage_bytes((int)K);
+    if (!occ1[dev].load()) {
+        if (cudaFuncSetAttribute(gemv_kernel<NB, MAXSTEP, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemvSmemCap) != cudaSuccess)
             return TQ_ERR_CUDA;
-        if (per_sm < 1) per_sm = 1;
-        occ[dev].store(per_sm);
+        int a = 0, b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, gemv_kernel<NB, MAXSTEP, W>, W * 32,
+                                                          (size_t)sb) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, gemv_kernel<NB, MAXSTEP, W>, W * 32,
+                                                          (size_t)2 * sb) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        occ2[dev].store(b > 1 ? b : 1);
+        occ1[dev].store(a > 1 ? a : 1);
     }
-    const int64_t grid = nstrips < (int64_t)per_sm * sms ? nstrips : (int64_t)per_sm * sms;
-    gemv_kernel<NB, MAXSTEP><<<(unsigned)grid, kGemvWarps * 32, 0, st>>>(
-        xq, s_x, rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc);
-    return launch_status();
+    const int64_t nstrips = (N + 15) / 16;
+    const int64_t half1 = (int64_t)(occ1[dev].load() / 2 > 0 ? occ1[dev].load() / 2 : 1) * sms;
+    int64_t grid, per_cta;
+    int nstage;
+    if (nstrips <= half1) {
+        grid = nstrips;
+        per_cta = 1;
+        nstage = 1;
+    } else {
+        const int64_t half2 = (int64_t)(occ2[dev].load() / 2 > 0 ? occ2[dev].load() / 2 : 1) * sms;
+        grid = nstrips < half2 ? nstrips : half2;
+        per_cta = (nstrips + grid - 1) / grid;
+        nstage = per_cta < 2 ? 1 : 2;
+    }
+    const size_t smem = (size_t)nstage * sb;
+    return launch_pdl(gemv_kernel<NB, MAXSTEP, W>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq,
+                      s_x, rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, static_w,
+                      nstage);
 }
 
 template <int NW>
 void launch_prologue(const float *x, const ActParams &p, int64_t M, int8_t *xq, float *sx,
                      int32_t *rs, cudaStream_t st) {
-    prologue_fwht_kernel<NW><<<(unsigned)M, NW * 32, 0, st>>>(x, p, xq, sx, rs);
+    launch_pdl(prologue_fwht_kernel<NW>, dim3((unsigned)M), dim3(NW * 32), 0, st, x, p, xq, sx, rs);
 }
 
 typedef void (*PrologueFn)(const float *, const ActParams &, int64_t, int8_t *, float *, int32_t *,
@@ -183,17 +225,63 @@ constexpr int64_t kMaxFwhtFusedK = 512 * 32;
 void launch_act(const float *x, const ActParams &p, int64_t M, int64_t K, int8_t *xq, float *sx,
                 int32_t *rs, cudaStream_t st) {
     const int nv = (int)(K / 4);
-    const unsigned grid = (unsigned)M;
+    const dim3 grid((unsigned)M), block(kActThreads);
     if (nv <= 256)
-        act_quant_kernel<1><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+        launch_pdl(act_quant_kernel<1>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else if (nv <= 512)
-        act_quant_kernel<2><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+        launch_pdl(act_quant_kernel<2>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else if (nv <= 1024)
-        act_quant_kernel<4><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+        launch_pdl(act_quant_kernel<4>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else if (nv <= 2048)
-        act_quant_kernel<8><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+        launch_pdl(act_quant_kernel<8>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else
-        act_quant_kernel<0><<<grid, kActThreads, 0, st>>>(x, (int)K, p, xq, sx, rs);
+        launch_pdl(act_quant_kernel<0>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+}
+
+// Persistent pack grid: as many CTAs as fit on the device, at most one row per
+// team.  K <= 16384: a team of T warps holds a row in registers; larger K:
+// one warp streams the row twice.
+template <typename Kern>
+tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_cta, const float *w,
+                           int64_t N, int64_t K, uint8_t *packed, float *gamma, const float *t,
+                           int reverse, cudaStream_t st) {
+    int dev = 0, sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    cudaGetDevice(&dev);
+    int per_sm = occ[dev].load();
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPackThreads, 0) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        if (per_sm < 1) per_sm = 1;
+        occ[dev].store(per_sm);
+    }
+    const int64_t need = (N + rows_per_cta - 1) / rows_per_cta;
+    const int64_t cap = (int64_t)per_sm * sms;
+    const unsigned grid = (unsigned)(need < cap ? need : cap);
+    return launch_pdl(kern, dim3(grid), dim3(kPackThreads), 0, st, w, N, (int)K, 1.0 / (double)K,
+                      packed, gamma, t, reverse);
+}
+
+template <bool SAN>
+tq_status launch_pack_rows_s(const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
+                             const float *t, int reverse, cudaStream_t st) {
+    static std::atomic<int> occ[5][kMaxDevices];
+    const int64_t nv = K / 4;
+    if (nv <= 32 * kTeamVec * 1)
+        return launch_pack_grid(pack_team_kernel<1, SAN>, occ[0], kPackWarps / 1, w, N, K, packed, gamma, t, reverse, st);
+    if (nv <= 32 * kTeamVec * 2)
+        return launch_pack_grid(pack_team_kernel<2, SAN>, occ[1], kPackWarps / 2, w, N, K, packed, gamma, t, reverse, st);
+    if (nv <= 32 * kTeamVec * 4)
+        return launch_pack_grid(pack_team_kernel<4, SAN>, occ[2], kPackWarps / 4, w, N, K, packed, gamma, t, reverse, st);
+    if (nv <= 32 * kTeamVec * 8)
+        return launch_pack_grid(pack_team_kernel<8, SAN>, occ[3], kPackWarps / 8, w, N, K, packed, gamma, t, reverse, st);
+    return launch_pack_grid(pack_rows_kernel<SAN>, occ[4], kPackWarps, w, N, K, packed, gamma, t, reverse, st);
+}
+
+tq_status launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
+                           float *gamma, const float *t, int reverse, cudaStream_t st) {
+    return sanitize ? launch_pack_rows_s<true>(w, N, K, packed, gamma, t, reverse, st)
+                    : launch_pack_rows_s<false>(w, N, K, packed, gamma, t, reverse, st);
 }
 
 size_t pack_parts(int64_t nv) {
@@ -207,20 +295,25 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
                         const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
                         int64_t N, int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
     const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
+    const int static_w = (flags & TQ_FLAG_WEIGHTS_STATIC) ? 1 : 0;
     if (M <= 16 && K <= kGemvMaxK) {
-        const int steps = (int)((K / 4 + 64 * kGemvWarps - 1) / (64 * kGemvWarps));
+        const int nsteps = (int)((K / 4 + 63) / 64);  // 64-byte column steps per row
+#define TQ_GEMV(NB, MS, W) \
+    return launch_gemv<NB, MS, W>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, static_w, sms, st)
         if (M <= 8) {
-            if (steps <= 1) return launch_gemv<1, 1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
-            if (steps <= 2) return launch_gemv<1, 2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
-            return launch_gemv<1, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+            if (nsteps <= 4) TQ_GEMV(1, 1, 4);
+            if (nsteps <= 8) TQ_GEMV(1, 2, 4);
+            if (nsteps <= 16) TQ_GEMV(1, 4, 4);
+            TQ_GEMV(1, 4, 8);
         }
-        if (steps <= 1) return launch_gemv<2, 1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
-        if (steps <= 2) return launch_gemv<2, 2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
-        return launch_gemv<2, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+        if (nsteps <= 4) TQ_GEMV(2, 1, 4);
+        if (nsteps <= 8) TQ_GEMV(2, 2, 4);
+        if (nsteps <= 16) TQ_GEMV(2, 4, 4);
+        TQ_GEMV(2, 4, 8);
+#undef TQ_GEMV
     }
-    if (M <= 64) return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
-    if (M <= 128) return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
-    return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
+    if (M <= 64) return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+    return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
 }
 
 }  // namespace
@@ -275,32 +368,23 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     if (tq_status e = check_device(nullptr)) return e;
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
-    const int nv = (int)(K / 4);
-    auto rows = [&](const float *t, int reverse) {
-        const unsigned grid = (unsigned)N;
-        if (nv <= 256)
-            pack_rows_kernel<1><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-        else if (nv <= 512)
-            pack_rows_kernel<2><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-        else if (nv <= 1024)
-            pack_rows_kernel<4><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-        else if (nv <= 2048)
-            pack_rows_kernel<8><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-        else
-            pack_rows_kernel<0><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-    };
     if (per_row) {
-        rows(nullptr, 0);
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, st)) return e;
         return launch_status();
     }
     const int64_t total_v = N * K / 4;
     const size_t nparts = pack_parts(total_v);
     const int64_t chunk = (total_v + (int64_t)nparts - 1) / (int64_t)nparts;
-    DD *partial = reinterpret_cast<DD *>(workspace);
+    double *partial = reinterpret_cast<double *>(workspace);
     float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + nparts * sizeof(DD));
-    absum_partial_kernel<<<(unsigned)nparts, kPackThreads, 0, st>>>(w, total_v, chunk, sanitize, partial);
-    absum_finalize_kernel<<<1, kPackThreads, 0, st>>>(partial, (int)nparts, (double)N * (double)K, gamma, thresh);
-    rows(thresh, 1);
+    if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
+                                 st, w, total_v, chunk, sanitize, partial))
+        return e;
+    if (tq_status e = launch_pdl(absum_finalize_kernel, dim3(1), dim3(1024), 0, st, partial,
+                                 (int)nparts, absum_tree_height(chunk, (int)nparts), w, total_v,
+                                 sanitize, gamma, thresh))
+        return e;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, st)) return e;
     return launch_status();
 }
 
@@ -337,8 +421,8 @@ tq_status tq_fwht512(const float *x, float *y, int64_t rows, int64_t K, int norm
     if (x != y && overlap(x, b, y, b)) return TQ_ERR_ARG;
     if (tq_status e = check_device(nullptr)) return e;
     const int64_t nblocks = rows * (K / 512);
-    fwht512_kernel<<<(unsigned)((nblocks + 7) / 8), 256, 0, cs(stream)>>>(x, y, nblocks, normalize);
-    return launch_status();
+    return launch_pdl(fwht512_kernel, dim3((unsigned)((nblocks + 7) / 8)), dim3(256), 0, cs(stream),
+                      x, y, nblocks, normalize);
 }
 
 tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
@@ -347,7 +431,7 @@ tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *row
     if (!xq || !s_x || !rowsum || !packed || !gamma || !y) return TQ_ERR_NULL;
     if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
-    if (flags & ~TQ_GAMMA_PER_ROW) return TQ_ERR_ARG;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC)) return TQ_ERR_ARG;
     if (!aligned16(xq) || !aligned16(s_x) || !aligned16(rowsum) || !aligned16(packed) ||
         !aligned16(gamma) || !aligned16(y) || (acc && !aligned16(acc)))
         return TQ_ERR_ALIGN;
@@ -380,7 +464,7 @@ tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_ep
     if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
     const unsigned known = TQ_GAMMA_PER_ROW | TQ_FLAG_FWHT | TQ_FLAG_RMSNORM | TQ_FLAG_ETA_CLAMP |
-                           TQ_FLAG_SANITIZE_NONFINITE;
+                           TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_WEIGHTS_STATIC;
     if (flags & ~known) return TQ_ERR_ARG;
     if ((flags & TQ_FLAG_FWHT) && (K % 512 != 0 || K > kMaxFwhtFusedK)) return TQ_ERR_SHAPE;
     if ((flags & TQ_FLAG_ETA_CLAMP) && !(eta_min > 0.0f && eta_min <= eta_max)) return TQ_ERR_ARG;
@@ -429,7 +513,8 @@ tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_ep
     else
         launch_act(x, p, M, K, xq, sx, rs, st);
     if (tq_status e = launch_status()) return e;
-    return gemm_dispatch(xq, sx, rs, packed, gamma, flags & TQ_GAMMA_PER_ROW, M, N, K, y, nullptr,
+    return gemm_dispatch(xq, sx, rs, packed, gamma,
+                         flags & (TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC), M, N, K, y, nullptr,
                          sms, st);
 }
 
@@ -499,22 +584,6 @@ tq_status noalloc_scratch_addr(void **out) {
     return TQ_OK;
 }
 
-void launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
-                      float *gamma, const float *t, int reverse, cudaStream_t st) {
-    const int nv = (int)(K / 4);
-    const unsigned grid = (unsigned)N;
-    if (nv <= 256)
-        pack_rows_kernel<1><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-    else if (nv <= 512)
-        pack_rows_kernel<2><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-    else if (nv <= 1024)
-        pack_rows_kernel<4><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-    else if (nv <= 2048)
-        pack_rows_kernel<8><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-    else
-        pack_rows_kernel<0><<<grid, kPackThreads, 0, st>>>(w, N, (int)K, sanitize, packed, gamma, t, reverse);
-}
-
 }  // namespace
 
 extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N, int64_t K,
@@ -536,19 +605,22 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, st);
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, st)) return e;
         return launch_status();
     }
     void *scratch = nullptr;
     if (tq_status e = noalloc_scratch_addr(&scratch)) return e;
     const int64_t total_v = N * K / 4;
     const int64_t nparts = (total_v + kNoAllocChunk - 1) / kNoAllocChunk;  // <= kNoAllocSlots
-    DD *partial = reinterpret_cast<DD *>(scratch);
+    double *partial = reinterpret_cast<double *>(scratch);
     float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kNoAllocThreshOff);
-    absum_partial_kernel<<<(unsigned)nparts, kPackThreads, 0, st>>>(w, total_v, kNoAllocChunk,
-                                                                     sanitize, partial);
-    absum_finalize_kernel<<<1, kPackThreads, 0, st>>>(partial, (int)nparts,
-                                                      (double)N * (double)K, gamma, thresh);
-    launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, st);
+    if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
+                                 st, w, total_v, kNoAllocChunk, sanitize, partial))
+        return e;
+    if (tq_status e = launch_pdl(absum_finalize_kernel, dim3(1), dim3(1024), 0, st, partial,
+                                 (int)nparts, absum_tree_height(kNoAllocChunk, (int)nparts), w,
+                                 total_v, sanitize, gamma, thresh))
+        return e;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, st)) return e;
     return launch_status();
 }

@@ -4,14 +4,20 @@
 // "Ternary Format / Encoding"; Hetman-2b, src/quantization.py, section 2
 // (AbsmeanWeightQuantizer.forward) and section 5 (export_packed_weights).
 //
-// gamma is the fp32 nearest to the exact mean of |w|: every CTA sums |w| as a
-// double-double (TwoSum per element, error ~2^-100 relative), so the rounding
-// to fp32 does not depend on the reduction tree.  Codes come from a single
-// fp32 threshold per gamma (code_threshold), which is equivalent to rounding
-// the fp32 quotient w / gamma and clamping, without a divide per element.
+// gamma is the fp32 nearest to the exact mean of |w| (ties to even), then
+// max(., 1e-6).  Fast path: |w| is summed in plain fp64 over a fixed tree of
+// known height h, so the computed mean q is within eps = (h + 2) * 2^-53 * q of
+// the exact mean.  If q is farther than 2 * eps from both fp32 rounding
+// midpoints around fp32(q), fp32(q) is the correctly rounded mean.  Otherwise
+// (about one row in ten million on random data, and every row whose mean is an
+// exact midpoint) the sum is redone as a double-double (TwoSum per element,
+// ~2^-100 relative) and rounded with an explicit midpoint test.
 //
-// HBM traffic: read 4 B and write 0.25 B per weight (per-row gamma: one pass;
-// per-tensor gamma: a reduction pass, then the packing pass, which walks the
+// Codes come from one fp32 threshold per gamma (code_threshold), equivalent to
+// rounding the fp32 quotient w / gamma and clamping, without a divide.
+//
+// HBM traffic: read 4 B and write 0.25 B per weight.  Per-row gamma is one
+// pass; per-tensor gamma reads W twice (reduction, then packing walking the
 // rows in reverse so the tail of the first pass is still in L2).
 #pragma once
 
@@ -20,6 +26,7 @@
 namespace tq {
 
 constexpr int kPackThreads = 256;
+constexpr int kPackWarps = kPackThreads / 32;
 
 __device__ __forceinline__ float4 sanitize_w(float4 v) {
     auto f = [](float x) {
@@ -30,6 +37,13 @@ __device__ __forceinline__ float4 sanitize_w(float4 v) {
     return make_float4(f(v.x), f(v.y), f(v.z), f(v.w));
 }
 
+__device__ __forceinline__ double abs_sum4(float4 v) {
+    // left-to-right: ((|x| + |y|) + |z|) + |w|
+    return __dadd_rn(__dadd_rn(__dadd_rn((double)fabsf(v.x), (double)fabsf(v.y)),
+                               (double)fabsf(v.z)),
+                     (double)fabsf(v.w));
+}
+
 __device__ __forceinline__ void acc_abs4(DD &a, float4 v) {
     dd_acc(a, (double)fabsf(v.x));
     dd_acc(a, (double)fabsf(v.y));
@@ -37,101 +51,240 @@ __device__ __forceinline__ void acc_abs4(DD &a, float4 v) {
     dd_acc(a, (double)fabsf(v.w));
 }
 
+// Byte of four 2-bit codes: start from 0b01010101 (all zero codes) and move
+// each field up (+1 -> 0b10) or down (-1 -> 0b00).  NaN compares false: code 0.
 __device__ __forceinline__ uint32_t pack4(float4 v, float t) {
-    return ternary_field(v.x, t) | (ternary_field(v.y, t) << 2) | (ternary_field(v.z, t) << 4) |
-           (ternary_field(v.w, t) << 6);
+    uint32_t b = 0x55u;
+    b += (v.x >= t) ? 1u : 0u;
+    b -= (v.x <= -t) ? 1u : 0u;
+    b += (v.y >= t) ? 4u : 0u;
+    b -= (v.y <= -t) ? 4u : 0u;
+    b += (v.z >= t) ? 16u : 0u;
+    b -= (v.z <= -t) ? 16u : 0u;
+    b += (v.w >= t) ? 64u : 0u;
+    b -= (v.w <= -t) ? 64u : 0u;
+    return b;
 }
 
-// Sum over the CTA in a fixed order; the result is valid in every thread.
-__device__ __forceinline__ DD dd_block_sum(DD a, DD *red /* [kPackThreads/32] */) {
+__device__ __forceinline__ double warp_sum_dbl(double v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+
+// Plain fp64 block sum in a fixed order (5 + 3 tree levels); valid in every thread.
+__device__ __forceinline__ double block_sum_dbl(double a, double *red) {
+    a = warp_sum_dbl(a);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = a;
+    __syncthreads();
+    // lanes >= kPackWarps add exact zeros; every lane ends with the same value
+    double t = warp_sum_dbl(lane < kPackWarps ? red[lane] : 0.0);
+    __syncthreads();
+    return t;
+}
+
+// Double-double block sum in a fixed order; valid in every thread.
+__device__ __forceinline__ DD dd_block_sum(DD a, DD *red) {
     a = dd_warp_sum(a);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) red[warp] = a;
     __syncthreads();
     DD t = {0.0, 0.0};
-    if (lane < kPackThreads / 32) t = red[lane];
+    if (lane < kPackWarps) t = red[lane];
     t = dd_warp_sum(t);
     __syncthreads();
     return t;
 }
 
-// One CTA per row.  VEC > 0: each thread keeps VEC float4 of the row in
-// registers (K <= 1024 * VEC); VEC == 0: the row is streamed twice (any K).
-// per_tensor_t != nullptr: use that precomputed threshold instead of a row gamma.
-template <int VEC>
+// fp32(q) if the exact mean, known to lie within q * (1 +- eps), must round to
+// it; otherwise a negative value (caller falls back to the exact sum).
+__device__ __forceinline__ float mean_fast_or_fail(double q, double eps) {
+    if (!(q > 0.0)) return 0.0f;  // all zero: exact
+    const float f = __double2float_rn(q);
+    if (!(f > 0.0f) || isinf(f)) return -1.0f;  // tiny or huge: let the exact path decide
+    const float up = __int_as_float(__float_as_int(f) + 1);  // neighbours of a positive finite f
+    const float dn = __int_as_float(__float_as_int(f) - 1);
+    const double mu = 0.5 * ((double)f + (double)up);
+    const double ml = 0.5 * ((double)f + (double)dn);
+    const double margin = 2.0 * eps * q;
+    if (mu - q > margin && q - ml > margin) return f;
+    return -1.0f;
+}
+
+// Relative error bound of a plain fp64 sum of non-negative terms over a tree of
+// height h, followed by a multiply with a rounded reciprocal of n: h + 2
+// roundings of relative error 2^-53 each, with slack.
+__device__ __forceinline__ double sum_error_bound(int h) { return (double)(h + 3) * 0x1p-53 * 1.01; }
+
+// ---------------------------------------------------------------------------
+// Per-row gamma (or a precomputed per-tensor threshold) + packing, one warp per
+// row, persistent warps walking rows (warp id, + total warps, ...).
+//   pass 1: stream the row once (8 float4 per lane in flight), sum |w| in plain
+//           fp64 per lane, fold the 32 lanes with shuffles (fixed order);
+//           every lane derives the same gamma and code threshold; the rare
+//           rows whose mean sits within the error bound of a midpoint are
+//           re-summed exactly (double-double) by the same warp.
+//   pass 2: re-read the row (L2 hit: pass 1 left it there) and write one byte
+//           per float4; a warp stores 32 consecutive bytes per instruction.
+// No block-level synchronisation: warps are independent.
+// ---------------------------------------------------------------------------
+constexpr int kPackUnroll = 8;
+
+template <bool SAN>
 __global__ void __launch_bounds__(kPackThreads)
-    pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, int sanitize,
+    pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const float *__restrict__ per_tensor_t, int reverse) {
-    __shared__ DD red[kPackThreads / 32];
-    __shared__ float s_t;
-    const int64_t n = reverse ? (N - 1 - (int64_t)blockIdx.x) : (int64_t)blockIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * kPackWarps;
     const int nv = K >> 2;
-    const float4 *src = reinterpret_cast<const float4 *>(w + n * (int64_t)K);
-    uint8_t *dst = packed + n * (int64_t)(K >> 2);
-    const int tid = threadIdx.x;
+    const float t_tensor = per_tensor_t ? __ldg(per_tensor_t) : 0.0f;
+    // per-lane chain length (float4) of pass 1, for the error bound
+    const int chain = (nv + 31) / 32;
+    const double eps = sum_error_bound(4 * chain + 5);
 
-    float4 v[VEC > 0 ? VEC : 1];
-    if (VEC > 0) {
+    for (int64_t i = (int64_t)blockIdx.x * kPackWarps + (threadIdx.x >> 5); i < N; i += nwarps) {
+        const int64_t n = reverse ? (N - 1 - i) : i;
+        const float4 *src = reinterpret_cast<const float4 *>(w + n * (int64_t)K);
+        float t = t_tensor;
+        if (per_tensor_t == nullptr) {
+            double a = 0.0;
+            int c = lane;
+            for (; c + 32 * (kPackUnroll - 1) < nv; c += 32 * kPackUnroll) {
+                float4 x[kPackUnroll];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-            const int idx = tid + i * kPackThreads;
-            v[i] = idx < nv ? __ldcs(src + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (sanitize) v[i] = sanitize_w(v[i]);
-        }
-    }
-
-    float t;
-    if (per_tensor_t != nullptr) {
-        t = __ldg(per_tensor_t);
-    } else {
-        DD a = {0.0, 0.0};
-        if (VEC > 0) {
+                for (int u = 0; u < kPackUnroll; ++u) x[u] = __ldg(src + c + 32 * u);
 #pragma unroll
-            for (int i = 0; i < VEC; ++i) acc_abs4(a, v[i]);
-        } else {
-            for (int idx = tid; idx < nv; idx += kPackThreads) {
-                float4 x = __ldg(src + idx);
-                if (sanitize) x = sanitize_w(x);
-                acc_abs4(a, x);
+                for (int u = 0; u < kPackUnroll; ++u) a = __dadd_rn(a, abs_sum4(SAN ? sanitize_w(x[u]) : x[u]));
             }
-        }
-        a = dd_block_sum(a, red);
-        if (tid == 0) {
-            float g = dd_mean_to_f32(a, (double)K);
+            for (; c < nv; c += 32) {
+                const float4 x = __ldg(src + c);
+                a = __dadd_rn(a, abs_sum4(SAN ? sanitize_w(x) : x));
+            }
+            const double S = warp_sum_dbl(a);  // identical in every lane
+            float g = mean_fast_or_fail(__dmul_rn(S, inv_k), eps);
+            if (g < 0.0f) {  // rare: redo the sum exactly
+                DD d = {0.0, 0.0};
+                for (int cc = lane; cc < nv; cc += 32) {
+                    const float4 x = __ldg(src + cc);
+                    acc_abs4(d, SAN ? sanitize_w(x) : x);
+                }
+                d = dd_warp_sum(d);
+                g = dd_mean_to_f32(d, (double)K);
+            }
             g = g > 1e-6f ? g : 1e-6f;
-            gamma[n] = g;
-            s_t = code_threshold(g);
+            if (lane == 0) gamma[n] = g;
+            t = code_threshold(g);
         }
-        __syncthreads();
-        t = s_t;
-    }
-
-    if (VEC > 0) {
+        uint8_t *dst = packed + n * (int64_t)nv;
+        int c = lane;
+        for (; c + 32 * (kPackUnroll - 1) < nv; c += 32 * kPackUnroll) {
+            float4 x[kPackUnroll];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-            const int idx = tid + i * kPackThreads;
-            if (idx < nv) dst[idx] = (uint8_t)pack4(v[i], t);
+            for (int u = 0; u < kPackUnroll; ++u) x[u] = __ldcs(src + c + 32 * u);
+#pragma unroll
+            for (int u = 0; u < kPackUnroll; ++u) dst[c + 32 * u] = (uint8_t)pack4(SAN ? sanitize_w(x[u]) : x[u], t);
         }
-    } else {
-        for (int idx = tid; idx < nv; idx += kPackThreads) {
-            float4 x = __ldcs(src + idx);
-            if (sanitize) x = sanitize_w(x);
-            dst[idx] = (uint8_t)pack4(x, t);
+        for (; c < nv; c += 32) {
+            const float4 x = __ldcs(src + c);
+            dst[c] = (uint8_t)pack4(SAN ? sanitize_w(x) : x, t);
         }
     }
 }
 
-// Per-tensor gamma, pass 1: CTA b sums |w| over float4 range [b*chunk, ...)
-// into partial[b] (double-double).
+// ---------------------------------------------------------------------------
+// Team kernel (K <= 8192): T warps share a row, every thread holds 8 float4
+// of it in registers (read from HBM once).  Per row: per-lane fp64 chain,
+// warp shuffles, one named barrier for the T warp sums (double-buffered by row
+// parity), then each thread packs its own values.
+// ---------------------------------------------------------------------------
+constexpr int kTeamVec = 8;
+
+__device__ __forceinline__ void team_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int T, bool SAN>
+__global__ void __launch_bounds__(kPackThreads, 2)
+    pack_team_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
+                     uint8_t *__restrict__ packed, float *__restrict__ gamma,
+                     const float *__restrict__ per_tensor_t, int reverse) {
+    constexpr int TEAMS = kPackWarps / T;
+    __shared__ double tred[2][kPackWarps];
+    __shared__ DD tredd[kPackWarps];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int team = warp / T, tw = warp % T;
+    const int bar_id = 1 + team;
+    const int nv = K >> 2;
+    const int64_t nteams = (int64_t)gridDim.x * TEAMS;
+    const float t_tensor = per_tensor_t ? __ldg(per_tensor_t) : 0.0f;
+    const double eps = sum_error_bound(4 * kTeamVec + 5 + T);
+    int parity = 0;
+    for (int64_t i = (int64_t)blockIdx.x * TEAMS + team; i < N; i += nteams) {
+        const int64_t n = reverse ? (N - 1 - i) : i;
+        const float4 *src = reinterpret_cast<const float4 *>(w + n * (int64_t)K);
+        float4 v[kTeamVec];
+#pragma unroll
+        for (int j = 0; j < kTeamVec; ++j) {
+            const int idx = j * 32 * T + tw * 32 + lane;
+            v[j] = idx < nv ? __ldcs(src + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (SAN) v[j] = sanitize_w(v[j]);
+        }
+        float t = t_tensor;
+        if (per_tensor_t == nullptr) {
+            double a = 0.0;
+#pragma unroll
+            for (int j = 0; j < kTeamVec; ++j) a = __dadd_rn(a, abs_sum4(v[j]));
+            a = warp_sum_dbl(a);
+            if (lane == 0) tred[parity][warp] = a;
+            team_barrier(bar_id, 32 * T);
+            double S = 0.0;
+#pragma unroll
+            for (int u = 0; u < T; ++u) S = __dadd_rn(S, tred[parity][team * T + u]);
+            parity ^= 1;
+            float g = mean_fast_or_fail(__dmul_rn(S, inv_k), eps);
+            if (g < 0.0f) {  // rare: redo the sum exactly (team-uniform branch)
+                DD d = {0.0, 0.0};
+#pragma unroll
+                for (int j = 0; j < kTeamVec; ++j) acc_abs4(d, v[j]);
+                d = dd_warp_sum(d);
+                if (lane == 0) tredd[warp] = d;
+                team_barrier(bar_id, 32 * T);
+                DD e = {0.0, 0.0};
+                for (int u = 0; u < T; ++u) e = dd_add(e, tredd[team * T + u]);
+                team_barrier(bar_id, 32 * T);  // tredd may be rewritten by the next fallback
+                g = dd_mean_to_f32(e, (double)K);
+            }
+            g = g > 1e-6f ? g : 1e-6f;
+            if (tw == 0 && lane == 0) gamma[n] = g;
+            t = code_threshold(g);
+        }
+        uint8_t *dst = packed + n * (int64_t)nv;
+#pragma unroll
+        for (int j = 0; j < kTeamVec; ++j) {
+            const int idx = j * 32 * T + tw * 32 + lane;
+            if (idx < nv) dst[idx] = (uint8_t)pack4(v[j], t);
+        }
+    }
+}
+
+// Per-tensor gamma, pass 1: CTA b sums |w| over float4 range [b*chunk, ...) in
+// plain fp64 (each thread sequentially, then a fixed block tree).
 __global__ void __launch_bounds__(kPackThreads)
     absum_partial_kernel(const float *__restrict__ w, int64_t nv, int64_t chunk, int sanitize,
-                         DD *__restrict__ partial) {
-    __shared__ DD red[kPackThreads / 32];
+                         double *__restrict__ partial) {
+    __shared__ double red[kPackWarps];
+    pdl_wait();
+    pdl_trigger();
     const float4 *src = reinterpret_cast<const float4 *>(w);
     const int64_t beg = (int64_t)blockIdx.x * chunk;
     const int64_t end = min(nv, beg + chunk);
-    DD a = {0.0, 0.0};
+    double a0 = 0.0, a1 = 0.0;
     int64_t idx = beg + threadIdx.x;
     for (; idx + 3 * kPackThreads < end; idx += 4 * kPackThreads) {
         float4 x0 = __ldg(src + idx), x1 = __ldg(src + idx + kPackThreads),
@@ -142,31 +295,63 @@ __global__ void __launch_bounds__(kPackThreads)
             x2 = sanitize_w(x2);
             x3 = sanitize_w(x3);
         }
-        acc_abs4(a, x0);
-        acc_abs4(a, x1);
-        acc_abs4(a, x2);
-        acc_abs4(a, x3);
+        a0 = __dadd_rn(a0, __dadd_rn(abs_sum4(x0), abs_sum4(x1)));
+        a1 = __dadd_rn(a1, __dadd_rn(abs_sum4(x2), abs_sum4(x3)));
     }
     for (; idx < end; idx += kPackThreads) {
         float4 x = __ldg(src + idx);
         if (sanitize) x = sanitize_w(x);
-        acc_abs4(a, x);
+        a0 = __dadd_rn(a0, abs_sum4(x));
     }
-    a = dd_block_sum(a, red);
-    if (threadIdx.x == 0) partial[blockIdx.x] = a;
+    const double S = block_sum_dbl(__dadd_rn(a0, a1), red);
+    if (threadIdx.x == 0) partial[blockIdx.x] = S;
 }
 
-// Per-tensor gamma, pass 2: one CTA folds the partials in a fixed order and
-// writes gamma[0] and the code threshold.
-__global__ void __launch_bounds__(kPackThreads)
-    absum_finalize_kernel(const DD *__restrict__ partial, int nparts, double n,
+// Tree height of the per-tensor sum: per-thread chain over its float4 of a
+// chunk (two interleaved chains joined once, each float4 adding 4 levels),
+// the CTA tree, the finalize thread's chain over partials, the finalize tree.
+__host__ __device__ inline int absum_tree_height(int64_t chunk, int nparts) {
+    const int64_t per_thread = (chunk + kPackThreads - 1) / kPackThreads;  // float4
+    const int64_t parts_per_thread = (nparts + 1023) / 1024;
+    return (int)(per_thread + 4 + 1 + 8 + parts_per_thread + 10);
+}
+
+// Per-tensor gamma, pass 2: one CTA folds the partials in a fixed order,
+// checks the rounding margin, falls back to an exact double-double re-sum of
+// the whole tensor if needed, and writes gamma[0] and the code threshold.
+__global__ void __launch_bounds__(1024)
+    absum_finalize_kernel(const double *__restrict__ partial, int nparts, int height,
+                          const float *__restrict__ w, int64_t nv, int sanitize,
                           float *__restrict__ gamma, float *__restrict__ t_out) {
-    __shared__ DD red[kPackThreads / 32];
-    DD a = {0.0, 0.0};
-    for (int i = threadIdx.x; i < nparts; i += kPackThreads) a = dd_add(a, partial[i]);
-    a = dd_block_sum(a, red);
+    __shared__ double red[32];
+    __shared__ DD redd[32];
+    pdl_wait();
+    pdl_trigger();
+    double a = 0.0;
+    for (int i = threadIdx.x; i < nparts; i += 1024) a = __dadd_rn(a, partial[i]);
+    // fixed-order block tree over 32 warps
+    a = warp_sum_dbl(a);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = a;
+    __syncthreads();
+    double S = warp_sum_dbl(red[lane]);
+    const double n = 4.0 * (double)nv;
+    const double q = __ddiv_rn(S, n);
+    float g = mean_fast_or_fail(q, sum_error_bound(height));
+    if (g < 0.0f) {
+        const float4 *src = reinterpret_cast<const float4 *>(w);
+        DD d = {0.0, 0.0};
+        for (int64_t idx = threadIdx.x; idx < nv; idx += 1024) {
+            float4 x = __ldg(src + idx);
+            acc_abs4(d, sanitize ? sanitize_w(x) : x);
+        }
+        d = dd_warp_sum(d);
+        if (lane == 0) redd[warp] = d;
+        __syncthreads();
+        d = dd_warp_sum(redd[lane]);
+        g = dd_mean_to_f32(d, n);
+    }
     if (threadIdx.x == 0) {
-        float g = dd_mean_to_f32(a, n);
         g = g > 1e-6f ? g : 1e-6f;
         gamma[0] = g;
         *t_out = code_threshold(g);

@@ -359,3 +359,92 @@ def test_fused_full_size(cuda_lib):
 
 def test_device_status_clean(cuda_lib):
     assert cuda_lib.device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# exact-midpoint gamma (the double-double fallback) and launch ordering
+# ---------------------------------------------------------------------------
+
+def midpoint_rows(K, seed):
+    """Rows whose mean |w| is exactly an fp32 rounding midpoint (ties to even)."""
+    one, u = np.float32(1.0), np.float32(2.0 ** -23)
+    signs = np.where(S.normal((4, K), 1.0, seed, 77) > 0, 1.0, -1.0).astype(np.float32)
+    rows = np.empty((4, K), np.float32)
+    rows[0] = np.tile([one, one + u], K // 2)              # mean 1 + 2^-24  -> 1 (even)
+    rows[1] = np.tile([one + u, one + 2 * u], K // 2)      # mean 1 + 1.5u   -> 1 + 2u (even)
+    rows[2] = np.tile([np.float32(0.75), np.float32(0.75) + u / 2], K // 2)  # tie below 1
+    rows[3] = np.tile([np.float32(3.0), np.float32(3.0) + 2 * u], K // 2)    # mean 3 + u -> 3 (even)
+    return rows * signs
+
+
+@pytest.mark.parametrize("K", [512, 4096, 8256])
+def test_pack_midpoint_means_take_exact_path(cuda_lib, K):
+    W = midpoint_rows(K, K)
+    packed, gamma = cuda_lib.quantize_ternary_pack(dev(W), per_row=True)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=True)
+    assert g_ref.tolist() == [1.0, float(np.float32(1.0 + 2.0 ** -22)), 0.75, 3.0]
+    assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
+    # per tensor: the whole matrix's mean is a midpoint too when built from one row kind
+    Wt = np.tile(W[1:2], (64, 1))
+    packed, gamma = cuda_lib.quantize_ternary_pack(dev(Wt), per_row=False)
+    p_ref, g_ref = oracle.quantize_pack(Wt, per_row=False)
+    assert g_ref[0] == np.float32(1.0 + 2.0 ** -22)
+    assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (8, 1000, 4096), (16, 257, 8192), (3, 33, 192)])
+def test_gemv_static_weights_flag_same_result(cuda_lib, M, N, K):
+    tq = cuda_lib
+    W = S.normal((N, K), 0.02, 12, N)
+    X = S.decode_acts(M, K, seed=13)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=True)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    args = [dev(a) for a in (xq_ref, sx_ref, rs_ref, p_ref, g_ref)]
+    y0 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    y1 = torch.empty_like(y0)
+    tq.ternary_gemm_(*args, tq.GAMMA_PER_ROW, y0)
+    tq.ternary_gemm_(*args, tq.GAMMA_PER_ROW | tq.FLAG_WEIGHTS_STATIC, y1)
+    assert torch.equal(y0, y1)
+    acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
+    assert_y_close(host(y1), oracle.dequant(acc_ref, g_ref, sx_ref, True))
+
+
+def test_dependent_calls_back_to_back(cuda_lib):
+    """Re-pack into the same buffer and contract it five times without any host
+    synchronisation: every kernel must see its predecessor's writes (and not
+    overwrite what the predecessor is still reading)."""
+    tq = cuda_lib
+    N, K, M = 384, 2048, 8
+    X = dev(S.decode_acts(M, K, seed=21))
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty((1,), dtype=torch.float32, device="cuda")
+    ws = torch.empty((tq.pack_workspace_bytes(N, K, 0),), dtype=torch.uint8, device="cuda")
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sx = torch.empty((M,), dtype=torch.float32, device="cuda")
+    rs = torch.empty((M,), dtype=torch.int32, device="cuda")
+    ys = []
+    Ws = [S.normal((N, K), 0.02, 30 + i, 1) for i in range(5)]
+    for i, W in enumerate(Ws):
+        tq.quantize_ternary_pack_(dev(W), 0, packed, gamma, ws)
+        tq.quantize_act_int8_(X, 0, 0.05, 40.0, xq, sx, rs)
+        for Mi in (M, 40):  # GEMV and tcgen05 GEMM consumers of the same buffers
+            Xi = X if Mi == M else dev(S.decode_acts(Mi, K, seed=22))
+            if Mi != M:
+                xq2 = torch.empty((Mi, K), dtype=torch.int8, device="cuda")
+                sx2 = torch.empty((Mi,), dtype=torch.float32, device="cuda")
+                rs2 = torch.empty((Mi,), dtype=torch.int32, device="cuda")
+                tq.quantize_act_int8_(Xi, 0, 0.05, 40.0, xq2, sx2, rs2)
+                y = torch.empty((Mi, N), dtype=torch.float32, device="cuda")
+                tq.ternary_gemm_(xq2, sx2, rs2, packed, gamma, 0, y)
+            else:
+                y = torch.empty((Mi, N), dtype=torch.float32, device="cuda")
+                tq.ternary_gemm_(xq, sx, rs, packed, gamma, 0, y)
+            ys.append((i, Mi, y))
+    torch.cuda.synchronize()
+    for i, Mi, y in ys:
+        p_ref, g_ref = oracle.quantize_pack(Ws[i], per_row=False)
+        Xn = S.decode_acts(M, K, seed=21) if Mi == M else S.decode_acts(Mi, K, seed=22)
+        xq_ref, sx_ref, _ = oracle.act_quant(Xn)
+        acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
+        assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, False))
+    assert tq.device_status() == 0
