@@ -149,12 +149,16 @@ tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
     }
-    CUtensorMap tx;
-    if (!make_tmap_u8(&tx, xq, (uint64_t)K, (uint64_t)M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B))
+    // x_q [M][K] in 128-byte-swizzled [BT][128] boxes; packed weights [N][K/4]
+    // in plain [128][32] boxes (K % 64 == 0 keeps both row strides 16-byte multiples).
+    CUtensorMap tx, tw;
+    if (!make_tmap_u8(&tx, xq, (uint64_t)K, (uint64_t)M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_u8(&tw, packed, (uint64_t)(K / 4), (uint64_t)N, kTileK / 4, kTileN,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return TQ_ERR_CUDA;
     const int64_t tiles = ((M + BT - 1) / BT) * ((N + kTileN - 1) / kTileN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
-    return launch_pdl(gemm_kernel<BT>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, packed,
+    return launch_pdl(gemm_kernel<BT>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
                       s_x, rowsum, gamma, per_row, (int)M, (int)N, (int)K, y, acc);
 }
 
@@ -313,7 +317,8 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
 #undef TQ_GEMV
     }
     if (M <= 64) return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
-    return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+    if (M <= 128) return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+    return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
 }
 
 }  // namespace

@@ -6,30 +6,36 @@
 // as tcgen05.mma kind::i8 with int32 accumulators in tensor memory.
 //
 // Persistent: one CTA per SM walks output tiles of 128 features (the MMA's M,
-// taken by the weights) x BT tokens (the MMA's N), token blocks fastest so
-// that concurrently running CTAs share x_q and weight tiles in L2.  K is
-// consumed in steps of 128 codes.  Sixteen warps:
+// taken by the weights) x BT tokens (the MMA's N, up to 256), token blocks
+// fastest so that concurrently running CTAs share weight tiles in L2.  K is
+// consumed in steps of 128 codes; one step is four MMAs of K = 32 with both
+// operands in shared memory (128-byte swizzled, K-major).  Twenty warps:
 //
-//   warp 0      TMA producer: x_q tile [BT][128 B] (128-byte swizzle, the
-//               canonical K-major operand layout) into a shared-memory ring.
-//   warp 1      TMEM owner and single-thread MMA issuer: per step 4 MMAs of
-//               K = 32 with the weight operand read from tensor memory; the
+//   warp 0      x_q producer (lane 0): TMA of the x_q tile [BT][128 B] into
+//               stage s of the operand ring.
+//   warp 1      TMEM owner; lane 0 issues the MMAs.  Per step: one wait on
+//               full(s), four MMAs, one commit that frees stage s.  The
 //               accumulator alternates between two TMEM buffers per tile.
-//   warps 4-11  unpackers.  Warps 4-7 take even steps, 8-11 odd steps; thread
-//               r of quarter q owns TMEM lane 32q + r = weight row r of the
-//               tile: it loads its 32 packed bytes (prefetched one step ahead
-//               with 16-byte non-coherent loads), expands them to 128 unsigned
-//               codes c = q + 1 in natural K order and writes them with
-//               tcgen05.st into one of 8 TMEM operand slots.
-//   warps 12-15 epilogue: wait for a finished accumulator, read it with
+//   warp 2      weight producer (lane 0): TMA of the packed tile [128][32 B]
+//               into a deeper ring of its own, so that weights coming from
+//               HBM are requested well before they are needed.
+//   warps 4-11  unpackers: thread (row r, half h) expands 16 packed bytes to
+//               64 unsigned codes c = q + 1 in {0, 1, 2} and stores them into
+//               the code tile of stage s in the swizzled layout the MMA reads.
+//   warps 12-19 epilogue: wait for a finished accumulator, read it with
 //               tcgen05.ld (lane = feature, column = token), release it, and
 //               write y = (acc - rowsum) * gamma * s_x with evict-first
-//               128-byte stores -- overlapping the next tile's MMAs.
+//               stores -- overlapping the next tile's MMAs.
 //
-// Tensor memory: accumulators in columns [0, 2 BT), operand slots after them.
-// Every mbarrier wait is bounded (see mbar_wait); on a timeout the kernel
-// records it in the status word, skips the remaining work and still frees
-// its tensor memory.
+// The single-thread issue loops matter: an MMA-issuing warp that waits with
+// warp-wide votes or commits twice per step leaves the tensor pipe idle for
+// longer than a K = 32 MMA lasts.
+//
+// sum_k x * c = sum_k x * q + sum_k x, so the epilogue subtracts the token's
+// rowsum.  Zero-filled tails (tokens >= M, features >= N, codes >= K) carry
+// x = 0 or c = 0 and add nothing.  Every mbarrier wait is bounded (see
+// mbar_wait); on a timeout the kernel records it in the status word, skips
+// the remaining work, lets its copies land and still frees its tensor memory.
 #pragma once
 
 #include <cuda.h>
@@ -38,10 +44,14 @@
 
 namespace tq {
 
-constexpr int kGemmThreads = 512;
-constexpr int kGemmAStages = 8;  // tensor-memory slots for the unpacked weights
+constexpr int kGemmWarps = 20;
+constexpr int kGemmThreads = 32 * kGemmWarps;
+constexpr int kUnpackWarps = 8;  // warps 4 .. 11
+constexpr int kEpiWarps = 8;     // warps 12 .. 19
 constexpr int kTileN = 128;      // features per tile (MMA M)
 constexpr int kTileK = 128;      // codes (bytes of x_q) per step
+constexpr int kWStageBytes = kTileN * kTileK / 4;  // packed bytes of one step's weight tile
+constexpr int kAStageBytes = kTileN * kTileK;      // unpacked codes of one step
 
 __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t v) {
     uint32_t p = 32;
@@ -51,17 +61,24 @@ __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t v) {
 
 template <int BT>
 struct GemmLayout {
-    static constexpr int kStages = BT >= 128 ? 10 : 12;  // x_q ring
-    static constexpr int kB = BT * kTileK;               // x_q bytes per stage
-    static constexpr int offB = 0;
-    static constexpr int offBar = offB + kStages * kB;
-    // barriers: full[S], empty[S], a_full[SA], a_empty[SA], d_full[2], d_empty[2], mma_done
-    static constexpr int kBars = 2 * kStages + 2 * kGemmAStages + 5;
+    static constexpr int kWStages = 8;      // packed-weight ring
+    static constexpr int kB = BT * kTileK;  // x_q bytes per stage
+    static constexpr int kStage = kB + kAStageBytes;
+    // x_q + code ring: as many stages as fit beside the weight ring
+    // (4 for BT = 256, 6 for 128, 8 for 64)
+    static constexpr int kStagesFit = (232448 - 1024 - 512 - kWStages * kWStageBytes) / kStage;
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    static constexpr int offStage = 0;  // stage s: x_q tile, then code tile (both 1024-aligned)
+    static constexpr int offW = kStages * kStage;
+    static constexpr int offBar = offW + kWStages * kWStageBytes;
+    // barriers: full[S], empty[S], w_full[SW], w_empty[SW], d_full[2], d_empty[2], mma_done
+    static constexpr int kBars = 2 * kStages + 2 * kWStages + 5;
     static constexpr int offTmem = offBar + kBars * 8;
     static constexpr int kBytes = offTmem + 16;
     static constexpr int kDynamic = kBytes + 1024;  // slack for 1024-byte alignment
-    static constexpr uint32_t kACol = 2 * BT;       // first TMEM column of the operand slots
-    static constexpr uint32_t kTmemCols = pow2_at_least(2 * BT + kGemmAStages * (kTileK / 4));
+    static constexpr uint32_t kTmemCols = pow2_at_least(2 * BT);
+    static_assert(kDynamic <= 232448, "shared memory per CTA");
+    static_assert(kB % 1024 == 0 && kAStageBytes % 1024 == 0, "swizzle atoms stay aligned");
 };
 
 // Natural-order expansion of one 32-bit packed word (16 codes) into 16
@@ -77,22 +94,14 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
                       __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632));
 }
 
-__device__ __forceinline__ uint4 ldg_nc_u4(const void *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 template <int BT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restrict__ packed,
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
                 const float *__restrict__ gamma, int per_row, int M, int N, int K,
                 float *__restrict__ y, int32_t *__restrict__ acc_out) {
     using L = GemmLayout<BT>;
-    constexpr int S = L::kStages;
+    constexpr int S = L::kStages, SW = L::kWStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -100,35 +109,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t bar0 = sbase + L::offBar;
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (S + s); };
-    auto a_full = [&](int s) { return bar0 + 8u * (2 * S + s); };
-    auto a_empty = [&](int s) { return bar0 + 8u * (2 * S + kGemmAStages + s); };
-    auto d_full = [&](int b) { return bar0 + 8u * (2 * S + 2 * kGemmAStages + b); };
-    auto d_empty = [&](int b) { return bar0 + 8u * (2 * S + 2 * kGemmAStages + 2 + b); };
-    const uint32_t mma_done = bar0 + 8u * (2 * S + 2 * kGemmAStages + 4);
+    auto w_full = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    auto w_empty = [&](int s) { return bar0 + 8u * (2 * S + SW + s); };
+    auto d_full = [&](int b) { return bar0 + 8u * (2 * S + 2 * SW + b); };
+    auto d_empty = [&](int b) { return bar0 + 8u * (2 * S + 2 * SW + 2 + b); };
+    const uint32_t mma_done = bar0 + 8u * (2 * S + 2 * SW + 4);
+    auto x_stage = [&](int s) { return sbase + (uint32_t)(L::offStage + s * L::kStage); };
+    auto a_stage = [&](int s) { return x_stage(s) + (uint32_t)L::kB; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::offTmem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_m = (M + BT - 1) / BT, num_n = (N + kTileN - 1) / kTileN;
     const int ntiles = num_m * num_n;
     const int nkb = (K + kTileK - 1) / kTileK;
-    const int KB = K / 4;  // packed bytes per weight row
+    // steps this CTA runs: its tiles times the steps per tile
+    const int my_tiles = ntiles > (int)blockIdx.x
+                             ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                             : 0;
+    const int total = my_tiles * nkb;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full(s), 1);
+            mbar_init(full(s), 1 + kUnpackWarps);  // TMA bytes + one arrive per unpacker warp
             mbar_init(empty(s), 1);
         }
-        for (int s = 0; s < kGemmAStages; ++s) {
-            mbar_init(a_full(s), 4);
-            mbar_init(a_empty(s), 1);
+        for (int s = 0; s < SW; ++s) {
+            mbar_init(w_full(s), 1);
+            mbar_init(w_empty(s), kUnpackWarps);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(d_full(b), 1);
-            mbar_init(d_empty(b), 4);
+            mbar_init(d_empty(b), kEpiWarps);
         }
         mbar_init(mma_done, 1);
         fence_barrier_init();
         prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_w);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -144,140 +160,144 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- TMA producer (lane 0 issues; the warp stays converged) ----------------
-        int g = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const int m0 = (t % num_m) * BT;
-            for (int kb = 0; kb < nkb; ++kb, ++g) {
+        // ---------------- x_q producer ----------------
+        if (lane == 0) {
+            int g = 0;
+            for (; g < total; ++g) {
                 const int s = g % S, r = g / S;
-                if (!warp_wait(empty(s), (r & 1) ^ 1, lane)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(full(s), L::kB);
-                    tma_load_2d(sbase + L::offB + s * L::kB, &tm_x, kb * kTileK, m0, full(s));
-                }
-                __syncwarp();
+                const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
+                const int kb = g % nkb;
+                if (!mbar_wait(empty(s), (r & 1) ^ 1)) break;
+                mbar_arrive_expect_tx(full(s), L::kB);
+                tma_load_2d(x_stage(s), &tm_x, kb * kTileK, (t % num_m) * BT, full(s));
             }
+            // Own copies must have landed before the CTA may exit (already
+            // true unless a wait gave up).
+            for (int j = g - S < 0 ? 0 : g - S; j < g; ++j) mbar_wait(full(j % S), (j / S) & 1);
         }
-        // Own copies must have landed before the CTA may exit (already true
-        // unless a wait above gave up).
-        for (int j = g - S < 0 ? 0 : g - S; j < g; ++j) warp_wait(full(j % S), (j / S) & 1, lane);
+        __syncwarp();
+    } else if (warp == 2) {
+        // ---------------- packed-weight producer ----------------
+        if (lane == 0) {
+            int g = 0;
+            for (; g < total; ++g) {
+                const int s = g % SW, r = g / SW;
+                const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
+                const int kb = g % nkb;
+                if (!mbar_wait(w_empty(s), (r & 1) ^ 1)) break;
+                mbar_arrive_expect_tx(w_full(s), kWStageBytes);
+                tma_load_2d(sbase + (uint32_t)(L::offW + s * kWStageBytes), &tm_w, kb * (kTileK / 4),
+                            (t / num_m) * kTileN, w_full(s));
+            }
+            for (int j = g - SW < 0 ? 0 : g - SW; j < g; ++j) mbar_wait(w_full(j % SW), (j / SW) & 1);
+        }
+        __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer (lane 0 issues) ----------------
-        constexpr uint32_t idesc = idesc_i8_u8s8(kTileN, BT);
-        int g = 0, tl = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tl) {
-            const int b = tl & 1;
-            if (!warp_wait(d_empty(b), ((tl >> 1) & 1) ^ 1, lane)) break;
-            tc_fence_after();
-            const uint32_t d_col = tmem + (uint32_t)(b * BT);
-            for (int kb = 0; kb < nkb; ++kb, ++g) {
-                const int s = g % S, r = g / S;
-                const int sa = g % kGemmAStages, ra = g / kGemmAStages;
-                if (!warp_wait(full(s), r & 1, lane) || !warp_wait(a_full(sa), ra & 1, lane)) {
-                    ok = false;
-                    break;
-                }
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8_u8s8(kTileN, BT);
+            int g = 0;
+            bool ok = true;
+            for (int tl = 0; tl < my_tiles && ok; ++tl) {
+                const int b = tl & 1;
+                if (!mbar_wait(d_empty(b), ((tl >> 1) & 1) ^ 1)) break;
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t a_col = tmem + L::kACol + (uint32_t)sa * (kTileK / 4);
-                    const uint32_t b_addr = sbase + L::offB + s * L::kB;
+                const uint32_t d_col = tmem + (uint32_t)(b * BT);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    if (!mbar_wait(full(s), (g / S) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = a_stage(s), b_addr = x_stage(s);
 #pragma unroll
                     for (int kk = 0; kk < kTileK / 32; ++kk)
-                        mma_i8_ts(d_col, a_col + kk * 8, smem_desc_sw128(b_addr + kk * 32), idesc,
-                                  (kb | kk) != 0 ? 1u : 0u);
+                        mma_i8(d_col, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
+                               idesc, (kb | kk) != 0 ? 1u : 0u);
                     mma_commit(empty(s));
-                    mma_commit(a_empty(sa));
                 }
-                __syncwarp();
+                if (ok) mma_commit(d_full(b));  // accumulator b complete
             }
-            if (ok && lane == 0) mma_commit(d_full(b));  // accumulator b complete
-            __syncwarp();
+            // No MMA may still use TMEM when it is freed: this commit fires
+            // once every MMA issued above has completed.
+            mma_commit(mma_done);
+            mbar_wait(mma_done, 0);
         }
-        // No MMA may still use TMEM when it is freed: this commit fires once
-        // every MMA issued above has completed.
-        if (lane == 0) mma_commit(mma_done);
         __syncwarp();
-        warp_wait(mma_done, 0, lane);
-    } else if (warp >= 4 && warp < 12) {
-        // ---------------- unpack into tensor memory ----------------
-        const int q = warp & 3;            // TMEM lane quarter
-        const int par = (warp - 4) >> 2;   // steps g with g % 2 == par
-        const int r = 32 * q + lane;       // row of the tile = TMEM lane
-        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-        const int total = ((ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * nkb;
-        // packed bytes of step g for this thread's row (zeros past N or K)
-        auto load_step = [&](int gg, uint4 &v0, uint4 &v1) {
-            v0 = make_uint4(0u, 0u, 0u, 0u);
-            v1 = v0;
-            if (gg >= total) return;
-            const int tt = (int)blockIdx.x + (gg / nkb) * (int)gridDim.x;
-            const int kb = gg % nkb;
-            const int n = (tt / num_m) * kTileN + r;
-            if (n >= N) return;
-            const uint8_t *src = packed + (int64_t)n * KB + kb * 32;
-            if (kb * 32 + 16 <= KB) v0 = ldg_nc_u4(src);
-            if (kb * 32 + 32 <= KB) v1 = ldg_nc_u4(src + 16);
-        };
-        uint4 c0, c1, n0_, n1_;
-        load_step(par, c0, c1);
-        for (int g = par; g < total; g += 2) {
-            load_step(g + 2, n0_, n1_);  // prefetch this warp's next step
-            const int sa = g % kGemmAStages, ra = g / kGemmAStages;
-            const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            uint32_t cols[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 e = expand_word(words[c]);
-                cols[4 * c + 0] = e.x;
-                cols[4 * c + 1] = e.y;
-                cols[4 * c + 2] = e.z;
-                cols[4 * c + 3] = e.w;
-            }
-            if (!warp_wait(a_empty(sa), (ra & 1) ^ 1, lane)) break;
-            tc_fence_after();
-            tmem_st32(lane_addr + L::kACol + (uint32_t)sa * (kTileK / 4), cols);
-            tmem_st_wait();
-            tc_fence_before();
+    } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
+        // ---------------- unpack codes into the swizzled operand tile ----------------
+        const int u = (warp - 4) * 32 + lane;
+        const int r = u & (kTileN - 1);  // weight row of the tile
+        const int h = u >> 7;            // half of the step: codes [64 h, 64 h + 64)
+        const uint32_t w_off = (uint32_t)(L::offW + r * (kTileK / 4) + h * 16);
+        const uint32_t a_row = (uint32_t)(r * kTileK);
+        for (int g = 0; g < total; ++g) {
+            const int ws = g % SW, s = g % S;
+            if (!warp_wait(w_full(ws), (g / SW) & 1, lane)) break;
+            uint4 pw;
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(pw.x), "=r"(pw.y), "=r"(pw.z), "=r"(pw.w)
+                         : "r"(sbase + w_off + (uint32_t)(ws * kWStageBytes))
+                         : "memory");
+            const uint4 e0 = expand_word(pw.x), e1 = expand_word(pw.y);
+            const uint4 e2 = expand_word(pw.z), e3 = expand_word(pw.w);
             __syncwarp();
-            if (lane == 0) mbar_arrive(a_full(sa));
-            c0 = n0_;
-            c1 = n1_;
+            if (lane == 0) mbar_arrive(w_empty(ws));  // packed bytes are in registers
+            if (!warp_wait(empty(s), ((g / S) & 1) ^ 1, lane)) break;
+            // 16-byte chunk c of row r lives at chunk position c ^ (r & 7)
+            const uint32_t base = a_stage(s) + a_row;
+            const uint4 e[4] = {e0, e1, e2, e3};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t c = (uint32_t)(4 * h + i);
+                const uint32_t addr = base + (((c ^ (uint32_t)(r & 7)) & 7u) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(e[i].x),
+                             "r"(e[i].y), "r"(e[i].z), "r"(e[i].w)
+                             : "memory");
+            }
+            fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full(s));
         }
     } else if (warp >= 12) {
         // ---------------- epilogue ----------------
-        const int q = warp & 3;
+        constexpr int kHalf = BT / 2;          // tokens per epilogue warp and tile
+        constexpr int kChunks = kHalf / 32;
+        const int q = warp & 3;                // TMEM lane quarter
+        const int half = (warp - 12) >> 2;     // token half of the tile
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-        int tl = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
+        for (int tl = 0; tl < my_tiles; ++tl) {
+            const int t = (int)blockIdx.x + tl * (int)gridDim.x;
             const int b = tl & 1;
+            const int m0 = (t % num_m) * BT + half * kHalf, n0 = (t / num_m) * kTileN;
+            const int n = n0 + 32 * q + lane;
+            // per-tile scalars, loaded while the accumulator is still being computed
+            const float gn = n < N ? __ldg(gamma + (per_row ? n : 0)) : 0.0f;
+            float sxc[kChunks];
+            int rsc[kChunks];
+#pragma unroll
+            for (int cc = 0; cc < kChunks; ++cc) {
+                const int mj = m0 + cc * 32 + lane;  // lane j holds token m0 + 32 cc + j
+                sxc[cc] = mj < M ? __ldg(s_x + mj) : 0.0f;
+                rsc[cc] = mj < M ? __ldg(rowsum + mj) : 0;
+            }
             if (!warp_wait(d_full(b), (tl >> 1) & 1, lane)) break;
             tc_fence_after();
-            const int m0 = (t % num_m) * BT, n0 = (t / num_m) * kTileN;
-            const int n = n0 + 32 * q + lane;
-            const float gn = n < N ? __ldg(gamma + (per_row ? n : 0)) : 0.0f;
-#pragma unroll 1
-            for (int cc = 0; cc < BT / 32; ++cc) {
+#pragma unroll
+            for (int cc = 0; cc < kChunks; ++cc) {
                 uint32_t v[32];
-                tmem_ld32(lane_addr + (uint32_t)(b * BT + cc * 32), v);
-                // this chunk's 32 tokens: lane j holds token m0 + 32 cc + j
-                const int mj = m0 + cc * 32 + lane;
-                const float sxj = mj < M ? __ldg(s_x + mj) : 0.0f;
-                const int rsj = mj < M ? __ldg(rowsum + mj) : 0;
+                tmem_ld32(lane_addr + (uint32_t)(b * BT + half * kHalf + cc * 32), v);
                 tmem_ld_wait();
-                if (cc == BT / 32 - 1) {  // accumulator fully read: hand it back to the MMA warp
+                if (cc == kChunks - 1) {  // accumulator fully read: hand it back to the MMA warp
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(d_empty(b));
                 }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float sxm = __shfl_sync(0xffffffffu, sxj, j);
-                    const int rsm = __shfl_sync(0xffffffffu, rsj, j);
+                    const float sxm = __shfl_sync(0xffffffffu, sxc[cc], j);
+                    const int rsm = __shfl_sync(0xffffffffu, rsc[cc], j);
                     const int m = m0 + cc * 32 + j;
                     if (m < M && n < N) {
                         const int a = (int)v[j] - rsm;
