@@ -19,9 +19,10 @@
 //   warp 2      weight producer (lane 0): TMA of the packed tile [128][32 B]
 //               into a deeper ring of its own, so that weights coming from
 //               HBM are requested well before they are needed.
-//   warps 4-11  unpackers: thread (row r, half h) expands 16 packed bytes to
-//               64 unsigned codes c = q + 1 in {0, 1, 2} and stores them into
-//               the code tile of stage s in the swizzled layout the MMA reads.
+//   warps 4-11  unpackers, two groups of four taking alternate steps: thread
+//               r of a group expands row r's 32 packed bytes to 128 unsigned
+//               codes c = q + 1 in {0, 1, 2} and stores them into the code
+//               tile of stage s in the swizzled layout the MMA reads.
 //   warps 12-19 epilogue: wait for a finished accumulator, read it with
 //               tcgen05.ld (lane = feature, column = token), release it, and
 //               write y = (acc - rowsum) * gamma * s_x with evict-first
@@ -130,12 +131,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full(s), 1 + kUnpackWarps);  // TMA bytes + one arrive per unpacker warp
+            mbar_init(full(s), 1 + kUnpackWarps / 2);  // TMA bytes + the step's four unpacker warps
             mbar_init(empty(s), 1);
         }
         for (int s = 0; s < SW; ++s) {
             mbar_init(w_full(s), 1);
-            mbar_init(w_empty(s), kUnpackWarps);
+            mbar_init(w_empty(s), kUnpackWarps / 2);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(d_full(b), 1);
@@ -227,35 +228,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
         // ---------------- unpack codes into the swizzled operand tile ----------------
-        const int u = (warp - 4) * 32 + lane;
-        const int r = u & (kTileN - 1);  // weight row of the tile
-        const int h = u >> 7;            // half of the step: codes [64 h, 64 h + 64)
-        const uint32_t w_off = (uint32_t)(L::offW + r * (kTileK / 4) + h * 16);
-        const uint32_t a_row = (uint32_t)(r * kTileK);
-        for (int g = 0; g < total; ++g) {
+        // Two groups of four warps take alternate steps, so each has two steps'
+        // time for its waits, loads and stores; thread r of a group owns row r.
+        const int par = (warp - 4) >> 2;
+        const int r = 32 * (warp & 3) + lane;  // weight row of the tile
+        const uint32_t w_row = sbase + (uint32_t)(L::offW + r * (kTileK / 4));
+        const uint32_t a_row = (uint32_t)(r * kTileK), sw = (uint32_t)(r & 7);
+        for (int g = par; g < total; g += 2) {
             const int ws = g % SW, s = g % S;
             if (!warp_wait(w_full(ws), (g / SW) & 1, lane)) break;
-            uint4 pw;
+            uint4 p0, p1;
+            const uint32_t src = w_row + (uint32_t)(ws * kWStageBytes);
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                         : "=r"(pw.x), "=r"(pw.y), "=r"(pw.z), "=r"(pw.w)
-                         : "r"(sbase + w_off + (uint32_t)(ws * kWStageBytes))
+                         : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w)
+                         : "r"(src)
                          : "memory");
-            const uint4 e0 = expand_word(pw.x), e1 = expand_word(pw.y);
-            const uint4 e2 = expand_word(pw.z), e3 = expand_word(pw.w);
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w)
+                         : "r"(src + 16u)
+                         : "memory");
+            const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            uint4 e[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) e[c] = expand_word(words[c]);
             __syncwarp();
             if (lane == 0) mbar_arrive(w_empty(ws));  // packed bytes are in registers
             if (!warp_wait(empty(s), ((g / S) & 1) ^ 1, lane)) break;
             // 16-byte chunk c of row r lives at chunk position c ^ (r & 7)
             const uint32_t base = a_stage(s) + a_row;
-            const uint4 e[4] = {e0, e1, e2, e3};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t c = (uint32_t)(4 * h + i);
-                const uint32_t addr = base + (((c ^ (uint32_t)(r & 7)) & 7u) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(e[i].x),
-                             "r"(e[i].y), "r"(e[i].z), "r"(e[i].w)
+            for (int c = 0; c < 8; ++c)
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base + (((uint32_t)c ^ sw) << 4)),
+                             "r"(e[c].x), "r"(e[c].y), "r"(e[c].z), "r"(e[c].w)
                              : "memory");
-            }
             fence_proxy_async_smem();  // generic stores -> visible to the tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(full(s));
