@@ -77,16 +77,28 @@ typedef enum tq_status {
 #define TQ_FLAG_ETA_CLAMP (1u << 3)          /* clamp eta to [eta_min, eta_max]                */
 #define TQ_FLAG_SANITIZE_NONFINITE (1u << 4) /* quench NaN / +-Inf inputs first                */
 #define TQ_FLAG_WEIGHTS_STATIC (1u << 5)     /* see "Launch overlap" below                      */
+#define TQ_FLAG_INPUTS_READY (1u << 6)       /* see "Launch overlap" below                      */
 
 /*
  * Launch overlap.  Every kernel is launched with programmatic dependent launch:
- * it may be scheduled while the previous kernel on the stream is still
- * finishing, and waits for that kernel's results before reading or writing
- * any buffer.  With TQ_FLAG_WEIGHTS_STATIC (tq_ternary_gemm,
- * tq_bitlinear_fused) the caller promises that the packed weights and gamma
- * were not written by the immediately preceding work on the stream (true for
- * the layers of a model during inference); the small-M GEMV then starts
- * streaming weights before that wait.  Without the flag nothing is read early.
+ * it may be scheduled while earlier kernels on the stream are still finishing,
+ * and waits for the previous kernel's completion before reading or writing
+ * any buffer.  "In flight" below means: enqueued on the stream since the last
+ * point at which the stream was drained (a host synchronisation, an event
+ * wait, the start of a CUDA graph launch).
+ *
+ * TQ_FLAG_WEIGHTS_STATIC (tq_ternary_gemm, tq_bitlinear_fused): the caller
+ * promises that no work in flight writes the packed weights or gamma (true for
+ * the layers of a model during inference).  The small-M GEMV then starts
+ * streaming weights and gamma before the wait.
+ *
+ * TQ_FLAG_INPUTS_READY (tq_ternary_gemm): the caller promises that no work in
+ * flight writes any input of the call (xq, s_x, rowsum, packed, gamma) or
+ * reads or writes its outputs (y, acc) -- e.g. the independent projections of
+ * one decode step that share an activation (q/k/v, gate/up), each with its own
+ * output.  The kernel then reads and computes at once and waits for the
+ * previous kernel only before it exits, so any later call still sees every
+ * earlier result.  Without either flag nothing is read early.
  */
 
 /*
@@ -176,7 +188,8 @@ TQ_API tq_status tq_fwht512(const float *x, float *y, int64_t rows, int64_t K, i
  *                    ([M][K] int8, [M] fp32, [M] int32).
  *   packed, gamma    as written by tq_quantize_ternary_pack ([N][K/4], [N] or [1]).
  *   flags            TQ_GAMMA_PER_ROW selects gamma[N] (else gamma[0]);
- *                    TQ_FLAG_WEIGHTS_STATIC as described under "Launch overlap".
+ *                    TQ_FLAG_WEIGHTS_STATIC, TQ_FLAG_INPUTS_READY as described
+ *                    under "Launch overlap".
  *   y                [M][N] fp32, written: y = fp32(acc) * (gamma_n * s_x[m]).
  *   acc              [M][N] int32 or NULL: if given, the exact integer sums
  *                    acc[m][n] = sum_k xq[m][k] * q[n][k] are written too.

@@ -23,6 +23,7 @@ FLAG_RMSNORM = 1 << 2
 FLAG_ETA_CLAMP = 1 << 3
 FLAG_SANITIZE_NONFINITE = 1 << 4
 FLAG_WEIGHTS_STATIC = 1 << 5
+FLAG_INPUTS_READY = 1 << 6
 
 STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN", 4: "TQ_ERR_ARG",
           5: "TQ_ERR_CUDA", 6: "TQ_ERR_DEVICE", 7: "TQ_ERR_TIMEOUT"}

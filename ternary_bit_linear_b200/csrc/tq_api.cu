@@ -138,7 +138,7 @@ bool make_tmap_u8(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows
 template <int BT>
 tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
-                      int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
+                      int64_t K, float *y, int32_t *acc, int mode, int sms, cudaStream_t st) {
     using L = GemmLayout<BT>;
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
@@ -159,52 +159,44 @@ tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
     const int64_t tiles = ((M + BT - 1) / BT) * ((N + kTileN - 1) / kTileN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
     return launch_pdl(gemm_kernel<BT>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
-                      s_x, rowsum, gamma, per_row, (int)M, (int)N, (int)K, y, acc);
+                      s_x, rowsum, gamma, per_row, (int)M, (int)N, (int)K, y, acc, mode);
 }
 
-// Grid: at most half of the CTAs that fit on the device, so that the next
-// kernel's CTAs can be resident (and prefetching its weights under
-// programmatic dependent launch) while this one finishes; one strip per CTA
-// when that is enough, else a persistent ring of two stages.
-template <int NB, int MAXSTEP, int W>
+// Grid: one 16-row strip per CTA while that keeps the grid within the CTAs
+// that fit on the device at once (at most four per SM, so that several
+// layers' kernels can be resident together under programmatic dependent
+// launch); beyond that, runs of strips per CTA through a ring of up to
+// kGemvMaxStages stages.  Large x_q (M * K) costs shared memory per CTA and
+// L2 traffic per CTA, so it lowers the CTAs per SM and lengthens the runs.
+template <int NB, int W>
 tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
-                      int64_t K, float *y, int32_t *acc, int static_w, int sms, cudaStream_t st) {
-    static std::atomic<int> occ1[kMaxDevices], occ2[kMaxDevices];
+                      int64_t K, float *y, int32_t *acc, int mode, int sms, cudaStream_t st) {
+    static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
-    const int sb = gemv_stage_bytes((int)K);
-    if (!occ1[dev].load()) {
-        if (cudaFuncSetAttribute(gemv_kernel<NB, MAXSTEP, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!attr_done[dev].load()) {
+        if (cudaFuncSetAttribute(gemv_kernel<NB, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemvSmemCap) != cudaSuccess)
             return TQ_ERR_CUDA;
-        int a = 0, b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, gemv_kernel<NB, MAXSTEP, W>, W * 32,
-                                                          (size_t)sb) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, gemv_kernel<NB, MAXSTEP, W>, W * 32,
-                                                          (size_t)2 * sb) != cudaSuccess)
-            return TQ_ERR_CUDA;
-        occ2[dev].store(b > 1 ? b : 1);
-        occ1[dev].store(a > 1 ? a : 1);
+        attr_done[dev].store(1);
     }
     const int64_t nstrips = (N + 15) / 16;
-    const int64_t half1 = (int64_t)(occ1[dev].load() / 2 > 0 ? occ1[dev].load() / 2 : 1) * sms;
-    int64_t grid, per_cta;
-    int nstage;
-    if (nstrips <= half1) {
-        grid = nstrips;
-        per_cta = 1;
-        nstage = 1;
-    } else {
-        const int64_t half2 = (int64_t)(occ2[dev].load() / 2 > 0 ? occ2[dev].load() / 2 : 1) * sms;
-        grid = nstrips < half2 ? nstrips : half2;
-        per_cta = (nstrips + grid - 1) / grid;
-        nstage = per_cta < 2 ? 1 : 2;
-    }
-    const size_t smem = (size_t)nstage * sb;
-    return launch_pdl(gemv_kernel<NB, MAXSTEP, W>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq,
-                      s_x, rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, static_w,
-                      nstage);
+    const int xb = gemv_x_bytes((int)M, (int)K), sb = gemv_stage_bytes((int)K);
+    int64_t per_sm = kGemvSmemCap / (xb + sb);
+    if (per_sm > 4) per_sm = 4;
+    if (per_sm < 1) per_sm = 1;
+    const int64_t max_grid = per_sm * (int64_t)sms;
+    const int64_t per_cta = (nstrips + max_grid - 1) / max_grid;
+    const int64_t grid = (nstrips + per_cta - 1) / per_cta;
+    int64_t nstage = (kGemvSmemCap - xb) / sb;
+    if (nstage > per_cta) nstage = per_cta;
+    if (nstage > kGemvMaxStages) nstage = kGemvMaxStages;
+    if (nstage < 1) return TQ_ERR_SHAPE;  // cannot happen for K <= kGemvMaxK, M <= 16
+    const size_t smem = (size_t)xb + (size_t)nstage * sb;
+    return launch_pdl(gemv_kernel<NB, W>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq, s_x,
+                      rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, mode, (int)nstage,
+                      (int)per_cta);
 }
 
 template <int NW>
@@ -299,26 +291,23 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
                         const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
                         int64_t N, int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
     const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
-    const int static_w = (flags & TQ_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+    const int mode = ((flags & TQ_FLAG_WEIGHTS_STATIC) ? kModeWeightsStatic : 0) |
+                     ((flags & TQ_FLAG_INPUTS_READY) ? kModeInputsReady : 0);
     if (M <= 16 && K <= kGemvMaxK) {
-        const int nsteps = (int)((K / 4 + 63) / 64);  // 64-byte column steps per row
-#define TQ_GEMV(NB, MS, W) \
-    return launch_gemv<NB, MS, W>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, static_w, sms, st)
-        if (M <= 8) {
-            if (nsteps <= 4) TQ_GEMV(1, 1, 4);
-            if (nsteps <= 8) TQ_GEMV(1, 2, 4);
-            if (nsteps <= 16) TQ_GEMV(1, 4, 4);
-            TQ_GEMV(1, 4, 8);
-        }
-        if (nsteps <= 4) TQ_GEMV(2, 1, 4);
-        if (nsteps <= 8) TQ_GEMV(2, 2, 4);
-        if (nsteps <= 16) TQ_GEMV(2, 4, 4);
-        TQ_GEMV(2, 4, 8);
-#undef TQ_GEMV
+        // A dependent chain of layers waits on each kernel's critical path, so
+        // more warps share a strip; with ready inputs the kernels overlap and
+        // leaner CTAs let more of them be resident.
+        const int64_t nsteps = (K / 4 + 63) / 64;  // 64-byte column steps per row
+        const bool lean = nsteps <= 8 || ((mode & kModeInputsReady) && nsteps <= 16);
+        if (M <= 8)
+            return lean ? launch_gemv<1, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st)
+                        : launch_gemv<1, 8>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+        return lean ? launch_gemv<2, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st)
+                    : launch_gemv<2, 8>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
     }
-    if (M <= 64) return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
-    if (M <= 128) return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
-    return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, sms, st);
+    if (M <= 64) return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    if (M <= 128) return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
 }
 
 }  // namespace
@@ -436,7 +425,7 @@ tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *row
     if (!xq || !s_x || !rowsum || !packed || !gamma || !y) return TQ_ERR_NULL;
     if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
-    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC)) return TQ_ERR_ARG;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY)) return TQ_ERR_ARG;
     if (!aligned16(xq) || !aligned16(s_x) || !aligned16(rowsum) || !aligned16(packed) ||
         !aligned16(gamma) || !aligned16(y) || (acc && !aligned16(acc)))
         return TQ_ERR_ALIGN;

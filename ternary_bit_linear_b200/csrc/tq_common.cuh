@@ -23,6 +23,8 @@ constexpr unsigned kStatusTimeout = 1u;
 
 // A wait gives up after this much wall time (ns, %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+// Longest single sleep of a waiting thread (ns); the phase completing wakes it earlier.
+constexpr uint32_t kWaitHintNs = 1000000u;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;
@@ -38,6 +40,12 @@ __device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, kStatusTime
 // and lets the next kernel be scheduled early (pdl_trigger).  Without the
 // launch attribute both are no-ops.
 // ---------------------------------------------------------------------------
+// Launch modes of the contraction kernels (set from TQ_FLAG_WEIGHTS_STATIC and
+// TQ_FLAG_INPUTS_READY): weights may be read before the wait; no wait at all
+// before reading, only before exiting.
+constexpr int kModeWeightsStatic = 1;
+constexpr int kModeInputsReady = 2;
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -75,14 +83,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps until it completes (or the hint runs out) instead of spinning, so
+// waiting warps leave the issue slots to the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kWaitHintNs)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  Returns false (and sets
 // the timeout bit) if it did not complete within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (;;) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait_sleep(bar, parity)) return true;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             flag_timeout();
             return false;

@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
                 const float *__restrict__ gamma, int per_row, int M, int N, int K,
-                float *__restrict__ y, int32_t *__restrict__ acc_out) {
+                float *__restrict__ y, int32_t *__restrict__ acc_out, int mode) {
     using L = GemmLayout<BT>;
     constexpr int S = L::kStages, SW = L::kWStages;
     extern __shared__ uint8_t smem_raw[];
@@ -152,8 +152,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_relinquish();
     }
     // Everything above touched no global memory; inputs of the previous kernel
-    // on the stream are visible after this wait.
-    pdl_wait();
+    // on the stream are visible after this wait.  With ready inputs the kernel
+    // skips it here and waits before exiting instead (stream completion order).
+    if (!(mode & kModeInputsReady)) pdl_wait();
     pdl_trigger();
     tc_fence_before();
     __syncthreads();
@@ -313,6 +314,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     }
+    if (mode & kModeInputsReady) pdl_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

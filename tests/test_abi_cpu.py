@@ -33,6 +33,18 @@ def test_header_declares_the_five_calls_and_helpers():
     assert names == set(tq.SIGNATURES), "binding and header disagree"
 
 
+def test_header_flag_values_match_binding():
+    src = open(HEADER).read()
+    flags = dict((k, int(v)) for k, v in re.findall(r"#define\s+TQ_(\w+)\s+\(1u\s*<<\s*(\d+)\)", src))
+    py = {"GAMMA_PER_ROW": tq.GAMMA_PER_ROW, "FLAG_FWHT": tq.FLAG_FWHT, "FLAG_RMSNORM": tq.FLAG_RMSNORM,
+          "FLAG_ETA_CLAMP": tq.FLAG_ETA_CLAMP, "FLAG_SANITIZE_NONFINITE": tq.FLAG_SANITIZE_NONFINITE,
+          "FLAG_WEIGHTS_STATIC": tq.FLAG_WEIGHTS_STATIC, "FLAG_INPUTS_READY": tq.FLAG_INPUTS_READY}
+    for name, value in py.items():
+        assert name in flags, name
+        assert value == 1 << flags[name], name
+    assert len(set(py.values())) == len(py)
+
+
 def test_library_exports_every_declared_symbol(lib):
     for n in declared_functions():
         assert hasattr(lib, n), n

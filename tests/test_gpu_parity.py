@@ -448,3 +448,46 @@ def test_dependent_calls_back_to_back(cuda_lib):
         acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
         assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, False))
     assert tq.device_status() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (8, 1000, 4096), (16, 257, 8192), (300, 384, 1536)])
+def test_inputs_ready_flag_same_result_and_order(cuda_lib, M, N, K):
+    """Independent contractions that share one activation (q/k/v style), each
+    with its own output, launched with TQ_FLAG_INPUTS_READY back to back; then
+    a flag-less consumer re-packs into the first weight buffer.  Every result
+    must equal the flag-less one, and the re-pack must not overtake them."""
+    tq = cuda_lib
+    X = S.decode_acts(M, K, seed=41)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    xq, sx, rs = dev(xq_ref), dev(sx_ref), dev(rs_ref)
+    Ws = [S.normal((N, K), 0.02, 42 + i, N) for i in range(4)]
+    refs = [oracle.quantize_pack(W, per_row=True) for W in Ws]
+    P = [(dev(p), dev(g)) for p, g in refs]
+    fl = tq.GAMMA_PER_ROW | tq.FLAG_WEIGHTS_STATIC
+    torch.cuda.synchronize()
+    ys = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in Ws]
+    for (p, g), y in zip(P, ys):
+        tq.ternary_gemm_(xq, sx, rs, p, g, fl | tq.FLAG_INPUTS_READY, y)
+    # a flag-less call right behind them overwrites the first weights
+    ws = torch.empty((max(16, tq.pack_workspace_bytes(N, K, tq.GAMMA_PER_ROW)),), dtype=torch.uint8,
+                     device="cuda")
+    tq.quantize_ternary_pack_(dev(Ws[1]), tq.GAMMA_PER_ROW, P[0][0], P[0][1], ws)
+    y_after = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    tq.ternary_gemm_(xq, sx, rs, P[0][0], P[0][1], tq.GAMMA_PER_ROW, y_after)
+    for (p_ref, g_ref), y in zip(refs, ys):
+        acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
+        assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, True))
+    assert torch.equal(y_after, ys[1])
+    assert tq.device_status() == 0
+
+
+def test_inputs_ready_flag_rejected_by_fused(cuda_lib):
+    tq = cuda_lib
+    M, N, K = 4, 64, 512
+    x = torch.zeros((M, K), dtype=torch.float32, device="cuda")
+    packed = torch.zeros((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.ones((1,), dtype=torch.float32, device="cuda")
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    ws = torch.empty((max(16, tq.fused_workspace_bytes(M, K, 0)),), dtype=torch.uint8, device="cuda")
+    with pytest.raises(RuntimeError):
+        tq.bitlinear_fused_(x, packed, gamma, tq.FLAG_INPUTS_READY, y, ws)
