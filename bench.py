@@ -16,6 +16,14 @@ A ring of L = 64 distinct layers keeps every working set above L2: per step the
 batches are quantised, and each batch runs through the GEMV of all 64 layers.
 Metric: algorithmic HBM bytes of the step / step time (GB/s).
 
+The layers of the ring share the activation and have their own weights,
+outputs and workspaces, so the packs of one segment, and the contractions of
+one segment, are independent calls: they are issued with TQ_FLAG_INPUTS_READY
+(and TQ_FLAG_WEIGHTS_STATIC for the contractions), which lets consecutive
+kernels overlap.  For the small-M GEMVs the line also reports "chain": the
+same launches as a chain of dependent layers (each kernel waits for the
+previous one before reading), timed separately and not part of the step.
+
 Timing: CUDA graphs for each segment (pack, activation quantisation, GEMV
 M=1, GEMV M=8), CUDA events between segments on the launching stream, barrier
 + synchronize around the timed steps, max over ranks.  Per-kernel average
@@ -147,6 +155,7 @@ class Workload:
         self.name, self.tq, self.torch, self.dev = name, tq, torch, dev
         f32, u8, i8, i32 = torch.float32, torch.uint8, torch.int8, torch.int32
         self.segments = []  # (label, kernel_name, launches, algorithmic bytes or ops, [fns])
+        self.chains = []    # (label, launches, bytes per launch, [fns]): dependent-layer GEMV chains
         if name == "decode":
             N = K = 4096
             self.N, self.K, self.Ms, self.L = N, K, [1, 8], layers
@@ -181,10 +190,14 @@ class Workload:
             raise SystemExit(f"unknown workload {name}")
         N, K, L = self.N, self.K, self.L
         self.flags = tq.GAMMA_PER_ROW if self.per_row else 0
+        # the ring's layers share x and have their own weights and outputs:
+        # independent calls, so the contractions may overlap one another
+        self.ready_flags = self.flags | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY
         self.packed = [torch.empty((N, K // 4), dtype=u8, device=dev) for _ in range(L)]
         self.gamma = [torch.empty((N if self.per_row else 1,), dtype=f32, device=dev) for _ in range(L)]
         nws = tq.pack_workspace_bytes(N, K, self.flags)
-        self.pack_ws = torch.empty((max(nws, 16),), dtype=u8, device=dev)
+        # one workspace per layer: the ring's packs are independent calls
+        self.pack_ws = [torch.empty((max(nws, 16),), dtype=u8, device=dev) for _ in range(L)]
         self.Xd = {M: x.to(dev) for M, x in self.X.items()}
         self.xq = {M: torch.empty((M, K), dtype=i8, device=dev) for M in self.Ms}
         self.sx = {M: torch.empty((M,), dtype=f32, device=dev) for M in self.Ms}
@@ -199,8 +212,8 @@ class Workload:
         pack_bytes = 4 * N * K + N * K // 4 + 4 * (N if self.per_row else 1)
         pack_launches = 1 if self.per_row else 3
         self.segments.append(("pack", "pack", L, L * pack_bytes, L * pack_launches,
-                              [lambda l=l: tq.quantize_ternary_pack_(self.W[l], self.flags, self.packed[l],
-                                                                      self.gamma[l], self.pack_ws)
+                              [lambda l=l: tq.quantize_ternary_pack_(self.W[l], self.flags | tq.FLAG_INPUTS_READY,
+                                                                      self.packed[l], self.gamma[l], self.pack_ws[l])
                                for l in range(L)]))
         if name == "fused":
             M = self.Ms[0]
@@ -221,9 +234,14 @@ class Workload:
             self.segments.append(("gemv M=%d" % M if gemv else "gemm M=%d" % M,
                                   "gemv" if gemv else "gemm", L, L * work, L, [
                 lambda l=l, M=M: tq.ternary_gemm_(self.xq[M], self.sx[M], self.rs[M], self.packed[l],
-                                                  self.gamma[l], self.flags | tq.FLAG_WEIGHTS_STATIC,
-                                                  self.y[M][l])
+                                                  self.gamma[l], self.ready_flags, self.y[M][l])
                 for l in range(L)]))
+            if gemv:
+                self.chains.append(("gemv M=%d" % M, L, work, [
+                    lambda l=l, M=M: tq.ternary_gemm_(self.xq[M], self.sx[M], self.rs[M], self.packed[l],
+                                                      self.gamma[l], self.flags | tq.FLAG_WEIGHTS_STATIC,
+                                                      self.y[M][l])
+                    for l in range(L)]))
 
     def step_bytes(self):
         return sum(s[3] for s in self.segments if s[1] in ("pack", "act_quant", "gemv"))
@@ -295,6 +313,7 @@ def run_ours(args, rank, world, local_rank):
 
     # --- end to end through the public API with host buffers ---
     e2e = run_e2e(args, wl, tq, torch, stream, graphs, world)
+    chain = run_chains(args, wl, tq, torch, stream, world)
 
     pk = peaks()
     kernels = {}
@@ -338,6 +357,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
         "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
     }
+    if chain:
+        out["chain"] = chain
     if rank == 0:
         print(json.dumps(out), flush=True)
     del graphs
@@ -367,6 +388,42 @@ def config_for(name, layers, world):
 
 def wl_config(wl, world):
     return config_for(wl.name, wl.L, world)
+
+
+def run_chains(args, wl, tq, torch, stream, world):
+    """Dependent-layer GEMV chains: per-launch time when every kernel waits
+    for its predecessor's results (the latency-bound decode case)."""
+    import torch as _t
+    res = {}
+    pk = peaks()
+    for label, launches, work, fns in wl.chains:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for fn in fns:
+                fn()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for fn in fns:
+                    fn()
+            for _ in range(3):
+                g.replay()
+        torch.cuda.synchronize()
+        reps = max(3, min(args.steps, 20))
+        e0, e1 = _t.cuda.Event(enable_timing=True), _t.cuda.Event(enable_timing=True)
+        barrier(world)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = allreduce_max(e0.elapsed_time(e1), world) / (reps * launches)
+        ach = work / (ms * 1e-3) / 1e9
+        res[label] = {"us_per_launch": round(ms * 1e3, 3), "achieved": round(ach, 1), "unit": "GB/s",
+                      "frac": round(ach / pk["hbm"], 4)}
+        del g
+    assert tq.device_status(stream) == 0
+    return res
 
 
 def run_e2e(args, wl, tq, torch, stream, graphs, world):

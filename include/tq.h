@@ -92,13 +92,14 @@ typedef enum tq_status {
  * the layers of a model during inference).  The small-M GEMV then starts
  * streaming weights and gamma before the wait.
  *
- * TQ_FLAG_INPUTS_READY (tq_ternary_gemm): the caller promises that no work in
- * flight writes any input of the call (xq, s_x, rowsum, packed, gamma) or
- * reads or writes its outputs (y, acc) -- e.g. the independent projections of
- * one decode step that share an activation (q/k/v, gate/up), each with its own
- * output.  The kernel then reads and computes at once and waits for the
- * previous kernel only before it exits, so any later call still sees every
- * earlier result.  Without either flag nothing is read early.
+ * TQ_FLAG_INPUTS_READY (tq_ternary_gemm, tq_quantize_ternary_pack): the
+ * caller promises that no work in flight writes any input of the call or
+ * reads or writes its outputs or workspace -- e.g. the independent
+ * projections of one decode step that share an activation (q/k/v, gate/up),
+ * each with its own output, or the packing of a model's layers, each with its
+ * own buffers.  The first kernel of the call then reads and computes at once
+ * and waits for the previous kernel only before it exits, so any later call
+ * still sees every earlier result.  Without either flag nothing is read early.
  */
 
 /*
@@ -108,8 +109,9 @@ typedef enum tq_status {
  * variant is Foundry's per-channel granularity (fq_quantize_ternary_per_channel).
  *
  *   w       [N][K] fp32, read only.
- *   flags   TQ_GAMMA_PER_ROW and/or TQ_FLAG_SANITIZE_NONFINITE (nan -> 0,
- *           +-inf -> +-1 before anything else, Hetman-2b section 2).
+ *   flags   TQ_GAMMA_PER_ROW, TQ_FLAG_SANITIZE_NONFINITE (nan -> 0,
+ *           +-inf -> +-1 before anything else, Hetman-2b section 2),
+ *           TQ_FLAG_INPUTS_READY (see "Launch overlap").
  *   packed  [N][K/4] bytes, written: byte j of row n holds codes 4j..4j+3 in bits
  *           (0,1) (2,3) (4,5) (6,7); 0b11 is never produced.
  *   gamma   [N] (per row) or [1] (per tensor) fp32, written: the fp32 nearest to

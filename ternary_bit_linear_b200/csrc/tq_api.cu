@@ -235,49 +235,56 @@ void launch_act(const float *x, const ActParams &p, int64_t M, int64_t K, int8_t
 }
 
 // Persistent pack grid: as many CTAs as fit on the device, at most one row per
-// team.  K <= 16384: a team of T warps holds a row in registers; larger K:
-// one warp streams the row twice.
+// team.  K <= 8192: a team of T warps streams its rows through a shared-memory
+// ring (smem bytes per CTA); larger K: one warp streams each row twice.
 template <typename Kern>
-tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_cta, const float *w,
-                           int64_t N, int64_t K, uint8_t *packed, float *gamma, const float *t,
-                           int reverse, cudaStream_t st) {
+tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_cta, int smem,
+                           const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
+                           const float *t, int reverse, int ready, cudaStream_t st) {
     int dev = 0, sms = 0;
     if (tq_status e = check_device(&sms)) return e;
     cudaGetDevice(&dev);
-    int per_sm = occ[dev].load();
-    if (per_sm == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPackThreads, 0) != cudaSuccess)
+    // occupancy depends on smem, i.e. on K: cache it per (device, smem)
+    const int key = occ[dev].load();
+    int per_sm = 0;
+    if ((key >> 8) == smem + 1) {
+        per_sm = key & 0xff;
+    } else {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPackThreads, (size_t)smem) !=
+                cudaSuccess)
             return TQ_ERR_CUDA;
         if (per_sm < 1) per_sm = 1;
-        occ[dev].store(per_sm);
+        occ[dev].store(((smem + 1) << 8) | (per_sm & 0xff));
     }
     const int64_t need = (N + rows_per_cta - 1) / rows_per_cta;
     const int64_t cap = (int64_t)per_sm * sms;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
-    return launch_pdl(kern, dim3(grid), dim3(kPackThreads), 0, st, w, N, (int)K, 1.0 / (double)K,
-                      packed, gamma, t, reverse);
+    return launch_pdl(kern, dim3(grid), dim3(kPackThreads), (size_t)smem, st, w, N, (int)K,
+                      1.0 / (double)K, packed, gamma, t, reverse, ready);
 }
 
 template <bool SAN>
 tq_status launch_pack_rows_s(const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
-                             const float *t, int reverse, cudaStream_t st) {
+                             const float *t, int reverse, int ready, cudaStream_t st) {
     static std::atomic<int> occ[5][kMaxDevices];
     const int64_t nv = K / 4;
+    const int k = (int)K;
     if (nv <= 32 * kTeamVec * 1)
-        return launch_pack_grid(pack_team_kernel<1, SAN>, occ[0], kPackWarps / 1, w, N, K, packed, gamma, t, reverse, st);
+        return launch_pack_grid(pack_team_kernel<1, SAN>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, t, reverse, ready, st);
     if (nv <= 32 * kTeamVec * 2)
-        return launch_pack_grid(pack_team_kernel<2, SAN>, occ[1], kPackWarps / 2, w, N, K, packed, gamma, t, reverse, st);
+        return launch_pack_grid(pack_team_kernel<2, SAN>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, t, reverse, ready, st);
     if (nv <= 32 * kTeamVec * 4)
-        return launch_pack_grid(pack_team_kernel<4, SAN>, occ[2], kPackWarps / 4, w, N, K, packed, gamma, t, reverse, st);
+        return launch_pack_grid(pack_team_kernel<4, SAN>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, t, reverse, ready, st);
     if (nv <= 32 * kTeamVec * 8)
-        return launch_pack_grid(pack_team_kernel<8, SAN>, occ[3], kPackWarps / 8, w, N, K, packed, gamma, t, reverse, st);
-    return launch_pack_grid(pack_rows_kernel<SAN>, occ[4], kPackWarps, w, N, K, packed, gamma, t, reverse, st);
+        return launch_pack_grid(pack_team_kernel<8, SAN>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, t, reverse, ready, st);
+    return launch_pack_grid(pack_rows_kernel<SAN>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, t, reverse, ready, st);
 }
 
 tq_status launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
-                           float *gamma, const float *t, int reverse, cudaStream_t st) {
-    return sanitize ? launch_pack_rows_s<true>(w, N, K, packed, gamma, t, reverse, st)
-                    : launch_pack_rows_s<false>(w, N, K, packed, gamma, t, reverse, st);
+                           float *gamma, const float *t, int reverse, int ready, cudaStream_t st) {
+    return sanitize ? launch_pack_rows_s<true>(w, N, K, packed, gamma, t, reverse, ready, st)
+                    : launch_pack_rows_s<false>(w, N, K, packed, gamma, t, reverse, ready, st);
 }
 
 size_t pack_parts(int64_t nv) {
@@ -342,9 +349,10 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     if (!w || !packed || !gamma) return TQ_ERR_NULL;
     if (N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
-    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE)) return TQ_ERR_ARG;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_INPUTS_READY)) return TQ_ERR_ARG;
     if (!aligned16(w) || !aligned16(packed) || !aligned16(gamma)) return TQ_ERR_ALIGN;
     const bool per_row = flags & TQ_GAMMA_PER_ROW;
+    const int ready = (flags & TQ_FLAG_INPUTS_READY) ? 1 : 0;
     const size_t wbytes = (size_t)(N * K) * 4, pbytes = (size_t)(N * K / 4),
                  gbytes = (per_row ? (size_t)N : 1) * 4;
     if (overlap(w, wbytes, packed, pbytes) || overlap(w, wbytes, gamma, gbytes) ||
@@ -363,7 +371,7 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, st)) return e;
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, ready, st)) return e;
         return launch_status();
     }
     const int64_t total_v = N * K / 4;
@@ -372,13 +380,13 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     double *partial = reinterpret_cast<double *>(workspace);
     float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + nparts * sizeof(DD));
     if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
-                                 st, w, total_v, chunk, sanitize, partial))
+                                 st, w, total_v, chunk, sanitize, partial, ready))
         return e;
     if (tq_status e = launch_pdl(absum_finalize_kernel, dim3(1), dim3(1024), 0, st, partial,
                                  (int)nparts, absum_tree_height(chunk, (int)nparts), w, total_v,
                                  sanitize, gamma, thresh))
         return e;
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, st)) return e;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, 0, st)) return e;
     return launch_status();
 }
 
@@ -599,7 +607,7 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, st)) return e;
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, 0, st)) return e;
         return launch_status();
     }
     void *scratch = nullptr;
@@ -609,12 +617,12 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     double *partial = reinterpret_cast<double *>(scratch);
     float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kNoAllocThreshOff);
     if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
-                                 st, w, total_v, kNoAllocChunk, sanitize, partial))
+                                 st, w, total_v, kNoAllocChunk, sanitize, partial, 0))
         return e;
     if (tq_status e = launch_pdl(absum_finalize_kernel, dim3(1), dim3(1024), 0, st, partial,
                                  (int)nparts, absum_tree_height(kNoAllocChunk, (int)nparts), w,
                                  total_v, sanitize, gamma, thresh))
         return e;
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, st)) return e;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, 0, st)) return e;
     return launch_status();
 }

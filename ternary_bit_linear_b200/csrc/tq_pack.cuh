@@ -135,8 +135,8 @@ template <bool SAN>
 __global__ void __launch_bounds__(kPackThreads)
     pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
-                     const float *__restrict__ per_tensor_t, int reverse) {
-    pdl_wait();
+                     const float *__restrict__ per_tensor_t, int reverse, int ready) {
+    if (!ready) pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * kPackWarps;
@@ -193,56 +193,106 @@ __global__ void __launch_bounds__(kPackThreads)
             dst[c] = (uint8_t)pack4(SAN ? sanitize_w(x) : x, t);
         }
     }
+    if (ready) pdl_wait();  // complete no earlier than the previous kernel
 }
 
 // ---------------------------------------------------------------------------
-// Team kernel (K <= 8192): T warps share a row, every thread holds 8 float4
-// of it in registers (read from HBM once).  Per row: per-lane fp64 chain,
-// warp shuffles, one named barrier for the T warp sums (double-buffered by row
-// parity), then each thread packs its own values.
+// Team kernel (K <= 8192): T warps share a row.  The team's leader streams
+// its rows with 1-D bulk copies into a ring of kPackRing shared-memory row
+// buffers, kPackRing - 1 rows ahead, so HBM latency is hidden behind the
+// work on earlier rows; every thread takes 8 float4 of the row into
+// registers.  Per row: per-lane fp64 chain, warp shuffles, one named barrier
+// for the T warp sums (double-buffered by row parity; it also tells the
+// leader that the buffer is free again), then each thread packs its values.
 // ---------------------------------------------------------------------------
 constexpr int kTeamVec = 8;
+constexpr int kPackRing = 3;
 
 __device__ __forceinline__ void team_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier that also returns the AND of every participant's flag.
+__device__ __forceinline__ bool team_all(int id, int threads, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
+
+__host__ __device__ constexpr int pack_team_smem(int T, int K) {
+    return (kPackWarps / T) * kPackRing * (K / 4) * 16;
 }
 
 template <int T, bool SAN>
 __global__ void __launch_bounds__(kPackThreads, 2)
     pack_team_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
-                     const float *__restrict__ per_tensor_t, int reverse) {
+                     const float *__restrict__ per_tensor_t, int reverse, int ready) {
     constexpr int TEAMS = kPackWarps / T;
+    extern __shared__ __align__(16) float4 rowbuf[];  // [TEAMS][kPackRing][nv]
+    __shared__ uint64_t rbar[TEAMS][kPackRing];
     __shared__ double tred[2][kPackWarps];
     __shared__ DD tredd[kPackWarps];
-    pdl_wait();
-    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int team = warp / T, tw = warp % T;
     const int bar_id = 1 + team;
     const int nv = K >> 2;
     const int64_t nteams = (int64_t)gridDim.x * TEAMS;
+    const int64_t first = (int64_t)blockIdx.x * TEAMS + team;
+    const int64_t nmine = first < N ? (N - 1 - first) / nteams + 1 : 0;
+    const bool leader = tw == 0 && lane == 0;
+    float4 *ring = rowbuf + (size_t)team * kPackRing * nv;
+    if (threadIdx.x == 0) {
+        for (int u = 0; u < TEAMS; ++u)
+            for (int r = 0; r < kPackRing; ++r) mbar_init(smem_u32(&rbar[u][r]), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (!ready) pdl_wait();
+    pdl_trigger();
+    auto row_of = [&](int64_t k) {
+        const int64_t i = first + k * nteams;
+        return reverse ? (N - 1 - i) : i;
+    };
+    auto issue = [&](int64_t k) {  // leader: row k of this team into buffer k % kPackRing
+        const uint32_t bar = smem_u32(&rbar[team][k % kPackRing]);
+        mbar_arrive_expect_tx(bar, (uint32_t)(nv * 16));
+        bulk_g2s(smem_u32(ring + (k % kPackRing) * nv), w + row_of(k) * (int64_t)K, (uint32_t)(nv * 16), bar);
+    };
+    int64_t issued = nmine < kPackRing ? nmine : kPackRing;
+    if (leader)
+        for (int64_t k = 0; k < issued; ++k) issue(k);
     const float t_tensor = per_tensor_t ? __ldg(per_tensor_t) : 0.0f;
     const double eps = sum_error_bound(4 * kTeamVec + 5 + T);
     int parity = 0;
-    for (int64_t i = (int64_t)blockIdx.x * TEAMS + team; i < N; i += nteams) {
-        const int64_t n = reverse ? (N - 1 - i) : i;
-        const float4 *src = reinterpret_cast<const float4 *>(w + n * (int64_t)K);
+    int64_t k = 0;
+    for (; k < nmine; ++k) {
+        const int64_t n = row_of(k);
+        const bool ok = warp_wait(smem_u32(&rbar[team][k % kPackRing]), (uint32_t)((k / kPackRing) & 1), lane);
+        const float4 *src = ring + (k % kPackRing) * nv;
         float4 v[kTeamVec];
 #pragma unroll
         for (int j = 0; j < kTeamVec; ++j) {
             const int idx = j * 32 * T + tw * 32 + lane;
-            v[j] = idx < nv ? __ldcs(src + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[j] = idx < nv ? src[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
             if (SAN) v[j] = sanitize_w(v[j]);
         }
         float t = t_tensor;
+        bool all_ok;
         if (per_tensor_t == nullptr) {
             double a = 0.0;
 #pragma unroll
             for (int j = 0; j < kTeamVec; ++j) a = __dadd_rn(a, abs_sum4(v[j]));
             a = warp_sum_dbl(a);
             if (lane == 0) tred[parity][warp] = a;
-            team_barrier(bar_id, 32 * T);
+            all_ok = team_all(bar_id, 32 * T, ok);  // the buffer has been read, sums are in
             double S = 0.0;
 #pragma unroll
             for (int u = 0; u < T; ++u) S = __dadd_rn(S, tred[parity][team * T + u]);
@@ -261,9 +311,14 @@ __global__ void __launch_bounds__(kPackThreads, 2)
                 g = dd_mean_to_f32(e, (double)K);
             }
             g = g > 1e-6f ? g : 1e-6f;
-            if (tw == 0 && lane == 0) gamma[n] = g;
+            if (all_ok && tw == 0 && lane == 0) gamma[n] = g;
             t = code_threshold(g);
+        } else {
+            all_ok = team_all(bar_id, 32 * T, ok);  // the buffer has been read
         }
+        if (!all_ok) break;  // a copy never landed (timeout recorded)
+        if (leader && issued < nmine) issue(issued);
+        issued = issued < nmine ? issued + 1 : issued;
         uint8_t *dst = packed + n * (int64_t)nv;
 #pragma unroll
         for (int j = 0; j < kTeamVec; ++j) {
@@ -271,15 +326,21 @@ __global__ void __launch_bounds__(kPackThreads, 2)
             if (idx < nv) dst[idx] = (uint8_t)pack4(v[j], t);
         }
     }
+    // Copies in flight must land before the CTA exits (already true unless a
+    // wait gave up).
+    if (leader)
+        for (int64_t j = k; j < issued; ++j)
+            mbar_wait(smem_u32(&rbar[team][j % kPackRing]), (uint32_t)((j / kPackRing) & 1));
+    if (ready) pdl_wait();  // complete no earlier than the previous kernel
 }
 
 // Per-tensor gamma, pass 1: CTA b sums |w| over float4 range [b*chunk, ...) in
 // plain fp64 (each thread sequentially, then a fixed block tree).
 __global__ void __launch_bounds__(kPackThreads)
     absum_partial_kernel(const float *__restrict__ w, int64_t nv, int64_t chunk, int sanitize,
-                         double *__restrict__ partial) {
+                         double *__restrict__ partial, int ready) {
     __shared__ double red[kPackWarps];
-    pdl_wait();
+    if (!ready) pdl_wait();
     pdl_trigger();
     const float4 *src = reinterpret_cast<const float4 *>(w);
     const int64_t beg = (int64_t)blockIdx.x * chunk;
@@ -305,6 +366,7 @@ __global__ void __launch_bounds__(kPackThreads)
     }
     const double S = block_sum_dbl(__dadd_rn(a0, a1), red);
     if (threadIdx.x == 0) partial[blockIdx.x] = S;
+    if (ready) pdl_wait();  // complete no earlier than the previous kernel
 }
 
 // Tree height of the per-tensor sum: per-thread chain over its float4 of a

@@ -491,3 +491,35 @@ def test_inputs_ready_flag_rejected_by_fused(cuda_lib):
     ws = torch.empty((max(16, tq.fused_workspace_bytes(M, K, 0)),), dtype=torch.uint8, device="cuda")
     with pytest.raises(RuntimeError):
         tq.bitlinear_fused_(x, packed, gamma, tq.FLAG_INPUTS_READY, y, ws)
+
+
+@pytest.mark.parametrize("per_row", [True, False])
+def test_pack_inputs_ready_layers_then_dependent_reader(cuda_lib, per_row):
+    """Pack several layers with TQ_FLAG_INPUTS_READY (each with its own buffers
+    and workspace), then contract the last one right behind them without the
+    flag: bytes and gamma must equal the oracle's, in order."""
+    tq = cuda_lib
+    N, K, L = 1000, 2048, 5
+    Ws = [S.normal((N, K), 0.02, 60 + i, N) for i in range(L)]
+    flags = (tq.GAMMA_PER_ROW if per_row else 0)
+    nws = max(16, tq.pack_workspace_bytes(N, K, flags))
+    bufs = [(torch.empty((N, K // 4), dtype=torch.uint8, device="cuda"),
+             torch.empty((N if per_row else 1,), dtype=torch.float32, device="cuda"),
+             torch.empty((nws,), dtype=torch.uint8, device="cuda")) for _ in range(L)]
+    Wd = [dev(W) for W in Ws]
+    torch.cuda.synchronize()
+    for W, (p, g, ws) in zip(Wd, bufs):
+        tq.quantize_ternary_pack_(W, flags | tq.FLAG_INPUTS_READY, p, g, ws)
+    M = 8
+    X = S.decode_acts(M, K, seed=61)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    tq.ternary_gemm_(dev(xq_ref), dev(sx_ref), dev(rs_ref), bufs[-1][0], bufs[-1][1], flags, y)
+    for W, (p, g, _) in zip(Ws, bufs):
+        p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row)
+        assert np.array_equal(host(p), p_ref)
+        assert np.array_equal(host(g), g_ref)
+    p_ref, g_ref = oracle.quantize_pack(Ws[-1], per_row=per_row)
+    acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
+    assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, per_row))
+    assert tq.device_status() == 0
