@@ -117,9 +117,68 @@ __device__ __forceinline__ float rms_apply(float x, double r, const float *gain,
 }
 
 // ---------------------------------------------------------------------------
-// Per-token quantisation (optionally after RMSNorm), one CTA per token.
-// VEC > 0: the row lives in registers (K <= 1024*VEC); VEC == 0: streamed.
+// Per-token quantisation (optionally after RMSNorm) of one row that a CTA of
+// kActThreads holds in registers: thread tid has float4 tid + i * kActThreads
+// (i < VEC; zeros past the row).  Writes x_q, s_x[m] and rowsum[m].
 // ---------------------------------------------------------------------------
+template <int VEC>
+__device__ __forceinline__ void act_row_regs(float4 (&v)[VEC], int K, const ActParams &p, int64_t m,
+                                             int8_t *__restrict__ xq, float *__restrict__ s_x,
+                                             int32_t *__restrict__ rowsum, float *redf, int *redi,
+                                             double *redd) {
+    const int nv = K >> 2, tid = threadIdx.x;
+    uint32_t *dst = reinterpret_cast<uint32_t *>(xq + m * (int64_t)K);
+    if (p.rmsnorm) {
+        double ss = 0.0;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            ss = __fma_rn((double)v[i].x, (double)v[i].x, ss);
+            ss = __fma_rn((double)v[i].y, (double)v[i].y, ss);
+            ss = __fma_rn((double)v[i].z, (double)v[i].z, ss);
+            ss = __fma_rn((double)v[i].w, (double)v[i].w, ss);
+        }
+        ss = block_sum_d<kActThreads>(ss, redd);
+        const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            const int k = 4 * (tid + i * kActThreads);
+            v[i] = make_float4(rms_apply(v[i].x, r, p.rms_gain, k), rms_apply(v[i].y, r, p.rms_gain, k + 1),
+                               rms_apply(v[i].z, r, p.rms_gain, k + 2),
+                               rms_apply(v[i].w, r, p.rms_gain, k + 3));
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VEC; ++i)
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+    amax = block_max<kActThreads>(amax, redf);
+    const float eta = eta_of(amax, p);
+    const float scale = __fdiv_rn(127.0f, eta);
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        const int idx = tid + i * kActThreads;
+        if (idx < nv) {
+            const int a = quant_code(v[i].x, scale), b = quant_code(v[i].y, scale),
+                      c = quant_code(v[i].z, scale), d = quant_code(v[i].w, scale);
+            dst[idx] = pack_codes4(a, b, c, d);
+            sum += a + b + c + d;
+        }
+    }
+    sum = block_sum_i<kActThreads>(sum, redi);
+    if (tid == 0) {
+        s_x[m] = __fdiv_rn(eta, 127.0f);
+        if (rowsum) rowsum[m] = sum;
+    }
+}
+
+__device__ __forceinline__ float4 quench4(float4 v, const ActParams &p) {
+    return make_float4(quench(v.x, p.eta_max), quench(v.y, p.eta_max), quench(v.z, p.eta_max),
+                       quench(v.w, p.eta_max));
+}
+
+// One CTA per token.  VEC > 0: the row lives in registers (K <= 1024*VEC);
+// VEC == 0: streamed (two passes over the row, the second from cache).
 template <int VEC>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const float *__restrict__ x, int K, ActParams p, int8_t *__restrict__ xq,
@@ -132,105 +191,121 @@ __global__ void __launch_bounds__(kActThreads)
     const int64_t m = blockIdx.x;
     const int nv = K >> 2, tid = threadIdx.x;
     const float4 *src = reinterpret_cast<const float4 *>(x + m * (int64_t)K);
-    uint32_t *dst = reinterpret_cast<uint32_t *>(xq + m * (int64_t)K);
-
     auto load = [&](int idx) {
         float4 v = __ldg(src + idx);
-        if (p.sanitize)
-            v = make_float4(quench(v.x, p.eta_max), quench(v.y, p.eta_max), quench(v.z, p.eta_max),
-                            quench(v.w, p.eta_max));
+        if (p.sanitize) v = quench4(v, p);
         return v;
     };
-
-    float4 v[VEC > 0 ? VEC : 1];
-    double r = 1.0;
     if (VEC > 0) {
+        constexpr int V = VEC > 0 ? VEC : 1;
+        float4 v[V];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) {
+        for (int i = 0; i < V; ++i) {
             const int idx = tid + i * kActThreads;
             v[i] = idx < nv ? load(idx) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        act_row_regs<V>(v, K, p, m, xq, s_x, rowsum, redf, redi, redd);
+        return;
     }
+    uint32_t *dst = reinterpret_cast<uint32_t *>(xq + m * (int64_t)K);
+    double r = 1.0;
     if (p.rmsnorm) {
         double ss = 0.0;
-        if (VEC > 0) {
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) {
-                ss = __fma_rn((double)v[i].x, (double)v[i].x, ss);
-                ss = __fma_rn((double)v[i].y, (double)v[i].y, ss);
-                ss = __fma_rn((double)v[i].z, (double)v[i].z, ss);
-                ss = __fma_rn((double)v[i].w, (double)v[i].w, ss);
-            }
-        } else {
-            for (int idx = tid; idx < nv; idx += kActThreads) {
-                const float4 t = load(idx);
-                ss = __fma_rn((double)t.x, (double)t.x, ss);
-                ss = __fma_rn((double)t.y, (double)t.y, ss);
-                ss = __fma_rn((double)t.z, (double)t.z, ss);
-                ss = __fma_rn((double)t.w, (double)t.w, ss);
-            }
+        for (int idx = tid; idx < nv; idx += kActThreads) {
+            const float4 t = load(idx);
+            ss = __fma_rn((double)t.x, (double)t.x, ss);
+            ss = __fma_rn((double)t.y, (double)t.y, ss);
+            ss = __fma_rn((double)t.z, (double)t.z, ss);
+            ss = __fma_rn((double)t.w, (double)t.w, ss);
         }
         ss = block_sum_d<kActThreads>(ss, redd);
         r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
-        if (VEC > 0) {
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) {
-                const int k = 4 * (tid + i * kActThreads);
-                v[i] = make_float4(rms_apply(v[i].x, r, p.rms_gain, k),
-                                   rms_apply(v[i].y, r, p.rms_gain, k + 1),
-                                   rms_apply(v[i].z, r, p.rms_gain, k + 2),
-                                   rms_apply(v[i].w, r, p.rms_gain, k + 3));
-            }
-        }
     }
     auto normed = [&](int idx) {
         float4 t = load(idx);
         if (p.rmsnorm) {
             const int k = 4 * idx;
             t = make_float4(rms_apply(t.x, r, p.rms_gain, k), rms_apply(t.y, r, p.rms_gain, k + 1),
-                            rms_apply(t.z, r, p.rms_gain, k + 2),
-                            rms_apply(t.w, r, p.rms_gain, k + 3));
+                            rms_apply(t.z, r, p.rms_gain, k + 2), rms_apply(t.w, r, p.rms_gain, k + 3));
         }
         return t;
     };
-
     float amax = 0.0f;
-    if (VEC > 0) {
-#pragma unroll
-        for (int i = 0; i < VEC; ++i)
-            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)),
-                                     fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
-    } else {
-        for (int idx = tid; idx < nv; idx += kActThreads) {
-            const float4 t = normed(idx);
-            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
-        }
+    for (int idx = tid; idx < nv; idx += kActThreads) {
+        const float4 t = normed(idx);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
     }
     amax = block_max<kActThreads>(amax, redf);
     const float eta = eta_of(amax, p);
     const float scale = __fdiv_rn(127.0f, eta);
-
     int sum = 0;
-    auto emit = [&](int idx, float4 t) {
-        const int a = quant_code(t.x, scale), b = quant_code(t.y, scale),
-                  c = quant_code(t.z, scale), d = quant_code(t.w, scale);
+    for (int idx = tid; idx < nv; idx += kActThreads) {
+        const float4 t = normed(idx);
+        const int a = quant_code(t.x, scale), b = quant_code(t.y, scale), c = quant_code(t.z, scale),
+                  d = quant_code(t.w, scale);
         dst[idx] = pack_codes4(a, b, c, d);
         sum += a + b + c + d;
-    };
-    if (VEC > 0) {
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-            const int idx = tid + i * kActThreads;
-            if (idx < nv) emit(idx, v[i]);
-        }
-    } else {
-        for (int idx = tid; idx < nv; idx += kActThreads) emit(idx, normed(idx));
     }
     sum = block_sum_i<kActThreads>(sum, redi);
     if (tid == 0) {
         s_x[m] = __fdiv_rn(eta, 127.0f);
         if (rowsum) rowsum[m] = sum;
     }
+}
+
+// Many tokens (K <= 1024*VEC): a persistent grid; each CTA streams its tokens
+// m = blockIdx.x + j * gridDim.x through a ring of kActRing shared-memory row
+// buffers filled by 1-D bulk copies kActRing - 1 rows ahead, so HBM latency
+// hides behind the work on earlier rows.
+constexpr int kActRing = 4;
+
+template <int VEC>
+__global__ void __launch_bounds__(kActThreads)
+    act_ring_kernel(const float *__restrict__ x, int64_t M, int K, ActParams p,
+                    int8_t *__restrict__ xq, float *__restrict__ s_x, int32_t *__restrict__ rowsum) {
+    extern __shared__ __align__(16) float4 rowbuf[];  // [kActRing][nv]
+    __shared__ uint64_t rbar[kActRing];
+    __shared__ float redf[32];
+    __shared__ int redi[32];
+    __shared__ double redd[32];
+    const int nv = K >> 2, tid = threadIdx.x, lane = tid & 31;
+    const int64_t nmine = (int64_t)blockIdx.x < M ? (M - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    if (tid == 0) {
+        for (int r = 0; r < kActRing; ++r) mbar_init(smem_u32(&rbar[r]), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+    auto issue = [&](int64_t j) {  // thread 0: token j of this CTA into buffer j % kActRing
+        const uint32_t bar = smem_u32(&rbar[j % kActRing]);
+        mbar_arrive_expect_tx(bar, (uint32_t)(nv * 16));
+        bulk_g2s(smem_u32(rowbuf + (j % kActRing) * nv), x + ((int64_t)blockIdx.x + j * gridDim.x) * K,
+                 (uint32_t)(nv * 16), bar);
+    };
+    int64_t issued = nmine < kActRing ? nmine : kActRing;
+    if (tid == 0)
+        for (int64_t j = 0; j < issued; ++j) issue(j);
+    int64_t j = 0;
+    for (; j < nmine; ++j) {
+        const bool ok = warp_wait(smem_u32(&rbar[j % kActRing]), (uint32_t)((j / kActRing) & 1), lane);
+        const float4 *src = rowbuf + (j % kActRing) * nv;
+        float4 v[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            const int idx = tid + i * kActThreads;
+            v[i] = idx < nv ? src[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p.sanitize) v[i] = quench4(v[i], p);
+        }
+        if (!__syncthreads_and(ok)) break;  // buffer read by all; CTA-uniform timeout decision
+        if (tid == 0 && issued < nmine) issue(issued);
+        issued = issued < nmine ? issued + 1 : issued;
+        act_row_regs<VEC>(v, K, p, (int64_t)blockIdx.x + j * gridDim.x, xq, s_x, rowsum, redf, redi, redd);
+    }
+    // Copies in flight must land before the CTA exits (already true unless a
+    // wait gave up).
+    if (tid == 0)
+        for (int64_t u = j; u < issued; ++u) mbar_wait(smem_u32(&rbar[u % kActRing]), (uint32_t)((u / kActRing) & 1));
 }
 
 // ---------------------------------------------------------------------------

@@ -218,9 +218,45 @@ using Prologues = PrologueTable<1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 1
                                 20, 21, 22, 23, 24, 25, 26, 27, 28, 29, 30, 31, 32>;
 constexpr int64_t kMaxFwhtFusedK = 512 * 32;
 
+// Many tokens: persistent ring kernel (one CTA per SM share, rows streamed
+// through shared memory); few tokens: one CTA per token.
+template <int VEC>
+void launch_act_ring(const float *x, const ActParams &p, int64_t M, int64_t K, int8_t *xq, float *sx,
+                     int32_t *rs, int sms, cudaStream_t st) {
+    static std::atomic<int> per_sm_c[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int smem = kActRing * (int)(K / 4) * 16;
+    const int key = per_sm_c[dev].load();
+    int per_sm = 0;
+    if ((key >> 8) == smem + 1) {
+        per_sm = key & 0xff;
+    } else {
+        if (cudaFuncSetAttribute(act_ring_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_ring_kernel<VEC>, kActThreads,
+                                                          (size_t)smem) != cudaSuccess)
+            per_sm = 1;
+        if (per_sm < 1) per_sm = 1;
+        per_sm_c[dev].store(((smem + 1) << 8) | (per_sm & 0xff));
+    }
+    const int64_t cap = (int64_t)per_sm * sms;
+    const unsigned grid = (unsigned)(M < cap ? M : cap);
+    launch_pdl(act_ring_kernel<VEC>, dim3(grid), dim3(kActThreads), (size_t)smem, st, x, M, (int)K, p, xq,
+               sx, rs);
+}
+
 void launch_act(const float *x, const ActParams &p, int64_t M, int64_t K, int8_t *xq, float *sx,
                 int32_t *rs, cudaStream_t st) {
     const int nv = (int)(K / 4);
+    int sms = 0;
+    check_device(&sms);
+    if (M >= 2 * (int64_t)sms && nv <= 2048) {
+        if (nv <= 256) return launch_act_ring<1>(x, p, M, K, xq, sx, rs, sms, st);
+        if (nv <= 512) return launch_act_ring<2>(x, p, M, K, xq, sx, rs, sms, st);
+        if (nv <= 1024) return launch_act_ring<4>(x, p, M, K, xq, sx, rs, sms, st);
+        return launch_act_ring<8>(x, p, M, K, xq, sx, rs, sms, st);
+    }
     const dim3 grid((unsigned)M), block(kActThreads);
     if (nv <= 256)
         launch_pdl(act_quant_kernel<1>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);

@@ -99,18 +99,27 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Bounded wait for the phase with the given parity.  Returns false (and sets
-// the timeout bit) if it did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// the timeout bit) if it did not complete within kWaitLimitNs.  The spinning
+// form is for waits on a kernel's critical path; the sleeping form for warps
+// that wait long while others on the SM do the work.
+template <bool SLEEP>
+__device__ __forceinline__ bool mbar_wait_t(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (;;) {
-        for (int i = 0; i < 8; ++i)
-            if (mbar_try_wait_sleep(bar, parity)) return true;
+        for (int i = 0; i < (SLEEP ? 8 : 64); ++i)
+            if (SLEEP ? mbar_try_wait_sleep(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             flag_timeout();
             return false;
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    return mbar_wait_t<false>(bar, parity);
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity) {
+    return mbar_wait_t<true>(bar, parity);
 }
 
 // Warp-uniform bounded wait: lane 0 polls, every lane gets the same answer,
@@ -118,6 +127,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane) {
     int ok = 0;
     if (lane == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+__device__ __forceinline__ bool warp_wait_sleep(uint32_t bar, uint32_t parity, int lane) {
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait_sleep(bar, parity) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 

@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int s = g % S, r = g / S;
                 const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
                 const int kb = g % nkb;
-                if (!mbar_wait(empty(s), (r & 1) ^ 1)) break;
+                if (!mbar_wait_sleep(empty(s), (r & 1) ^ 1)) break;
                 mbar_arrive_expect_tx(full(s), L::kB);
                 tma_load_2d(x_stage(s), &tm_x, kb * kTileK, (t % num_m) * BT, full(s));
             }
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int s = g % SW, r = g / SW;
                 const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
                 const int kb = g % nkb;
-                if (!mbar_wait(w_empty(s), (r & 1) ^ 1)) break;
+                if (!mbar_wait_sleep(w_empty(s), (r & 1) ^ 1)) break;
                 mbar_arrive_expect_tx(w_full(s), kWStageBytes);
                 tma_load_2d(sbase + (uint32_t)(L::offW + s * kWStageBytes), &tm_w, kb * (kTileK / 4),
                             (t / num_m) * kTileN, w_full(s));
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t a_row = (uint32_t)(r * kTileK), sw = (uint32_t)(r & 7);
         for (int g = par; g < total; g += 2) {
             const int ws = g % SW, s = g % S;
-            if (!warp_wait(w_full(ws), (g / SW) & 1, lane)) break;
+            if (!warp_wait_sleep(w_full(ws), (g / SW) & 1, lane)) break;
             uint4 p0, p1;
             const uint32_t src = w_row + (uint32_t)(ws * kWStageBytes);
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int c = 0; c < 8; ++c) e[c] = expand_word(words[c]);
             __syncwarp();
             if (lane == 0) mbar_arrive(w_empty(ws));  // packed bytes are in registers
-            if (!warp_wait(empty(s), ((g / S) & 1) ^ 1, lane)) break;
+            if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
             // 16-byte chunk c of row r lives at chunk position c ^ (r & 7)
             const uint32_t base = a_stage(s) + a_row;
 #pragma unroll
@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 sxc[cc] = mj < M ? __ldg(s_x + mj) : 0.0f;
                 rsc[cc] = mj < M ? __ldg(rowsum + mj) : 0;
             }
-            if (!warp_wait(d_full(b), (tl >> 1) & 1, lane)) break;
+            if (!warp_wait_sleep(d_full(b), (tl >> 1) & 1, lane)) break;
             tc_fence_after();
 #pragma unroll
             for (int cc = 0; cc < kChunks; ++cc) {
@@ -300,15 +300,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(d_empty(b));
                 }
+                // Branch-free pass first (the shuffles of all 32 tokens can then
+                // overlap), then a pure store pass.
+                const int mb = m0 + cc * 32;
+                const int jmax = M - mb;  // tokens of this chunk inside [0, M)
+                if (!acc_out) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float sxm = __shfl_sync(0xffffffffu, sxc[cc], j);
-                    const int rsm = __shfl_sync(0xffffffffu, rsc[cc], j);
-                    const int m = m0 + cc * 32 + j;
-                    if (m < M && n < N) {
+                    for (int j = 0; j < 32; ++j) {
+                        const float sxm = __shfl_sync(0xffffffffu, sxc[cc], j);
+                        const int rsm = __shfl_sync(0xffffffffu, rsc[cc], j);
+                        v[j] = __float_as_uint(
+                            __fmul_rn(__int2float_rn((int)v[j] - rsm), __fmul_rn(gn, sxm)));
+                    }
+                    if (n < N) {
+                        float *yp = y + (int64_t)mb * N + n;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (j < jmax) __stcs(yp + (int64_t)j * N, __uint_as_float(v[j]));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float sxm = __shfl_sync(0xffffffffu, sxc[cc], j);
+                        const int rsm = __shfl_sync(0xffffffffu, rsc[cc], j);
                         const int a = (int)v[j] - rsm;
-                        __stcs(y + (int64_t)m * N + n, __fmul_rn(__int2float_rn(a), __fmul_rn(gn, sxm)));
-                        if (acc_out) __stcs(acc_out + (int64_t)m * N + n, a);
+                        if (j < jmax && n < N) {
+                            __stcs(y + (int64_t)(mb + j) * N + n,
+                                   __fmul_rn(__int2float_rn(a), __fmul_rn(gn, sxm)));
+                            __stcs(acc_out + (int64_t)(mb + j) * N + n, a);
+                        }
                     }
                 }
             }

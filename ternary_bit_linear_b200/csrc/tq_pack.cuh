@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kPackThreads, 2)
     int64_t k = 0;
     for (; k < nmine; ++k) {
         const int64_t n = row_of(k);
-        const bool ok = warp_wait(smem_u32(&rbar[team][k % kPackRing]), (uint32_t)((k / kPackRing) & 1), lane);
+        const bool ok = warp_wait_sleep(smem_u32(&rbar[team][k % kPackRing]), (uint32_t)((k / kPackRing) & 1), lane);
         const float4 *src = ring + (k % kPackRing) * nv;
         float4 v[kTeamVec];
 #pragma unroll

@@ -138,7 +138,9 @@ def test_pack_full_size(cuda_lib, which):
 # activation quantisation and FWHT
 # ---------------------------------------------------------------------------
 
-ACT_SHAPES = [(1, 64), (3, 192), (4, 512), (8, 4096), (17, 4160), (2, 8192), (5, 8256), (3, 65536)]
+ACT_SHAPES = [(1, 64), (3, 192), (4, 512), (8, 4096), (17, 4160), (2, 8192), (5, 8256), (3, 65536),
+              # many tokens: the persistent ring kernel (rows streamed through shared memory)
+              (300, 64), (401, 1088), (297, 4160), (600, 8192), (1000, 2048)]
 
 
 @pytest.mark.parametrize("M,K", ACT_SHAPES)
@@ -164,6 +166,17 @@ def test_act_quant_golden_ties_and_sanitize(cuda_lib):
     xs = oracle.sanitize_acts(x, 40.0)
     xq_ref, sx_ref, rs_ref = oracle.act_quant(xs)
     assert xq_ref[0, :8].tolist() == [127, 64, -64, 32, 16, -127, 0, 95]
+    assert np.array_equal(host(xq), xq_ref) and np.array_equal(host(sx), sx_ref)
+    assert np.array_equal(host(rs), rs_ref)
+
+
+def test_act_quant_many_tokens_sanitize(cuda_lib):
+    M, K = 700, 4096
+    X = S.decode_acts(M, K, seed=12)
+    X[5, 3], X[40, 9], X[41, 10], X[699, 4095] = np.nan, np.inf, -np.inf, np.nan
+    X[6] = np.inf
+    xq, sx, rs = cuda_lib.quantize_act_int8(dev(X), sanitize=True, eta_max=40.0)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(oracle.sanitize_acts(X, 40.0))
     assert np.array_equal(host(xq), xq_ref) and np.array_equal(host(sx), sx_ref)
     assert np.array_equal(host(rs), rs_ref)
 
