@@ -330,6 +330,25 @@ size_t pack_parts(int64_t nv) {
     return (size_t)((nv + chunk - 1) / chunk);
 }
 
+// Tokens per GEMM tile.  Cost model: rounds of tiles over the SMs times the
+// time of one K-step, 4 MMAs of BT/2 cycles each but no faster than the
+// single-thread issue rate (about 72 cycles per MMA); ties go to the smaller
+// tile (less padding and x_q traffic).
+int gemm_tile_tokens(int64_t M, int64_t N, int sms) {
+    int best = 64;
+    int64_t best_cost = -1;
+    for (int bt : {64, 128, 192, 256}) {
+        const int64_t tiles = ((M + bt - 1) / bt) * ((N + kTileN - 1) / kTileN);
+        const int64_t rounds = (tiles + sms - 1) / sms;
+        const int64_t cost = rounds * (bt / 2 > 72 ? bt / 2 : 72);
+        if (best_cost < 0 || cost < best_cost) {
+            best = bt;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
 tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                         const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
                         int64_t N, int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
@@ -348,9 +367,12 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
         return lean ? launch_gemv<2, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st)
                     : launch_gemv<2, 8>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
     }
-    if (M <= 64) return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    if (M <= 128) return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    switch (gemm_tile_tokens(M, N, sms)) {
+    case 64: return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    case 128: return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    case 192: return launch_gemm<192>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    default: return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    }
 }
 
 }  // namespace

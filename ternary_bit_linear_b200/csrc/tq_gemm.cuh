@@ -6,7 +6,8 @@
 // as tcgen05.mma kind::i8 with int32 accumulators in tensor memory.
 //
 // Persistent: one CTA per SM walks output tiles of 128 features (the MMA's M,
-// taken by the weights) x BT tokens (the MMA's N, up to 256), token blocks
+// taken by the weights) x BT tokens (the MMA's N: 64, 128, 192 or 256, chosen
+// per problem by the launcher to fill the SMs), token blocks
 // fastest so that concurrently running CTAs share weight tiles in L2.  K is
 // consumed in steps of 128 codes; one step is four MMAs of K = 32 with both
 // operands in shared memory (128-byte swizzled, K-major).  Twenty warps:
@@ -77,7 +78,9 @@ struct GemmLayout {
     static constexpr int offTmem = offBar + kBars * 8;
     static constexpr int kBytes = offTmem + 16;
     static constexpr int kDynamic = kBytes + 1024;  // slack for 1024-byte alignment
-    static constexpr uint32_t kTmemCols = pow2_at_least(2 * BT);
+    // accumulator buffers start at multiples of kDStride TMEM columns
+    static constexpr int kDStride = BT <= 128 ? BT : 256;
+    static constexpr uint32_t kTmemCols = pow2_at_least(BT + kDStride);
     static_assert(kDynamic <= 232448, "shared memory per CTA");
     static_assert(kB % 1024 == 0 && kAStageBytes % 1024 == 0, "swizzle atoms stay aligned");
 };
@@ -152,9 +155,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_relinquish();
     }
     // Everything above touched no global memory; inputs of the previous kernel
-    // on the stream are visible after this wait.  With ready inputs the kernel
-    // skips it here and waits before exiting instead (stream completion order).
-    if (!(mode & kModeInputsReady)) pdl_wait();
+    // on the stream are visible after this wait.  With static weights only the
+    // roles that read x_q, s_x, rowsum or write y wait (the weight producer,
+    // the unpackers and the MMA issuer start at once); with ready inputs no
+    // role waits here and the kernel waits before exiting instead (stream
+    // completion order).
+    const bool ready = (mode & kModeInputsReady) != 0;
+    const bool w_early = (mode & (kModeWeightsStatic | kModeInputsReady)) != 0;
+    if (!w_early) pdl_wait();
     pdl_trigger();
     tc_fence_before();
     __syncthreads();
@@ -163,6 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == 0) {
         // ---------------- x_q producer ----------------
+        if (w_early && !ready) pdl_wait();
         if (lane == 0) {
             int g = 0;
             for (; g < total; ++g) {
@@ -204,7 +213,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int b = tl & 1;
                 if (!mbar_wait(d_empty(b), ((tl >> 1) & 1) ^ 1)) break;
                 tc_fence_after();
-                const uint32_t d_col = tmem + (uint32_t)(b * BT);
+                const uint32_t d_col = tmem + (uint32_t)(b * L::kDStride);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % S;
                     if (!mbar_wait(full(s), (g / S) & 1)) {
@@ -268,6 +277,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp >= 12) {
         // ---------------- epilogue ----------------
+        if (w_early && !ready) pdl_wait();
         constexpr int kHalf = BT / 2;          // tokens per epilogue warp and tile
         constexpr int kChunks = kHalf / 32;
         const int q = warp & 3;                // TMEM lane quarter
@@ -293,7 +303,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int cc = 0; cc < kChunks; ++cc) {
                 uint32_t v[32];
-                tmem_ld32(lane_addr + (uint32_t)(b * BT + half * kHalf + cc * 32), v);
+                tmem_ld32(lane_addr + (uint32_t)(b * L::kDStride + half * kHalf + cc * 32), v);
                 tmem_ld_wait();
                 if (cc == kChunks - 1) {  // accumulator fully read: hand it back to the MMA warp
                     tc_fence_before();
@@ -334,7 +344,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     }
-    if (mode & kModeInputsReady) pdl_wait();
+    if (ready || w_early) pdl_wait();  // no-op for roles that already waited
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

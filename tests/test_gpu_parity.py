@@ -536,3 +536,13 @@ def test_pack_inputs_ready_layers_then_dependent_reader(cuda_lib, per_row):
     acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
     assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, per_row))
     assert tq.device_status() == 0
+
+
+# Shapes whose tile choice (tokens per tile, from the launcher's cost model on
+# 148 SMs) is 128, 192 and 256 respectively, all ragged in M, N and K.
+@pytest.mark.parametrize("M,N,K", [(383, 11000, 192), (500, 5600, 320), (1000, 4000, 192)])
+def test_gemm_tile_sizes_sampled(cuda_lib, M, N, K):
+    W = S.normal((N, K), 0.02, 70, N)
+    X = S.decode_acts(M, K, seed=71)
+    sample = np.unique(np.r_[0, 1, np.arange(5, M, max(1, M // 17)), M - 2, M - 1])
+    sampled_gemm_check(cuda_lib, W, X, False, sample)
