@@ -12,15 +12,16 @@ RMSNorm + FWHT prologue).
 Default workload ("decode"): K = N = 4096, per-row gamma, W ~ N(0, 0.02),
 activations ~ N(0, 1) with 0.1 % outliers x20, token batches M = 1 and M = 8.
 A ring of L = 64 distinct layers keeps every working set above L2: per step the
-64 fp32 weights (4 GiB) are re-packed (the packed ring is 256 MiB), both
-batches are quantised, and each batch runs through the GEMV of all 64 layers.
+64 fp32 weights (4 GiB) are re-packed (the packed ring is 256 MiB), each layer's
+activation batches (its own buffers) are quantised, and each batch runs through
+the GEMV of its layer.
 Metric: algorithmic HBM bytes of the step / step time (GB/s).
 
-The layers of the ring share the activation and have their own weights,
-outputs and workspaces, so the packs of one segment, and the contractions of
-one segment, are independent calls: they are issued with TQ_FLAG_INPUTS_READY
-(and TQ_FLAG_WEIGHTS_STATIC for the contractions), which lets consecutive
-kernels overlap.  For the small-M GEMVs the line also reports "chain": the
+The layers of the ring have their own weights, activations, outputs and
+workspaces, so the calls within one segment (packs, activation quantisations,
+contractions) are independent: they are issued with TQ_FLAG_INPUTS_READY (and
+TQ_FLAG_WEIGHTS_STATIC for the contractions), which lets consecutive kernels
+overlap.  For the small-M GEMVs the line also reports "chain": the
 same launches as a chain of dependent layers (each kernel waits for the
 previous one before reading), timed separately and not part of the step.
 
@@ -198,10 +199,11 @@ class Workload:
         nws = tq.pack_workspace_bytes(N, K, self.flags)
         # one workspace per layer: the ring's packs are independent calls
         self.pack_ws = [torch.empty((max(nws, 16),), dtype=u8, device=dev) for _ in range(L)]
-        self.Xd = {M: x.to(dev) for M, x in self.X.items()}
-        self.xq = {M: torch.empty((M, K), dtype=i8, device=dev) for M in self.Ms}
-        self.sx = {M: torch.empty((M,), dtype=f32, device=dev) for M in self.Ms}
-        self.rs = {M: torch.empty((M,), dtype=i32, device=dev) for M in self.Ms}
+        # every layer of the ring has its own activation batch (same values)
+        self.Xd = {M: [x.to(dev) for _ in range(L)] for M, x in self.X.items()}
+        self.xq = {M: [torch.empty((M, K), dtype=i8, device=dev) for _ in range(L)] for M in self.Ms}
+        self.sx = {M: [torch.empty((M,), dtype=f32, device=dev) for _ in range(L)] for M in self.Ms}
+        self.rs = {M: [torch.empty((M,), dtype=i32, device=dev) for _ in range(L)] for M in self.Ms}
         self.y = {M: [torch.empty((M, N), dtype=f32, device=dev) for _ in range(L)] for M in self.Ms}
         if name == "fused":
             fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM
@@ -219,28 +221,30 @@ class Workload:
             M = self.Ms[0]
             ops = 2 * M * N * K
             self.segments.append(("fused M=%d" % M, "fused", L, L * ops, 2 * L, [
-                lambda l=l: tq.bitlinear_fused_(self.Xd[M], self.packed[l], self.gamma[l],
+                lambda l=l: tq.bitlinear_fused_(self.Xd[M][l], self.packed[l], self.gamma[l],
                                                 self.fused_flags, self.y[M][l], self.fused_ws)
                 for l in range(L)]))
             return
-        act_bytes = sum(4 * M * K + M * K + 8 * M for M in self.Ms)
-        self.segments.append(("act", "act_quant", len(self.Ms), act_bytes, len(self.Ms), [
-            lambda M=M: tq.quantize_act_int8_(self.Xd[M], 0, 0.05, 40.0, self.xq[M], self.sx[M], self.rs[M])
-            for M in self.Ms]))
+        act_bytes = L * sum(4 * M * K + M * K + 8 * M for M in self.Ms)
+        nact = L * len(self.Ms)
+        self.segments.append(("act", "act_quant", nact, act_bytes, nact, [
+            lambda M=M, l=l: tq.quantize_act_int8_(self.Xd[M][l], tq.FLAG_INPUTS_READY, 0.05, 40.0,
+                                                   self.xq[M][l], self.sx[M][l], self.rs[M][l])
+            for M in self.Ms for l in range(L)]))
         for M in self.Ms:
             gemv = M <= 16
             work = (N * K // 4 + 4 * N * (1 if self.per_row else 0) + M * K + 8 * M + 4 * M * N) if gemv \
                 else 2 * M * N * K
             self.segments.append(("gemv M=%d" % M if gemv else "gemm M=%d" % M,
                                   "gemv" if gemv else "gemm", L, L * work, L, [
-                lambda l=l, M=M: tq.ternary_gemm_(self.xq[M], self.sx[M], self.rs[M], self.packed[l],
+                lambda l=l, M=M: tq.ternary_gemm_(self.xq[M][l], self.sx[M][l], self.rs[M][l], self.packed[l],
                                                   self.gamma[l], self.ready_flags, self.y[M][l])
                 for l in range(L)]))
             if gemv:
                 self.chains.append(("gemv M=%d" % M, L, work, [
-                    lambda l=l, M=M: tq.ternary_gemm_(self.xq[M], self.sx[M], self.rs[M], self.packed[l],
-                                                      self.gamma[l], self.flags | tq.FLAG_WEIGHTS_STATIC,
-                                                      self.y[M][l])
+                    lambda l=l, M=M: tq.ternary_gemm_(self.xq[M][l], self.sx[M][l], self.rs[M][l],
+                                                      self.packed[l], self.gamma[l],
+                                                      self.flags | tq.FLAG_WEIGHTS_STATIC, self.y[M][l])
                     for l in range(L)]))
 
     def step_bytes(self):
@@ -432,13 +436,14 @@ def run_e2e(args, wl, tq, torch, stream, graphs, world):
     host_x = {M: x.pin_memory() for M, x in wl.X.items()}
     outs = [y for M in wl.Ms for y in wl.y[M]]
     host_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in outs]
-    h2d = sum(x.numel() * 4 for x in host_x.values())
+    h2d = sum(x.numel() * 4 * wl.L for x in host_x.values())
     d2h = sum(y.numel() * 4 for y in outs)
     steps = max(3, min(args.steps, 50))
 
     def one():
         for M in wl.Ms:
-            wl.Xd[M].copy_(host_x[M], non_blocking=True)
+            for xd in wl.Xd[M]:
+                xd.copy_(host_x[M], non_blocking=True)
         for g in graphs:
             g.replay()
         for y, hy in zip(outs, host_y):

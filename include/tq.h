@@ -92,7 +92,8 @@ typedef enum tq_status {
  * the layers of a model during inference).  The small-M GEMV then starts
  * streaming weights and gamma before the wait.
  *
- * TQ_FLAG_INPUTS_READY (tq_ternary_gemm, tq_quantize_ternary_pack): the
+ * TQ_FLAG_INPUTS_READY (tq_ternary_gemm, tq_quantize_ternary_pack,
+ * tq_quantize_act_int8): the
  * caller promises that no work in flight writes any input of the call or
  * reads or writes its outputs or workspace -- e.g. the independent
  * projections of one decode step that share an activation (q/k/v, gate/up),
@@ -160,7 +161,8 @@ TQ_API tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N, int
  *
  *   x       [M][K] fp32, read only.
  *   flags   TQ_FLAG_ETA_CLAMP (eta clamped to [eta_min, eta_max] after the 1e-6
- *           floor), TQ_FLAG_SANITIZE_NONFINITE (nan -> 0, +-inf -> +-eta_max).
+ *           floor), TQ_FLAG_SANITIZE_NONFINITE (nan -> 0, +-inf -> +-eta_max),
+ *           TQ_FLAG_INPUTS_READY (see "Launch overlap").
  *   xq      [M][K] int8, written, values in [-127, 127].
  *   s_x     [M] fp32, written.
  *   rowsum  [M] int32, written: sum_k xq[m][k].  tq_ternary_gemm needs it.

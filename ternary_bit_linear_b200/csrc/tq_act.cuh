@@ -32,6 +32,8 @@ struct ActParams {
     int rmsnorm;     // (fused prologue only)
     float rms_eps;
     const float *rms_gain;  // [K] or nullptr
+    int ready;       // inputs complete and outputs untouched by work in flight:
+                     // read at once, wait for the previous kernel before exiting
 };
 
 __device__ __forceinline__ float quench(float x, float eta_max) {
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kActThreads)
     __shared__ float redf[32];
     __shared__ int redi[32];
     __shared__ double redd[32];
-    pdl_wait();
+    if (!p.ready) pdl_wait();
     pdl_trigger();
     const int64_t m = blockIdx.x;
     const int nv = K >> 2, tid = threadIdx.x;
@@ -205,6 +207,7 @@ __global__ void __launch_bounds__(kActThreads)
             v[i] = idx < nv ? load(idx) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         act_row_regs<V>(v, K, p, m, xq, s_x, rowsum, redf, redi, redd);
+        if (p.ready) pdl_wait();  // complete no earlier than the previous kernel
         return;
     }
     uint32_t *dst = reinterpret_cast<uint32_t *>(xq + m * (int64_t)K);
@@ -251,6 +254,7 @@ __global__ void __launch_bounds__(kActThreads)
         s_x[m] = __fdiv_rn(eta, 127.0f);
         if (rowsum) rowsum[m] = sum;
     }
+    if (p.ready) pdl_wait();  // complete no earlier than the previous kernel
 }
 
 // Many tokens (K <= 1024*VEC): a persistent grid; each CTA streams its tokens
@@ -275,7 +279,7 @@ __global__ void __launch_bounds__(kActThreads)
         fence_barrier_init();
     }
     __syncthreads();
-    pdl_wait();
+    if (!p.ready) pdl_wait();
     pdl_trigger();
     auto issue = [&](int64_t j) {  // thread 0: token j of this CTA into buffer j % kActRing
         const uint32_t bar = smem_u32(&rbar[j % kActRing]);
@@ -306,6 +310,7 @@ __global__ void __launch_bounds__(kActThreads)
     // wait gave up).
     if (tid == 0)
         for (int64_t u = j; u < issued; ++u) mbar_wait(smem_u32(&rbar[u % kActRing]), (uint32_t)((u / kActRing) & 1));
+    if (p.ready) pdl_wait();  // complete no earlier than the previous kernel
 }
 
 // ---------------------------------------------------------------------------

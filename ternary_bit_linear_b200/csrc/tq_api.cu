@@ -454,7 +454,7 @@ tq_status tq_quantize_act_int8(const float *x, int64_t M, int64_t K, unsigned fl
     if (!x || !xq || !s_x || !rowsum) return TQ_ERR_NULL;
     if (M < 1 || M > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
-    if (flags & ~(TQ_FLAG_ETA_CLAMP | TQ_FLAG_SANITIZE_NONFINITE)) return TQ_ERR_ARG;
+    if (flags & ~(TQ_FLAG_ETA_CLAMP | TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_INPUTS_READY)) return TQ_ERR_ARG;
     if ((flags & TQ_FLAG_ETA_CLAMP) && !(eta_min > 0.0f && eta_min <= eta_max)) return TQ_ERR_ARG;
     if ((flags & TQ_FLAG_SANITIZE_NONFINITE) && !(eta_max > 0.0f && eta_max < 3.0e38f)) return TQ_ERR_ARG;
     if (!aligned16(x) || !aligned16(xq) || !aligned16(s_x) || !aligned16(rowsum)) return TQ_ERR_ALIGN;
@@ -468,6 +468,7 @@ tq_status tq_quantize_act_int8(const float *x, int64_t M, int64_t K, unsigned fl
     p.clamp_eta = (flags & TQ_FLAG_ETA_CLAMP) ? 1 : 0;
     p.eta_min = eta_min;
     p.eta_max = eta_max;
+    p.ready = (flags & TQ_FLAG_INPUTS_READY) ? 1 : 0;
     launch_act(x, p, M, K, xq, s_x, rowsum, cs(stream));
     return launch_status();
 }

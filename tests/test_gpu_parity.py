@@ -546,3 +546,32 @@ def test_gemm_tile_sizes_sampled(cuda_lib, M, N, K):
     X = S.decode_acts(M, K, seed=71)
     sample = np.unique(np.r_[0, 1, np.arange(5, M, max(1, M // 17)), M - 2, M - 1])
     sampled_gemm_check(cuda_lib, W, X, False, sample)
+
+
+@pytest.mark.parametrize("M,K", [(8, 4096), (700, 4096)])
+def test_act_inputs_ready_then_dependent_reader(cuda_lib, M, K):
+    """Independent activation quantisations with TQ_FLAG_INPUTS_READY, then a
+    flag-less contraction of the last batch right behind them."""
+    tq = cuda_lib
+    L = 5
+    Xs = [S.decode_acts(M, K, seed=80 + i) for i in range(L)]
+    outs = [(torch.empty((M, K), dtype=torch.int8, device="cuda"),
+             torch.empty((M,), dtype=torch.float32, device="cuda"),
+             torch.empty((M,), dtype=torch.int32, device="cuda")) for _ in range(L)]
+    Xd = [dev(X) for X in Xs]
+    N = 300
+    W = S.normal((N, K), 0.02, 81, N)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=True)
+    packed, gamma = dev(p_ref), dev(g_ref)
+    torch.cuda.synchronize()
+    for x, (xq, sx, rs) in zip(Xd, outs):
+        tq.quantize_act_int8_(x, tq.FLAG_INPUTS_READY, 0.05, 40.0, xq, sx, rs)
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    tq.ternary_gemm_(outs[-1][0], outs[-1][1], outs[-1][2], packed, gamma, tq.GAMMA_PER_ROW, y)
+    for X, (xq, sx, rs) in zip(Xs, outs):
+        xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+        assert np.array_equal(host(xq), xq_ref) and np.array_equal(host(sx), sx_ref)
+        assert np.array_equal(host(rs), rs_ref)
+    xq_ref, sx_ref, _ = oracle.act_quant(Xs[-1])
+    assert_y_close(host(y), oracle.dequant(oracle.matmul_addsub(xq_ref, p_ref), g_ref, sx_ref, True))
+    assert tq.device_status() == 0
