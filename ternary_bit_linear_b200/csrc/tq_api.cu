@@ -270,13 +270,21 @@ void launch_act(const float *x, const ActParams &p, int64_t M, int64_t K, int8_t
         launch_pdl(act_quant_kernel<0>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
 }
 
+// Per-tensor mode of the pack pass: the partial sums of absum_partial_kernel
+// and the height of the whole summation tree (partial == nullptr: per row).
+struct PerTensor {
+    const double *partial = nullptr;
+    int nparts = 0;
+    int height = 0;
+};
+
 // Persistent pack grid: as many CTAs as fit on the device, at most one row per
 // team.  K <= 8192: a team of T warps streams its rows through a shared-memory
 // ring (smem bytes per CTA); larger K: one warp streams each row twice.
 template <typename Kern>
 tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_cta, int smem,
                            const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
-                           const float *t, int reverse, int ready, cudaStream_t st) {
+                           const PerTensor &pt, int reverse, int ready, cudaStream_t st) {
     int dev = 0, sms = 0;
     if (tq_status e = check_device(&sms)) return e;
     cudaGetDevice(&dev);
@@ -297,30 +305,30 @@ tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_ct
     const int64_t cap = (int64_t)per_sm * sms;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
     return launch_pdl(kern, dim3(grid), dim3(kPackThreads), (size_t)smem, st, w, N, (int)K,
-                      1.0 / (double)K, packed, gamma, t, reverse, ready);
+                      1.0 / (double)K, packed, gamma, pt.partial, pt.nparts, pt.height, reverse, ready);
 }
 
 template <bool SAN>
 tq_status launch_pack_rows_s(const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
-                             const float *t, int reverse, int ready, cudaStream_t st) {
+                             const PerTensor &pt, int reverse, int ready, cudaStream_t st) {
     static std::atomic<int> occ[5][kMaxDevices];
     const int64_t nv = K / 4;
     const int k = (int)K;
     if (nv <= 32 * kTeamVec * 1)
-        return launch_pack_grid(pack_team_kernel<1, SAN>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, t, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<1, SAN>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, pt, reverse, ready, st);
     if (nv <= 32 * kTeamVec * 2)
-        return launch_pack_grid(pack_team_kernel<2, SAN>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, t, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<2, SAN>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, pt, reverse, ready, st);
     if (nv <= 32 * kTeamVec * 4)
-        return launch_pack_grid(pack_team_kernel<4, SAN>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, t, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<4, SAN>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, pt, reverse, ready, st);
     if (nv <= 32 * kTeamVec * 8)
-        return launch_pack_grid(pack_team_kernel<8, SAN>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, t, reverse, ready, st);
-    return launch_pack_grid(pack_rows_kernel<SAN>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, t, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<8, SAN>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, pt, reverse, ready, st);
+    return launch_pack_grid(pack_rows_kernel<SAN>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, ready, st);
 }
 
 tq_status launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
-                           float *gamma, const float *t, int reverse, int ready, cudaStream_t st) {
-    return sanitize ? launch_pack_rows_s<true>(w, N, K, packed, gamma, t, reverse, ready, st)
-                    : launch_pack_rows_s<false>(w, N, K, packed, gamma, t, reverse, ready, st);
+                           float *gamma, const PerTensor &pt, int reverse, int ready, cudaStream_t st) {
+    return sanitize ? launch_pack_rows_s<true>(w, N, K, packed, gamma, pt, reverse, ready, st)
+                    : launch_pack_rows_s<false>(w, N, K, packed, gamma, pt, reverse, ready, st);
 }
 
 size_t pack_parts(int64_t nv) {
@@ -429,22 +437,21 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, ready, st)) return e;
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, ready, st)) return e;
         return launch_status();
     }
     const int64_t total_v = N * K / 4;
     const size_t nparts = pack_parts(total_v);
     const int64_t chunk = (total_v + (int64_t)nparts - 1) / (int64_t)nparts;
     double *partial = reinterpret_cast<double *>(workspace);
-    float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + nparts * sizeof(DD));
     if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
                                  st, w, total_v, chunk, sanitize, partial, ready))
         return e;
-    if (tq_status e = launch_pdl(absum_finalize_kernel, dim3(1), dim3(1024), 0, st, partial,
-                                 (int)nparts, absum_tree_height(chunk, (int)nparts), w, total_v,
-                                 sanitize, gamma, thresh))
-        return e;
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, 0, st)) return e;
+    PerTensor pt;
+    pt.partial = partial;
+    pt.nparts = (int)nparts;
+    pt.height = absum_tree_height(chunk, (int)nparts);
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, 0, st)) return e;
     return launch_status();
 }
 
@@ -666,7 +673,7 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, nullptr, 0, 0, st)) return e;
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, 0, st)) return e;
         return launch_status();
     }
     void *scratch = nullptr;
@@ -674,14 +681,13 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     const int64_t total_v = N * K / 4;
     const int64_t nparts = (total_v + kNoAllocChunk - 1) / kNoAllocChunk;  // <= kNoAllocSlots
     double *partial = reinterpret_cast<double *>(scratch);
-    float *thresh = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(scratch) + kNoAllocThreshOff);
     if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
                                  st, w, total_v, kNoAllocChunk, sanitize, partial, 0))
         return e;
-    if (tq_status e = launch_pdl(absum_finalize_kernel, dim3(1), dim3(1024), 0, st, partial,
-                                 (int)nparts, absum_tree_height(kNoAllocChunk, (int)nparts), w,
-                                 total_v, sanitize, gamma, thresh))
-        return e;
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, thresh, 1, 0, st)) return e;
+    PerTensor pt;
+    pt.partial = partial;
+    pt.nparts = (int)nparts;
+    pt.height = absum_tree_height(kNoAllocChunk, (int)nparts);
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, 0, st)) return e;
     return launch_status();
 }

@@ -127,6 +127,51 @@ __device__ __forceinline__ double sum_error_bound(int h) { return (double)(h + 3
 //           re-summed exactly (double-double) by the same warp.
 //   pass 2: re-read the row (L2 hit: pass 1 left it there) and write one byte
 //           per float4; a warp stores 32 consecutive bytes per instruction.
+// ---------------------------------------------------------------------------
+// Per-tensor gamma from the partial sums of absum_partial_kernel, computed by
+// every CTA of the pack pass (all kPackThreads threads take part): a fixed
+// thread-strided chain over the partials and a fixed block tree, then the
+// rounding-margin check of mean_fast_or_fail with the error bound of the
+// whole summation tree (height); in the rare case that the mean lies too close
+// to an fp32 rounding boundary, an exact double-double re-sum of the tensor.
+// All CTAs therefore agree on gamma (it is the correctly rounded exact mean).
+// CTA 0 writes gamma[0].  Returns the code threshold.
+// ---------------------------------------------------------------------------
+__device__ __noinline__ float per_tensor_threshold(const double *__restrict__ partial, int nparts, int height,
+                                                   const float *__restrict__ w, int64_t nv, int sanitize,
+                                                   float *__restrict__ gamma) {
+    __shared__ double red[kPackWarps];
+    __shared__ DD redd[kPackWarps];
+    __shared__ float g_s;
+    double a = 0.0;
+    for (int i = threadIdx.x; i < nparts; i += kPackThreads) a = __dadd_rn(a, partial[i]);
+    const double S = block_sum_dbl(a, red);
+    const double n = 4.0 * (double)nv;
+    float g = mean_fast_or_fail(__ddiv_rn(S, n), sum_error_bound(height));
+    if (g < 0.0f) {  // CTA-uniform: every thread holds the same S
+        const float4 *src = reinterpret_cast<const float4 *>(w);
+        DD d = {0.0, 0.0};
+        for (int64_t idx = threadIdx.x; idx < nv; idx += kPackThreads) {
+            float4 x = __ldg(src + idx);
+            acc_abs4(d, sanitize ? sanitize_w(x) : x);
+        }
+        d = dd_warp_sum(d);
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        if (lane == 0) redd[warp] = d;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            DD e = {0.0, 0.0};
+            for (int u = 0; u < kPackWarps; ++u) e = dd_add(e, redd[u]);
+            g_s = dd_mean_to_f32(e, n);
+        }
+        __syncthreads();
+        g = g_s;
+    }
+    g = g > 1e-6f ? g : 1e-6f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) gamma[0] = g;
+    return code_threshold(g);
+}
+
 // No block-level synchronisation: warps are independent.
 // ---------------------------------------------------------------------------
 constexpr int kPackUnroll = 8;
@@ -135,13 +180,16 @@ template <bool SAN>
 __global__ void __launch_bounds__(kPackThreads)
     pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
-                     const float *__restrict__ per_tensor_t, int reverse, int ready) {
+                     const double *__restrict__ partial, int nparts, int height, int reverse,
+                     int ready) {
     if (!ready) pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * kPackWarps;
     const int nv = K >> 2;
-    const float t_tensor = per_tensor_t ? __ldg(per_tensor_t) : 0.0f;
+    const bool per_tensor = partial != nullptr;
+    const float t_tensor =
+        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma) : 0.0f;
     // per-lane chain length (float4) of pass 1, for the error bound
     const int chain = (nv + 31) / 32;
     const double eps = sum_error_bound(4 * chain + 5);
@@ -150,7 +198,7 @@ __global__ void __launch_bounds__(kPackThreads)
         const int64_t n = reverse ? (N - 1 - i) : i;
         const float4 *src = reinterpret_cast<const float4 *>(w + n * (int64_t)K);
         float t = t_tensor;
-        if (per_tensor_t == nullptr) {
+        if (!per_tensor) {
             double a = 0.0;
             int c = lane;
             for (; c + 32 * (kPackUnroll - 1) < nv; c += 32 * kPackUnroll) {
@@ -234,7 +282,8 @@ template <int T, bool SAN>
 __global__ void __launch_bounds__(kPackThreads, 2)
     pack_team_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
-                     const float *__restrict__ per_tensor_t, int reverse, int ready) {
+                     const double *__restrict__ partial, int nparts, int height, int reverse,
+                     int ready) {
     constexpr int TEAMS = kPackWarps / T;
     extern __shared__ __align__(16) float4 rowbuf[];  // [TEAMS][kPackRing][nv]
     __shared__ uint64_t rbar[TEAMS][kPackRing];
@@ -269,7 +318,10 @@ __global__ void __launch_bounds__(kPackThreads, 2)
     int64_t issued = nmine < kPackRing ? nmine : kPackRing;
     if (leader)
         for (int64_t k = 0; k < issued; ++k) issue(k);
-    const float t_tensor = per_tensor_t ? __ldg(per_tensor_t) : 0.0f;
+    // the first rows are in flight: now the per-tensor threshold (if any)
+    const bool per_tensor = partial != nullptr;
+    const float t_tensor =
+        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma) : 0.0f;
     const double eps = sum_error_bound(4 * kTeamVec + 5 + T);
     int parity = 0;
     int64_t k = 0;
@@ -286,7 +338,7 @@ __global__ void __launch_bounds__(kPackThreads, 2)
         }
         float t = t_tensor;
         bool all_ok;
-        if (per_tensor_t == nullptr) {
+        if (!per_tensor) {
             double a = 0.0;
 #pragma unroll
             for (int j = 0; j < kTeamVec; ++j) a = __dadd_rn(a, abs_sum4(v[j]));
@@ -348,16 +400,18 @@ __global__ void __launch_bounds__(kPackThreads)
     double a0 = 0.0, a1 = 0.0;
     int64_t idx = beg + threadIdx.x;
     for (; idx + 3 * kPackThreads < end; idx += 4 * kPackThreads) {
-        float4 x0 = __ldg(src + idx), x1 = __ldg(src + idx + kPackThreads),
-               x2 = __ldg(src + idx + 2 * kPackThreads), x3 = __ldg(src + idx + 3 * kPackThreads);
+        float4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = __ldg(src + idx + u * kPackThreads);
         if (sanitize) {
-            x0 = sanitize_w(x0);
-            x1 = sanitize_w(x1);
-            x2 = sanitize_w(x2);
-            x3 = sanitize_w(x3);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = sanitize_w(x[u]);
         }
-        a0 = __dadd_rn(a0, __dadd_rn(abs_sum4(x0), abs_sum4(x1)));
-        a1 = __dadd_rn(a1, __dadd_rn(abs_sum4(x2), abs_sum4(x3)));
+#pragma unroll
+        for (int u = 0; u < 4; u += 2) {
+            a0 = __dadd_rn(a0, abs_sum4(x[u]));
+            a1 = __dadd_rn(a1, abs_sum4(x[u + 1]));
+        }
     }
     for (; idx < end; idx += kPackThreads) {
         float4 x = __ldg(src + idx);
@@ -369,55 +423,14 @@ __global__ void __launch_bounds__(kPackThreads)
     if (ready) pdl_wait();  // complete no earlier than the previous kernel
 }
 
-// Tree height of the per-tensor sum: per-thread chain over its float4 of a
-// chunk (two interleaved chains joined once, each float4 adding 4 levels),
-// the CTA tree, the finalize thread's chain over partials, the finalize tree.
+// Tree height of the per-tensor sum (the longest chain of additions any term
+// goes through): a thread's chain over its float4 of a chunk (each float4
+// adds 4 levels, two interleaved chains joined once), the partial kernel's
+// block tree (8), the pack CTA's chain over partials and its block tree (8).
 __host__ __device__ inline int absum_tree_height(int64_t chunk, int nparts) {
     const int64_t per_thread = (chunk + kPackThreads - 1) / kPackThreads;  // float4
-    const int64_t parts_per_thread = (nparts + 1023) / 1024;
-    return (int)(per_thread + 4 + 1 + 8 + parts_per_thread + 10);
-}
-
-// Per-tensor gamma, pass 2: one CTA folds the partials in a fixed order,
-// checks the rounding margin, falls back to an exact double-double re-sum of
-// the whole tensor if needed, and writes gamma[0] and the code threshold.
-__global__ void __launch_bounds__(1024)
-    absum_finalize_kernel(const double *__restrict__ partial, int nparts, int height,
-                          const float *__restrict__ w, int64_t nv, int sanitize,
-                          float *__restrict__ gamma, float *__restrict__ t_out) {
-    __shared__ double red[32];
-    __shared__ DD redd[32];
-    pdl_wait();
-    pdl_trigger();
-    double a = 0.0;
-    for (int i = threadIdx.x; i < nparts; i += 1024) a = __dadd_rn(a, partial[i]);
-    // fixed-order block tree over 32 warps
-    a = warp_sum_dbl(a);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) red[warp] = a;
-    __syncthreads();
-    double S = warp_sum_dbl(red[lane]);
-    const double n = 4.0 * (double)nv;
-    const double q = __ddiv_rn(S, n);
-    float g = mean_fast_or_fail(q, sum_error_bound(height));
-    if (g < 0.0f) {
-        const float4 *src = reinterpret_cast<const float4 *>(w);
-        DD d = {0.0, 0.0};
-        for (int64_t idx = threadIdx.x; idx < nv; idx += 1024) {
-            float4 x = __ldg(src + idx);
-            acc_abs4(d, sanitize ? sanitize_w(x) : x);
-        }
-        d = dd_warp_sum(d);
-        if (lane == 0) redd[warp] = d;
-        __syncthreads();
-        d = dd_warp_sum(redd[lane]);
-        g = dd_mean_to_f32(d, n);
-    }
-    if (threadIdx.x == 0) {
-        g = g > 1e-6f ? g : 1e-6f;
-        gamma[0] = g;
-        *t_out = code_threshold(g);
-    }
+    const int64_t parts_per_thread = (nparts + kPackThreads - 1) / kPackThreads;
+    return (int)(per_thread + 4 + 1 + 8 + parts_per_thread + 8);
 }
 
 }  // namespace tq

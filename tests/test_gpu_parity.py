@@ -575,3 +575,23 @@ def test_act_inputs_ready_then_dependent_reader(cuda_lib, M, K):
     xq_ref, sx_ref, _ = oracle.act_quant(Xs[-1])
     assert_y_close(host(y), oracle.dequant(oracle.matmul_addsub(xq_ref, p_ref), g_ref, sx_ref, True))
     assert tq.device_status() == 0
+
+
+@pytest.mark.parametrize("odd, expect", [(1.25, 1.0), (1.75, 1.0 + 2.0 ** -22)])
+@pytest.mark.parametrize("sanitize", [False, True])
+def test_pack_per_tensor_midpoint_many_ctas(cuda_lib, odd, expect, sanitize):
+    """1024 x 4096 ones and one odd value: the mean is 1 + 2^-24 (ties to 1) or
+    1 + 3 * 2^-24 (ties to 1 + 2^-22), so every pack CTA must take the exact
+    path and all must agree with the oracle."""
+    N, K = 1024, 4096
+    W = np.ones((N, K), np.float32)
+    W[N // 2, 7] = odd
+    W[::3] *= -1.0
+    if sanitize:
+        W[5, 5], W[6, 6] = np.nan, np.nan  # quenched to 0: the mean drops by 2/(N K)
+        W[7, 7] = 1.0
+    packed, gamma = cuda_lib.quantize_ternary_pack(dev(W), per_row=False, sanitize=sanitize)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=False, sanitize=sanitize)
+    if not sanitize:
+        assert g_ref[0] == np.float32(expect)
+    assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)

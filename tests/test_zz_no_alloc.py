@@ -37,8 +37,11 @@ def noalloc_pack(tq, w, flags):
 def test_noalloc_matches_workspace_version_twice(cuda_lib, per_row):
     tq = cuda_lib
     flags = tq.GAMMA_PER_ROW if per_row else 0
+    tie = np.ones((1024, 4096), np.float32)
+    tie[512, 7] = 1.25  # per-tensor mean 1 + 2^-24: an exact fp32 tie (exact path)
     cases = [S.normal((2048, 4096), 0.02, 0, 61),        # many partial sums
-             S.laplace((129, 4160), 0.05, 0, 62)]        # ragged, few partial sums
+             S.laplace((129, 4160), 0.05, 0, 62),        # ragged, few partial sums
+             tie]
     for W in cases:  # two calls in a row share the library's scratch
         w = torch.from_numpy(W).cuda()
         rc, packed, gamma = noalloc_pack(tq, w, flags)
