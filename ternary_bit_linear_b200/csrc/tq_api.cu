@@ -162,41 +162,40 @@ tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       s_x, rowsum, gamma, per_row, (int)M, (int)N, (int)K, y, acc, mode);
 }
 
-// Grid: one 16-row strip per CTA while that keeps the grid within the CTAs
-// that fit on the device at once (at most four per SM, so that several
-// layers' kernels can be resident together under programmatic dependent
-// launch); beyond that, runs of strips per CTA through a ring of up to
-// kGemvMaxStages stages.  Large x_q (M * K) costs shared memory per CTA and
-// L2 traffic per CTA, so it lowers the CTAs per SM and lengthens the runs.
-template <int NB, int W>
+// Grid: one CTA per 16-row strip.  Dynamic shared memory holds x_q only.
+template <int NB, int W, int SPW>
 tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
-                      int64_t K, float *y, int32_t *acc, int mode, int sms, cudaStream_t st) {
+                      int64_t K, float *y, int32_t *acc, int mode, cudaStream_t st) {
+    static_assert(256 * W * SPW >= kGemvMaxK / 2, "shape covers K");
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemv_kernel<NB, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemvSmemCap) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemv_kernel<NB, W, SPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemv_x_bytes(8 * NB, kGemvMaxK)) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
     }
-    const int64_t nstrips = (N + 15) / 16;
-    const int xb = gemv_x_bytes((int)M, (int)K), sb = gemv_stage_bytes((int)K);
-    int64_t per_sm = kGemvSmemCap / (xb + sb);
-    if (per_sm > 4) per_sm = 4;
-    if (per_sm < 1) per_sm = 1;
-    const int64_t max_grid = per_sm * (int64_t)sms;
-    const int64_t per_cta = (nstrips + max_grid - 1) / max_grid;
-    const int64_t grid = (nstrips + per_cta - 1) / per_cta;
-    int64_t nstage = (kGemvSmemCap - xb) / sb;
-    if (nstage > per_cta) nstage = per_cta;
-    if (nstage > kGemvMaxStages) nstage = kGemvMaxStages;
-    if (nstage < 1) return TQ_ERR_SHAPE;  // cannot happen for K <= kGemvMaxK, M <= 16
-    const size_t smem = (size_t)xb + (size_t)nstage * sb;
-    return launch_pdl(gemv_kernel<NB, W>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq, s_x,
-                      rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, mode, (int)nstage,
-                      (int)per_cta);
+    const int64_t grid = (N + 15) / 16;
+    const size_t smem = (size_t)gemv_x_bytes((int)M, (int)K);
+    return launch_pdl(gemv_kernel<NB, W, SPW>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq, s_x,
+                      rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, mode);
+}
+
+// Independent calls (inputs ready) overlap one another: lean CTAs (four
+// steps per warp) keep several layers resident.  Otherwise, for K <= 4096,
+// the time after the wait is the critical path: twice the warps, two steps
+// each.  Larger K keeps the lean shape (16-warp CTAs measured slower).
+template <int NB>
+tq_status gemv_shape(const int8_t *xq, const float *s_x, const int32_t *rowsum, const uint8_t *packed,
+                     const float *gamma, int per_row, int64_t M, int64_t N, int64_t K, float *y,
+                     int32_t *acc, int mode, cudaStream_t st) {
+    const bool lean = (mode & kModeInputsReady) != 0;
+    if (K <= kGemvMaxK / 2)
+        return lean ? launch_gemv<NB, 4, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st)
+                    : launch_gemv<NB, 8, 2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+    return launch_gemv<NB, 8, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
 }
 
 template <int NW>
@@ -364,16 +363,8 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
     const int mode = ((flags & TQ_FLAG_WEIGHTS_STATIC) ? kModeWeightsStatic : 0) |
                      ((flags & TQ_FLAG_INPUTS_READY) ? kModeInputsReady : 0);
     if (M <= 16 && K <= kGemvMaxK) {
-        // A dependent chain of layers waits on each kernel's critical path, so
-        // more warps share a strip; with ready inputs the kernels overlap and
-        // leaner CTAs let more of them be resident.
-        const int64_t nsteps = (K / 4 + 63) / 64;  // 64-byte column steps per row
-        const bool lean = nsteps <= 8 || ((mode & kModeInputsReady) && nsteps <= 16);
-        if (M <= 8)
-            return lean ? launch_gemv<1, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st)
-                        : launch_gemv<1, 8>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-        return lean ? launch_gemv<2, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st)
-                    : launch_gemv<2, 8>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+        if (M <= 8) return gemv_shape<1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+        return gemv_shape<2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
     }
     switch (gemm_tile_tokens(M, N, sms)) {
     case 64: return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
