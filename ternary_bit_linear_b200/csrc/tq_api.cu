@@ -183,6 +183,29 @@ tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, mode);
 }
 
+// Independent calls: a narrow grid of about 32 CTAs streaming runs of strips
+// (at least one strip per group), so that consecutive calls run side by side.
+tq_status launch_gemv_stream(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                             const uint8_t *packed, const float *gamma, int per_row, int64_t M,
+                             int64_t N, int64_t K, float *y, int32_t *acc, cudaStream_t st) {
+    static std::atomic<int> attr_done[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev].load()) {
+        if (cudaFuncSetAttribute(gemv_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemv_x_bytes(8, kStreamMaxK)) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        attr_done[dev].store(1);
+    }
+    const int64_t nstrips = (N + 15) / 16;
+    int64_t per_cta = (nstrips + 31) / 32;
+    if (per_cta < kStreamGroups) per_cta = kStreamGroups;
+    const int64_t grid = (nstrips + per_cta - 1) / per_cta;
+    const size_t smem = (size_t)gemv_x_bytes((int)M, (int)K);
+    return launch_pdl(gemv_stream_kernel, dim3((unsigned)grid), dim3(kStreamThreads), smem, st, xq, s_x,
+                      rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, (int)per_cta);
+}
+
 // Independent calls (inputs ready) overlap one another: lean CTAs (four
 // steps per warp) keep several layers resident.  Otherwise, for K <= 4096,
 // the time after the wait is the critical path: twice the warps, two steps
@@ -363,6 +386,8 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
     const int mode = ((flags & TQ_FLAG_WEIGHTS_STATIC) ? kModeWeightsStatic : 0) |
                      ((flags & TQ_FLAG_INPUTS_READY) ? kModeInputsReady : 0);
     if (M <= 16 && K <= kGemvMaxK) {
+        if ((mode & kModeInputsReady) && M <= 8 && K <= kStreamMaxK)
+            return launch_gemv_stream(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
         if (M <= 8) return gemv_shape<1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
         return gemv_shape<2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
     }

@@ -241,6 +241,33 @@ def test_gemm_matches_oracle(cuda_lib, M, N, K, per_row):
     assert_y_close(y, oracle.dequant(acc_ref, g_ref, sx_ref, per_row))
 
 
+# Independent calls (TQ_FLAG_INPUTS_READY, M <= 8, K <= 4096) take the narrow
+# streaming GEMV: runs of strips per CTA, one group of warps per strip, two
+# strips in flight per group.  Shapes: one 64-byte step, a ragged last step,
+# ragged last strips, runs shorter than the groups, and long runs (N = 16400:
+# 33 strips per CTA, a ragged tail run).
+STREAM_CASES = [(1, 1, 64), (3, 17, 1088), (8, 1000, 4096), (1, 4096, 4096), (5, 16400, 2048),
+                (8, 64, 256), (2, 16384, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", STREAM_CASES)
+@pytest.mark.parametrize("per_row", [True, False])
+def test_gemv_stream_matches_oracle(cuda_lib, M, N, K, per_row):
+    tq = cuda_lib
+    W = S.normal((N, K), 0.02, 7, 2000 + N)
+    X = S.decode_acts(M, K, seed=8)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    fl = (tq.GAMMA_PER_ROW if per_row else 0) | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY
+    tq.ternary_gemm_(dev(xq_ref), dev(sx_ref), dev(rs_ref), dev(p_ref), dev(g_ref), fl, y, acc)
+    acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
+    assert np.array_equal(host(acc), acc_ref)
+    assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, per_row))
+    assert tq.device_status() == 0
+
+
 def test_gemm_extreme_codes(cuda_lib):
     # all +1 / all -1 / all 0 weight rows and +-127 activations: |acc| = 127*K
     K, N, M = 4096, 130, 40
