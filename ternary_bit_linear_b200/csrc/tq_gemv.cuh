@@ -26,15 +26,16 @@
 //     j < SPW, and loads them straight into registers (no shared-memory
 //     staging, no barrier in front of the weight stream).
 //   * x_q (M <= 16 rows) is copied into shared memory with cp.async (no
-//     registers held), rows padded so that the reads below are free of bank
-//     conflicts; gamma, s_x and rowsum are requested early.
+//     registers held); gamma, s_x and rowsum are requested early.
 //   * A 32-bit word holds 16 codes; (word >> 2j) & 0x03030303 spreads codes
 //     {j, 4+j, 8+j, 12+j} into bytes as unsigned values c = q + 1 in
-//     {0, 1, 2}; the matching 16 activations are transposed the same way, so
-//     the pairing of codes and activations is exact.  Threads with t >= 2
-//     walk their four words in rotated order (a relabelling of k that is the
-//     same for codes and activations), which spreads a quarter-warp's
-//     activation reads over all 32 banks.
+//     {0, 1, 2}.  The matching 16 activations are the 16-byte chunk of x_q
+//     transposed 4 x 4 the same way, so the pairing of codes and activations
+//     is exact.  The streaming kernel, whose CTAs use x_q for many strips,
+//     transposes every chunk once, in place, right after it lands.  Chunk c
+//     of a row sits at position c ^ (((c >> 3) & 1) << 1) and rows are 16
+//     bytes past a multiple of 128 apart, which makes a quarter-warp's chunk
+//     reads (8 threads, 2 rows x 4 column offsets) free of bank conflicts.
 //   * mma.sync m16n8k32 (u8 x s8 -> s32) reduces 32 codes per row and token;
 //     sum_k x*c - sum_k x = sum_k x*q removes the offset (rowsum).
 //   * The warps' partial sums meet in shared memory; each thread finishes one
@@ -47,8 +48,10 @@ namespace tq {
 
 constexpr int kGemvMaxK = 8192;
 
-// Padded shared-memory row stride of x_q: 32 bytes past a multiple of 128.
-__host__ __device__ inline int gemv_x_stride(int K) { return K + ((32 - K % 128) + 128) % 128; }
+// Shared-memory row stride of x_q (16 bytes past a multiple of 128) and the
+// swizzled position of 16-byte chunk c inside a row.
+__host__ __device__ inline int gemv_x_stride(int K) { return K + ((16 - K % 128) + 128) % 128; }
+__device__ __forceinline__ uint32_t x_chunk(int c) { return (uint32_t)(c ^ (((c >> 3) & 1) << 1)) << 4; }
 __host__ __device__ inline int gemv_x_bytes(int M, int K) { return M * gemv_x_stride(K); }
 
 // 4x4 byte transpose: out word j = (in0.byte j, in1.byte j, in2.byte j, in3.byte j).
@@ -119,12 +122,14 @@ __device__ __forceinline__ void load_strip(StripRegs<SPW> &r, const uint8_t *__r
 }
 
 // Partial sums of one warp over its column steps: d[chain][nb][fragment].
-template <int NB, int W, int SPW, int CH>
+// XT: the x_q chunks in shared memory are already transposed (else each
+// chunk is transposed here, after it is read).
+template <int NB, int W, int SPW, int CH, bool XT>
 __device__ __forceinline__ void strip_mma(const StripRegs<SPW> &r, int (&d)[CH][NB][4], int w, int lane,
                                           uint32_t x_s, int XS, int M, int KB) {
     const int g = lane >> 2, t = lane & 3;
     const int nsteps = (KB + 63) >> 6;
-    const int rot = t >> 1;  // rotated word order for t >= 2
+    const uint32_t xsw = (uint32_t)(t & 2) << 4;  // chunk swizzle of this thread's columns
 #pragma unroll
     for (int i = 0; i < CH; ++i)
 #pragma unroll
@@ -138,9 +143,7 @@ __device__ __forceinline__ void strip_mma(const StripRegs<SPW> &r, int (&d)[CH][
             const uint32_t b4[4] = {r.b[j].x, r.b[j].y, r.b[j].z, r.b[j].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int ii = (i + rot) & 3;
-                const uint32_t ar = rot ? a4[(i + 1) & 3] : a4[i];
-                const uint32_t br = rot ? b4[(i + 1) & 3] : b4[i];
+                const uint32_t ar = a4[i], br = b4[i];
                 uint32_t ua[4], ub[4];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
@@ -150,9 +153,11 @@ __device__ __forceinline__ void strip_mma(const StripRegs<SPW> &r, int (&d)[CH][
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb) {
                     const int m = g + 8 * nb;
-                    uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-                    if (m < M && bo < KB) xv = lds128(x_s + (uint32_t)(m * XS + 4 * bo + 16 * ii));
-                    const uint4 xt = transpose_bytes4x4(xv);
+                    // chunk c = bo / 4 + i, at x_chunk(c) = 16 * (bo / 4 + (i ^ (t & 2)))
+                    uint4 xt = make_uint4(0u, 0u, 0u, 0u);
+                    if (m < M && bo < KB)
+                        xt = lds128(x_s + (uint32_t)(m * XS + 4 * bo) + ((uint32_t)(i << 4) ^ xsw));
+                    if (!XT) xt = transpose_bytes4x4(xt);
                     mma_16x8x32_u8s8(d[i % CH][nb], ua[0], ub[0], ua[1], ub[1], xt.x, xt.y);
                     mma_16x8x32_u8s8(d[i % CH][nb], ua[2], ub[2], ua[3], ub[3], xt.z, xt.w);
                 }
@@ -167,13 +172,25 @@ __device__ __forceinline__ void strip_mma(const StripRegs<SPW> &r, int (&d)[CH][
 __device__ __forceinline__ int fin_row(int e) { return ((e & 31) >> 2) + (((e >> 5) & 2) ? 8 : 0); }
 __device__ __forceinline__ int fin_tok(int e) { return 8 * (e >> 7) + 2 * (e & 3) + ((e >> 5) & 1); }
 
-// x_q rows into padded shared memory, 16 bytes per copy, by `nthr` threads.
+// x_q rows into shared memory (swizzled chunks), 16 bytes per copy, by
+// `nthr` threads; then, once landed, each thread transposes the chunks it
+// copied (its own cp.async writes are complete after the wait).
 __device__ __forceinline__ void copy_x(uint32_t x_s, const int8_t *__restrict__ xq, int M, int K, int XS,
                                        int tid, int nthr) {
     const int cpr = K >> 4;
     for (int i = tid; i < M * cpr; i += nthr) {
         const int m = i / cpr, c = i - m * cpr;
-        cp_async16(x_s + (uint32_t)(m * XS + 16 * c), xq + (int64_t)m * K + 16 * c);
+        cp_async16(x_s + (uint32_t)(m * XS) + x_chunk(c), xq + (int64_t)m * K + 16 * c);
+    }
+}
+__device__ __forceinline__ void transpose_x(uint32_t x_s, int M, int K, int XS, int tid, int nthr) {
+    const int cpr = K >> 4;
+    for (int i = tid; i < M * cpr; i += nthr) {
+        const int m = i / cpr, c = i - m * cpr;
+        const uint32_t a = x_s + (uint32_t)(m * XS) + x_chunk(c);
+        const uint4 v = transpose_bytes4x4(lds128(a));
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                     : "memory");
     }
 }
 
@@ -245,10 +262,11 @@ __global__ void __launch_bounds__(W * 32, gemv_min_blocks(NB, W))
         load_strip<SPW, W>(wr, packed, r0, N, KB, warp, lane);
     }
     cp_async_wait_all();
-    __syncthreads();  // x_q is in shared memory
+    __syncthreads();  // x_q is in shared memory (each chunk is used once here:
+                      // transposed where it is read, off the wait's critical path)
 
     int d[CH][NB][4];
-    strip_mma<NB, W, SPW, CH>(wr, d, warp, lane, x_s, XS, M, KB);
+    strip_mma<NB, W, SPW, CH, false>(wr, d, warp, lane, x_s, XS, M, KB);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -329,12 +347,13 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
     if (k < nmine) load_strip<SPW, GW>(w0, packed, (s0 + k) * 16, N, KB, gw, lane);
     float g0 = gamma_of(k);
     cp_async_wait_all();
-    __syncthreads();  // x_q is in shared memory
+    transpose_x(x_s, M, K, XS, threadIdx.x, kStreamThreads);
+    __syncthreads();  // x_q is in shared memory, transposed
 
     int par = 0;
     auto one = [&](const StripRegs<SPW> &w, int kk, float gn) {
         int d[CH][1][4];
-        strip_mma<1, GW, SPW, CH>(w, d, gw, lane, x_s, XS, M, KB);
+        strip_mma<1, GW, SPW, CH, true>(w, d, gw, lane, x_s, XS, M, KB);
 #pragma unroll
         for (int c = 0; c < 4; ++c) red[group][par][gw][c][lane] = d[0][0][c] + d[1][0][c];
         group_sync(group);
