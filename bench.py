@@ -69,24 +69,30 @@ def peaks():
                 "source": "fallback"}
 
 
-def kernel_source_hash():
+KERNEL_FILES = {  # sources that decide a kernel's memory traffic (besides tq_common.cuh, tq_api.cu)
+    "pack": ["tq_pack.cuh"], "act_quant": ["tq_act.cuh"], "gemv": ["tq_gemv.cuh"],
+    "gemm": ["tq_gemm.cuh"], "fused": ["tq_act.cuh", "tq_gemm.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ternary_bit_linear_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in ["tq_common.cuh", "tq_api.cu"] + KERNEL_FILES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, or None if the
-    kernels changed since it was taken."""
+def traffic_for(key: str):
+    """DRAM bytes per launch ("kernel:workload") from the committed ncu
+    summary, or None if that kernel's sources changed since it was taken."""
     try:
         with open(TRAFFIC_FILE) as f:
-            t = json.load(f)
-        if t.get("source_hash") != kernel_source_hash():
+            t = json.load(f)["kernels"][key]
+        if t["source_hash"] != kernel_source_hash(key.split(":")[0]):
             return None
-        return t["kernels"].get(kernel)
+        return t["bytes"]
     except Exception:
         return None
 

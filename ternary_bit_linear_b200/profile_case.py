@@ -1,7 +1,7 @@
 """Run one kernel of the hot path a few times on a chosen shape -- the small,
 self-contained command that ncu captures are taken on.
 
-    python -m ternary_bit_linear_b200.profile_case --kernel gemv --M 8 --N 4096 --K 4096 --reps 3
+    python -m ternary_bit_linear_b200.profile_case --kernel gemv --M 8 --N 4096 --K 4096 --reps 3 [--ready]
 
 Inputs are random device tensors of the workloads' distributions (values do
 not affect timing); every call goes through the C ABI.  Exits non-zero if a
@@ -24,6 +24,8 @@ def main():
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--ready", action="store_true",
+                    help="contractions with TQ_FLAG_INPUTS_READY (independent calls: the streaming GEMV)")
     a = ap.parse_args()
     tq.load()
     dev = torch.device("cuda", 0)
@@ -49,7 +51,8 @@ def main():
         elif a.kernel == "fwht":
             tq.fwht512_(X, Xr)
         elif a.kernel in ("gemv", "gemm"):
-            tq.ternary_gemm_(xq, sx, rs, packed, gamma, flags, y)
+            ready = tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY if a.ready else 0
+            tq.ternary_gemm_(xq, sx, rs, packed, gamma, flags | ready, y)
         else:
             tq.bitlinear_fused_(X, packed, gamma, tq.FLAG_FWHT | tq.FLAG_RMSNORM, y, ws)
     torch.cuda.synchronize()
