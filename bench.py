@@ -213,8 +213,10 @@ class Workload:
         self.y = {M: [torch.empty((M, N), dtype=f32, device=dev) for _ in range(L)] for M in self.Ms}
         if name == "fused":
             fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM
-            self.fused_flags = fl | tq.FLAG_WEIGHTS_STATIC
-            self.fused_ws = torch.empty((tq.fused_workspace_bytes(self.Ms[0], K, fl),), dtype=u8, device=dev)
+            # the ring's layers have their own x, y and workspace: independent calls
+            self.fused_flags = fl | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY
+            self.fused_ws = [torch.empty((tq.fused_workspace_bytes(self.Ms[0], K, fl),), dtype=u8, device=dev)
+                             for _ in range(L)]
 
         # --- segments of one step ---
         pack_bytes = 4 * N * K + N * K // 4 + 4 * (N if self.per_row else 1)
@@ -228,7 +230,7 @@ class Workload:
             ops = 2 * M * N * K
             self.segments.append(("fused M=%d" % M, "fused", L, L * ops, 2 * L, [
                 lambda l=l: tq.bitlinear_fused_(self.Xd[M][l], self.packed[l], self.gamma[l],
-                                                self.fused_flags, self.y[M][l], self.fused_ws)
+                                                self.fused_flags, self.y[M][l], self.fused_ws[l])
                 for l in range(L)]))
             return
         act_bytes = L * sum(4 * M * K + M * K + 8 * M for M in self.Ms)

@@ -93,14 +93,20 @@ typedef enum tq_status {
  * streaming weights and gamma before the wait.
  *
  * TQ_FLAG_INPUTS_READY (tq_ternary_gemm, tq_quantize_ternary_pack,
- * tq_quantize_act_int8): the
- * caller promises that no work in flight writes any input of the call or
- * reads or writes its outputs or workspace -- e.g. the independent
- * projections of one decode step that share an activation (q/k/v, gate/up),
- * each with its own output, or the packing of a model's layers, each with its
- * own buffers.  The first kernel of the call then reads and computes at once
- * and waits for the previous kernel only before it exits, so any later call
- * still sees every earlier result.  Without either flag nothing is read early.
+ * tq_quantize_act_int8, tq_bitlinear_fused): the caller promises that no work
+ * in flight writes any input of the call or reads or writes its outputs or
+ * workspace -- e.g. the independent projections of one decode step that share
+ * an activation (q/k/v, gate/up), each with its own output, or the packing of
+ * a model's layers, each with its own buffers.  The first kernel of the call
+ * then reads and computes at once and waits for the previous kernel only
+ * before it exits, so any later call still sees every earlier result (it
+ * implies TQ_FLAG_WEIGHTS_STATIC).  For the small-M contraction it also
+ * selects a narrow streaming grid built for many such calls in flight; a
+ * lone call is quicker without the flag.  Without either flag nothing is read
+ * early.  A flagged call may still be running while later calls on the stream
+ * start, so its buffers must not be recycled by a stream-ordered allocator
+ * (which assumes that work on one stream runs in order) until the stream has
+ * been drained.
  */
 
 /*

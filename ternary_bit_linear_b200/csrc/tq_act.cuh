@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(NW * 32)
     __shared__ int redi[32];
     __shared__ double redd[32];
     constexpr int K = 512 * NW;
-    pdl_wait();
+    if (!p.ready) pdl_wait();
     pdl_trigger();
     const int64_t m = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -453,6 +453,9 @@ __global__ void __launch_bounds__(NW * 32)
         s_x[m] = __fdiv_rn(eta, 127.0f);
         rowsum[m] = sum;
     }
+    // Inputs ready: complete no earlier than the previous kernel (one CTA
+    // waits; the others free their slots at once).
+    if (p.ready && blockIdx.x == gridDim.x - 1) pdl_wait();
 }
 
 }  // namespace tq

@@ -548,7 +548,7 @@ tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_ep
     if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
     const unsigned known = TQ_GAMMA_PER_ROW | TQ_FLAG_FWHT | TQ_FLAG_RMSNORM | TQ_FLAG_ETA_CLAMP |
-                           TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_WEIGHTS_STATIC;
+                           TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY;
     if (flags & ~known) return TQ_ERR_ARG;
     if ((flags & TQ_FLAG_FWHT) && (K % 512 != 0 || K > kMaxFwhtFusedK)) return TQ_ERR_SHAPE;
     if ((flags & TQ_FLAG_ETA_CLAMP) && !(eta_min > 0.0f && eta_min <= eta_max)) return TQ_ERR_ARG;
@@ -592,14 +592,17 @@ tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_ep
     p.rmsnorm = (flags & TQ_FLAG_RMSNORM) ? 1 : 0;
     p.rms_eps = rms_eps;
     p.rms_gain = rms_gain;
+    // Inputs ready: the activation pass reads x at once; the contraction still
+    // waits for it (x_q is made here), but may stream its weights early.
+    p.ready = (flags & TQ_FLAG_INPUTS_READY) ? 1 : 0;
     if (flags & TQ_FLAG_FWHT)
         Prologues::fns[K / 512 - 1](x, p, M, xq, sx, rs, st);
     else
         launch_act(x, p, M, K, xq, sx, rs, st);
     if (tq_status e = launch_status()) return e;
-    return gemm_dispatch(xq, sx, rs, packed, gamma,
-                         flags & (TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC), M, N, K, y, nullptr,
-                         sms, st);
+    const unsigned cflags = (flags & (TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC)) |
+                            ((flags & TQ_FLAG_INPUTS_READY) ? TQ_FLAG_WEIGHTS_STATIC : 0u);
+    return gemm_dispatch(xq, sx, rs, packed, gamma, cflags, M, N, K, y, nullptr, sms, st);
 }
 
 tq_status tq_get_device_status(tq_stream_t stream) {

@@ -261,7 +261,8 @@ def test_gemv_stream_matches_oracle(cuda_lib, M, N, K, per_row):
     y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
     fl = (tq.GAMMA_PER_ROW if per_row else 0) | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY
-    tq.ternary_gemm_(dev(xq_ref), dev(sx_ref), dev(rs_ref), dev(p_ref), dev(g_ref), fl, y, acc)
+    ins = [dev(a) for a in (xq_ref, sx_ref, rs_ref, p_ref, g_ref)]  # alive until the sync below
+    tq.ternary_gemm_(*ins, fl, y, acc)
     acc_ref = oracle.matmul_addsub(xq_ref, p_ref)
     assert np.array_equal(host(acc), acc_ref)
     assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, per_row))
@@ -521,16 +522,45 @@ def test_inputs_ready_flag_same_result_and_order(cuda_lib, M, N, K):
     assert tq.device_status() == 0
 
 
-def test_inputs_ready_flag_rejected_by_fused(cuda_lib):
+@pytest.mark.parametrize("M,K", [(4, 512), (512, 2048)])
+def test_fused_inputs_ready_same_result_and_order(cuda_lib, M, K):
+    """Independent fused layers (own x, y and workspace; N = K) launched with
+    TQ_FLAG_INPUTS_READY back to back, then a flag-less fused call that takes
+    the first layer's output as its input: every result equals the flag-less
+    one, and the dependent call sees the finished output."""
     tq = cuda_lib
-    M, N, K = 4, 64, 512
-    x = torch.zeros((M, K), dtype=torch.float32, device="cuda")
-    packed = torch.zeros((N, K // 4), dtype=torch.uint8, device="cuda")
-    gamma = torch.ones((1,), dtype=torch.float32, device="cuda")
-    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
-    ws = torch.empty((max(16, tq.fused_workspace_bytes(M, K, 0)),), dtype=torch.uint8, device="cuda")
-    with pytest.raises(RuntimeError):
-        tq.bitlinear_fused_(x, packed, gamma, tq.FLAG_INPUTS_READY, y, ws)
+    N = K
+    fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM
+    p_ref, g_ref = oracle.quantize_pack(S.normal((N, K), 0.02, 61, N), per_row=False)
+    packed, gamma = dev(p_ref), dev(g_ref)
+    xs = [dev(S.student_t3((M, K), 62 + i, 4 * M)) for i in range(3)]
+
+    def new_ws():
+        return torch.empty((tq.fused_workspace_bytes(M, K, fl),), dtype=torch.uint8, device="cuda")
+
+    def new_y():
+        return torch.empty((M, N), dtype=torch.float32, device="cuda")
+
+    torch.cuda.synchronize()
+    # every buffer of a flagged call stays allocated until the stream is
+    # drained: the caching allocator would hand a freed block to the next
+    # call on the same stream while the flagged call may still run
+    ys = [new_y() for _ in xs]
+    wss = [new_ws() for _ in xs]
+    for x, y, ws in zip(xs, ys, wss):
+        tq.bitlinear_fused_(x, packed, gamma, fl | tq.FLAG_INPUTS_READY, y, ws)
+    y_dep = new_y()
+    tq.bitlinear_fused_(ys[0], packed, gamma, fl, y_dep, new_ws())
+    torch.cuda.synchronize()
+    refs = [new_y() for _ in xs]
+    for x, r in zip(xs, refs):
+        tq.bitlinear_fused_(x, packed, gamma, fl, r, new_ws())
+    r_dep = new_y()
+    tq.bitlinear_fused_(refs[0], packed, gamma, fl, r_dep, new_ws())
+    for i, (y, r) in enumerate(zip(ys + [y_dep], refs + [r_dep])):
+        bad = (y != r).sum().item()
+        assert bad == 0, "call %d: %d of %d outputs differ" % (i, bad, y.numel())
+    assert tq.device_status() == 0
 
 
 @pytest.mark.parametrize("per_row", [True, False])
