@@ -56,6 +56,10 @@ def _load():
         _lib.tqo_unpack.argtypes = [P, I64, I64, P]
         _lib.tqo_unpack.restype = I64
         _lib.tqo_quantize_pack.argtypes = [P, I64, I64, I, I, P, P]
+        _lib.tqo_quantize_pack_format.argtypes = [P, I64, I64, I, I, I, P, P]
+        _lib.tqo_pack_format.argtypes = [P, I64, I64, I, P]
+        _lib.tqo_unpack_format.argtypes = [P, I64, I64, I, P]
+        _lib.tqo_matmul_addsub_format.argtypes = [P, P, I64, I64, I64, I, P]
         _lib.tqo_act_quant.argtypes = [P, I64, I64, I, F, F, P, P, P]
         _lib.tqo_matmul_dense.argtypes = [P, P, I64, I64, I64, P]
         _lib.tqo_matmul_addsub.argtypes = [P, P, I64, I64, I64, P]
@@ -118,16 +122,35 @@ def unpack(packed, K: int):
     return q, int(n_res)
 
 
-def quantize_pack(w, per_row: bool, sanitize: bool = False):
-    """Returns (packed uint8 [N, K/4], gamma float32 [N] or [1])."""
+def quantize_pack(w, per_row: bool, sanitize: bool = False, encoding: int = 0):
+    """Returns (packed uint8 [N, K/4], gamma float32 [N] or [1]).  encoding:
+    0 Foundry's layout, 1 Hetman-2b "Format 0", 2 Hetman-2b "Format 1"."""
     w, pw = _c(w, np.float32)
     N, K = w.shape
     packed = np.empty((N, K // 4), np.uint8)
     gamma = np.empty((N if per_row else 1,), np.float32)
-    _load().tqo_quantize_pack(pw, N, K, int(per_row), int(sanitize),
-                              packed.ctypes.data_as(ctypes.c_void_p),
-                              gamma.ctypes.data_as(ctypes.c_void_p))
+    _load().tqo_quantize_pack_format(pw, N, K, int(per_row), int(sanitize), int(encoding),
+                                     packed.ctypes.data_as(ctypes.c_void_p),
+                                     gamma.ctypes.data_as(ctypes.c_void_p))
     return packed, gamma
+
+
+def pack_format(q, encoding: int):
+    q, pq = _c(q, np.int8)
+    N, K = q.shape
+    assert K % 4 == 0
+    out = np.empty((N, K // 4), np.uint8)
+    _load().tqo_pack_format(pq, N, K, int(encoding), out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def unpack_format(packed, K: int, encoding: int):
+    packed, pp = _c(packed, np.uint8)
+    N = packed.shape[0]
+    assert packed.shape[1] * 4 == K
+    q = np.empty((N, K), np.int8)
+    _load().tqo_unpack_format(pp, N, K, int(encoding), q.ctypes.data_as(ctypes.c_void_p))
+    return q
 
 
 # --------------------------------------------------------------------------
@@ -165,6 +188,17 @@ def matmul_addsub(xq, packed):
     assert packed.shape[1] * 4 == K
     acc = np.empty((M, N), np.int32)
     _load().tqo_matmul_addsub(px, pp, M, N, K, acc.ctypes.data_as(ctypes.c_void_p))
+    return acc
+
+
+def matmul_addsub_format(xq, packed, encoding: int):
+    xq, px = _c(xq, np.int8)
+    packed, pp = _c(packed, np.uint8)
+    M, K = xq.shape
+    N = packed.shape[0]
+    assert packed.shape[1] * 4 == K
+    acc = np.empty((M, N), np.int32)
+    _load().tqo_matmul_addsub_format(px, pp, M, N, K, int(encoding), acc.ctypes.data_as(ctypes.c_void_p))
     return acc
 
 

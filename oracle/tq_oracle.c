@@ -222,11 +222,58 @@ int64_t tqo_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *q)
     return reserved;
 }
 
+/* The other two layouts of [H] section 3 (PackedTernaryStorage), four codes
+ * per byte LSB-first as above:
+ *   format 1 ("Format 0", the arithmetic-optimised default there): the low
+ *            two bits of the int8 code, -1 -> 0b11, 0 -> 0b00, +1 -> 0b01;
+ *   format 2 ("Format 1"): -1 -> 0b10, 0 -> 0b00, +1 -> 0b01.
+ * format 0 is [F]'s layout (tqo_pack).  The numbering is this library's. */
+void tqo_pack_format(const int8_t *q, int64_t N, int64_t K, int format, uint8_t *packed)
+{
+    if (format == 0) {
+        tqo_pack(q, N, K, packed);
+        return;
+    }
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 4; ++j) {
+            unsigned b = 0;
+            for (int i = 0; i < 4; ++i) {
+                int c = q[n * K + 4 * j + i];
+                unsigned v;
+                if (format == 1) v = (unsigned)(c & 3); /* two's complement -1 = ...11 */
+                else v = c == -1 ? 2u : (c == 1 ? 1u : 0u);
+                b |= v << (2 * i);
+            }
+            packed[n * (K / 4) + j] = (uint8_t)b;
+        }
+}
+
+/* Decoding of [H] section 3 unpack_torch, per 2-bit field f: P = f & 1,
+ * N = (f >> 1) & 1; "Format 0": v = P - 2 (P & N); "Format 1": v = P - N.
+ * The unassigned field (0b10, resp. 0b11) decodes to 0 by these formulas
+ * (the page's "reserved / NOP").  format 0 ([F]) decodes as tqo_unpack. */
+static int decode_field(unsigned f, int format)
+{
+    int P = (int)(f & 1u), Nb = (int)((f >> 1) & 1u);
+    if (format == 1) return P - 2 * (P & Nb);
+    if (format == 2) return P - Nb;
+    return f == 0 ? -1 : (f == 2 ? 1 : 0);
+}
+
+void tqo_unpack_format(const uint8_t *packed, int64_t N, int64_t K, int format, int8_t *q)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 4; ++j) {
+            unsigned b = packed[n * (K / 4) + j];
+            for (int i = 0; i < 4; ++i) q[n * K + 4 * j + i] = (int8_t)decode_field((b >> (2 * i)) & 3u, format);
+        }
+}
+
 /* gamma (per tensor, or per row) then codes then packing: the export path of
  * [H] section 5 BitLinear.export_packed_weights, with the per-row gamma of
  * [F] fq_quantize_ternary_per_channel as the alternative granularity. */
-void tqo_quantize_pack(const float *w_in, int64_t N, int64_t K, int per_row,
-                       int sanitize, uint8_t *packed, float *gamma)
+void tqo_quantize_pack_format(const float *w_in, int64_t N, int64_t K, int per_row,
+                              int sanitize, int format, uint8_t *packed, float *gamma)
 {
     const float *w = w_in;
     float *tmp = NULL;
@@ -242,9 +289,15 @@ void tqo_quantize_pack(const float *w_in, int64_t N, int64_t K, int per_row,
     }
     int8_t *q = (int8_t *)malloc((size_t)(N * K));
     tqo_ternary_codes(w, N, K, gamma, per_row, q);
-    tqo_pack(q, N, K, packed);
+    tqo_pack_format(q, N, K, format, packed);
     free(q);
     free(tmp);
+}
+
+void tqo_quantize_pack(const float *w_in, int64_t N, int64_t K, int per_row,
+                       int sanitize, uint8_t *packed, float *gamma)
+{
+    tqo_quantize_pack_format(w_in, N, K, per_row, sanitize, 0, packed, gamma);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -331,6 +384,27 @@ void tqo_matmul_addsub(const int8_t *xq, const uint8_t *packed, int64_t M, int64
                     int64_t xv = xq[m * K + 4 * j + i];
                     if (v == 2) plus += xv;       /* +1 */
                     else if (v == 0) minus += xv; /* -1 */
+                }
+            }
+            acc[m * N + n] = (int32_t)(plus - minus);
+        }
+}
+
+/* The same add/subtract/skip walk for a packed row in any of the three
+ * layouts, each field decoded by the layout's own rule (decode_field). */
+void tqo_matmul_addsub_format(const int8_t *xq, const uint8_t *packed, int64_t M, int64_t N,
+                              int64_t K, int format, int32_t *acc)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t plus = 0, minus = 0;
+            for (int64_t j = 0; j < K / 4; ++j) {
+                unsigned b = packed[n * (K / 4) + j];
+                for (int i = 0; i < 4; ++i) {
+                    int v = decode_field((b >> (2 * i)) & 3u, format);
+                    int64_t xv = xq[m * K + 4 * j + i];
+                    if (v == 1) plus += xv;
+                    else if (v == -1) minus += xv;
                 }
             }
             acc[m * N + n] = (int32_t)(plus - minus);

@@ -80,6 +80,65 @@ def test_unpack_flags_reserved_code():
     assert back.tolist() == [[0, 0, 0, 0, 0, 0, 0, 0]]
 
 
+# Hetman-2b section 3 layouts ("Format 0" = encoding 1, "Format 1" = encoding 2)
+FORMATS = {"F0": 1, "F1": 2}
+
+
+def test_pack_formats_hand_worked_bytes():
+    for ln in golden_lines("pack_bytes_formats.txt"):
+        fmt, *vals, byte = ln.split()
+        q = np.array([[int(v) for v in vals]], np.int8)
+        assert oracle.pack_format(q, FORMATS[fmt])[0, 0] == int(byte, 16), ln
+
+
+def test_pack_formats_test13_round_trip_and_all_tuples():
+    # Hetman-2b section 8 Test 13 (Format 1 round trip), and the same for
+    # every 4-tuple in both layouts
+    t13 = np.array([[-1, 0, 1, -1], [1, -1, 0, 1]], np.int8)
+    vals = np.array(np.meshgrid(*[[-1, 0, 1]] * 4, indexing="ij")).reshape(4, -1).T.astype(np.int8)
+    for enc in (1, 2):
+        assert np.array_equal(oracle.unpack_format(oracle.pack_format(t13, enc), 4, enc), t13)
+        packed = oracle.pack_format(vals.reshape(1, -1), enc)
+        assert len(set(packed[0].tolist())) == 81
+        assert np.array_equal(oracle.unpack_format(packed, 324, enc).reshape(-1, 4), vals)
+
+
+def test_unpack_formats_every_byte_against_the_code_table():
+    # the page's stated codes (reserved field reads as 0), not its formulas
+    table = {1: {0b00: 0, 0b01: 1, 0b11: -1, 0b10: 0}, 2: {0b00: 0, 0b01: 1, 0b10: -1, 0b11: 0},
+             0: {0b00: -1, 0b01: 0, 0b10: 1, 0b11: 0}}
+    allb = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    for enc, tab in table.items():
+        got = oracle.unpack_format(allb, 1024, enc).reshape(256, 4)
+        want = np.array([[tab[(b >> (2 * i)) & 3] for i in range(4)] for b in range(256)], np.int8)
+        assert np.array_equal(got, want), enc
+
+
+def test_contraction_in_every_layout_equals_dense():
+    rng = np.random.default_rng(11)
+    q = rng.integers(-1, 2, (7, 192)).astype(np.int8)
+    xq = rng.integers(-127, 128, (5, 192)).astype(np.int8)
+    dense = xq.astype(np.int64) @ q.astype(np.int64).T
+    for enc in (0, 1, 2):
+        acc = oracle.matmul_addsub_format(xq, oracle.pack_format(q, enc), enc)
+        assert np.array_equal(acc, dense), enc
+    # reserved fields contribute nothing: a row of them gives 0
+    res = {1: 0xAA, 2: 0xFF}
+    for enc, b in res.items():
+        packed = np.full((1, 48), b, np.uint8)
+        assert np.all(oracle.matmul_addsub_format(xq, packed, enc) == 0)
+
+
+def test_quantize_pack_layouts_carry_the_same_codes():
+    W = S.normal((9, 256), 0.02, 12, 9)
+    p0, g0 = oracle.quantize_pack(W, per_row=True)
+    q0, _ = oracle.unpack(p0, 256)
+    for enc in (1, 2):
+        p, g = oracle.quantize_pack(W, per_row=True, encoding=enc)
+        assert np.array_equal(g, g0)
+        assert np.array_equal(oracle.unpack_format(p, 256, enc), q0)
+
+
 def test_packed_size_and_compression():
     for ln in golden_lines("sizes.txt"):
         N, K, nbytes, f32bytes = map(int, ln.split())
