@@ -79,6 +79,21 @@ typedef enum tq_status {
 #define TQ_FLAG_WEIGHTS_STATIC (1u << 5)     /* see "Launch overlap" below                      */
 #define TQ_FLAG_INPUTS_READY (1u << 6)       /* see "Launch overlap" below                      */
 
+/* Packed-code layout (flag bits 7-8; tq_quantize_ternary_pack[_noalloc],
+ * tq_ternary_gemm, tq_bitlinear_fused).  Four codes per byte, LSB first.
+ *   TQ_ENC_FOUNDRY  -1 = 0b00, 0 = 0b01, +1 = 0b10 (Foundry, docs/quantization.md,
+ *                   "Ternary Format / Encoding"; the default; 0b11 is never
+ *                   produced and undefined on input).
+ *   TQ_ENC_FORMAT0  0 = 0b00, +1 = 0b01, -1 = 0b11, 0b10 reads as 0 (Hetman-2b,
+ *                   src/quantization.py, section 3, "Format 0").
+ *   TQ_ENC_FORMAT1  0 = 0b00, +1 = 0b01, -1 = 0b10, 0b11 reads as 0 (same, "Format 1").
+ * A contraction must be given the layout its weights were packed in.  The
+ * value 3 << 7 is rejected (TQ_ERR_ARG). */
+#define TQ_ENC_FOUNDRY (0u << 7)
+#define TQ_ENC_FORMAT0 (1u << 7)
+#define TQ_ENC_FORMAT1 (2u << 7)
+#define TQ_ENC_MASK (3u << 7)
+
 /*
  * Launch overlap.  Every kernel is launched with programmatic dependent launch:
  * it may be scheduled while earlier kernels on the stream are still finishing,

@@ -24,6 +24,11 @@ FLAG_ETA_CLAMP = 1 << 3
 FLAG_SANITIZE_NONFINITE = 1 << 4
 FLAG_WEIGHTS_STATIC = 1 << 5
 FLAG_INPUTS_READY = 1 << 6
+# packed-code layouts (flag bits 7-8): Foundry's (default), Hetman-2b "Format 0" and "Format 1"
+ENC_FOUNDRY = 0 << 7
+ENC_FORMAT0 = 1 << 7
+ENC_FORMAT1 = 2 << 7
+ENC_MASK = 3 << 7
 
 STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN", 4: "TQ_ERR_ARG",
           5: "TQ_ERR_CUDA", 6: "TQ_ERR_DEVICE", 7: "TQ_ERR_TIMEOUT"}

@@ -89,6 +89,12 @@ tq_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
                : TQ_ERR_CUDA;
 }
 
+// Packed-code layout from the flags (kEnc*), or -1 for the reserved value.
+inline int flag_encoding(unsigned flags) {
+    const int e = (int)((flags & TQ_ENC_MASK) >> 7);
+    return e == 3 ? -1 : e;
+}
+
 inline tq_status check_k(int64_t K) {
     if (K < 64 || K > kMaxK || (K % 64) != 0) return TQ_ERR_SHAPE;
     return TQ_OK;
@@ -135,7 +141,7 @@ bool make_tmap_u8(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows
 // ---------------------------------------------------------------------------
 // Launch helpers
 // ---------------------------------------------------------------------------
-template <int BT>
+template <int BT, bool CONV>
 tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
                       int64_t K, float *y, int32_t *acc, int mode, int sms, cudaStream_t st) {
@@ -144,7 +150,7 @@ tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemm_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_kernel<BT, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  L::kDynamic) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
@@ -158,12 +164,12 @@ tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
         return TQ_ERR_CUDA;
     const int64_t tiles = ((M + BT - 1) / BT) * ((N + kTileN - 1) / kTileN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
-    return launch_pdl(gemm_kernel<BT>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
+    return launch_pdl(gemm_kernel<BT, CONV>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
                       s_x, rowsum, gamma, per_row, (int)M, (int)N, (int)K, y, acc, mode);
 }
 
 // Grid: one CTA per 16-row strip.  Dynamic shared memory holds x_q only.
-template <int NB, int W, int SPW>
+template <int NB, int W, int SPW, bool CONV>
 tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                       const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
                       int64_t K, float *y, int32_t *acc, int mode, cudaStream_t st) {
@@ -172,27 +178,28 @@ tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemv_kernel<NB, W, SPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemv_kernel<NB, W, SPW, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemv_x_bytes(8 * NB, kGemvMaxK)) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
     }
     const int64_t grid = (N + 15) / 16;
     const size_t smem = (size_t)gemv_x_bytes((int)M, (int)K);
-    return launch_pdl(gemv_kernel<NB, W, SPW>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq, s_x,
+    return launch_pdl(gemv_kernel<NB, W, SPW, CONV>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq, s_x,
                       rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, mode);
 }
 
 // Independent calls: a narrow grid of about 32 CTAs streaming runs of strips
 // (at least one strip per group), so that consecutive calls run side by side.
-tq_status launch_gemv_stream(const int8_t *xq, const float *s_x, const int32_t *rowsum,
-                             const uint8_t *packed, const float *gamma, int per_row, int64_t M,
-                             int64_t N, int64_t K, float *y, int32_t *acc, cudaStream_t st) {
+template <int ENC>
+tq_status launch_gemv_stream_t(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                               const uint8_t *packed, const float *gamma, int per_row, int64_t M,
+                               int64_t N, int64_t K, float *y, int32_t *acc, cudaStream_t st) {
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemv_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemv_stream_kernel<ENC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemv_x_bytes(8, kStreamMaxK)) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
@@ -202,23 +209,33 @@ tq_status launch_gemv_stream(const int8_t *xq, const float *s_x, const int32_t *
     if (per_cta < kStreamGroups) per_cta = kStreamGroups;
     const int64_t grid = (nstrips + per_cta - 1) / per_cta;
     const size_t smem = (size_t)gemv_x_bytes((int)M, (int)K);
-    return launch_pdl(gemv_stream_kernel, dim3((unsigned)grid), dim3(kStreamThreads), smem, st, xq, s_x,
-                      rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, (int)per_cta);
+    return launch_pdl(gemv_stream_kernel<ENC>, dim3((unsigned)grid), dim3(kStreamThreads), smem, st, xq,
+                      s_x, rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, (int)per_cta);
+}
+
+tq_status launch_gemv_stream(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                             const uint8_t *packed, const float *gamma, int per_row, int64_t M,
+                             int64_t N, int64_t K, float *y, int32_t *acc, int enc, cudaStream_t st) {
+    if (enc == kEncFormat0)
+        return launch_gemv_stream_t<kEncFormat0>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
+    if (enc == kEncFormat1)
+        return launch_gemv_stream_t<kEncFormat1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
+    return launch_gemv_stream_t<kEncFoundry>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
 }
 
 // Independent calls (inputs ready) overlap one another: lean CTAs (four
 // steps per warp) keep several layers resident.  Otherwise, for K <= 4096,
 // the time after the wait is the critical path: twice the warps, two steps
 // each.  Larger K keeps the lean shape (16-warp CTAs measured slower).
-template <int NB>
+template <int NB, bool CONV>
 tq_status gemv_shape(const int8_t *xq, const float *s_x, const int32_t *rowsum, const uint8_t *packed,
                      const float *gamma, int per_row, int64_t M, int64_t N, int64_t K, float *y,
                      int32_t *acc, int mode, cudaStream_t st) {
     const bool lean = (mode & kModeInputsReady) != 0;
     if (K <= kGemvMaxK / 2)
-        return lean ? launch_gemv<NB, 4, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st)
-                    : launch_gemv<NB, 8, 2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
-    return launch_gemv<NB, 8, 4>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+        return lean ? launch_gemv<NB, 4, 4, CONV>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st)
+                    : launch_gemv<NB, 8, 2, CONV>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+    return launch_gemv<NB, 8, 4, CONV>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
 }
 
 template <int NW>
@@ -306,7 +323,7 @@ struct PerTensor {
 template <typename Kern>
 tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_cta, int smem,
                            const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
-                           const PerTensor &pt, int reverse, int ready, cudaStream_t st) {
+                           const PerTensor &pt, int reverse, int opts, cudaStream_t st) {
     int dev = 0, sms = 0;
     if (tq_status e = check_device(&sms)) return e;
     cudaGetDevice(&dev);
@@ -327,30 +344,36 @@ tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_ct
     const int64_t cap = (int64_t)per_sm * sms;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
     return launch_pdl(kern, dim3(grid), dim3(kPackThreads), (size_t)smem, st, w, N, (int)K,
-                      1.0 / (double)K, packed, gamma, pt.partial, pt.nparts, pt.height, reverse, ready);
+                      1.0 / (double)K, packed, gamma, pt.partial, pt.nparts, pt.height, reverse, opts);
 }
 
-template <bool SAN>
+template <bool SAN, bool CONV>
 tq_status launch_pack_rows_s(const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
-                             const PerTensor &pt, int reverse, int ready, cudaStream_t st) {
+                             const PerTensor &pt, int reverse, int opts, cudaStream_t st) {
     static std::atomic<int> occ[5][kMaxDevices];
     const int64_t nv = K / 4;
     const int k = (int)K;
     if (nv <= 32 * kTeamVec * 1)
-        return launch_pack_grid(pack_team_kernel<1, SAN>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, pt, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<1, SAN, CONV>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, pt, reverse, opts, st);
     if (nv <= 32 * kTeamVec * 2)
-        return launch_pack_grid(pack_team_kernel<2, SAN>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, pt, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<2, SAN, CONV>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, pt, reverse, opts, st);
     if (nv <= 32 * kTeamVec * 4)
-        return launch_pack_grid(pack_team_kernel<4, SAN>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, pt, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<4, SAN, CONV>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, pt, reverse, opts, st);
     if (nv <= 32 * kTeamVec * 8)
-        return launch_pack_grid(pack_team_kernel<8, SAN>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, pt, reverse, ready, st);
-    return launch_pack_grid(pack_rows_kernel<SAN>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, ready, st);
+        return launch_pack_grid(pack_team_kernel<8, SAN, CONV>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, pt, reverse, opts, st);
+    return launch_pack_grid(pack_rows_kernel<SAN, CONV>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, opts, st);
 }
 
+// Options word of the pack kernels: bit 0 inputs ready, bits 1-2 layout.
+inline int pack_opts(int ready, int enc) { return (ready ? 1 : 0) | (enc << 1); }
+
 tq_status launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
-                           float *gamma, const PerTensor &pt, int reverse, int ready, cudaStream_t st) {
-    return sanitize ? launch_pack_rows_s<true>(w, N, K, packed, gamma, pt, reverse, ready, st)
-                    : launch_pack_rows_s<false>(w, N, K, packed, gamma, pt, reverse, ready, st);
+                           float *gamma, const PerTensor &pt, int reverse, int opts, cudaStream_t st) {
+    if (opts >> 1)  // a layout other than Foundry's
+        return sanitize ? launch_pack_rows_s<true, true>(w, N, K, packed, gamma, pt, reverse, opts, st)
+                        : launch_pack_rows_s<false, true>(w, N, K, packed, gamma, pt, reverse, opts, st);
+    return sanitize ? launch_pack_rows_s<true, false>(w, N, K, packed, gamma, pt, reverse, opts, st)
+                    : launch_pack_rows_s<false, false>(w, N, K, packed, gamma, pt, reverse, opts, st);
 }
 
 size_t pack_parts(int64_t nv) {
@@ -383,19 +406,33 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
                         const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
                         int64_t N, int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
     const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
+    const int enc = flag_encoding(flags);
     const int mode = ((flags & TQ_FLAG_WEIGHTS_STATIC) ? kModeWeightsStatic : 0) |
-                     ((flags & TQ_FLAG_INPUTS_READY) ? kModeInputsReady : 0);
+                     ((flags & TQ_FLAG_INPUTS_READY) ? kModeInputsReady : 0) | (enc << kModeEncShift);
     if (M <= 16 && K <= kGemvMaxK) {
         if ((mode & kModeInputsReady) && M <= 8 && K <= kStreamMaxK)
-            return launch_gemv_stream(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, st);
-        if (M <= 8) return gemv_shape<1>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
-        return gemv_shape<2>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+            return launch_gemv_stream(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, enc, st);
+        if (enc != kEncFoundry) {
+            if (M <= 8) return gemv_shape<1, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+            return gemv_shape<2, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+        }
+        if (M <= 8) return gemv_shape<1, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+        return gemv_shape<2, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
     }
-    switch (gemm_tile_tokens(M, N, sms)) {
-    case 64: return launch_gemm<64>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    case 128: return launch_gemm<128>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    case 192: return launch_gemm<192>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    default: return launch_gemm<256>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    const int bt = gemm_tile_tokens(M, N, sms);
+    if (enc != kEncFoundry) {
+        switch (bt) {
+        case 64: return launch_gemm<64, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+        case 128: return launch_gemm<128, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+        case 192: return launch_gemm<192, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+        default: return launch_gemm<256, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+        }
+    }
+    switch (bt) {
+    case 64: return launch_gemm<64, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    case 128: return launch_gemm<128, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    case 192: return launch_gemm<192, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
+    default: return launch_gemm<256, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
     }
 }
 
@@ -431,7 +468,10 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     if (!w || !packed || !gamma) return TQ_ERR_NULL;
     if (N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
-    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_INPUTS_READY)) return TQ_ERR_ARG;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_INPUTS_READY | TQ_ENC_MASK))
+        return TQ_ERR_ARG;
+    const int enc = flag_encoding(flags);
+    if (enc < 0) return TQ_ERR_ARG;
     if (!aligned16(w) || !aligned16(packed) || !aligned16(gamma)) return TQ_ERR_ALIGN;
     const bool per_row = flags & TQ_GAMMA_PER_ROW;
     const int ready = (flags & TQ_FLAG_INPUTS_READY) ? 1 : 0;
@@ -453,7 +493,9 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, ready, st)) return e;
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0,
+                                           pack_opts(ready, enc), st))
+            return e;
         return launch_status();
     }
     const int64_t total_v = N * K / 4;
@@ -467,7 +509,8 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     pt.partial = partial;
     pt.nparts = (int)nparts;
     pt.height = absum_tree_height(chunk, (int)nparts);
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, 0, st)) return e;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, pack_opts(0, enc), st))
+        return e;
     return launch_status();
 }
 
@@ -515,7 +558,9 @@ tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *row
     if (!xq || !s_x || !rowsum || !packed || !gamma || !y) return TQ_ERR_NULL;
     if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
-    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY)) return TQ_ERR_ARG;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY | TQ_ENC_MASK))
+        return TQ_ERR_ARG;
+    if (flag_encoding(flags) < 0) return TQ_ERR_ARG;
     if (!aligned16(xq) || !aligned16(s_x) || !aligned16(rowsum) || !aligned16(packed) ||
         !aligned16(gamma) || !aligned16(y) || (acc && !aligned16(acc)))
         return TQ_ERR_ALIGN;
@@ -548,8 +593,10 @@ tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_ep
     if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
     const unsigned known = TQ_GAMMA_PER_ROW | TQ_FLAG_FWHT | TQ_FLAG_RMSNORM | TQ_FLAG_ETA_CLAMP |
-                           TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY;
+                           TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY |
+                           TQ_ENC_MASK;
     if (flags & ~known) return TQ_ERR_ARG;
+    if (flag_encoding(flags) < 0) return TQ_ERR_ARG;
     if ((flags & TQ_FLAG_FWHT) && (K % 512 != 0 || K > kMaxFwhtFusedK)) return TQ_ERR_SHAPE;
     if ((flags & TQ_FLAG_ETA_CLAMP) && !(eta_min > 0.0f && eta_min <= eta_max)) return TQ_ERR_ARG;
     if ((flags & TQ_FLAG_SANITIZE_NONFINITE) && !(eta_max > 0.0f && eta_max < 3.0e38f)) return TQ_ERR_ARG;
@@ -600,7 +647,7 @@ tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_ep
     else
         launch_act(x, p, M, K, xq, sx, rs, st);
     if (tq_status e = launch_status()) return e;
-    const unsigned cflags = (flags & (TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC)) |
+    const unsigned cflags = (flags & (TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC | TQ_ENC_MASK)) |
                             ((flags & TQ_FLAG_INPUTS_READY) ? TQ_FLAG_WEIGHTS_STATIC : 0u);
     return gemm_dispatch(xq, sx, rs, packed, gamma, cflags, M, N, K, y, nullptr, sms, st);
 }

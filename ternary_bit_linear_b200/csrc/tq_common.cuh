@@ -45,6 +45,7 @@ __device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, kStatusTime
 // before reading, only before exiting.
 constexpr int kModeWeightsStatic = 1;
 constexpr int kModeInputsReady = 2;
+constexpr int kModeEncShift = 2;  // bits 2-3: packed-code layout (kEnc*, below)
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
@@ -382,6 +383,36 @@ __device__ __forceinline__ float code_threshold(float gamma) {
 // 2-bit code (-1 -> 0b00, 0 -> 0b01, +1 -> 0b10) of one weight.
 __device__ __forceinline__ uint32_t ternary_field(float w, float t) {
     return 1u + (w >= t ? 1u : 0u) - (w <= -t ? 1u : 0u);
+}
+
+// Packed-code layouts.  Foundry (docs/quantization.md, "Ternary Format /
+// Encoding"): -1 = 0b00, 0 = 0b01, +1 = 0b10, the field being q + 1 -- the
+// form the kernels compute with.  Hetman-2b (src/quantization.py, section 3,
+// PackedTernaryStorage) "Format 0": 0 = 0b00, +1 = 0b01, -1 = 0b11 (0b10 reads
+// as 0); "Format 1": 0 = 0b00, +1 = 0b01, -1 = 0b10 (0b11 reads as 0).
+constexpr int kEncFoundry = 0, kEncFormat0 = 1, kEncFormat1 = 2;
+
+// The 16 fields of a word in layout `enc`, rewritten in Foundry's layout.
+// With p, n the low and high bit of a field, Foundry's field is
+// (p & ~n) << 1 | (Format 0: ~p, Format 1: ~(p ^ n)) -- the page's decodes
+// p - 2(p & n) and p - n, plus one.  A warp-uniform branch for the default.
+__device__ __forceinline__ uint32_t codes_to_foundry(uint32_t w, int enc) {
+    if (enc == kEncFoundry) return w;
+    const uint32_t M = 0x55555555u;
+    const uint32_t p = w & M, n = (w >> 1) & M;
+    const uint32_t lo = enc == kEncFormat0 ? (~p & M) : (~(p ^ n) & M);
+    return ((p & ~n) << 1) | lo;
+}
+
+// Inverse for the packer (its Foundry-layout fields are never 0b11): with
+// f0, f1 the low and high bit, a -1 (both clear) gets the high bit, and the
+// low bit is ~f0 (Format 0) or f1 (Format 1).
+__device__ __forceinline__ uint32_t codes_from_foundry(uint32_t f, int enc) {
+    if (enc == kEncFoundry) return f;
+    const uint32_t M = 0x55555555u;
+    const uint32_t f0 = f & M, f1 = (f >> 1) & M;
+    const uint32_t lo = enc == kEncFormat0 ? (~f0 & M) : f1;
+    return lo | ((~f0 & ~f1 & M) << 1);
 }
 
 }  // namespace tq

@@ -98,7 +98,10 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
                       __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632));
 }
 
-template <int BT>
+// CONV: the weights are packed in one of Hetman-2b's layouts (mode bits
+// 2-3) and every word is rewritten in Foundry's layout before the unpack; the
+// default layout compiles without that step.
+template <int BT, bool CONV>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
@@ -241,6 +244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // Two groups of four warps take alternate steps, so each has two steps'
         // time for its waits, loads and stores; thread r of a group owns row r.
         const int par = (warp - 4) >> 2;
+        const int enc = (mode >> kModeEncShift) & 3;  // packed-code layout
         const int r = 32 * (warp & 3) + lane;  // weight row of the tile
         const uint32_t w_row = sbase + (uint32_t)(L::offW + r * (kTileK / 4));
         const uint32_t a_row = (uint32_t)(r * kTileK), sw = (uint32_t)(r & 7);
@@ -257,7 +261,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                          : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w)
                          : "r"(src + 16u)
                          : "memory");
-            const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            if (CONV) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) words[c] = codes_to_foundry(words[c], enc);
+            }
             uint4 e[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) e[c] = expand_word(words[c]);

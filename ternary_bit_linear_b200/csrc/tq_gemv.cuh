@@ -124,9 +124,9 @@ __device__ __forceinline__ void load_strip(StripRegs<SPW> &r, const uint8_t *__r
 // Partial sums of one warp over its column steps: d[chain][nb][fragment].
 // XT: the x_q chunks in shared memory are already transposed (else each
 // chunk is transposed here, after it is read).
-template <int NB, int W, int SPW, int CH, bool XT>
+template <int NB, int W, int SPW, int CH, bool XT, bool CONV>
 __device__ __forceinline__ void strip_mma(const StripRegs<SPW> &r, int (&d)[CH][NB][4], int w, int lane,
-                                          uint32_t x_s, int XS, int M, int KB) {
+                                          uint32_t x_s, int XS, int M, int KB, int enc) {
     const int g = lane >> 2, t = lane & 3;
     const int nsteps = (KB + 63) >> 6;
     const uint32_t xsw = (uint32_t)(t & 2) << 4;  // chunk swizzle of this thread's columns
@@ -143,7 +143,9 @@ __device__ __forceinline__ void strip_mma(const StripRegs<SPW> &r, int (&d)[CH][
             const uint32_t b4[4] = {r.b[j].x, r.b[j].y, r.b[j].z, r.b[j].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t ar = a4[i], br = b4[i];
+                // codes in Foundry's layout (field = q + 1); other layouts (CONV) converted here
+                const uint32_t ar = CONV ? codes_to_foundry(a4[i], enc) : a4[i];
+                const uint32_t br = CONV ? codes_to_foundry(b4[i], enc) : b4[i];
                 uint32_t ua[4], ub[4];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
@@ -195,7 +197,8 @@ __device__ __forceinline__ void transpose_x(uint32_t x_s, int M, int K, int XS, 
 }
 
 // NB: token blocks of 8 (M <= 8 * NB).  W: warps per CTA.  SPW: 64-byte
-// column steps per warp (K <= 256 * W * SPW).
+// column steps per warp (K <= 256 * W * SPW).  CONV: weights in one of
+// Hetman-2b's layouts (mode bits 2-3), rewritten in Foundry's as they are used.
 //
 // mode & kModeWeightsStatic: the packed weights and gamma are not written by
 // work still in flight on the stream, so they are requested before the
@@ -205,7 +208,7 @@ __device__ __forceinline__ void transpose_x(uint32_t x_s, int M, int K, int XS, 
 // One CTA (the last) waits for the previous kernel before it exits, so this
 // kernel still completes after its predecessor and later work sees the
 // stream's results in order; the other CTAs leave as soon as they are done.
-template <int NB, int W, int SPW>
+template <int NB, int W, int SPW, bool CONV>
 __global__ void __launch_bounds__(W * 32, gemv_min_blocks(NB, W))
     gemv_kernel(const int8_t *__restrict__ xq, const float *__restrict__ s_x,
                 const int32_t *__restrict__ rowsum, const uint8_t *__restrict__ packed,
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(W * 32, gemv_min_blocks(NB, W))
                       // transposed where it is read, off the wait's critical path)
 
     int d[CH][NB][4];
-    strip_mma<NB, W, SPW, CH, false>(wr, d, warp, lane, x_s, XS, M, KB);
+    strip_mma<NB, W, SPW, CH, false, CONV>(wr, d, warp, lane, x_s, XS, M, KB, (mode >> kModeEncShift) & 3);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -314,6 +317,9 @@ __device__ __forceinline__ void group_sync(int group) {
     asm volatile("bar.sync %0, 128;" ::"r"(1 + group) : "memory");
 }
 
+// ENC: packed-code layout (kEnc*), a template argument here: registers are at
+// the two-CTAs-per-SM limit.
+template <int ENC>
 __global__ void __launch_bounds__(kStreamThreads, 2)
     gemv_stream_kernel(const int8_t *__restrict__ xq, const float *__restrict__ s_x,
                        const int32_t *__restrict__ rowsum, const uint8_t *__restrict__ packed,
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
     int par = 0;
     auto one = [&](const StripRegs<SPW> &w, int kk, float gn) {
         int d[CH][1][4];
-        strip_mma<1, GW, SPW, CH, true>(w, d, gw, lane, x_s, XS, M, KB);
+        strip_mma<1, GW, SPW, CH, true, ENC != kEncFoundry>(w, d, gw, lane, x_s, XS, M, KB, ENC);
 #pragma unroll
         for (int c = 0; c < 4; ++c) red[group][par][gw][c][lane] = d[0][0][c] + d[1][0][c];
         group_sync(group);

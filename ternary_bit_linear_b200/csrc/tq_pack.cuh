@@ -53,6 +53,12 @@ __device__ __forceinline__ void acc_abs4(DD &a, float4 v) {
 
 // Byte of four 2-bit codes: start from 0b01010101 (all zero codes) and move
 // each field up (+1 -> 0b10) or down (-1 -> 0b00).  NaN compares false: code 0.
+// The packed byte in the requested layout (CONV: one of Hetman-2b's).
+template <bool CONV>
+__device__ __forceinline__ uint32_t out_codes(uint32_t foundry_byte, int enc) {
+    return CONV ? codes_from_foundry(foundry_byte, enc) : foundry_byte;
+}
+
 __device__ __forceinline__ uint32_t pack4(float4 v, float t) {
     uint32_t b = 0x55u;
     b += (v.x >= t) ? 1u : 0u;
@@ -176,12 +182,13 @@ __device__ __noinline__ float per_tensor_threshold(const double *__restrict__ pa
 // ---------------------------------------------------------------------------
 constexpr int kPackUnroll = 8;
 
-template <bool SAN>
+template <bool SAN, bool CONV>
 __global__ void __launch_bounds__(kPackThreads)
     pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
-                     int ready) {
+                     int opts) {
+    const int ready = opts & 1, enc = opts >> 1;  // inputs ready; packed-code layout
     if (!ready) pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -234,11 +241,12 @@ __global__ void __launch_bounds__(kPackThreads)
 #pragma unroll
             for (int u = 0; u < kPackUnroll; ++u) x[u] = __ldcs(src + c + 32 * u);
 #pragma unroll
-            for (int u = 0; u < kPackUnroll; ++u) dst[c + 32 * u] = (uint8_t)pack4(SAN ? sanitize_w(x[u]) : x[u], t);
+            for (int u = 0; u < kPackUnroll; ++u)
+                dst[c + 32 * u] = (uint8_t)out_codes<CONV>(pack4(SAN ? sanitize_w(x[u]) : x[u], t), enc);
         }
         for (; c < nv; c += 32) {
             const float4 x = __ldcs(src + c);
-            dst[c] = (uint8_t)pack4(SAN ? sanitize_w(x) : x, t);
+            dst[c] = (uint8_t)out_codes<CONV>(pack4(SAN ? sanitize_w(x) : x, t), enc);
         }
     }
     if (ready) pdl_wait();  // complete no earlier than the previous kernel
@@ -278,12 +286,13 @@ __host__ __device__ constexpr int pack_team_smem(int T, int K) {
     return (kPackWarps / T) * kPackRing * (K / 4) * 16;
 }
 
-template <int T, bool SAN>
+template <int T, bool SAN, bool CONV>
 __global__ void __launch_bounds__(kPackThreads, 2)
     pack_team_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
-                     int ready) {
+                     int opts) {
+    const int ready = opts & 1, enc = opts >> 1;  // inputs ready; packed-code layout
     constexpr int TEAMS = kPackWarps / T;
     extern __shared__ __align__(16) float4 rowbuf[];  // [TEAMS][kPackRing][nv]
     __shared__ uint64_t rbar[TEAMS][kPackRing];
@@ -375,7 +384,7 @@ __global__ void __launch_bounds__(kPackThreads, 2)
 #pragma unroll
         for (int j = 0; j < kTeamVec; ++j) {
             const int idx = j * 32 * T + tw * 32 + lane;
-            if (idx < nv) dst[idx] = (uint8_t)pack4(v[j], t);
+            if (idx < nv) dst[idx] = (uint8_t)out_codes<CONV>(pack4(v[j], t), enc);
         }
     }
     // Copies in flight must land before the CTA exits (already true unless a

@@ -43,6 +43,10 @@ def test_header_flag_values_match_binding():
         assert name in flags, name
         assert value == 1 << flags[name], name
     assert len(set(py.values())) == len(py)
+    enc = dict((k, int(v) << int(sh)) for k, v, sh in re.findall(r"#define\s+TQ_(ENC_\w+)\s+\((\d+)u\s*<<\s*(\d+)\)", src))
+    assert enc == {"ENC_FOUNDRY": tq.ENC_FOUNDRY, "ENC_FORMAT0": tq.ENC_FORMAT0, "ENC_FORMAT1": tq.ENC_FORMAT1,
+                   "ENC_MASK": tq.ENC_MASK}
+    assert all(not (tq.ENC_MASK & v) for v in py.values())
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -77,7 +81,8 @@ def test_pack_validation(lib):
     assert f(P(), 4, 60, 1, P(1 << 20), P(2 << 20), None, 0, None) == 2      # K % 64
     assert f(P(), 0, 64, 1, P(1 << 20), P(2 << 20), None, 0, None) == 2      # N = 0
     assert f(P(4), 4, 64, 1, P(1 << 20), P(2 << 20), None, 0, None) == 3     # misaligned
-    assert f(P(), 4, 64, 1 << 7, P(1 << 20), P(2 << 20), None, 0, None) == 4  # unknown flag
+    assert f(P(), 4, 64, 1 << 9, P(1 << 20), P(2 << 20), None, 0, None) == 4  # unknown flag
+    assert f(P(), 4, 64, 1 | 3 << 7, P(1 << 20), P(2 << 20), None, 0, None) == 4  # reserved layout
     assert f(P(), 4, 64, 1, P(16), P(2 << 20), None, 0, None) == 4           # overlap w/packed
     assert f(P(), 4, 64, 0, P(1 << 20), P(2 << 20), None, 0, None) == 1      # needs workspace
     assert f(P(), 4, 64, 0, P(1 << 20), P(2 << 20), P(3 << 20), 8, None) == 4  # too small
@@ -100,6 +105,8 @@ def test_gemm_and_fused_validation(lib):
     bad = list(args)
     bad[5] = 4
     assert f(*bad) == 4
+    bad[5] = 3 << 7  # reserved layout
+    assert f(*bad) == 4
     bad = list(args)
     bad[8] = 32
     assert f(*bad) == 2
@@ -116,3 +123,6 @@ def test_gemm_and_fused_validation(lib):
     fused[10] = 512
     fused[15] = 16
     assert h(*fused) == 4  # workspace too small
+    fused[15] = 1 << 20
+    fused[5] = tq.FLAG_FWHT | 3 << 7
+    assert h(*fused) == 4  # reserved layout

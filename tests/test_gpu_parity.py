@@ -652,3 +652,80 @@ def test_pack_per_tensor_midpoint_many_ctas(cuda_lib, odd, expect, sanitize):
     if not sanitize:
         assert g_ref[0] == np.float32(expect)
     assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
+
+
+# ---------------------------------------------------------------------------
+# Packed-code layouts: Hetman-2b section 3 "Format 0" / "Format 1" beside
+# Foundry's (the default).  Bytes bit-exact against the oracle's packer;
+# contractions (both GEMV shapes and the tcgen05 GEMM) bit-exact against the
+# oracle's add/subtract walk in the same layout, with reserved fields mixed in
+# (they read as 0).
+# ---------------------------------------------------------------------------
+LAYOUTS = [1, 2]  # oracle numbering; flag = layout << 7
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("N,K,per_row", [(33, 512, True), (129, 4160, False), (5, 8256, True), (64, 2048, False)])
+def test_pack_layouts_match_oracle(cuda_lib, layout, N, K, per_row):
+    tq = cuda_lib
+    W = S.normal((N, K), 0.02, 90, N)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=per_row, encoding=layout)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty((N if per_row else 1,), dtype=torch.float32, device="cuda")
+    flags = (tq.GAMMA_PER_ROW if per_row else 0) | (layout << 7)
+    ws = torch.empty((max(16, tq.pack_workspace_bytes(N, K, flags)),), dtype=torch.uint8, device="cuda")
+    tq.quantize_ternary_pack_(dev(W), flags, packed, gamma, ws)
+    assert np.array_equal(host(packed), p_ref)
+    assert np.array_equal(host(gamma), g_ref)
+
+
+def _with_reserved(packed, layout, seed):
+    """Replace about 5 % of the fields with the layout's reserved code."""
+    rng = np.random.default_rng(seed)
+    res = 0b10 if layout == 1 else 0b11
+    out = packed.copy()
+    mask = rng.random(out.shape + (4,)) < 0.05
+    for i in range(4):
+        m = mask[..., i]
+        out[m] = (out[m] & ~np.uint8(3 << (2 * i))) | np.uint8(res << (2 * i))
+    return out
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("M,N,K,ready", [(1, 300, 4096, False), (5, 129, 1088, True), (8, 1000, 4096, True),
+                                         (12, 64, 8192, False), (64, 256, 1024, False), (300, 384, 1536, False)])
+def test_contraction_layouts_match_oracle(cuda_lib, layout, M, N, K, ready):
+    tq = cuda_lib
+    W = S.normal((N, K), 0.02, 91, N)
+    X = S.decode_acts(M, K, seed=92)
+    p_lay, g_ref = oracle.quantize_pack(W, per_row=True, encoding=layout)
+    p_lay = _with_reserved(p_lay, layout, 93)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    acc_ref = oracle.matmul_addsub_format(xq_ref, p_lay, layout)
+    ins = [dev(a) for a in (xq_ref, sx_ref, rs_ref, p_lay, g_ref)]
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    fl = tq.GAMMA_PER_ROW | (layout << 7) | (tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY if ready else 0)
+    tq.ternary_gemm_(*ins, fl, y, acc)
+    assert np.array_equal(host(acc), acc_ref)
+    assert_y_close(host(y), oracle.dequant(acc_ref, g_ref, sx_ref, True))
+    assert tq.device_status() == 0
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_fused_layouts_equal_default_layout(cuda_lib, layout):
+    tq = cuda_lib
+    M, N, K = 512, 640, 2048
+    W = S.normal((N, K), 0.02, 94, N)
+    fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM
+    x = dev(S.student_t3((M, K), 95, M))
+    outs = []
+    for lay in (0, layout):
+        p_ref, g_ref = oracle.quantize_pack(W, per_row=False, encoding=lay)
+        packed, gamma = dev(p_ref), dev(g_ref)
+        y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        ws = torch.empty((tq.fused_workspace_bytes(M, K, fl),), dtype=torch.uint8, device="cuda")
+        tq.bitlinear_fused_(x, packed, gamma, fl | (lay << 7), y, ws)
+        outs.append(host(y))
+    assert np.array_equal(outs[0], outs[1])
+    assert tq.device_status() == 0
