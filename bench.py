@@ -158,7 +158,7 @@ class ClockSampler:
 class Workload:
     """Builds device buffers and the per-segment launch lists of one step."""
 
-    def __init__(self, name, tq, S, torch, dev, layers):
+    def __init__(self, name, tq, S, torch, dev, layers, layout=0):
         self.name, self.tq, self.torch, self.dev = name, tq, torch, dev
         f32, u8, i8, i32 = torch.float32, torch.uint8, torch.int8, torch.int32
         self.segments = []  # (label, kernel_name, launches, algorithmic bytes or ops, [fns])
@@ -196,7 +196,9 @@ class Workload:
         else:
             raise SystemExit(f"unknown workload {name}")
         N, K, L = self.N, self.K, self.L
-        self.flags = tq.GAMMA_PER_ROW if self.per_row else 0
+        # packed-code layout (0 Foundry, 1 Hetman-2b Format 0, 2 Format 1) on every pack and contraction
+        self.layout = layout
+        self.flags = (tq.GAMMA_PER_ROW if self.per_row else 0) | (layout << 7)
         # the ring's layers share x and have their own weights and outputs:
         # independent calls, so the contractions may overlap one another
         self.ready_flags = self.flags | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY
@@ -214,7 +216,7 @@ class Workload:
         if name == "fused":
             fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM
             # the ring's layers have their own x, y and workspace: independent calls
-            self.fused_flags = fl | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY
+            self.fused_flags = fl | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY | (layout << 7)
             self.fused_ws = [torch.empty((tq.fused_workspace_bytes(self.Ms[0], K, fl),), dtype=u8, device=dev)
                              for _ in range(L)]
 
@@ -274,7 +276,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     tq.load()
-    wl = Workload(args.workload, tq, S, torch, dev, args.layers or WORKLOAD_SHAPES[args.workload][3])
+    wl = Workload(args.workload, tq, S, torch, dev, args.layers or WORKLOAD_SHAPES[args.workload][3],
+                  LAYOUTS.index(args.layout))
     stream = torch.cuda.Stream(device=dev)
     graphs = []
     with torch.cuda.stream(stream):
@@ -384,7 +387,10 @@ WORKLOAD_SHAPES = {  # name -> (Ms, N, K, default ring of layers, per_row)
 }
 
 
-def config_for(name, layers, world):
+LAYOUTS = ["foundry", "format0", "format1"]  # packed-code layouts, flag value = index << 7
+
+
+def config_for(name, layers, world, layout="foundry"):
     Ms, N, K, L, per_row = WORKLOAD_SHAPES[name]
     L = layers or L
     desc = {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers" % L,
@@ -392,14 +398,14 @@ def config_for(name, layers, world):
             "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512, ring of %d layers" % L,
             "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L}[name]
     return {"workload": desc, "M": Ms, "N": N, "K": K, "layers": L,
-            "gamma": "per-row" if per_row else "per-tensor",
+            "gamma": "per-row" if per_row else "per-tensor", "layout": layout,
             "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
                 L * N * K * 4 >> 20, L * N * K // 4 >> 20),
             "parallelism": "replicas x%d" % world if world > 1 else "single GPU"}
 
 
 def wl_config(wl, world):
-    return config_for(wl.name, wl.L, world)
+    return config_for(wl.name, wl.L, world, LAYOUTS[wl.layout])
 
 
 def run_chains(args, wl, tq, torch, stream, world):
@@ -556,7 +562,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic", "config": dict(config_for(args.workload, args.layers, world), sample=what),
+        "data": "synthetic", "config": dict(config_for(args.workload, args.layers, world, args.layout), sample=what),
         "cpu_baseline": {"value": round(v, 6), "unit": unit, "cores": 1, "kind": "oracle",
                          "sample": what + " per step"},
         "e2e": {"value": round(v, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -588,6 +594,8 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fused", "sweep"])
+    ap.add_argument("--layout", default="foundry", choices=LAYOUTS,
+                    help="packed-code layout: Foundry's (default) or Hetman-2b's Format 0 / Format 1")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0, help="ring of distinct layers (0: workload default)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
