@@ -57,6 +57,8 @@ def _load():
         _lib.tqo_unpack.restype = I64
         _lib.tqo_quantize_pack.argtypes = [P, I64, I64, I, I, P, P]
         _lib.tqo_quantize_pack_format.argtypes = [P, I64, I64, I, I, I, P, P]
+        _lib.tqo_quantize_pack_threshold.argtypes = [P, I64, I64, I, I, I, F, P, P]
+        _lib.tqo_ternary_codes_threshold.argtypes = [P, I64, I64, P, I, F, P]
         _lib.tqo_pack_format.argtypes = [P, I64, I64, I, P]
         _lib.tqo_unpack_format.argtypes = [P, I64, I64, I, P]
         _lib.tqo_matmul_addsub_format.argtypes = [P, P, I64, I64, I64, I, P]
@@ -132,6 +134,29 @@ def quantize_pack(w, per_row: bool, sanitize: bool = False, encoding: int = 0):
     _load().tqo_quantize_pack_format(pw, N, K, int(per_row), int(sanitize), int(encoding),
                                      packed.ctypes.data_as(ctypes.c_void_p),
                                      gamma.ctypes.data_as(ctypes.c_void_p))
+    return packed, gamma
+
+
+def ternary_codes_threshold(w, gamma, per_row: bool, ratio: float):
+    w, pw = _c(w, np.float32)
+    N, K = w.shape
+    g, pg = _c(np.atleast_1d(gamma), np.float32)
+    q = np.empty((N, K), np.int8)
+    _load().tqo_ternary_codes_threshold(pw, N, K, pg, int(per_row), float(ratio),
+                                        q.ctypes.data_as(ctypes.c_void_p))
+    return q
+
+
+def quantize_pack_threshold(w, per_row: bool, ratio: float, sanitize: bool = False, encoding: int = 0):
+    """Threshold rule (code = sign(w) where |w| > fp32(ratio * gamma)); returns
+    (packed, gamma) like quantize_pack."""
+    w, pw = _c(w, np.float32)
+    N, K = w.shape
+    packed = np.empty((N, K // 4), np.uint8)
+    gamma = np.empty((N if per_row else 1,), np.float32)
+    _load().tqo_quantize_pack_threshold(pw, N, K, int(per_row), int(sanitize), int(encoding), float(ratio),
+                                        packed.ctypes.data_as(ctypes.c_void_p),
+                                        gamma.ctypes.data_as(ctypes.c_void_p))
     return packed, gamma
 
 

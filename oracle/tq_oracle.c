@@ -186,6 +186,24 @@ void tqo_ternary_codes(const float *w, int64_t N, int64_t K, const float *gamma,
     }
 }
 
+/* Threshold ternarisation: tau = fp32(ratio * gamma), code = +1 if w > tau,
+ * -1 if w < -tau, else 0 (strict comparisons).  ratio = 1 is [F] "Absmean
+ * Thresholding (BitNet b1.58)" (threshold = mean |w|); ratio = 0.55 with
+ * per-row gamma is [B] ternarize_weight (w > threshold * scale, scale = the
+ * row's mean |w|).  gamma as for tqo_ternary_codes. */
+void tqo_ternary_codes_threshold(const float *w, int64_t N, int64_t K, const float *gamma,
+                                 int per_row, float ratio, int8_t *q)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        float g = per_row ? gamma[n] : gamma[0];
+        float tau = ratio * g;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = w[n * K + k];
+            q[n * K + k] = (int8_t)(v > tau ? 1 : (v < -tau ? -1 : 0));
+        }
+    }
+}
+
 /* byte[n][j] = (v3 << 6) | (v2 << 4) | (v1 << 2) | v0 with v = code + 1,
  * i.e. -1 -> 0b00, 0 -> 0b01, +1 -> 0b10, value 4j+i in bits 2i..2i+1.
  * [F] "Ternary Format / Encoding".  Rows are K-contiguous, K % 4 == 0. */
@@ -272,8 +290,9 @@ void tqo_unpack_format(const uint8_t *packed, int64_t N, int64_t K, int format, 
 /* gamma (per tensor, or per row) then codes then packing: the export path of
  * [H] section 5 BitLinear.export_packed_weights, with the per-row gamma of
  * [F] fq_quantize_ternary_per_channel as the alternative granularity. */
-void tqo_quantize_pack_format(const float *w_in, int64_t N, int64_t K, int per_row,
-                              int sanitize, int format, uint8_t *packed, float *gamma)
+void tqo_quantize_pack_threshold(const float *w_in, int64_t N, int64_t K, int per_row,
+                                 int sanitize, int format, float ratio, uint8_t *packed,
+                                 float *gamma)
 {
     const float *w = w_in;
     float *tmp = NULL;
@@ -288,10 +307,20 @@ void tqo_quantize_pack_format(const float *w_in, int64_t N, int64_t K, int per_r
         gamma[0] = tqo_absmean_gamma(w, N * K, TQO_EPS);
     }
     int8_t *q = (int8_t *)malloc((size_t)(N * K));
-    tqo_ternary_codes(w, N, K, gamma, per_row, q);
+    if (ratio > 0.0f)
+        tqo_ternary_codes_threshold(w, N, K, gamma, per_row, ratio, q);
+    else
+        tqo_ternary_codes(w, N, K, gamma, per_row, q);
     tqo_pack_format(q, N, K, format, packed);
     free(q);
     free(tmp);
+}
+
+/* ratio 0: the round/clamp rule of tqo_ternary_codes. */
+void tqo_quantize_pack_format(const float *w_in, int64_t N, int64_t K, int per_row,
+                              int sanitize, int format, uint8_t *packed, float *gamma)
+{
+    tqo_quantize_pack_threshold(w_in, N, K, per_row, sanitize, format, 0.0f, packed, gamma);
 }
 
 void tqo_quantize_pack(const float *w_in, int64_t N, int64_t K, int per_row,

@@ -139,6 +139,43 @@ def test_quantize_pack_layouts_carry_the_same_codes():
         assert np.array_equal(oracle.unpack_format(p, 256, enc), q0)
 
 
+def test_threshold_rule_hand_worked_rows():
+    for ln in golden_lines("threshold_codes.txt"):
+        ratio, ws, codes = [f.strip() for f in ln.split("|")]
+        w = np.array([[float(v) for v in ws.split()]], np.float32)
+        p, g = oracle.quantize_pack_threshold(w, per_row=True, ratio=float(ratio))
+        q, n_res = oracle.unpack(p, 4)
+        assert n_res == 0
+        assert q[0].tolist() == [int(c) for c in codes.split()], ln
+
+
+def test_threshold_rule_one_half_matches_round_rule_off_ties():
+    # ratio 0.5: w > gamma/2 is the round rule's |w/gamma| > 0.5 except where the
+    # fp32 quotient lands exactly on 0.5 (the round rule then gives 0, as strict > does,
+    # unless the quotient rounded up onto 0.5 from below or down from above)
+    W = S.normal((64, 512), 0.02, 21, 64)
+    for per_row in (True, False):
+        p_round, g = oracle.quantize_pack(W, per_row=per_row)
+        q_round, _ = oracle.unpack(p_round, 512)
+        p_thr, g2 = oracle.quantize_pack_threshold(W, per_row=per_row, ratio=0.5)
+        q_thr, _ = oracle.unpack(p_thr, 512)
+        assert np.array_equal(g, g2)
+        gg = np.broadcast_to(g[:, None] if per_row else g, W.shape).astype(np.float32)
+        tie = np.abs(W / gg) == np.float32(0.5)
+        assert np.array_equal(q_round[~tie], q_thr[~tie])
+
+
+def test_threshold_rule_boundaries_are_strict():
+    # a row whose mean is exactly 1: w = 1 is not above tau = 1, the next float is
+    w = np.array([[1.0, 1.0, 1.0, 1.0, 0.5, 1.5, 1.0, 1.0]], np.float32)  # mean |w| = 1
+    q = oracle.ternary_codes_threshold(w, np.array([1.0], np.float32), True, 1.0)
+    assert q[0].tolist() == [0, 0, 0, 0, 0, 1, 0, 0]
+    up = np.nextafter(np.float32(1.0), np.float32(2.0))
+    q = oracle.ternary_codes_threshold(np.array([[up, -up, 1.0, -1.0]], np.float32),
+                                       np.array([1.0], np.float32), True, 1.0)
+    assert q[0].tolist() == [1, -1, 0, 0]
+
+
 def test_packed_size_and_compression():
     for ln in golden_lines("sizes.txt"):
         N, K, nbytes, f32bytes = map(int, ln.split())
