@@ -158,7 +158,7 @@ class ClockSampler:
 class Workload:
     """Builds device buffers and the per-segment launch lists of one step."""
 
-    def __init__(self, name, tq, S, torch, dev, layers, layout=0):
+    def __init__(self, name, tq, S, torch, dev, layers, layout=0, ratio=0.0):
         self.name, self.tq, self.torch, self.dev = name, tq, torch, dev
         f32, u8, i8, i32 = torch.float32, torch.uint8, torch.int8, torch.int32
         self.segments = []  # (label, kernel_name, launches, algorithmic bytes or ops, [fns])
@@ -197,7 +197,7 @@ class Workload:
             raise SystemExit(f"unknown workload {name}")
         N, K, L = self.N, self.K, self.L
         # packed-code layout (0 Foundry, 1 Hetman-2b Format 0, 2 Format 1) on every pack and contraction
-        self.layout = layout
+        self.layout, self.ratio = layout, ratio
         self.flags = (tq.GAMMA_PER_ROW if self.per_row else 0) | (layout << 7)
         # the ring's layers share x and have their own weights and outputs:
         # independent calls, so the contractions may overlap one another
@@ -223,10 +223,15 @@ class Workload:
         # --- segments of one step ---
         pack_bytes = 4 * N * K + N * K // 4 + 4 * (N if self.per_row else 1)
         pack_launches = 1 if self.per_row else 3
-        self.segments.append(("pack", "pack", L, L * pack_bytes, L * pack_launches,
-                              [lambda l=l: tq.quantize_ternary_pack_(self.W[l], self.flags | tq.FLAG_INPUTS_READY,
-                                                                      self.packed[l], self.gamma[l], self.pack_ws[l])
-                               for l in range(L)]))
+        if ratio > 0:  # threshold ternarisation (w > ratio * gamma) instead of round/clamp
+            pack_fns = [lambda l=l: tq.quantize_ternary_pack_threshold_(
+                self.W[l], self.flags | tq.FLAG_INPUTS_READY, ratio, self.packed[l], self.gamma[l], self.pack_ws[l])
+                for l in range(L)]
+        else:
+            pack_fns = [lambda l=l: tq.quantize_ternary_pack_(self.W[l], self.flags | tq.FLAG_INPUTS_READY,
+                                                              self.packed[l], self.gamma[l], self.pack_ws[l])
+                        for l in range(L)]
+        self.segments.append(("pack", "pack", L, L * pack_bytes, L * pack_launches, pack_fns))
         if name == "fused":
             M = self.Ms[0]
             ops = 2 * M * N * K
@@ -277,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     tq.load()
     wl = Workload(args.workload, tq, S, torch, dev, args.layers or WORKLOAD_SHAPES[args.workload][3],
-                  LAYOUTS.index(args.layout))
+                  LAYOUTS.index(args.layout), args.ratio)
     stream = torch.cuda.Stream(device=dev)
     graphs = []
     with torch.cuda.stream(stream):
@@ -390,7 +395,7 @@ WORKLOAD_SHAPES = {  # name -> (Ms, N, K, default ring of layers, per_row)
 LAYOUTS = ["foundry", "format0", "format1"]  # packed-code layouts, flag value = index << 7
 
 
-def config_for(name, layers, world, layout="foundry"):
+def config_for(name, layers, world, layout="foundry", ratio=0.0):
     Ms, N, K, L, per_row = WORKLOAD_SHAPES[name]
     L = layers or L
     desc = {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers" % L,
@@ -399,13 +404,14 @@ def config_for(name, layers, world, layout="foundry"):
             "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L}[name]
     return {"workload": desc, "M": Ms, "N": N, "K": K, "layers": L,
             "gamma": "per-row" if per_row else "per-tensor", "layout": layout,
+            "ternarise": "threshold w > %g * gamma" % ratio if ratio > 0 else "round/clamp",
             "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
                 L * N * K * 4 >> 20, L * N * K // 4 >> 20),
             "parallelism": "replicas x%d" % world if world > 1 else "single GPU"}
 
 
 def wl_config(wl, world):
-    return config_for(wl.name, wl.L, world, LAYOUTS[wl.layout])
+    return config_for(wl.name, wl.L, world, LAYOUTS[wl.layout], wl.ratio)
 
 
 def run_chains(args, wl, tq, torch, stream, world):
@@ -594,6 +600,8 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fused", "sweep"])
+    ap.add_argument("--ratio", type=float, default=0.0,
+                    help="threshold ternarisation w > ratio * gamma (0: the round/clamp rule)")
     ap.add_argument("--layout", default="foundry", choices=LAYOUTS,
                     help="packed-code layout: Foundry's (default) or Hetman-2b's Format 0 / Format 1")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -148,8 +148,23 @@ TQ_API tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, 
                                    uint8_t *packed, float *gamma, void *workspace,
                                    size_t workspace_bytes, tq_stream_t stream);
 
-/* Scratch bytes tq_quantize_ternary_pack needs for these arguments. */
+/* Scratch bytes tq_quantize_ternary_pack needs for these arguments (the same
+ * for tq_quantize_ternary_pack_threshold). */
 TQ_API size_t tq_pack_workspace_bytes(int64_t N, int64_t K, unsigned flags);
+
+/*
+ * Threshold ternarisation with the same gamma: tau = fp32(ratio * gamma),
+ * code = +1 if w > tau, -1 if w < -tau, else 0 (strict).  Foundry,
+ * docs/quantization.md, "Absmean Thresholding (BitNet b1.58)" is ratio = 1
+ * (threshold = mean |w|, scale = threshold); BitRASP, core_math.py,
+ * ternarize_weight is ratio = 0.55 with TQ_GAMMA_PER_ROW (scale = the row's
+ * mean |w|).  Arguments, flags, layout, workspace and errors as for
+ * tq_quantize_ternary_pack; ratio must lie in (0, 64] (else TQ_ERR_ARG).
+ */
+TQ_API tq_status tq_quantize_ternary_pack_threshold(const float *w, int64_t N, int64_t K,
+                                             unsigned flags, float ratio, uint8_t *packed,
+                                             float *gamma, void *workspace,
+                                             size_t workspace_bytes, tq_stream_t stream);
 
 /*
  * Same result as tq_quantize_ternary_pack, for callers that cannot allocate

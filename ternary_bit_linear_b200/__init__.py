@@ -39,6 +39,7 @@ _P, _I64, _U, _F, _I, _SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint, cty
 SIGNATURES = {
     "tq_quantize_ternary_pack": (_I, [_P, _I64, _I64, _U, _P, _P, _P, _SZ, _P]),
     "tq_pack_workspace_bytes": (_SZ, [_I64, _I64, _U]),
+    "tq_quantize_ternary_pack_threshold": (_I, [_P, _I64, _I64, _U, _F, _P, _P, _P, _SZ, _P]),
     "tq_quantize_ternary_pack_noalloc": (_I, [_P, _I64, _I64, _U, _P, _P, _P]),
     "tq_quantize_act_int8": (_I, [_P, _I64, _I64, _U, _F, _F, _P, _P, _P, _P]),
     "tq_fwht512": (_I, [_P, _P, _I64, _I64, _I, _P]),
@@ -124,6 +125,20 @@ def quantize_ternary_pack_(w, flags, packed, gamma, workspace=None, stream=None)
     _check("tq_quantize_ternary_pack",
            load().tq_quantize_ternary_pack(_ptr(w), N, K, flags, _ptr(packed), _ptr(gamma),
                                            _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def quantize_ternary_pack_threshold_(w, flags, ratio, packed, gamma, workspace=None, stream=None):
+    import torch
+
+    N, K = w.shape
+    _need(w, torch.float32, (N, K), "w")
+    _need(packed, torch.uint8, (N, K // 4), "packed")
+    _need(gamma, torch.float32, (N if flags & GAMMA_PER_ROW else 1,), "gamma")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("tq_quantize_ternary_pack_threshold",
+           load().tq_quantize_ternary_pack_threshold(_ptr(w), N, K, flags, float(ratio), _ptr(packed),
+                                                     _ptr(gamma), _ptr(workspace), ws_bytes,
+                                                     _stream(stream)))
 
 
 def quantize_act_int8_(x, flags, eta_min, eta_max, xq, s_x, rowsum, stream=None):

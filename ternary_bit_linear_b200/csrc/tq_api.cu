@@ -323,7 +323,7 @@ struct PerTensor {
 template <typename Kern>
 tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_cta, int smem,
                            const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
-                           const PerTensor &pt, int reverse, int opts, cudaStream_t st) {
+                           const PerTensor &pt, int reverse, int opts, float ratio, cudaStream_t st) {
     int dev = 0, sms = 0;
     if (tq_status e = check_device(&sms)) return e;
     cudaGetDevice(&dev);
@@ -344,36 +344,36 @@ tq_status launch_pack_grid(Kern kern, std::atomic<int> *occ, int64_t rows_per_ct
     const int64_t cap = (int64_t)per_sm * sms;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
     return launch_pdl(kern, dim3(grid), dim3(kPackThreads), (size_t)smem, st, w, N, (int)K,
-                      1.0 / (double)K, packed, gamma, pt.partial, pt.nparts, pt.height, reverse, opts);
+                      1.0 / (double)K, packed, gamma, pt.partial, pt.nparts, pt.height, reverse, opts, ratio);
 }
 
 template <bool SAN, bool CONV>
 tq_status launch_pack_rows_s(const float *w, int64_t N, int64_t K, uint8_t *packed, float *gamma,
-                             const PerTensor &pt, int reverse, int opts, cudaStream_t st) {
+                             const PerTensor &pt, int reverse, int opts, float ratio, cudaStream_t st) {
     static std::atomic<int> occ[5][kMaxDevices];
     const int64_t nv = K / 4;
     const int k = (int)K;
     if (nv <= 32 * kTeamVec * 1)
-        return launch_pack_grid(pack_team_kernel<1, SAN, CONV>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, pt, reverse, opts, st);
+        return launch_pack_grid(pack_team_kernel<1, SAN, CONV>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
     if (nv <= 32 * kTeamVec * 2)
-        return launch_pack_grid(pack_team_kernel<2, SAN, CONV>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, pt, reverse, opts, st);
+        return launch_pack_grid(pack_team_kernel<2, SAN, CONV>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
     if (nv <= 32 * kTeamVec * 4)
-        return launch_pack_grid(pack_team_kernel<4, SAN, CONV>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, pt, reverse, opts, st);
+        return launch_pack_grid(pack_team_kernel<4, SAN, CONV>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
     if (nv <= 32 * kTeamVec * 8)
-        return launch_pack_grid(pack_team_kernel<8, SAN, CONV>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, pt, reverse, opts, st);
-    return launch_pack_grid(pack_rows_kernel<SAN, CONV>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, opts, st);
+        return launch_pack_grid(pack_team_kernel<8, SAN, CONV>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
+    return launch_pack_grid(pack_rows_kernel<SAN, CONV>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
 }
 
 // Options word of the pack kernels: bit 0 inputs ready, bits 1-2 layout.
 inline int pack_opts(int ready, int enc) { return (ready ? 1 : 0) | (enc << 1); }
 
 tq_status launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
-                           float *gamma, const PerTensor &pt, int reverse, int opts, cudaStream_t st) {
+                           float *gamma, const PerTensor &pt, int reverse, int opts, float ratio, cudaStream_t st) {
     if (opts >> 1)  // a layout other than Foundry's
-        return sanitize ? launch_pack_rows_s<true, true>(w, N, K, packed, gamma, pt, reverse, opts, st)
-                        : launch_pack_rows_s<false, true>(w, N, K, packed, gamma, pt, reverse, opts, st);
-    return sanitize ? launch_pack_rows_s<true, false>(w, N, K, packed, gamma, pt, reverse, opts, st)
-                    : launch_pack_rows_s<false, false>(w, N, K, packed, gamma, pt, reverse, opts, st);
+        return sanitize ? launch_pack_rows_s<true, true>(w, N, K, packed, gamma, pt, reverse, opts, ratio, st)
+                        : launch_pack_rows_s<false, true>(w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
+    return sanitize ? launch_pack_rows_s<true, false>(w, N, K, packed, gamma, pt, reverse, opts, ratio, st)
+                    : launch_pack_rows_s<false, false>(w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
 }
 
 size_t pack_parts(int64_t nv) {
@@ -462,9 +462,10 @@ size_t tq_pack_workspace_bytes(int64_t N, int64_t K, unsigned flags) {
     return pack_parts(N * K / 4) * sizeof(DD) + 16;
 }
 
-tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigned flags,
-                                   uint8_t *packed, float *gamma, void *workspace,
-                                   size_t workspace_bytes, tq_stream_t stream) {
+// Shared body of the two packing entry points; ratio 0 selects the round rule.
+static tq_status pack_impl(const float *w, int64_t N, int64_t K, unsigned flags, float ratio,
+                           uint8_t *packed, float *gamma, void *workspace, size_t workspace_bytes,
+                           tq_stream_t stream) {
     if (!w || !packed || !gamma) return TQ_ERR_NULL;
     if (N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
@@ -494,7 +495,7 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     cudaStream_t st = cs(stream);
     if (per_row) {
         if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0,
-                                           pack_opts(ready, enc), st))
+                                           pack_opts(ready, enc), ratio, st))
             return e;
         return launch_status();
     }
@@ -509,9 +510,23 @@ tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigne
     pt.partial = partial;
     pt.nparts = (int)nparts;
     pt.height = absum_tree_height(chunk, (int)nparts);
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, pack_opts(0, enc), st))
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, pack_opts(0, enc), ratio, st))
         return e;
     return launch_status();
+}
+
+tq_status tq_quantize_ternary_pack(const float *w, int64_t N, int64_t K, unsigned flags,
+                                   uint8_t *packed, float *gamma, void *workspace,
+                                   size_t workspace_bytes, tq_stream_t stream) {
+    return pack_impl(w, N, K, flags, 0.0f, packed, gamma, workspace, workspace_bytes, stream);
+}
+
+tq_status tq_quantize_ternary_pack_threshold(const float *w, int64_t N, int64_t K, unsigned flags,
+                                             float ratio, uint8_t *packed, float *gamma,
+                                             void *workspace, size_t workspace_bytes,
+                                             tq_stream_t stream) {
+    if (!(ratio > 0.0f && ratio <= 64.0f)) return TQ_ERR_ARG;  // NaN fails too
+    return pack_impl(w, N, K, flags, ratio, packed, gamma, workspace, workspace_bytes, stream);
 }
 
 tq_status tq_quantize_act_int8(const float *x, int64_t M, int64_t K, unsigned flags, float eta_min,
@@ -739,7 +754,7 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, 0, st)) return e;
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, 0, 0.0f, st)) return e;
         return launch_status();
     }
     void *scratch = nullptr;
@@ -754,6 +769,6 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     pt.partial = partial;
     pt.nparts = (int)nparts;
     pt.height = absum_tree_height(kNoAllocChunk, (int)nparts);
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, 0, st)) return e;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, 0, 0.0f, st)) return e;
     return launch_status();
 }

@@ -380,6 +380,14 @@ __device__ __forceinline__ float code_threshold(float gamma) {
     return t;
 }
 
+// Code threshold t for one gamma (a weight is +1 iff w >= t, -1 iff w <= -t):
+// the round rule (ratio <= 0; code_threshold) or the threshold rule
+// w > fp32(ratio * gamma), strict, i.e. t = the next float above it.
+__device__ __forceinline__ float pack_threshold(float gamma, float ratio) {
+    if (ratio > 0.0f) return nextafterf(__fmul_rn(ratio, gamma), __int_as_float(0x7f800000));
+    return code_threshold(gamma);
+}
+
 // 2-bit code (-1 -> 0b00, 0 -> 0b01, +1 -> 0b10) of one weight.
 __device__ __forceinline__ uint32_t ternary_field(float w, float t) {
     return 1u + (w >= t ? 1u : 0u) - (w <= -t ? 1u : 0u);

@@ -14,7 +14,9 @@
 // ~2^-100 relative) and rounded with an explicit midpoint test.
 //
 // Codes come from one fp32 threshold per gamma (code_threshold), equivalent to
-// rounding the fp32 quotient w / gamma and clamping, without a divide.
+// rounding the fp32 quotient w / gamma and clamping, without a divide; or, for
+// the threshold rule (Foundry "Absmean Thresholding", BitRASP ternarize_weight),
+// from w > fp32(ratio * gamma) (pack_threshold).
 //
 // HBM traffic: read 4 B and write 0.25 B per weight.  Per-row gamma is one
 // pass; per-tensor gamma reads W twice (reduction, then packing walking the
@@ -145,7 +147,7 @@ __device__ __forceinline__ double sum_error_bound(int h) { return (double)(h + 3
 // ---------------------------------------------------------------------------
 __device__ __noinline__ float per_tensor_threshold(const double *__restrict__ partial, int nparts, int height,
                                                    const float *__restrict__ w, int64_t nv, int sanitize,
-                                                   float *__restrict__ gamma) {
+                                                   float *__restrict__ gamma, float ratio) {
     __shared__ double red[kPackWarps];
     __shared__ DD redd[kPackWarps];
     __shared__ float g_s;
@@ -175,7 +177,7 @@ __device__ __noinline__ float per_tensor_threshold(const double *__restrict__ pa
     }
     g = g > 1e-6f ? g : 1e-6f;
     if (blockIdx.x == 0 && threadIdx.x == 0) gamma[0] = g;
-    return code_threshold(g);
+    return pack_threshold(g, ratio);
 }
 
 // No block-level synchronisation: warps are independent.
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(kPackThreads)
     pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
-                     int opts) {
+                     int opts, float ratio) {
     const int ready = opts & 1, enc = opts >> 1;  // inputs ready; packed-code layout
     if (!ready) pdl_wait();
     pdl_trigger();
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(kPackThreads)
     const int nv = K >> 2;
     const bool per_tensor = partial != nullptr;
     const float t_tensor =
-        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma) : 0.0f;
+        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma, ratio) : 0.0f;
     // per-lane chain length (float4) of pass 1, for the error bound
     const int chain = (nv + 31) / 32;
     const double eps = sum_error_bound(4 * chain + 5);
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kPackThreads)
             }
             g = g > 1e-6f ? g : 1e-6f;
             if (lane == 0) gamma[n] = g;
-            t = code_threshold(g);
+            t = pack_threshold(g, ratio);
         }
         uint8_t *dst = packed + n * (int64_t)nv;
         int c = lane;
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(kPackThreads, 2)
     pack_team_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
-                     int opts) {
+                     int opts, float ratio) {
     const int ready = opts & 1, enc = opts >> 1;  // inputs ready; packed-code layout
     constexpr int TEAMS = kPackWarps / T;
     extern __shared__ __align__(16) float4 rowbuf[];  // [TEAMS][kPackRing][nv]
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kPackThreads, 2)
     // the first rows are in flight: now the per-tensor threshold (if any)
     const bool per_tensor = partial != nullptr;
     const float t_tensor =
-        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma) : 0.0f;
+        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma, ratio) : 0.0f;
     const double eps = sum_error_bound(4 * kTeamVec + 5 + T);
     int parity = 0;
     int64_t k = 0;
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(kPackThreads, 2)
             }
             g = g > 1e-6f ? g : 1e-6f;
             if (all_ok && tw == 0 && lane == 0) gamma[n] = g;
-            t = code_threshold(g);
+            t = pack_threshold(g, ratio);
         } else {
             all_ok = team_all(bar_id, 32 * T, ok);  // the buffer has been read
         }

@@ -88,6 +88,21 @@ def test_pack_validation(lib):
     assert f(P(), 4, 64, 0, P(1 << 20), P(2 << 20), P(3 << 20), 8, None) == 4  # too small
 
 
+def test_pack_threshold_validation(lib):
+    f = lib.tq_quantize_ternary_pack_threshold
+    ok = [P(), 4, 64, 1, 0.55, P(1 << 20), P(2 << 20), None, 0, None]
+    for bad_ratio in (0.0, -1.0, 65.0, float("nan"), float("inf")):
+        args = list(ok)
+        args[4] = bad_ratio
+        assert f(*args) == 4, bad_ratio
+    args = list(ok)
+    args[0] = None
+    assert f(*args) == 1
+    args = list(ok)
+    args[3] = 1 << 9
+    assert f(*args) == 4
+
+
 def test_act_and_fwht_validation(lib):
     f = lib.tq_quantize_act_int8
     assert f(P(), 2, 64, 0, 0.05, 40.0, P(1 << 20), P(2 << 20), None, None) == 1

@@ -729,3 +729,47 @@ def test_fused_layouts_equal_default_layout(cuda_lib, layout):
         outs.append(host(y))
     assert np.array_equal(outs[0], outs[1])
     assert tq.device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# Threshold ternarisation (Foundry "Absmean Thresholding": ratio 1; BitRASP
+# ternarize_weight: ratio 0.55 per row), bytes and gamma bit-exact.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("ratio", [1.0, 0.55, 0.5, 2.0])
+@pytest.mark.parametrize("N,K,per_row", [(17, 512, True), (129, 4160, False), (5, 8256, True), (40, 2048, True),
+                                         (300, 1024, False)])
+def test_pack_threshold_matches_oracle(cuda_lib, ratio, N, K, per_row):
+    tq = cuda_lib
+    W = S.normal((N, K), 0.02, 96, N)
+    p_ref, g_ref = oracle.quantize_pack_threshold(W, per_row=per_row, ratio=ratio)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty((N if per_row else 1,), dtype=torch.float32, device="cuda")
+    flags = tq.GAMMA_PER_ROW if per_row else 0
+    ws = torch.empty((max(16, tq.pack_workspace_bytes(N, K, flags)),), dtype=torch.uint8, device="cuda")
+    tq.quantize_ternary_pack_threshold_(dev(W), flags, ratio, packed, gamma, ws)
+    assert np.array_equal(host(packed), p_ref)
+    assert np.array_equal(host(gamma), g_ref)
+
+
+def test_pack_threshold_boundaries_and_layout(cuda_lib):
+    """Rows whose mean |w| is exactly 1 (so tau = ratio exactly for ratio 1 and
+    0.5) holding weights at tau, just above and just below it, in both signs;
+    packed in Hetman-2b's Format 1 as well."""
+    tq = cuda_lib
+    K = 512
+    base = np.ones((8, K), np.float32)
+    up, dn = np.nextafter(np.float32(1), np.float32(2)), np.nextafter(np.float32(1), np.float32(0))
+    h_up, h_dn = np.nextafter(np.float32(0.5), np.float32(1)), np.nextafter(np.float32(0.5), np.float32(0))
+    vals = np.array([1.0, -1.0, up, -up, dn, -dn, 0.5, -0.5, h_up, -h_up, h_dn, -h_dn], np.float32)
+    base[:, :vals.size] = vals
+    base[:, vals.size:2 * vals.size] = 2.0 - np.abs(vals)  # keeps the row's mean |w| at exactly 1
+    W = base
+    for ratio in (1.0, 0.5):
+        for layout in (0, 2):
+            p_ref, g_ref = oracle.quantize_pack_threshold(W, per_row=True, ratio=ratio, encoding=layout)
+            assert np.all(g_ref == 1.0)
+            packed = torch.empty((8, K // 4), dtype=torch.uint8, device="cuda")
+            gamma = torch.empty((8,), dtype=torch.float32, device="cuda")
+            tq.quantize_ternary_pack_threshold_(dev(W), tq.GAMMA_PER_ROW | (layout << 7), ratio, packed, gamma)
+            assert np.array_equal(host(packed), p_ref), (ratio, layout)
+            assert np.array_equal(host(gamma), g_ref)
