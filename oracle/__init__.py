@@ -58,6 +58,9 @@ def _load():
         _lib.tqo_quantize_pack.argtypes = [P, I64, I64, I, I, P, P]
         _lib.tqo_quantize_pack_format.argtypes = [P, I64, I64, I, I, I, P, P]
         _lib.tqo_quantize_pack_threshold.argtypes = [P, I64, I64, I, I, I, F, P, P]
+        _lib.tqo_dequant_bias.argtypes = [P, P, I, P, P, I64, I64, P]
+        _lib.tqo_int_epilogue.argtypes = [P, P, I, I64, I64, P]
+        _lib.tqo_fwht_roundtrip.argtypes = [P, I64, I64, F, F, P, P]
         _lib.tqo_ternary_codes_threshold.argtypes = [P, I64, I64, P, I, F, P]
         _lib.tqo_pack_format.argtypes = [P, I64, I64, I, P]
         _lib.tqo_unpack_format.argtypes = [P, I64, I64, I, P]
@@ -262,6 +265,42 @@ def fwht512(x, normalize: bool = True):
     y = np.empty_like(x)
     _load().tqo_fwht512(px, y.ctypes.data_as(ctypes.c_void_p), rows, K, int(normalize))
     return y
+
+
+def dequant_bias(acc, gamma, s_x, per_row: bool, bias=None):
+    acc, pa = _c(acc, np.int32)
+    M, N = acc.shape
+    g, pg = _c(np.atleast_1d(gamma), np.float32)
+    sx, ps = _c(s_x, np.float32)
+    pb = None
+    if bias is not None:
+        bias, pb = _c(bias, np.float32)
+    y = np.empty((M, N), np.float32)
+    _load().tqo_dequant_bias(pa, pg, int(per_row), ps, pb, M, N, y.ctypes.data_as(ctypes.c_void_p))
+    return y
+
+
+def int_epilogue(acc, bias=None, out_shift: int = 0):
+    acc, pa = _c(acc, np.int32)
+    M, N = acc.shape
+    pb = None
+    if bias is not None:
+        bias, pb = _c(bias, np.int32)
+    out = np.empty((M, N), np.int32)
+    _load().tqo_int_epilogue(pa, pb, int(out_shift), M, N, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def fwht_roundtrip(x, eta_min: float = 0.05, eta_max: float = 40.0):
+    """Returns (y float32 [rows, K], eta float32 [rows])."""
+    x, px = _c(x, np.float32)
+    rows, K = x.shape
+    assert K % 512 == 0
+    y = np.empty_like(x)
+    eta = np.empty((rows,), np.float32)
+    _load().tqo_fwht_roundtrip(px, rows, K, float(eta_min), float(eta_max), y.ctypes.data_as(ctypes.c_void_p),
+                               eta.ctypes.data_as(ctypes.c_void_p))
+    return y, eta
 
 
 def bitlinear(x, packed, gamma, per_row: bool, rms_gain=None, rms_eps: float = 1e-6,

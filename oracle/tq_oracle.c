@@ -453,6 +453,38 @@ void tqo_dequant(const int32_t *acc, const float *gamma, int per_row, const floa
         }
 }
 
+/* Epilogue variants.
+ * [H] section 5 BitLinear.forward step 6: y = y_int32 * scale_fusion, then
+ * "+ self.bias" when the layer has one: here y = acc * gamma_n * s_x[m] +
+ * bias[n], computed in fp64 and rounded once (bias may be NULL).
+ * [B] additive_ternary_linear_int8: acc += bias[o] (int32), then, for
+ * out_shift > 0, acc >>= out_shift (arithmetic shift): the integer output. */
+void tqo_dequant_bias(const int32_t *acc, const float *gamma, int per_row, const float *s_x,
+                      const float *bias, int64_t M, int64_t N, float *y)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double g = per_row ? (double)gamma[n] : (double)gamma[0];
+            double b = bias ? (double)bias[n] : 0.0;
+            y[m * N + n] = (float)((double)acc[m * N + n] * g * (double)s_x[m] + b);
+        }
+}
+
+void tqo_int_epilogue(const int32_t *acc, const int32_t *bias, int out_shift, int64_t M, int64_t N,
+                      int32_t *out)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t v = (int64_t)acc[m * N + n] + (bias ? (int64_t)bias[n] : 0);
+            if (out_shift > 0) {
+                /* floor division by 2^out_shift: the arithmetic right shift */
+                int64_t d = (int64_t)1 << out_shift;
+                v = v >= 0 ? v / d : -((-v + d - 1) / d);
+            }
+            out[m * N + n] = (int32_t)v;
+        }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Prologue: quench, RMSNorm, FWHT-512                                        */
 /* ------------------------------------------------------------------------ */
@@ -508,6 +540,47 @@ void tqo_fwht512(const float *x, float *y, int64_t rows, int64_t K, int normaliz
                     }
             for (int i = 0; i < 512; ++i) dst[i] = normalize ? buf[i] * norm : buf[i];
         }
+}
+
+/* [H] section 1 FastWalshHadamardTransform.forward (the quantisation round
+ * trip of the module, per row of K, K % 512 == 0):
+ *   0. nan -> 0, +inf -> eta_max, -inf -> -eta_max (nan_to_num);
+ *   1. x_rot = FWHT-512 (normalised) of every block;
+ *   2. eta = max_k |x_rot| + 1e-5 (fp32), clamped to [eta_min, eta_max];
+ *   3. x_q = clamp(round(x_rot * (127 / eta)), -127, 127) (fp32, half to even),
+ *      dequantised as x_q * fp32(eta / 127) -- the straight-through form
+ *      x_s + (x_q - x_s) is exactly x_q in fp32, since x_q - x_s is exact;
+ *   4. y = FWHT-512 (normalised) of the dequantised row.
+ * eta_out[row] receives the clamped eta (the module reports their mean). */
+void tqo_fwht_roundtrip(const float *x, int64_t rows, int64_t K, float eta_min, float eta_max,
+                        float *y, float *eta_out)
+{
+    float *t = (float *)malloc((size_t)K * sizeof(float));
+    float *u = (float *)malloc((size_t)K * sizeof(float));
+    for (int64_t r = 0; r < rows; ++r) {
+        tqo_sanitize_acts(x + r * K, K, eta_max, t);
+        tqo_fwht512(t, u, 1, K, 1);
+        float a = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = fabsf(u[k]);
+            if (v > a) a = v;
+        }
+        float eta = a + 1e-5f;
+        if (eta < eta_min) eta = eta_min;
+        if (eta > eta_max) eta = eta_max;
+        float scale = 127.0f / eta;
+        float back = eta / 127.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float q = rintf(u[k] * scale);
+            if (q > 127.0f) q = 127.0f;
+            if (q < -127.0f) q = -127.0f;
+            t[k] = q * back;
+        }
+        tqo_fwht512(t, y + r * K, 1, K, 1);
+        if (eta_out) eta_out[r] = eta;
+    }
+    free(t);
+    free(u);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -395,6 +395,32 @@ def test_dequant_correct_rounding_and_zero():
             assert np.sign(y[m, n]) == np.sign(float(exact))
 
 
+def test_dequant_bias_correct_rounding():
+    # [H] section 5 step 6 with the layer bias: acc * gamma * s_x + bias, one rounding
+    rng = np.random.default_rng(19)
+    acc = rng.integers(-500000, 500000, (5, 7)).astype(np.int32)
+    acc[0, 0] = 0
+    g = (rng.random(7) * 0.05 + 1e-3).astype(np.float32)
+    sx = (rng.random(5) * 0.1 + 1e-3).astype(np.float32)
+    b = (rng.standard_normal(7) * 0.5).astype(np.float32)
+    y = oracle.dequant_bias(acc, g, sx, True, b)
+    assert y[0, 0] == b[0]
+    for m in range(5):
+        for n in range(7):
+            exact = Fraction(int(acc[m, n])) * Fraction(float(g[n])) * Fraction(float(sx[m])) + Fraction(float(b[n]))
+            r = f32_round_rational(abs(exact))
+            assert abs(y[m, n]) in (r, np.nextafter(r, np.float32(0)), np.nextafter(r, np.float32(np.inf)))
+            assert np.sign(y[m, n]) == np.sign(float(exact))
+    assert np.array_equal(oracle.dequant_bias(acc, g, sx, True, None), oracle.dequant(acc, g, sx, True))
+
+
+def test_int_epilogue_hand_worked():
+    for ln in golden_lines("int_epilogue.txt"):
+        a, b, sh, want = map(int, ln.split())
+        out = oracle.int_epilogue(np.array([[a]], np.int32), np.array([b], np.int32), sh)
+        assert out[0, 0] == want, ln
+
+
 # --------------------------------------------------------------------------
 # FWHT-512
 # --------------------------------------------------------------------------
@@ -435,6 +461,48 @@ def test_fwht_spike_attenuation_golden():
     assert np.abs(y).max() <= float(max_peak)
     c = np.float32(float(val)) * F32_ONE_OVER_SQRT512
     assert np.all(y[:256] == c) and np.all(y[256:] == -c)  # row 256 of H: + then -
+
+
+def test_fwht_roundtrip_spike_closed_form():
+    # Hetman-2b section 1 FastWalshHadamardTransform: a spike of 100 at 256 rotates to
+    # +-100/sqrt(512) everywhere, eta = that + 1e-5, every code is +-127 (the value
+    # sits 1e-5 below eta), the dequantised +-eta rotates back to a spike of
+    # 512 * eta / sqrt(512) = 100 + 1e-5 * sqrt(512) and exact zeros elsewhere
+    x = np.zeros((1, 512), np.float32)
+    x[0, 256] = 100.0
+    y, eta = oracle.fwht_roundtrip(x)
+    c = float(F32_ONE_OVER_SQRT512)
+    assert abs(float(eta[0]) - (100.0 * c + 1e-5)) < 1e-6
+    assert abs(float(y[0, 256]) - (100.0 + 1e-5 * math.sqrt(512))) < 5e-5
+    assert np.count_nonzero(y[0]) == 1
+
+
+def test_fwht_roundtrip_gain_clamp_and_quench():
+    # eta below eta_min / above eta_max is clamped; NaN reads as 0, +-inf as +-eta_max
+    z, eta = oracle.fwht_roundtrip(np.zeros((1, 512), np.float32))
+    assert eta[0] == np.float32(0.05) and not z.any()
+    x = np.zeros((1, 512), np.float32)
+    x[0, 0] = 1000.0  # rotates to 44.19 > eta_max = 40: codes saturate at 127
+    y, eta = oracle.fwht_roundtrip(x)
+    assert eta[0] == np.float32(40.0)
+    step = np.float32(40.0) / np.float32(127.0)
+    assert abs(float(y[0, 0]) - 512 * float(np.float32(127.0) * step) * float(F32_ONE_OVER_SQRT512)) < 1e-3
+    xn = np.zeros((1, 512), np.float32)
+    xn[0, 3] = np.nan
+    xn[0, 7] = np.inf
+    xf = np.zeros((1, 512), np.float32)
+    xf[0, 7] = 40.0
+    assert np.array_equal(oracle.fwht_roundtrip(xn)[0], oracle.fwht_roundtrip(xf)[0])
+
+
+def test_fwht_roundtrip_error_bound():
+    # the rotation is orthonormal, so ||y - x||_2 = ||dequant - x_rot||_2 <= sqrt(K) * step / 2
+    X = S.student_t3((6, 1024), 22, 6)
+    Y, eta = oracle.fwht_roundtrip(X)
+    for r in range(6):
+        step = float(eta[r]) / 127.0
+        err = float(np.linalg.norm(Y[r].astype(np.float64) - X[r].astype(np.float64)))
+        assert err <= math.sqrt(1024) * step / 2 * 1.001 + 1e-5
 
 
 def test_fwht_blocks_are_independent():
