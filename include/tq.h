@@ -241,6 +241,25 @@ TQ_API tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32
                           tq_stream_t stream);
 
 /*
+ * tq_ternary_gemm with the pages' other epilogues.
+ *   bias      [N] fp32 or NULL: y = acc * gamma * s_x + bias[n] (Hetman-2b
+ *             section 5, BitLinear.forward, "y_out + self.bias").
+ *   acc_bias  [N] int32 or NULL, out_shift in [0, 31]: the int32 output becomes
+ *             (acc + acc_bias[n]) >> out_shift, an arithmetic shift (BitRASP,
+ *             core_math.py, additive_ternary_linear_int8: acc += bias[o];
+ *             acc >>= out_shift).  Applies to `acc` only; y uses the plain sum.
+ * Other arguments, flags and errors as for tq_ternary_gemm (bias and acc_bias
+ * 16-byte aligned, not overlapping the outputs; out_shift outside [0, 31] is
+ * TQ_ERR_ARG).  Small M runs the per-strip GEMV shapes even with
+ * TQ_FLAG_INPUTS_READY.
+ */
+TQ_API tq_status tq_ternary_gemm_ex(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                                    const uint8_t *packed, const float *gamma, unsigned flags,
+                                    int64_t M, int64_t N, int64_t K, const float *bias,
+                                    const int32_t *acc_bias, int out_shift, float *y, int32_t *acc,
+                                    tq_stream_t stream);
+
+/*
  * Whole layer on pre-packed weights: [quench] -> [RMSNorm] -> [FWHT-512] ->
  * per-token int8 -> contraction -> rescale.  Hetman-2b section 5
  * BitLinear.forward steps 0-6.
@@ -268,6 +287,25 @@ TQ_API tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float
 
 /* Scratch bytes tq_bitlinear_fused needs for these arguments. */
 TQ_API size_t tq_fused_workspace_bytes(int64_t M, int64_t K, unsigned flags);
+
+/*
+ * The FWHT module's quantisation round trip.  Hetman-2b section 1,
+ * FastWalshHadamardTransform.forward: per row of K, nan -> 0 and +-inf ->
+ * +-eta_max, then x_rot = FWHT-512 (normalised) of every 512-block, eta =
+ * max_k |x_rot| + 1e-5 clamped to [eta_min, eta_max] (the Hadamard gain
+ * clamp; 0.05 and 40 on the page), x_q = clamp(round(x_rot * 127 / eta),
+ * -127, 127) half to even, y = FWHT-512 of x_q * (eta / 127).  All in fp32, in
+ * the definition's order (bit-identical to it).
+ *
+ *   x, y      [rows][K] fp32; y may equal x (in place), else no overlap.
+ *   K         multiple of 512, at most 16384.
+ *   eta_out   [rows] fp32 or NULL: each row's clamped eta (the module reports
+ *             their mean).
+ * Errors: TQ_ERR_SHAPE, TQ_ERR_ARG (eta bounds not 0 < min <= max < 3e38, or
+ * overlap), TQ_ERR_ALIGN (16 bytes).
+ */
+TQ_API tq_status tq_fwht_roundtrip(const float *x, float *y, int64_t rows, int64_t K, float eta_min,
+                                   float eta_max, float *eta_out, tq_stream_t stream);
 
 /*
  * Waits for `stream`, then returns and clears the current device's status word:

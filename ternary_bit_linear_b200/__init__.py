@@ -43,7 +43,9 @@ SIGNATURES = {
     "tq_quantize_ternary_pack_noalloc": (_I, [_P, _I64, _I64, _U, _P, _P, _P]),
     "tq_quantize_act_int8": (_I, [_P, _I64, _I64, _U, _F, _F, _P, _P, _P, _P]),
     "tq_fwht512": (_I, [_P, _P, _I64, _I64, _I, _P]),
+    "tq_fwht_roundtrip": (_I, [_P, _P, _I64, _I64, _F, _F, _P, _P]),
     "tq_ternary_gemm": (_I, [_P, _P, _P, _P, _P, _U, _I64, _I64, _I64, _P, _P, _P]),
+    "tq_ternary_gemm_ex": (_I, [_P, _P, _P, _P, _P, _U, _I64, _I64, _I64, _P, _P, _I, _P, _P, _P]),
     "tq_bitlinear_fused": (_I, [_P, _P, _F, _F, _F, _U, _P, _P, _I64, _I64, _I64, _P, _P, _P,
                                 _P, _SZ, _P]),
     "tq_fused_workspace_bytes": (_SZ, [_I64, _I64, _U]),
@@ -178,6 +180,24 @@ def ternary_gemm_(xq, s_x, rowsum, packed, gamma, flags, y, acc=None, stream=Non
                                   flags, M, N, K, _ptr(y), _ptr(acc), _stream(stream)))
 
 
+def ternary_gemm_ex_(xq, s_x, rowsum, packed, gamma, flags, y, acc=None, bias=None, acc_bias=None,
+                     out_shift=0, stream=None):
+    import torch
+
+    M, K = xq.shape
+    N = packed.shape[0]
+    _need(xq, torch.int8, (M, K), "xq")
+    _need(packed, torch.uint8, (N, K // 4), "packed")
+    _need(y, torch.float32, (M, N), "y")
+    _need(acc, torch.int32, (M, N), "acc")
+    _need(bias, torch.float32, (N,), "bias")
+    _need(acc_bias, torch.int32, (N,), "acc_bias")
+    _check("tq_ternary_gemm_ex",
+           load().tq_ternary_gemm_ex(_ptr(xq), _ptr(s_x), _ptr(rowsum), _ptr(packed), _ptr(gamma), flags, M, N, K,
+                                     _ptr(bias), _ptr(acc_bias), int(out_shift), _ptr(y), _ptr(acc),
+                                     _stream(stream)))
+
+
 def bitlinear_fused_(x, packed, gamma, flags, y, workspace, rms_gain=None, rms_eps=1e-6,
                      eta_min=0.05, eta_max=40.0, xq_out=None, s_x_out=None, stream=None):
     import torch
@@ -192,6 +212,18 @@ def bitlinear_fused_(x, packed, gamma, flags, y, workspace, rms_gain=None, rms_e
                                      _ptr(s_x_out), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(),
                                      _stream(stream)))
+
+
+def fwht_roundtrip_(x, y, eta_min=0.05, eta_max=40.0, eta_out=None, stream=None):
+    import torch
+
+    rows, K = x.shape
+    _need(x, torch.float32, (rows, K), "x")
+    _need(y, torch.float32, (rows, K), "y")
+    _need(eta_out, torch.float32, (rows,), "eta_out")
+    _check("tq_fwht_roundtrip",
+           load().tq_fwht_roundtrip(_ptr(x), _ptr(y), rows, K, float(eta_min), float(eta_max), _ptr(eta_out),
+                                    _stream(stream)))
 
 
 def device_status(stream=None) -> int:

@@ -389,6 +389,56 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
+// Hetman-2b section 1 FastWalshHadamardTransform.forward: the module's int8
+// round trip between two rotations.  One CTA per row, one warp per 512-block
+// (K = 512 * blockDim.x / 32): quench (nan -> 0, +-inf -> +-eta_max), FWHT,
+// eta = max|x_rot| + 1e-5 clamped to [eta_min, eta_max], x_q =
+// clamp(round(x_rot * fp32(127 / eta)), +-127), dequantised by fp32(eta / 127),
+// FWHT again -- every step the fp32 operation the definition names, so the
+// result is bit-identical to it.  y may alias x (a CTA reads its row before
+// it writes it).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+    fwht_roundtrip_kernel(const float *x, float *y, float eta_min, float eta_max,
+                          float *__restrict__ eta_out) {
+    __shared__ float redf[32];
+    pdl_wait();
+    pdl_trigger();
+    const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t K = 512 * (int64_t)nw;
+    const float *row = x + (int64_t)blockIdx.x * K + warp * 512;
+    float f[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float4 v = reinterpret_cast<const float4 *>(row)[j * 32 + lane];
+        f[4 * j + 0] = quench(v.x, eta_max);
+        f[4 * j + 1] = quench(v.y, eta_max);
+        f[4 * j + 2] = quench(v.z, eta_max);
+        f[4 * j + 3] = quench(v.w, eta_max);
+    }
+    fwht512_regs(f, true);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = warp_max(amax);
+    if (lane == 0) redf[warp] = amax;
+    __syncthreads();
+    amax = warp_max(lane < nw ? redf[lane] : 0.0f);
+    const float eta = fminf(fmaxf(__fadd_rn(amax, 1e-5f), eta_min), eta_max);
+    const float scale = __fdiv_rn(127.0f, eta), back = __fdiv_rn(eta, 127.0f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float q = fminf(fmaxf(rintf(__fmul_rn(f[i], scale)), -127.0f), 127.0f);
+        f[i] = __fmul_rn(q, back);
+    }
+    fwht512_regs(f, true);
+    float4 *dst = reinterpret_cast<float4 *>(y + (int64_t)blockIdx.x * K + warp * 512);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[j * 32 + lane] = make_float4(f[4 * j + 0], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+    if (eta_out && threadIdx.x == 0) eta_out[blockIdx.x] = eta;
+}
+
+// ---------------------------------------------------------------------------
 // Fused prologue of the whole layer: [quench] -> [RMSNorm] -> FWHT-512 ->
 // per-token int8.  One CTA per token, one warp per 512-block (K = 512 * NW).
 // ---------------------------------------------------------------------------

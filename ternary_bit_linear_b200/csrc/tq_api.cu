@@ -141,16 +141,29 @@ bool make_tmap_u8(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows
 // ---------------------------------------------------------------------------
 // Launch helpers
 // ---------------------------------------------------------------------------
-template <int BT, bool CONV>
-tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
-                      const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
-                      int64_t K, float *y, int32_t *acc, int mode, int sms, cudaStream_t st) {
+// Arguments of one contraction call, as the kernels take them.
+struct GemmArgs {
+    const int8_t *xq;
+    const float *s_x;
+    const int32_t *rowsum;
+    const uint8_t *packed;
+    const float *gamma;
+    int per_row;
+    int64_t M, N, K;
+    float *y;
+    int32_t *acc;
+    int mode;
+    Epilogue ep;
+};
+
+template <int BT, bool CONV, bool EPI>
+tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
     using L = GemmLayout<BT>;
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemm_kernel<BT, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_kernel<BT, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  L::kDynamic) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
@@ -158,35 +171,35 @@ tq_status launch_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
     // x_q [M][K] in 128-byte-swizzled [BT][128] boxes; packed weights [N][K/4]
     // in plain [128][32] boxes (K % 64 == 0 keeps both row strides 16-byte multiples).
     CUtensorMap tx, tw;
-    if (!make_tmap_u8(&tx, xq, (uint64_t)K, (uint64_t)M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_u8(&tw, packed, (uint64_t)(K / 4), (uint64_t)N, kTileK / 4, kTileN,
+    if (!make_tmap_u8(&tx, a.xq, (uint64_t)a.K, (uint64_t)a.M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_u8(&tw, a.packed, (uint64_t)(a.K / 4), (uint64_t)a.N, kTileK / 4, kTileN,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return TQ_ERR_CUDA;
-    const int64_t tiles = ((M + BT - 1) / BT) * ((N + kTileN - 1) / kTileN);
+    const int64_t tiles = ((a.M + BT - 1) / BT) * ((a.N + kTileN - 1) / kTileN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
-    return launch_pdl(gemm_kernel<BT, CONV>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
-                      s_x, rowsum, gamma, per_row, (int)M, (int)N, (int)K, y, acc, mode);
+    return launch_pdl(gemm_kernel<BT, CONV, EPI>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
+                      a.s_x, a.rowsum, a.gamma, a.per_row, (int)a.M, (int)a.N, (int)a.K, a.y, a.acc, a.mode,
+                      a.ep);
 }
 
 // Grid: one CTA per 16-row strip.  Dynamic shared memory holds x_q only.
-template <int NB, int W, int SPW, bool CONV>
-tq_status launch_gemv(const int8_t *xq, const float *s_x, const int32_t *rowsum,
-                      const uint8_t *packed, const float *gamma, int per_row, int64_t M, int64_t N,
-                      int64_t K, float *y, int32_t *acc, int mode, cudaStream_t st) {
+template <int NB, int W, int SPW, bool CONV, bool EPI>
+tq_status launch_gemv(const GemmArgs &a, cudaStream_t st) {
     static_assert(256 * W * SPW >= kGemvMaxK / 2, "shape covers K");
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemv_kernel<NB, W, SPW, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemv_kernel<NB, W, SPW, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemv_x_bytes(8 * NB, kGemvMaxK)) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
     }
-    const int64_t grid = (N + 15) / 16;
-    const size_t smem = (size_t)gemv_x_bytes((int)M, (int)K);
-    return launch_pdl(gemv_kernel<NB, W, SPW, CONV>, dim3((unsigned)grid), dim3(W * 32), smem, st, xq, s_x,
-                      rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, mode);
+    const int64_t grid = (a.N + 15) / 16;
+    const size_t smem = (size_t)gemv_x_bytes((int)a.M, (int)a.K);
+    return launch_pdl(gemv_kernel<NB, W, SPW, CONV, EPI>, dim3((unsigned)grid), dim3(W * 32), smem, st, a.xq,
+                      a.s_x, a.rowsum, a.packed, a.gamma, a.per_row, (int)a.M, a.N, (int)a.K, a.y, a.acc,
+                      a.mode, a.ep);
 }
 
 // Independent calls: a narrow grid of about 32 CTAs streaming runs of strips
@@ -227,15 +240,12 @@ tq_status launch_gemv_stream(const int8_t *xq, const float *s_x, const int32_t *
 // steps per warp) keep several layers resident.  Otherwise, for K <= 4096,
 // the time after the wait is the critical path: twice the warps, two steps
 // each.  Larger K keeps the lean shape (16-warp CTAs measured slower).
-template <int NB, bool CONV>
-tq_status gemv_shape(const int8_t *xq, const float *s_x, const int32_t *rowsum, const uint8_t *packed,
-                     const float *gamma, int per_row, int64_t M, int64_t N, int64_t K, float *y,
-                     int32_t *acc, int mode, cudaStream_t st) {
-    const bool lean = (mode & kModeInputsReady) != 0;
-    if (K <= kGemvMaxK / 2)
-        return lean ? launch_gemv<NB, 4, 4, CONV>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st)
-                    : launch_gemv<NB, 8, 2, CONV>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
-    return launch_gemv<NB, 8, 4, CONV>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
+template <int NB, bool CONV, bool EPI>
+tq_status gemv_shape(const GemmArgs &a, cudaStream_t st) {
+    const bool lean = (a.mode & kModeInputsReady) != 0;
+    if (a.K <= kGemvMaxK / 2)
+        return lean ? launch_gemv<NB, 4, 4, CONV, EPI>(a, st) : launch_gemv<NB, 8, 2, CONV, EPI>(a, st);
+    return launch_gemv<NB, 8, 4, CONV, EPI>(a, st);
 }
 
 template <int NW>
@@ -402,38 +412,34 @@ int gemm_tile_tokens(int64_t M, int64_t N, int sms) {
     return best;
 }
 
+template <bool CONV, bool EPI>
+tq_status contraction(const GemmArgs &a, int sms, cudaStream_t st) {
+    if (a.M <= 16 && a.K <= kGemvMaxK)
+        return a.M <= 8 ? gemv_shape<1, CONV, EPI>(a, st) : gemv_shape<2, CONV, EPI>(a, st);
+    switch (gemm_tile_tokens(a.M, a.N, sms)) {
+    case 64: return launch_gemm<64, CONV, EPI>(a, sms, st);
+    case 128: return launch_gemm<128, CONV, EPI>(a, sms, st);
+    case 192: return launch_gemm<192, CONV, EPI>(a, sms, st);
+    default: return launch_gemm<256, CONV, EPI>(a, sms, st);
+    }
+}
+
+// ep: the extra epilogue of tq_ternary_gemm_ex, or nullptr.
 tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsum,
                         const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
-                        int64_t N, int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st) {
+                        int64_t N, int64_t K, float *y, int32_t *acc, int sms, cudaStream_t st,
+                        const Epilogue *ep = nullptr) {
     const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
     const int enc = flag_encoding(flags);
     const int mode = ((flags & TQ_FLAG_WEIGHTS_STATIC) ? kModeWeightsStatic : 0) |
                      ((flags & TQ_FLAG_INPUTS_READY) ? kModeInputsReady : 0) | (enc << kModeEncShift);
-    if (M <= 16 && K <= kGemvMaxK) {
-        if ((mode & kModeInputsReady) && M <= 8 && K <= kStreamMaxK)
-            return launch_gemv_stream(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, enc, st);
-        if (enc != kEncFoundry) {
-            if (M <= 8) return gemv_shape<1, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
-            return gemv_shape<2, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
-        }
-        if (M <= 8) return gemv_shape<1, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
-        return gemv_shape<2, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, st);
-    }
-    const int bt = gemm_tile_tokens(M, N, sms);
-    if (enc != kEncFoundry) {
-        switch (bt) {
-        case 64: return launch_gemm<64, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-        case 128: return launch_gemm<128, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-        case 192: return launch_gemm<192, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-        default: return launch_gemm<256, true>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-        }
-    }
-    switch (bt) {
-    case 64: return launch_gemm<64, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    case 128: return launch_gemm<128, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    case 192: return launch_gemm<192, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    default: return launch_gemm<256, false>(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode, sms, st);
-    }
+    if (!ep && M <= 8 && K <= kStreamMaxK && (mode & kModeInputsReady))
+        return launch_gemv_stream(xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, enc, st);
+    const GemmArgs a{xq, s_x, rowsum, packed, gamma, per_row, M, N, K, y, acc, mode,
+                     ep ? *ep : Epilogue{nullptr, nullptr, 0}};
+    const bool conv = enc != kEncFoundry;
+    if (ep) return conv ? contraction<true, true>(a, sms, st) : contraction<false, true>(a, sms, st);
+    return conv ? contraction<true, false>(a, sms, st) : contraction<false, false>(a, sms, st);
 }
 
 }  // namespace
@@ -567,9 +573,26 @@ tq_status tq_fwht512(const float *x, float *y, int64_t rows, int64_t K, int norm
                       x, y, nblocks, normalize);
 }
 
-tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
-                          const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
-                          int64_t N, int64_t K, float *y, int32_t *acc, tq_stream_t stream) {
+tq_status tq_fwht_roundtrip(const float *x, float *y, int64_t rows, int64_t K, float eta_min,
+                            float eta_max, float *eta_out, tq_stream_t stream) {
+    if (!x || !y) return TQ_ERR_NULL;
+    if (rows < 1 || rows > INT32_MAX || K < 512 || K % 512 != 0 || K > kMaxFwhtFusedK) return TQ_ERR_SHAPE;
+    if (!(eta_min > 0.0f && eta_min <= eta_max && eta_max < 3.0e38f)) return TQ_ERR_ARG;
+    if (!aligned16(x) || !aligned16(y) || (eta_out && !aligned16(eta_out))) return TQ_ERR_ALIGN;
+    const size_t b = (size_t)(rows * K) * 4;
+    if (x != y && overlap(x, b, y, b)) return TQ_ERR_ARG;
+    if (eta_out && (overlap(eta_out, (size_t)rows * 4, x, b) || overlap(eta_out, (size_t)rows * 4, y, b)))
+        return TQ_ERR_ARG;
+    if (tq_status e = check_device(nullptr)) return e;
+    return launch_pdl(fwht_roundtrip_kernel, dim3((unsigned)rows), dim3((unsigned)(K / 512 * 32)), 0, cs(stream),
+                      x, y, eta_min, eta_max, eta_out);
+}
+
+// Shared body of tq_ternary_gemm and tq_ternary_gemm_ex (ep: the extra epilogue or nullptr).
+static tq_status gemm_impl(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                           const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
+                           int64_t N, int64_t K, float *y, int32_t *acc, tq_stream_t stream,
+                           const Epilogue *ep) {
     if (!xq || !s_x || !rowsum || !packed || !gamma || !y) return TQ_ERR_NULL;
     if (M < 1 || N < 1 || M > INT32_MAX || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
@@ -588,7 +611,27 @@ tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *row
     if (acc && overlap(acc, yb, y, yb)) return TQ_ERR_ARG;
     int sms = 0;
     if (tq_status e = check_device(&sms)) return e;
-    return gemm_dispatch(xq, s_x, rowsum, packed, gamma, flags, M, N, K, y, acc, sms, cs(stream));
+    return gemm_dispatch(xq, s_x, rowsum, packed, gamma, flags, M, N, K, y, acc, sms, cs(stream), ep);
+}
+
+tq_status tq_ternary_gemm(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                          const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
+                          int64_t N, int64_t K, float *y, int32_t *acc, tq_stream_t stream) {
+    return gemm_impl(xq, s_x, rowsum, packed, gamma, flags, M, N, K, y, acc, stream, nullptr);
+}
+
+tq_status tq_ternary_gemm_ex(const int8_t *xq, const float *s_x, const int32_t *rowsum,
+                             const uint8_t *packed, const float *gamma, unsigned flags, int64_t M,
+                             int64_t N, int64_t K, const float *bias, const int32_t *acc_bias,
+                             int out_shift, float *y, int32_t *acc, tq_stream_t stream) {
+    if (out_shift < 0 || out_shift > 31) return TQ_ERR_ARG;
+    if ((bias && !aligned16(bias)) || (acc_bias && !aligned16(acc_bias))) return TQ_ERR_ALIGN;
+    const size_t yb = (size_t)(M > 0 && N > 0 ? M * N : 0) * 4, nb = (size_t)(N > 0 ? N : 0) * 4;
+    if ((bias && (overlap(bias, nb, y, yb) || (acc && overlap(bias, nb, acc, yb)))) ||
+        (acc_bias && (overlap(acc_bias, nb, y, yb) || (acc && overlap(acc_bias, nb, acc, yb)))))
+        return TQ_ERR_ARG;
+    const Epilogue ep{bias, acc_bias, out_shift};
+    return gemm_impl(xq, s_x, rowsum, packed, gamma, flags, M, N, K, y, acc, stream, &ep);
 }
 
 size_t tq_fused_workspace_bytes(int64_t M, int64_t K, unsigned flags) {

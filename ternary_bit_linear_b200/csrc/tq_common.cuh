@@ -47,6 +47,15 @@ constexpr int kModeWeightsStatic = 1;
 constexpr int kModeInputsReady = 2;
 constexpr int kModeEncShift = 2;  // bits 2-3: packed-code layout (kEnc*, below)
 
+// Extra epilogue of a contraction (tq_ternary_gemm_ex): y gets + bias[n]
+// (Hetman-2b BitLinear's bias), the int32 accumulator output (acc + acc_bias[n])
+// >> shift (BitRASP's integer epilogue).  NULL pointers add nothing.
+struct Epilogue {
+    const float *bias;
+    const int32_t *acc_bias;
+    int shift;
+};
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -100,13 +100,14 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
 
 // CONV: the weights are packed in one of Hetman-2b's layouts (mode bits
 // 2-3) and every word is rewritten in Foundry's layout before the unpack; the
-// default layout compiles without that step.
-template <int BT, bool CONV>
+// default layout compiles without that step.  EPI: the extra epilogue `ep`
+// (bias, integer bias and shift) is applied.
+template <int BT, bool CONV, bool EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
                 const float *__restrict__ gamma, int per_row, int M, int N, int K,
-                float *__restrict__ y, int32_t *__restrict__ acc_out, int mode) {
+                float *__restrict__ y, int32_t *__restrict__ acc_out, int mode, Epilogue ep) {
     using L = GemmLayout<BT>;
     constexpr int S = L::kStages, SW = L::kWStages;
     extern __shared__ uint8_t smem_raw[];
@@ -298,6 +299,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int n = n0 + 32 * q + lane;
             // per-tile scalars, loaded while the accumulator is still being computed
             const float gn = n < N ? __ldg(gamma + (per_row ? n : 0)) : 0.0f;
+            const float bn = (EPI && n < N && ep.bias) ? __ldg(ep.bias + n) : 0.0f;
+            const int abn = (EPI && n < N && ep.acc_bias) ? __ldg(ep.acc_bias + n) : 0;
             float sxc[kChunks];
             int rsc[kChunks];
 #pragma unroll
@@ -327,8 +330,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int j = 0; j < 32; ++j) {
                         const float sxm = __shfl_sync(0xffffffffu, sxc[cc], j);
                         const int rsm = __shfl_sync(0xffffffffu, rsc[cc], j);
-                        v[j] = __float_as_uint(
-                            __fmul_rn(__int2float_rn((int)v[j] - rsm), __fmul_rn(gn, sxm)));
+                        const float yv = __fmul_rn(__int2float_rn((int)v[j] - rsm), __fmul_rn(gn, sxm));
+                        v[j] = __float_as_uint(EPI ? __fadd_rn(yv, bn) : yv);
                     }
                     if (n < N) {
                         float *yp = y + (int64_t)mb * N + n;
@@ -343,9 +346,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const int rsm = __shfl_sync(0xffffffffu, rsc[cc], j);
                         const int a = (int)v[j] - rsm;
                         if (j < jmax && n < N) {
-                            __stcs(y + (int64_t)(mb + j) * N + n,
-                                   __fmul_rn(__int2float_rn(a), __fmul_rn(gn, sxm)));
-                            __stcs(acc_out + (int64_t)(mb + j) * N + n, a);
+                            const float yv = __fmul_rn(__int2float_rn(a), __fmul_rn(gn, sxm));
+                            __stcs(y + (int64_t)(mb + j) * N + n, EPI ? __fadd_rn(yv, bn) : yv);
+                            __stcs(acc_out + (int64_t)(mb + j) * N + n, EPI ? (a + abn) >> ep.shift : a);
                         }
                     }
                 }

@@ -199,6 +199,7 @@ __device__ __forceinline__ void transpose_x(uint32_t x_s, int M, int K, int XS, 
 // NB: token blocks of 8 (M <= 8 * NB).  W: warps per CTA.  SPW: 64-byte
 // column steps per warp (K <= 256 * W * SPW).  CONV: weights in one of
 // Hetman-2b's layouts (mode bits 2-3), rewritten in Foundry's as they are used.
+// EPI: the extra epilogue `ep` (bias, integer bias and shift) is applied.
 //
 // mode & kModeWeightsStatic: the packed weights and gamma are not written by
 // work still in flight on the stream, so they are requested before the
@@ -208,12 +209,12 @@ __device__ __forceinline__ void transpose_x(uint32_t x_s, int M, int K, int XS, 
 // One CTA (the last) waits for the previous kernel before it exits, so this
 // kernel still completes after its predecessor and later work sees the
 // stream's results in order; the other CTAs leave as soon as they are done.
-template <int NB, int W, int SPW, bool CONV>
+template <int NB, int W, int SPW, bool CONV, bool EPI>
 __global__ void __launch_bounds__(W * 32, gemv_min_blocks(NB, W))
     gemv_kernel(const int8_t *__restrict__ xq, const float *__restrict__ s_x,
                 const int32_t *__restrict__ rowsum, const uint8_t *__restrict__ packed,
                 const float *__restrict__ gamma, int per_row, int M, int64_t N, int K,
-                float *__restrict__ y, int32_t *__restrict__ acc_out, int mode) {
+                float *__restrict__ y, int32_t *__restrict__ acc_out, int mode, Epilogue ep) {
     constexpr int CH = 8 / SPW;                              // independent MMA chains
     constexpr int FPT = (128 * NB + W * 32 - 1) / (W * 32);  // outputs finished per thread
     extern __shared__ __align__(128) uint8_t dsm[];
@@ -229,14 +230,19 @@ __global__ void __launch_bounds__(W * 32, gemv_min_blocks(NB, W))
     const bool ready = (mode & kModeInputsReady) != 0;
     const bool early_w = (mode & (kModeWeightsStatic | kModeInputsReady)) != 0;
 
-    float gv[FPT], sxv[FPT];
-    int rsv[FPT];
-    auto load_gamma = [&]() {
+    float gv[FPT], sxv[FPT], bv[FPT];
+    int rsv[FPT], abv[FPT];
+    auto load_gamma = [&]() {  // and, with EPI, the row's biases
 #pragma unroll
         for (int q = 0; q < FPT; ++q) {
             const int e = threadIdx.x + q * W * 32;
             const int64_t n = r0 + fin_row(e);
-            gv[q] = (e < 128 * NB && n < N) ? __ldg(gamma + (per_row ? n : 0)) : 0.0f;
+            const bool ok = e < 128 * NB && n < N;
+            gv[q] = ok ? __ldg(gamma + (per_row ? n : 0)) : 0.0f;
+            if (EPI) {
+                bv[q] = (ok && ep.bias) ? __ldg(ep.bias + n) : 0.0f;
+                abv[q] = (ok && ep.acc_bias) ? __ldg(ep.acc_bias + n) : 0;
+            }
         }
     };
     auto load_tok = [&]() {
@@ -291,8 +297,9 @@ __global__ void __launch_bounds__(W * 32, gemv_min_blocks(NB, W))
             for (int ww = 0; ww < W; ++ww) tot += red[ww][(e >> 7) * 4 + ((e >> 5) & 3)][e & 31];
             if (m < M && n < N) {
                 const int a = tot - rsv[q];
-                y[(int64_t)m * N + n] = __fmul_rn(__int2float_rn(a), __fmul_rn(gv[q], sxv[q]));
-                if (acc_out) acc_out[(int64_t)m * N + n] = a;
+                const float v = __fmul_rn(__int2float_rn(a), __fmul_rn(gv[q], sxv[q]));
+                y[(int64_t)m * N + n] = EPI ? __fadd_rn(v, bv[q]) : v;
+                if (acc_out) acc_out[(int64_t)m * N + n] = EPI ? (a + abv[q]) >> ep.shift : a;
             }
         }
     }

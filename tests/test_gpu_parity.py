@@ -773,3 +773,69 @@ def test_pack_threshold_boundaries_and_layout(cuda_lib):
             tq.quantize_ternary_pack_threshold_(dev(W), tq.GAMMA_PER_ROW | (layout << 7), ratio, packed, gamma)
             assert np.array_equal(host(packed), p_ref), (ratio, layout)
             assert np.array_equal(host(gamma), g_ref)
+
+
+# ---------------------------------------------------------------------------
+# NEXT row N2: the FWHT module's quantisation round trip (Hetman-2b section 1,
+# FastWalshHadamardTransform.forward) and the contraction's extra epilogues
+# (BitLinear bias; BitRASP's integer bias + arithmetic shift).
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("rows,K", [(1, 512), (7, 1536), (300, 4096), (3, 16384)])
+def test_fwht_roundtrip_bit_exact(cuda_lib, rows, K):
+    tq = cuda_lib
+    X = S.student_t3((rows, K), 97, rows)
+    X[0, 5] = np.nan
+    X[-1, 9] = np.inf
+    X[-1, 11] = -np.inf
+    y_ref, eta_ref = oracle.fwht_roundtrip(X, 0.05, 40.0)
+    x = dev(X)
+    y = torch.empty_like(x)
+    eta = torch.empty((rows,), dtype=torch.float32, device="cuda")
+    tq.fwht_roundtrip_(x, y, 0.05, 40.0, eta)
+    assert np.array_equal(host(y), y_ref)
+    assert np.array_equal(host(eta), eta_ref)
+    tq.fwht_roundtrip_(x, x, 0.05, 40.0)  # in place
+    assert np.array_equal(host(x), y_ref)
+
+
+def test_fwht_roundtrip_gain_clamp_both_ends(cuda_lib):
+    tq = cuda_lib
+    X = np.zeros((3, 1024), np.float32)
+    X[1, 0] = 1000.0  # rotates above eta_max
+    X[2] = S.normal((1, 1024), 1e-4, 98, 1)[0]  # eta below eta_min
+    for lo, hi in ((0.05, 40.0), (0.5, 2.0)):
+        y_ref, eta_ref = oracle.fwht_roundtrip(X, lo, hi)
+        x = dev(X)
+        y = torch.empty_like(x)
+        eta = torch.empty((3,), dtype=torch.float32, device="cuda")
+        tq.fwht_roundtrip_(x, y, lo, hi, eta)
+        assert np.array_equal(host(y), y_ref) and np.array_equal(host(eta), eta_ref)
+        assert host(eta)[1] == np.float32(hi) and host(eta)[0] == np.float32(lo)
+
+
+@pytest.mark.parametrize("M,N,K,layout", [(1, 300, 4096, 0), (8, 129, 1088, 1), (16, 64, 8192, 0),
+                                          (64, 256, 1024, 2), (300, 384, 1536, 0)])
+def test_gemm_ex_bias_and_integer_epilogue(cuda_lib, M, N, K, layout):
+    tq = cuda_lib
+    W = S.normal((N, K), 0.02, 99, N)
+    X = S.decode_acts(M, K, seed=100)
+    p_ref, g_ref = oracle.quantize_pack(W, per_row=True, encoding=layout)
+    xq_ref, sx_ref, rs_ref = oracle.act_quant(X)
+    acc_ref = oracle.matmul_addsub_format(xq_ref, p_ref, layout)
+    rng = np.random.default_rng(101)
+    bias = (rng.standard_normal(N) * 0.3).astype(np.float32)
+    abias = rng.integers(-5000, 5000, N).astype(np.int32)
+    for shift in (0, 3):
+        ins = [dev(a) for a in (xq_ref, sx_ref, rs_ref, p_ref, g_ref)]
+        bd, abd = dev(bias), dev(abias)
+        y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+        tq.ternary_gemm_ex_(*ins, tq.GAMMA_PER_ROW | (layout << 7), y, acc, bd, abd, shift)
+        assert np.array_equal(host(acc), oracle.int_epilogue(acc_ref, abias, shift))
+        y_ref = oracle.dequant_bias(acc_ref, g_ref, sx_ref, True, bias)
+        y0 = np.abs(oracle.dequant(acc_ref, g_ref, sx_ref, True).astype(np.float64))
+        # two fp32 roundings (product, then the sum) against one: within 1e-5 of the
+        # terms' magnitude, not of a possibly cancelled sum
+        err = np.abs(host(y).astype(np.float64) - y_ref.astype(np.float64))
+        assert np.all(err <= REL * (y0 + np.abs(bias)[None, :]) + 1e-30)
+    assert tq.device_status() == 0
