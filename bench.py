@@ -158,10 +158,11 @@ class ClockSampler:
 class Workload:
     """Builds device buffers and the per-segment launch lists of one step."""
 
-    def __init__(self, name, tq, S, torch, dev, layers, layout=0, ratio=0.0):
+    def __init__(self, name, tq, S, torch, dev, layers, layout=0, ratio=0.0, bias=False):
         self.name, self.tq, self.torch, self.dev = name, tq, torch, dev
         f32, u8, i8, i32 = torch.float32, torch.uint8, torch.int8, torch.int32
         self.segments = []  # (label, kernel_name, launches, algorithmic bytes or ops, [fns])
+        self.bias = None
         self.chains = []    # (label, launches, bytes per launch, [fns]): dependent-layer GEMV chains
         if name == "decode":
             N = K = 4096
@@ -193,6 +194,20 @@ class Workload:
             W = torch.from_numpy(S.sweep_weights(N, K, seed=0))
             self.W = [W.to(dev) for _ in range(self.L)]
             self.X = {M: torch.from_numpy(S.sweep_acts(M, K, seed=0)) for M in self.Ms}
+        elif name == "roundtrip":
+            # the FWHT module's int8 round trip on the fused configuration's activations
+            M, K = 512, 2048
+            self.N, self.K, self.Ms, self.L = 0, K, [M], layers
+            self.per_row = False
+            self.layout, self.ratio = layout, ratio
+            X = torch.from_numpy(S.fused(M, 16, K, seed=0)[1])
+            self.X = {M: X}
+            self.Xd = {M: [X.to(dev) for _ in range(layers)]}
+            self.yr = [torch.empty((M, K), dtype=torch.float32, device=dev) for _ in range(layers)]
+            self.y = {M: self.yr}
+            self.segments.append(("fwht roundtrip", "roundtrip", layers, layers * 8 * M * K, layers, [
+                lambda l=l: tq.fwht_roundtrip_(self.Xd[M][l], self.yr[l], 0.05, 40.0) for l in range(layers)]))
+            return
         else:
             raise SystemExit(f"unknown workload {name}")
         N, K, L = self.N, self.K, self.L
@@ -246,15 +261,23 @@ class Workload:
             lambda M=M, l=l: tq.quantize_act_int8_(self.Xd[M][l], tq.FLAG_INPUTS_READY, 0.05, 40.0,
                                                    self.xq[M][l], self.sx[M][l], self.rs[M][l])
             for M in self.Ms for l in range(L)]))
+        self.bias = [torch.full((N,), 0.25, dtype=f32, device=dev) for _ in range(L)] if bias else None
         for M in self.Ms:
             gemv = M <= 16
             work = (N * K // 4 + 4 * N * (1 if self.per_row else 0) + M * K + 8 * M + 4 * M * N) if gemv \
                 else 2 * M * N * K
+            if bias:  # the extra epilogue (y + bias[n]) through tq_ternary_gemm_ex
+                fns = [lambda l=l, M=M: tq.ternary_gemm_ex_(self.xq[M][l], self.sx[M][l], self.rs[M][l],
+                                                            self.packed[l], self.gamma[l], self.ready_flags,
+                                                            self.y[M][l], bias=self.bias[l])
+                       for l in range(L)]
+            else:
+                fns = [lambda l=l, M=M: tq.ternary_gemm_(self.xq[M][l], self.sx[M][l], self.rs[M][l],
+                                                         self.packed[l], self.gamma[l], self.ready_flags,
+                                                         self.y[M][l])
+                       for l in range(L)]
             self.segments.append(("gemv M=%d" % M if gemv else "gemm M=%d" % M,
-                                  "gemv" if gemv else "gemm", L, L * work, L, [
-                lambda l=l, M=M: tq.ternary_gemm_(self.xq[M][l], self.sx[M][l], self.rs[M][l], self.packed[l],
-                                                  self.gamma[l], self.ready_flags, self.y[M][l])
-                for l in range(L)]))
+                                  "gemv" if gemv else "gemm", L, L * work, L, fns))
             if gemv:
                 self.chains.append(("gemv M=%d" % M, L, work, [
                     lambda l=l, M=M: tq.ternary_gemm_(self.xq[M][l], self.sx[M][l], self.rs[M][l],
@@ -263,7 +286,7 @@ class Workload:
                     for l in range(L)]))
 
     def step_bytes(self):
-        return sum(s[3] for s in self.segments if s[1] in ("pack", "act_quant", "gemv"))
+        return sum(s[3] for s in self.segments if s[1] in ("pack", "act_quant", "gemv", "roundtrip"))
 
     def step_ops(self):
         return sum(s[3] for s in self.segments if s[1] in ("gemm", "fused"))
@@ -282,7 +305,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     tq.load()
     wl = Workload(args.workload, tq, S, torch, dev, args.layers or WORKLOAD_SHAPES[args.workload][3],
-                  LAYOUTS.index(args.layout), args.ratio)
+                  LAYOUTS.index(args.layout), args.ratio, args.bias)
     stream = torch.cuda.Stream(device=dev)
     graphs = []
     with torch.cuda.stream(stream):
@@ -357,7 +380,7 @@ def run_ours(args, rank, world, local_rank):
                 "traffic": traffic_for(dom[1] + ":" + args.workload), "kernel": dom[0],
                 "peak_source": pk["source"] + (" hbm_gbs (copy, burst)" if dk["bound"] == "hbm"
                                                else " bf16_tflops x2 (nominal int8/bf16 ratio)")}
-    if wl.name in ("decode",):
+    if wl.name in ("decode", "roundtrip"):
         value = wl.step_bytes() * world / (ms_per_step * 1e-3) / 1e9
         unit = "GB/s"
     else:
@@ -389,29 +412,32 @@ WORKLOAD_SHAPES = {  # name -> (Ms, N, K, default ring of layers, per_row)
     "prefill": ([2048], 11008, 4096, 4, False),
     "fused": ([512], 5632, 2048, 8, False),
     "sweep": ([1, 4, 16, 64, 512, 4096], 8192, 8192, 8, True),
+    "roundtrip": ([512], 0, 2048, 64, False),
 }
 
 
 LAYOUTS = ["foundry", "format0", "format1"]  # packed-code layouts, flag value = index << 7
 
 
-def config_for(name, layers, world, layout="foundry", ratio=0.0):
+def config_for(name, layers, world, layout="foundry", ratio=0.0, bias=False):
     Ms, N, K, L, per_row = WORKLOAD_SHAPES[name]
     L = layers or L
     desc = {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers" % L,
             "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma, ring of %d layers" % L,
             "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512, ring of %d layers" % L,
-            "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L}[name]
+            "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L,
+            "roundtrip": "FWHT module int8 round trip: 512 x 2048 Student-t(3), ring of %d batches" % L}[name]
     return {"workload": desc, "M": Ms, "N": N, "K": K, "layers": L,
             "gamma": "per-row" if per_row else "per-tensor", "layout": layout,
             "ternarise": "threshold w > %g * gamma" % ratio if ratio > 0 else "round/clamp",
+            "epilogue": "y + bias (tq_ternary_gemm_ex)" if bias else "y",
             "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
                 L * N * K * 4 >> 20, L * N * K // 4 >> 20),
             "parallelism": "replicas x%d" % world if world > 1 else "single GPU"}
 
 
 def wl_config(wl, world):
-    return config_for(wl.name, wl.L, world, LAYOUTS[wl.layout], wl.ratio)
+    return config_for(wl.name, wl.L, world, LAYOUTS[wl.layout], wl.ratio, wl.bias is not None)
 
 
 def run_chains(args, wl, tq, torch, stream, world):
@@ -482,7 +508,7 @@ def run_e2e(args, wl, tq, torch, stream, graphs, world):
         t1.record(stream)
     torch.cuda.synchronize()
     ms = allreduce_max(t0.elapsed_time(t1), world) / steps
-    if wl.name == "decode":
+    if wl.name in ("decode", "roundtrip"):
         v, u = wl.step_bytes() * world / (ms * 1e-3) / 1e9, "GB/s"
     else:
         v, u = wl.step_ops() * world / (ms * 1e-3) / 1e12, "TOPS"
@@ -511,6 +537,14 @@ def oracle_sample(workload):
         work = (4 * N * K + N * K // 4 + 4 * N) + sum(
             4 * M * K + M * K + 8 * M + N * K // 4 + 4 * N + M * K + 8 * M + 4 * M * N for M in (1, 8))
         return fn, work, "one full layer of the step (pack 4096x4096 per-row, act-quant + GEMV for M=1 and M=8)", "GB/s"
+    if workload == "roundtrip":
+        M, K = 512, 2048
+        X = S.fused(M, 16, K, seed=0)[1]
+        rows = 64
+
+        def fn():
+            oracle.fwht_roundtrip(X[:rows])
+        return fn, 8 * rows * K, "%d of the 512 rows of one batch" % rows, "GB/s"
     if workload in ("prefill", "fused", "sweep"):
         if workload == "prefill":
             M, N, K, per_row = 2048, 11008, 4096, False
@@ -599,7 +633,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fused", "sweep"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fused", "sweep", "roundtrip"])
+    ap.add_argument("--bias", action="store_true",
+                    help="contractions through tq_ternary_gemm_ex with a bias (the extra epilogue)")
     ap.add_argument("--ratio", type=float, default=0.0,
                     help="threshold ternarisation w > ratio * gamma (0: the round/clamp rule)")
     ap.add_argument("--layout", default="foundry", choices=LAYOUTS,
