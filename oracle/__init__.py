@@ -61,6 +61,7 @@ def _load():
         _lib.tqo_dequant_bias.argtypes = [P, P, I, P, P, I64, I64, P]
         _lib.tqo_int_epilogue.argtypes = [P, P, I, I64, I64, P]
         _lib.tqo_fwht_roundtrip.argtypes = [P, I64, I64, F, F, P, P]
+        _lib.tqo_swiglu_act.argtypes = [P, P, I64, F, P]
         _lib.tqo_ternary_codes_threshold.argtypes = [P, I64, I64, P, I, F, P]
         _lib.tqo_pack_format.argtypes = [P, I64, I64, I, P]
         _lib.tqo_unpack_format.argtypes = [P, I64, I64, I, P]
@@ -325,3 +326,25 @@ def bitlinear(x, packed, gamma, per_row: bool, rms_gain=None, rms_eps: float = 1
                           y.ctypes.data_as(ctypes.c_void_p), xq.ctypes.data_as(ctypes.c_void_p),
                           sx.ctypes.data_as(ctypes.c_void_p), acc.ctypes.data_as(ctypes.c_void_p))
     return y, xq, sx, acc
+
+
+def swiglu_act(gate, up, clamp_val: float = 10.0):
+    gate, pg = _c(gate, np.float32)
+    up, pu = _c(up, np.float32)
+    assert gate.shape == up.shape
+    out = np.empty_like(gate)
+    _load().tqo_swiglu_act(pg, pu, gate.size, float(clamp_val), out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def swiglu_mlp(x, gate, up, down, per_row: bool, clamp_val: float = 10.0, use_rmsnorm: bool = True,
+               use_fwht: bool = True):
+    """Hetman-2b section 6 SwiGLUClamped.forward with three BitLinear layers
+    (each: bitlinear above) on pre-packed (packed, gamma) pairs.  Returns
+    (y, activated-and-clamped, x_q of the down projection)."""
+    kw = dict(use_rmsnorm=use_rmsnorm, use_fwht=use_fwht)
+    yg = bitlinear(x, gate[0], gate[1], per_row, **kw)[0]
+    yu = bitlinear(x, up[0], up[1], per_row, **kw)[0]
+    act = swiglu_act(yg, yu, clamp_val)
+    y, xq, _, _ = bitlinear(act, down[0], down[1], per_row, **kw)
+    return y, act, xq, yg, yu

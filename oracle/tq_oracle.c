@@ -485,6 +485,21 @@ void tqo_int_epilogue(const int32_t *acc, const int32_t *bias, int out_shift, in
         }
 }
 
+/* [H] section 6 SwiGLUClamped.forward, between the projections:
+ *   activated = SiLU(gate) * up,  SiLU(v) = v * sigmoid(v) = v / (1 + e^-v),
+ *   clamped   = clamp(activated, -clamp_val, +clamp_val)   (10.0 on the page).
+ * Computed in fp64 and rounded once to fp32. */
+void tqo_swiglu_act(const float *gate, const float *up, int64_t n, float clamp_val, float *out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        double g = (double)gate[i];
+        double a = g / (1.0 + exp(-g)) * (double)up[i];
+        if (a > (double)clamp_val) a = (double)clamp_val;
+        if (a < -(double)clamp_val) a = -(double)clamp_val;
+        out[i] = (float)a;
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Prologue: quench, RMSNorm, FWHT-512                                        */
 /* ------------------------------------------------------------------------ */

@@ -421,6 +421,37 @@ def test_int_epilogue_hand_worked():
         assert out[0, 0] == want, ln
 
 
+def test_swiglu_act_closed_forms_and_clamp():
+    # Hetman-2b section 6 SwiGLUClamped: clamp(SiLU(gate) * up, -10, 10).
+    # sigmoid(ln 3) = 3/4 exactly; SiLU(v) - SiLU(-v) = v; SiLU(0) = 0.
+    ln3 = math.log(3.0)
+    a = oracle.swiglu_act(np.array([0.0, ln3], np.float32), np.array([1.0, 1.0], np.float32))
+    assert a[0] == 0.0
+    assert abs(float(a[1]) - 0.75 * float(np.float32(ln3))) <= 2e-7
+    v = S.normal((1, 257), 2.0, 23, 1)[0]
+    ones = np.ones_like(v)
+    diff = oracle.swiglu_act(v, ones, 1e6).astype(np.float64) - oracle.swiglu_act(-v, ones, 1e6).astype(np.float64)
+    assert np.all(np.abs(diff - v.astype(np.float64)) <= 3e-7 * np.maximum(1.0, np.abs(v)))
+    # the clamp bounds both signs; it is the last step (large gate, opposite signs)
+    big = oracle.swiglu_act(np.array([10.0, 5.0, 50.0], np.float32), np.array([10.0, -5.0, 0.1], np.float32))
+    assert big[0] == 10.0 and big[1] == -10.0 and abs(float(big[2]) - 5.0) < 1e-5
+    assert np.array_equal(oracle.swiglu_act(np.array([3.0], np.float32), np.array([1.0], np.float32), 1.5),
+                          np.array([1.5], np.float32))
+
+
+def test_swiglu_mlp_is_the_composition():
+    # gate and up see the same x; the down projection sees the clamped activation
+    M, d, f = 3, 512, 1024
+    X = S.student_t3((M, d), 24, M)
+    packs = [oracle.quantize_pack(S.normal(shape, 0.02, 25 + i, shape[0]), per_row=False)
+             for i, shape in enumerate([(f, d), (f, d), (d, f)])]
+    y, act, xq, yg, yu = oracle.swiglu_mlp(X, packs[0], packs[1], packs[2], per_row=False)
+    assert np.array_equal(yg, oracle.bitlinear(X, *packs[0], False)[0])
+    assert np.array_equal(act, oracle.swiglu_act(yg, yu))
+    assert np.abs(act).max() <= 10.0
+    assert np.array_equal(y, oracle.bitlinear(act, *packs[2], False)[0])
+
+
 # --------------------------------------------------------------------------
 # FWHT-512
 # --------------------------------------------------------------------------
