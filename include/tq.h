@@ -308,6 +308,31 @@ TQ_API tq_status tq_fwht_roundtrip(const float *x, float *y, int64_t rows, int64
                                    float eta_max, float *eta_out, tq_stream_t stream);
 
 /*
+ * Clamped SwiGLU feed-forward block of three BitLinear layers.  Hetman-2b
+ * section 6, SwiGLUClamped.forward: gate = SiLU(W_gate(x)), up = W_up(x),
+ * y = W_down(clamp(gate * up, -clamp_val, +clamp_val)) (clamp_val 10 on the
+ * page), every W_* a BitLinear as in tq_bitlinear_fused (with TQ_FLAG_FWHT,
+ * which is required here, and TQ_FLAG_RMSNORM if given, eps 1e-6, unit gain).
+ *
+ *   x          [M][d_model] fp32.  d_model, d_ffn multiples of 512, at most 16384.
+ *   gate_*, up_*   packed [d_ffn][d_model/4] and gamma; down_* packed
+ *              [d_model][d_ffn/4] and gamma (all per row with TQ_GAMMA_PER_ROW,
+ *              in the layout the flags name).
+ *   y          [M][d_model] fp32, written.
+ *   act_out    [M][d_ffn] fp32 or NULL: the clamped activation.
+ *   workspace  tq_swiglu_workspace_bytes(M, d_model, d_ffn, flags) bytes.
+ * flags: TQ_FLAG_FWHT (required), TQ_FLAG_RMSNORM, TQ_GAMMA_PER_ROW,
+ * TQ_FLAG_SANITIZE_NONFINITE, TQ_FLAG_WEIGHTS_STATIC, TQ_ENC_*.  SiLU is
+ * computed in fp32 (v / (1 + e^-v)), within a few ulp of its exact value.
+ */
+TQ_API tq_status tq_swiglu_mlp(const float *x, int64_t M, int64_t d_model, int64_t d_ffn, unsigned flags,
+                               float clamp_val, const uint8_t *gate_packed, const float *gate_gamma,
+                               const uint8_t *up_packed, const float *up_gamma, const uint8_t *down_packed,
+                               const float *down_gamma, float *y, float *act_out, void *workspace,
+                               size_t workspace_bytes, tq_stream_t stream);
+TQ_API size_t tq_swiglu_workspace_bytes(int64_t M, int64_t d_model, int64_t d_ffn, unsigned flags);
+
+/*
  * Waits for `stream`, then returns and clears the current device's status word:
  * TQ_OK, or TQ_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the
  * last call.  TQ_ERR_CUDA if the synchronisation itself failed.

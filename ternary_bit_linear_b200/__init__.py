@@ -49,6 +49,8 @@ SIGNATURES = {
     "tq_bitlinear_fused": (_I, [_P, _P, _F, _F, _F, _U, _P, _P, _I64, _I64, _I64, _P, _P, _P,
                                 _P, _SZ, _P]),
     "tq_fused_workspace_bytes": (_SZ, [_I64, _I64, _U]),
+    "tq_swiglu_mlp": (_I, [_P, _I64, _I64, _I64, _U, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tq_swiglu_workspace_bytes": (_SZ, [_I64, _I64, _I64, _U]),
     "tq_get_device_status": (_I, [_P]),
     "tq_status_string": (ctypes.c_char_p, [_I]),
     "tq_version": (_I, []),
@@ -224,6 +226,28 @@ def fwht_roundtrip_(x, y, eta_min=0.05, eta_max=40.0, eta_out=None, stream=None)
     _check("tq_fwht_roundtrip",
            load().tq_fwht_roundtrip(_ptr(x), _ptr(y), rows, K, float(eta_min), float(eta_max), _ptr(eta_out),
                                     _stream(stream)))
+
+
+def swiglu_workspace_bytes(M: int, d_model: int, d_ffn: int, flags: int) -> int:
+    return int(load().tq_swiglu_workspace_bytes(M, d_model, d_ffn, flags))
+
+
+def swiglu_mlp_(x, gate, up, down, flags, y, workspace, clamp_val=10.0, act_out=None, stream=None):
+    """gate, up, down: (packed, gamma) pairs."""
+    import torch
+
+    M, D = x.shape
+    F = gate[0].shape[0]
+    _need(x, torch.float32, (M, D), "x")
+    _need(y, torch.float32, (M, D), "y")
+    _need(act_out, torch.float32, (M, F), "act_out")
+    _need(gate[0], torch.uint8, (F, D // 4), "gate packed")
+    _need(up[0], torch.uint8, (F, D // 4), "up packed")
+    _need(down[0], torch.uint8, (D, F // 4), "down packed")
+    _check("tq_swiglu_mlp",
+           load().tq_swiglu_mlp(_ptr(x), M, D, F, flags, float(clamp_val), _ptr(gate[0]), _ptr(gate[1]),
+                                _ptr(up[0]), _ptr(up[1]), _ptr(down[0]), _ptr(down[1]), _ptr(y), _ptr(act_out),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def device_status(stream=None) -> int:

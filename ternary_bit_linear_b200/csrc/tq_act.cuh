@@ -439,6 +439,97 @@ __global__ void __launch_bounds__(1024)
 }
 
 // ---------------------------------------------------------------------------
+// Between the projections of Hetman-2b's clamped SwiGLU (section 6,
+// SwiGLUClamped.forward), fused with the down projection's activation pass:
+// a = clamp(SiLU(gate) * up, +-clamp_val) (SiLU(v) = v / (1 + e^-v), fp32),
+// then [quench] -> [RMSNorm] -> FWHT-512 -> per-token int8, as
+// prologue_fwht_kernel.  One CTA per token, one warp per 512-block
+// (K = 512 * blockDim.x / 32).  act_out (or NULL) receives a.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float swiglu_one(float g, float u, float c) {
+    const float a = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+    return fminf(fmaxf(a, -c), c);
+}
+
+__global__ void __launch_bounds__(1024)
+    swiglu_prologue_kernel(const float *__restrict__ gate, const float *__restrict__ up, float clamp_val,
+                           ActParams p, int8_t *__restrict__ xq, float *__restrict__ s_x,
+                           int32_t *__restrict__ rowsum, float *__restrict__ act_out) {
+    __shared__ float redf[32];
+    __shared__ int redi[32];
+    __shared__ double redd[32];
+    pdl_wait();
+    pdl_trigger();
+    const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t K = 512 * (int64_t)nw;
+    const int64_t m = blockIdx.x;
+    const int64_t off = m * K + warp * 512;
+    float f[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 g = reinterpret_cast<const float4 *>(gate + off)[j * 32 + lane];
+        const float4 u = reinterpret_cast<const float4 *>(up + off)[j * 32 + lane];
+        float4 a = make_float4(swiglu_one(g.x, u.x, clamp_val), swiglu_one(g.y, u.y, clamp_val),
+                               swiglu_one(g.z, u.z, clamp_val), swiglu_one(g.w, u.w, clamp_val));
+        if (act_out) reinterpret_cast<float4 *>(act_out + off)[j * 32 + lane] = a;
+        if (p.sanitize)
+            a = make_float4(quench(a.x, p.eta_max), quench(a.y, p.eta_max), quench(a.z, p.eta_max),
+                            quench(a.w, p.eta_max));
+        f[4 * j + 0] = a.x;
+        f[4 * j + 1] = a.y;
+        f[4 * j + 2] = a.z;
+        f[4 * j + 3] = a.w;
+    }
+    if (p.rmsnorm) {
+        double ss = 0.0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ss = __fma_rn((double)f[i], (double)f[i], ss);
+        ss = warp_sum_d(ss);
+        if (lane == 0) redd[warp] = ss;
+        __syncthreads();
+        ss = warp_sum_d(lane < nw ? redd[lane] : 0.0);
+        const double r =
+            __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)p.rms_eps)));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = warp * 512 + j * 128 + lane * 4 + e;
+                f[4 * j + e] = rms_apply(f[4 * j + e], r, p.rms_gain, k);
+            }
+    }
+    fwht512_regs(f, true);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = warp_max(amax);
+    if (lane == 0) redf[warp] = amax;
+    __syncthreads();
+    amax = warp_max(lane < nw ? redf[lane] : 0.0f);
+    const float eta = eta_of(amax, p);
+    const float scale = __fdiv_rn(127.0f, eta);
+    int sum = 0;
+    uint32_t *dst = reinterpret_cast<uint32_t *>(xq + off);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int a = quant_code(f[4 * j + 0], scale), b = quant_code(f[4 * j + 1], scale),
+                  c = quant_code(f[4 * j + 2], scale), d = quant_code(f[4 * j + 3], scale);
+        dst[j * 32 + lane] = pack_codes4(a, b, c, d);
+        sum += a + b + c + d;
+    }
+    sum = warp_sum_i(sum);
+    if (lane == 0) redi[warp] = sum;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        sum = warp_sum_i(lane < nw ? redi[lane] : 0);
+        if (lane == 0) {
+            s_x[m] = __fdiv_rn(eta, 127.0f);
+            rowsum[m] = sum;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Fused prologue of the whole layer: [quench] -> [RMSNorm] -> FWHT-512 ->
 // per-token int8.  One CTA per token, one warp per 512-block (K = 512 * NW).
 // ---------------------------------------------------------------------------

@@ -710,6 +710,100 @@ tq_status tq_bitlinear_fused(const float *x, const float *rms_gain, float rms_ep
     return gemm_dispatch(xq, sx, rs, packed, gamma, cflags, M, N, K, y, nullptr, sms, st);
 }
 
+// Workspace of tq_swiglu_mlp: the first projection's x_q, s_x, rowsum; the
+// gate and up outputs; the down projection's x_q, s_x, rowsum (each 256-byte
+// aligned).
+static size_t swiglu_parts(int64_t M, int64_t D, int64_t F, size_t off[8]) {
+    auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
+    const size_t sz[8] = {al((size_t)(M * D)), al((size_t)M * 4), al((size_t)M * 4), al((size_t)(M * F) * 4),
+                          al((size_t)(M * F) * 4), al((size_t)(M * F)), al((size_t)M * 4), al((size_t)M * 4)};
+    size_t t = 0;
+    for (int i = 0; i < 8; ++i) {
+        off[i] = t;
+        t += sz[i];
+    }
+    return t;
+}
+
+size_t tq_swiglu_workspace_bytes(int64_t M, int64_t d_model, int64_t d_ffn, unsigned flags) {
+    (void)flags;
+    if (M <= 0 || d_model <= 0 || d_ffn <= 0) return 0;
+    size_t off[8];
+    return swiglu_parts(M, d_model, d_ffn, off);
+}
+
+tq_status tq_swiglu_mlp(const float *x, int64_t M, int64_t d_model, int64_t d_ffn, unsigned flags,
+                        float clamp_val, const uint8_t *gate_packed, const float *gate_gamma,
+                        const uint8_t *up_packed, const float *up_gamma, const uint8_t *down_packed,
+                        const float *down_gamma, float *y, float *act_out, void *workspace,
+                        size_t workspace_bytes, tq_stream_t stream) {
+    if (!x || !gate_packed || !gate_gamma || !up_packed || !up_gamma || !down_packed || !down_gamma || !y ||
+        !workspace)
+        return TQ_ERR_NULL;
+    if (M < 1 || M > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(d_model)) return e;
+    if (tq_status e = check_k(d_ffn)) return e;
+    if (d_model % 512 || d_ffn % 512 || d_model > kMaxFwhtFusedK || d_ffn > kMaxFwhtFusedK) return TQ_ERR_SHAPE;
+    const unsigned known = TQ_GAMMA_PER_ROW | TQ_FLAG_FWHT | TQ_FLAG_RMSNORM | TQ_FLAG_SANITIZE_NONFINITE |
+                           TQ_FLAG_WEIGHTS_STATIC | TQ_ENC_MASK;
+    if ((flags & ~known) || !(flags & TQ_FLAG_FWHT) || flag_encoding(flags) < 0) return TQ_ERR_ARG;
+    if (!(clamp_val > 0.0f && clamp_val < 3.0e38f)) return TQ_ERR_ARG;
+    const void *al16[10] = {x, gate_packed, gate_gamma, up_packed, up_gamma, down_packed, down_gamma, y, workspace,
+                            act_out};
+    for (const void *q : al16)
+        if (q && !aligned16(q)) return TQ_ERR_ALIGN;
+    size_t off[8];
+    const size_t need = swiglu_parts(M, d_model, d_ffn, off);
+    if (workspace_bytes < need) return TQ_ERR_ARG;
+    const size_t yb = (size_t)(M * d_model) * 4, ab = (size_t)(M * d_ffn) * 4;
+    const bool pr = flags & TQ_GAMMA_PER_ROW;
+    const void *ins[7] = {x, gate_packed, gate_gamma, up_packed, up_gamma, down_packed, down_gamma};
+    const size_t inb[7] = {yb, (size_t)(d_ffn * d_model / 4), (pr ? (size_t)d_ffn : 1) * 4,
+                           (size_t)(d_ffn * d_model / 4), (pr ? (size_t)d_ffn : 1) * 4,
+                           (size_t)(d_model * d_ffn / 4), (pr ? (size_t)d_model : 1) * 4};
+    const void *outs[3] = {y, workspace, act_out};
+    const size_t outb[3] = {yb, need, ab};
+    for (int o = 0; o < 3; ++o) {
+        if (!outs[o]) continue;
+        for (int i = 0; i < 7; ++i)
+            if (overlap(outs[o], outb[o], ins[i], inb[i])) return TQ_ERR_ARG;
+        for (int o2 = o + 1; o2 < 3; ++o2)
+            if (outs[o2] && overlap(outs[o], outb[o], outs[o2], outb[o2])) return TQ_ERR_ARG;
+    }
+    int sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    cudaStream_t st = cs(stream);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    int8_t *xq1 = reinterpret_cast<int8_t *>(ws + off[0]);
+    float *sx1 = reinterpret_cast<float *>(ws + off[1]);
+    int32_t *rs1 = reinterpret_cast<int32_t *>(ws + off[2]);
+    float *yg = reinterpret_cast<float *>(ws + off[3]);
+    float *yu = reinterpret_cast<float *>(ws + off[4]);
+    int8_t *xq2 = reinterpret_cast<int8_t *>(ws + off[5]);
+    float *sx2 = reinterpret_cast<float *>(ws + off[6]);
+    int32_t *rs2 = reinterpret_cast<int32_t *>(ws + off[7]);
+    ActParams p{};
+    p.sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
+    p.eta_max = 40.0f;  // the quench bound of Hetman-2b's BitLinear (step 0)
+    p.eta_min = 0.05f;
+    p.rmsnorm = (flags & TQ_FLAG_RMSNORM) ? 1 : 0;
+    p.rms_eps = 1e-6f;
+    const unsigned cflags = flags & (TQ_GAMMA_PER_ROW | TQ_FLAG_WEIGHTS_STATIC | TQ_ENC_MASK);
+    // gate and up see the same x: one activation pass for both
+    Prologues::fns[d_model / 512 - 1](x, p, M, xq1, sx1, rs1, st);
+    if (tq_status e = launch_status()) return e;
+    if (tq_status e = gemm_dispatch(xq1, sx1, rs1, gate_packed, gate_gamma, cflags, M, d_ffn, d_model, yg,
+                                    nullptr, sms, st))
+        return e;
+    if (tq_status e = gemm_dispatch(xq1, sx1, rs1, up_packed, up_gamma, cflags, M, d_ffn, d_model, yu, nullptr,
+                                    sms, st))
+        return e;
+    if (tq_status e = launch_pdl(swiglu_prologue_kernel, dim3((unsigned)M), dim3((unsigned)(d_ffn / 512 * 32)), 0,
+                                 st, (const float *)yg, (const float *)yu, clamp_val, p, xq2, sx2, rs2, act_out))
+        return e;
+    return gemm_dispatch(xq2, sx2, rs2, down_packed, down_gamma, cflags, M, d_model, d_ffn, y, nullptr, sms, st);
+}
+
 tq_status tq_get_device_status(tq_stream_t stream) {
     if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return TQ_ERR_CUDA;
     unsigned v = 0, zero = 0;

@@ -839,3 +839,36 @@ def test_gemm_ex_bias_and_integer_epilogue(cuda_lib, M, N, K, layout):
         err = np.abs(host(y).astype(np.float64) - y_ref.astype(np.float64))
         assert np.all(err <= REL * (y0 + np.abs(bias)[None, :]) + 1e-30)
     assert tq.device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# NEXT row N3: Hetman-2b's clamped SwiGLU block of three BitLinear layers.
+# gate/up projections within 1e-5 (through the clamped activation, compared
+# to the oracle's within a few ulp of SiLU's fp32 evaluation); the block's
+# output equals the fused layer run on its own activation, which in turn is
+# checked against the oracle with the fused path's rule.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,D,F,per_row", [(5, 512, 1024, False), (64, 1536, 6144, False), (33, 1024, 2048, True)])
+def test_swiglu_mlp(cuda_lib, M, D, F, per_row):
+    tq = cuda_lib
+    X = S.student_t3((M, D), 110, M)
+    Ws = [S.normal(shape, 0.02, 111 + i, shape[0]) for i, shape in enumerate([(F, D), (F, D), (D, F)])]
+    packs = [oracle.quantize_pack(W, per_row=per_row) for W in Ws]
+    y_ref, act_ref, _, yg_ref, yu_ref = oracle.swiglu_mlp(X, packs[0], packs[1], packs[2], per_row)
+    fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM | (tq.GAMMA_PER_ROW if per_row else 0)
+    dp = [(dev(p), dev(g)) for p, g in packs]
+    y = torch.empty((M, D), dtype=torch.float32, device="cuda")
+    act = torch.empty((M, F), dtype=torch.float32, device="cuda")
+    ws = torch.empty((tq.swiglu_workspace_bytes(M, D, F, fl),), dtype=torch.uint8, device="cuda")
+    tq.swiglu_mlp_(dev(X), dp[0], dp[1], dp[2], fl, y, ws, 10.0, act)
+    act_h = host(act)
+    assert np.abs(act_h).max() <= 10.0
+    err = np.abs(act_h.astype(np.float64) - act_ref.astype(np.float64))
+    assert np.all(err <= 2e-5 * np.abs(act_ref.astype(np.float64)) + 1e-6)
+    # the down projection: the fused layer on the block's own activation, bit for bit
+    y_chk = torch.empty_like(y)
+    fws = torch.empty((tq.fused_workspace_bytes(M, F, fl),), dtype=torch.uint8, device="cuda")
+    tq.bitlinear_fused_(act, dp[2][0], dp[2][1], fl, y_chk, fws)
+    assert torch.equal(y, y_chk)
+    check_fused(tq, act_h, Ws[2], per_row)
+    assert tq.device_status() == 0
