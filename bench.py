@@ -194,6 +194,37 @@ class Workload:
             W = torch.from_numpy(S.sweep_weights(N, K, seed=0))
             self.W = [W.to(dev) for _ in range(self.L)]
             self.X = {M: torch.from_numpy(S.sweep_acts(M, K, seed=0)) for M in self.Ms}
+        elif name == "mlp":
+            # Hetman-2b's clamped SwiGLU block: d_model 1536, d_ffn 4 * 1536, 512 tokens
+            M, D, F = 512, 1536, 6144
+            self.N, self.K, self.Ms, self.L = D, D, [M], layers
+            self.per_row = False
+            self.layout, self.ratio = layout, ratio
+            fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM | (layout << 7)
+            X = torch.from_numpy(S.fused(M, 16, D, seed=0)[1])
+            shapes = [(F, D), (F, D), (D, F)]
+            Wf = [torch.from_numpy(S.normal(sh, 0.02, 7 + i, sh[0])) for i, sh in enumerate(shapes)]
+            self.W3 = [[w.to(dev) for w in Wf] for _ in range(layers)]
+            self.P3 = [[(torch.empty((sh[0], sh[1] // 4), dtype=torch.uint8, device=dev),
+                         torch.empty((1,), dtype=torch.float32, device=dev)) for sh in shapes] for _ in range(layers)]
+            wsz = max(tq.pack_workspace_bytes(sh[0], sh[1], 0) for sh in shapes)
+            self.pws3 = [torch.empty((wsz,), dtype=torch.uint8, device=dev) for _ in range(layers)]
+            self.X = {M: X}
+            self.Xd = {M: [X.to(dev) for _ in range(layers)]}
+            self.y = {M: [torch.empty((M, D), dtype=torch.float32, device=dev) for _ in range(layers)]}
+            self.mws = [torch.empty((tq.swiglu_workspace_bytes(M, D, F, fl),), dtype=torch.uint8, device=dev)
+                        for _ in range(layers)]
+            pack_bytes = sum(4 * a * b + a * b // 4 + 4 for a, b in shapes)
+            self.segments.append(("pack", "pack", 3 * layers, layers * pack_bytes, 6 * layers, [
+                lambda l=l, i=i: tq.quantize_ternary_pack_(self.W3[l][i], (layout << 7), self.P3[l][i][0],
+                                                          self.P3[l][i][1], self.pws3[l])
+                for l in range(layers) for i in range(3)]))
+            ops = 2 * M * 3 * D * F
+            self.segments.append(("mlp M=%d" % M, "mlp", layers, layers * ops, 5 * layers, [
+                lambda l=l: tq.swiglu_mlp_(self.Xd[M][l], self.P3[l][0], self.P3[l][1], self.P3[l][2],
+                                           fl | tq.FLAG_WEIGHTS_STATIC, self.y[M][l], self.mws[l])
+                for l in range(layers)]))
+            return
         elif name == "roundtrip":
             # the FWHT module's int8 round trip on the fused configuration's activations
             M, K = 512, 2048
@@ -237,7 +268,7 @@ class Workload:
 
         # --- segments of one step ---
         pack_bytes = 4 * N * K + N * K // 4 + 4 * (N if self.per_row else 1)
-        pack_launches = 1 if self.per_row else 3
+        pack_launches = 1 if self.per_row else 2  # per tensor: partial sums, then the pack pass
         if ratio > 0:  # threshold ternarisation (w > ratio * gamma) instead of round/clamp
             pack_fns = [lambda l=l: tq.quantize_ternary_pack_threshold_(
                 self.W[l], self.flags | tq.FLAG_INPUTS_READY, ratio, self.packed[l], self.gamma[l], self.pack_ws[l])
@@ -289,7 +320,7 @@ class Workload:
         return sum(s[3] for s in self.segments if s[1] in ("pack", "act_quant", "gemv", "roundtrip"))
 
     def step_ops(self):
-        return sum(s[3] for s in self.segments if s[1] in ("gemm", "fused"))
+        return sum(s[3] for s in self.segments if s[1] in ("gemm", "fused", "mlp"))
 
 
 def run_ours(args, rank, world, local_rank):
@@ -362,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
     kernels = {}
     for (label, kname, launches, work, nlaunch, _), ms in zip(wl.segments, seg_ms):
         per_launch_ms = ms / args.steps / launches
-        if kname in ("gemm", "fused"):
+        if kname in ("gemm", "fused", "mlp"):
             ach = work / launches / (per_launch_ms * 1e-3) / 1e12
             peak = pk["bf16"] * INT8_OVER_BF16
             kernels[label] = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
@@ -413,6 +444,7 @@ WORKLOAD_SHAPES = {  # name -> (Ms, N, K, default ring of layers, per_row)
     "fused": ([512], 5632, 2048, 8, False),
     "sweep": ([1, 4, 16, 64, 512, 4096], 8192, 8192, 8, True),
     "roundtrip": ([512], 0, 2048, 64, False),
+    "mlp": ([512], 1536, 1536, 8, False),
 }
 
 
@@ -426,7 +458,8 @@ def config_for(name, layers, world, layout="foundry", ratio=0.0, bias=False):
             "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma, ring of %d layers" % L,
             "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512, ring of %d layers" % L,
             "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L,
-            "roundtrip": "FWHT module int8 round trip: 512 x 2048 Student-t(3), ring of %d batches" % L}[name]
+            "roundtrip": "FWHT module int8 round trip: 512 x 2048 Student-t(3), ring of %d batches" % L,
+            "mlp": "clamped SwiGLU block of 3 BitLinears: 512 tokens, d_model 1536, d_ffn 6144, ring of %d" % L}[name]
     return {"workload": desc, "M": Ms, "N": N, "K": K, "layers": L,
             "gamma": "per-row" if per_row else "per-tensor", "layout": layout,
             "ternarise": "threshold w > %g * gamma" % ratio if ratio > 0 else "round/clamp",
@@ -537,6 +570,16 @@ def oracle_sample(workload):
         work = (4 * N * K + N * K // 4 + 4 * N) + sum(
             4 * M * K + M * K + 8 * M + N * K // 4 + 4 * N + M * K + 8 * M + 4 * M * N for M in (1, 8))
         return fn, work, "one full layer of the step (pack 4096x4096 per-row, act-quant + GEMV for M=1 and M=8)", "GB/s"
+    if workload == "mlp":
+        M, D, F = 512, 1536, 6144
+        X = S.fused(M, 16, D, seed=0)[1]
+        shapes = [(F, D), (F, D), (D, F)]
+        packs = [oracle.quantize_pack(S.normal(sh, 0.02, 7 + i, sh[0]), per_row=False) for i, sh in enumerate(shapes)]
+        rows = 2
+
+        def fn():
+            oracle.swiglu_mlp(X[:rows], packs[0], packs[1], packs[2], False)
+        return fn, 2 * rows * 3 * D * F, "%d tokens through the block (weights pre-packed)" % rows, "TOPS"
     if workload == "roundtrip":
         M, K = 512, 2048
         X = S.fused(M, 16, K, seed=0)[1]
@@ -633,7 +676,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fused", "sweep", "roundtrip"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill", "fused", "sweep", "roundtrip", "mlp"])
     ap.add_argument("--bias", action="store_true",
                     help="contractions through tq_ternary_gemm_ex with a bias (the extra epilogue)")
     ap.add_argument("--ratio", type=float, default=0.0,
