@@ -73,6 +73,13 @@ def _load():
         _lib.tqo_sanitize_acts.argtypes = [P, I64, F, P]
         _lib.tqo_rmsnorm.argtypes = [P, P, I64, I64, F, P]
         _lib.tqo_fwht512.argtypes = [P, P, I64, I64, I]
+        U64P = ctypes.POINTER(ctypes.c_uint64)
+        _lib.tqo_backward_input.argtypes = [P, P, I, P, I, P, I, I64, I64, I64, P]
+        _lib.tqo_ste_backward.argtypes = [P, P, P, I, F, I, I64, I64, P]
+        _lib.tqo_xorshift64.argtypes = [U64P]
+        _lib.tqo_xorshift64.restype = ctypes.c_uint64
+        _lib.tqo_seed.argtypes = [U64P, ctypes.c_uint64]
+        _lib.tqo_stochastic_flip.argtypes = [P, I, P, F, I64, I64, U64P]
         _lib.tqo_bitlinear.argtypes = [P, P, F, I, I, I, I, F, F, P, P, I, I64, I64, I64,
                                        P, P, P, P]
     return _lib
@@ -348,3 +355,62 @@ def swiglu_mlp(x, gate, up, down, per_row: bool, clamp_val: float = 10.0, use_rm
     act = swiglu_act(yg, yu, clamp_val)
     y, xq, _, _ = bitlinear(act, down[0], down[1], per_row, **kw)
     return y, act, xq, yg, yu
+
+
+# ---------------------------------------------------------------------------
+# Training: gradient through the layer, STE, stochastic flip (tq_oracle.c)
+# ---------------------------------------------------------------------------
+def backward_input(dY, packed, gamma, per_row: bool, K: int, row_scale=None, dX_in=None, encoding: int = 0):
+    """dX [M, K] float32 = (dX_in or 0) + row_scale[m] * sum_n fp32(dY[m, n] * gamma_n) * q[n, k]
+    (Foundry fq_matmul_ternary_backward_input)."""
+    dY, pd = _c(dY, np.float32)
+    M, N = dY.shape
+    packed, pp = _c(packed, np.uint8)
+    assert packed.shape == (N, K // 4)
+    g, pg = _c(np.atleast_1d(gamma), np.float32)
+    pr = None
+    if row_scale is not None:
+        row_scale, pr = _c(row_scale, np.float32)
+    dX = np.zeros((M, K), np.float32) if dX_in is None else np.array(dX_in, dtype=np.float32, order="C", copy=True)
+    _load().tqo_backward_input(pd, pp, int(encoding), pg, int(per_row), pr, int(dX_in is not None), M, N, K,
+                               dX.ctypes.data_as(ctypes.c_void_p))
+    return dX
+
+
+def ste_backward(grad, w, gamma, per_row: bool, tau: float = 1.0, sanitize: bool = False):
+    """Hetman-2b AbsmeanWeightQuantizer.backward: (grad / gamma) * (1 or 0.1)."""
+    grad, pgr = _c(grad, np.float32)
+    w, pw = _c(w, np.float32)
+    N, K = w.shape
+    assert grad.shape == w.shape
+    g, pg = _c(np.atleast_1d(gamma), np.float32)
+    out = np.empty_like(w)
+    _load().tqo_ste_backward(pgr, pw, pg, int(per_row), float(tau), int(sanitize), N, K,
+                             out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def seed(value: int) -> int:
+    st = ctypes.c_uint64(0)
+    _load().tqo_seed(ctypes.byref(st), ctypes.c_uint64(value))
+    return st.value
+
+
+def xorshift64(state: int, count: int = 1):
+    """Returns (list of `count` outputs, state after them)."""
+    st = ctypes.c_uint64(state)
+    out = [_load().tqo_xorshift64(ctypes.byref(st)) for _ in range(count)]
+    return out, st.value
+
+
+def stochastic_flip(packed, grad, temperature: float, state: int, encoding: int = 0):
+    """Foundry fq_ternary_stochastic_flip on a copy of `packed`.  Returns
+    (new packed, state after the N*K draws)."""
+    grad, pgr = _c(grad, np.float32)
+    N, K = grad.shape
+    out = np.array(packed, dtype=np.uint8, order="C", copy=True)
+    assert out.shape == (N, K // 4)
+    st = ctypes.c_uint64(state)
+    _load().tqo_stochastic_flip(out.ctypes.data_as(ctypes.c_void_p), int(encoding), pgr, float(temperature),
+                                N, K, ctypes.byref(st))
+    return out, st.value

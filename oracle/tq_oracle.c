@@ -13,12 +13,15 @@
  *   [F]  Foundry, docs/quantization.md -- "Ternary Format / Encoding" and
  *        "Ternary Quantization (BitNet b1.58) / How It Works" (absmean gamma,
  *        round+clamp, 00=-1 01=0 10=+1 packing four per byte LSB-first,
- *        add/subtract/skip matmul scaled by gamma).
+ *        add/subtract/skip matmul scaled by gamma); "Ternary Training
+ *        (Backward Pass + Stochastic Flip)" (backward_input, xorshift64
+ *        stochastic flip, seed).
  *   [H]  Hetman-2b, src/quantization.py -- section 1 (FWHT B=512: nine
  *        butterfly stages h = 1..256, then 1/sqrt(512)), section 2
  *        (AbsmeanWeightQuantizer.forward, SymmetricActivationQuantizer.forward),
  *        section 4 (SubLayerRMSNorm.forward), section 5 (BitLinear.forward
- *        steps 0-6), section 7 (simulate_hardware_bitnet_gemv).
+ *        steps 0-6), section 7 (simulate_hardware_bitnet_gemv); section 2
+ *        AbsmeanWeightQuantizer.backward (the STE) for training.
  *   [B]  BitRASP, core_math.py -- additive_ternary_linear_int8
  *        (y[o] = sum of x where W=+1 minus sum of x where W=-1).
  *
@@ -631,4 +634,124 @@ void tqo_bitlinear(const float *x, const float *rms_gain, float rms_eps, int use
     free(sx);
     free(xq);
     free(a);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Training: gradient through the layer, STE, stochastic flip               */
+/* ------------------------------------------------------------------------ */
+
+/* [F] "Ternary Training (Backward Pass + Stochastic Flip) / Backward Pass",
+ * fq_matmul_ternary_backward_input: the gradient of Y = scale * X W_ternary
+ * with respect to X, formed with the same unpacking as the forward and summed
+ * over the output features.  W is stored [N][K] here (row = output feature n),
+ * so, with scale_n = gamma_n (per row) or gamma_0 (per tensor),
+ *
+ *   g[m][n]  = fp32(dY[m][n] * scale_n)                 (one fp32 product)
+ *   dX[m][k] = fp32( (accumulate ? dX[m][k] : 0) + row_scale[m] * sum_n g[m][n] q[n][k] )
+ *
+ * The sum is taken in fp64 (terms are fp32 values times -1, 0 or +1) and the
+ * result rounded once.  accumulate = 1 is the page's "+=" (the caller zeroes
+ * d_input first); row_scale (NULL = 1) is the per-token factor of [H]
+ * section 5 BitLinear.forward step 6 (y_int32 * gamma / scale_x): the
+ * gradient reaching x_q there is dY * gamma * s_x W, which section 2's
+ * identity STE passes on unchanged. */
+void tqo_backward_input(const float *dY, const uint8_t *packed, int format, const float *gamma,
+                        int per_row, const float *row_scale, int accumulate, int64_t M, int64_t N,
+                        int64_t K, float *dX)
+{
+    int8_t *q = (int8_t *)malloc((size_t)(N * K));
+    double *s = (double *)malloc((size_t)K * sizeof(double));
+    tqo_unpack_format(packed, N, K, format, q);
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) s[k] = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            float sc = per_row ? gamma[n] : gamma[0];
+            float g = dY[m * N + n] * sc;
+            for (int64_t k = 0; k < K; ++k) s[k] += (double)g * (double)q[n * K + k];
+        }
+        double rs = row_scale ? (double)row_scale[m] : 1.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double v = rs * s[k];
+            if (accumulate) v += (double)dX[m * K + k];
+            dX[m * K + k] = (float)v;
+        }
+    }
+    free(s);
+    free(q);
+}
+
+/* [H] section 2, AbsmeanWeightQuantizer.backward.  The forward saved
+ * w_scaled = w / gamma (fp32, after the quarantine nan -> 0, +inf -> 1,
+ * -inf -> -1 when the weights held any); the gradient of the latent weights is
+ *
+ *   grad_w = (grad_w_ternary / gamma) * (|w_scaled| <= tau ? 1 : 0.1)
+ *
+ * every operation in fp32 as the page computes it (0.1 is the fp32 constant).
+ * gamma per tensor on the page; per row as the per-channel variant. */
+void tqo_ste_backward(const float *grad, const float *w, const float *gamma, int per_row, float tau,
+                      int sanitize, int64_t N, int64_t K, float *out)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        float gm = per_row ? gamma[n] : gamma[0];
+        for (int64_t k = 0; k < K; ++k) {
+            float wv = w[n * K + k];
+            if (sanitize) {
+                if (isnan(wv)) wv = 0.0f;
+                else if (isinf(wv)) wv = wv > 0 ? 1.0f : -1.0f;
+            }
+            float ws = wv / gm;
+            float damp = fabsf(ws) <= tau ? 1.0f : 0.1f;
+            float gw = grad[n * K + k] / gm;
+            out[n * K + k] = gw * damp;
+        }
+    }
+}
+
+/* [F] "Stochastic Weight Flip": the generator is xorshift64 on a 64-bit
+ * state the caller owns.  G. Marsaglia, "Xorshift RNGs", Journal of
+ * Statistical Software 8(14), 2003: the 64-bit generator with the shift
+ * triple (13, 7, 17) -- x ^= x << 13; x ^= x >> 7; x ^= x << 17 -- whose
+ * new state is also the output. */
+uint64_t tqo_xorshift64(uint64_t *state)
+{
+    uint64_t x = *state;
+    x ^= x << 13;
+    x ^= x >> 7;
+    x ^= x << 17;
+    *state = x;
+    return x;
+}
+
+/* [F] fq_seed.  The page does not say how the seed becomes the state; here
+ * the state is the seed itself, except that 0 (a fixed point of xorshift)
+ * becomes 0x9E3779B97F4A7C15. */
+void tqo_seed(uint64_t *state, uint64_t seed)
+{
+    *state = seed ? seed : 0x9E3779B97F4A7C15ull;
+}
+
+/* [F] fq_ternary_stochastic_flip, for every weight in storage order (row n,
+ * then k), one draw each:
+ *   x = xorshift64(state), u = (x >> 40) * 2^-24      (a uniform fp32 in [0, 1))
+ *   p = clamp(|grad| * temperature, 0, 1)              (fp32; NaN never flips)
+ *   if u < p: q = clamp(q - sign(grad), -1, 1)         (one step toward -grad)
+ * Codes are read and written in `format` (see tqo_pack_format); the state is
+ * left after the last draw. */
+void tqo_stochastic_flip(uint8_t *packed, int format, const float *grad, float temperature,
+                         int64_t N, int64_t K, uint64_t *state)
+{
+    int8_t *q = (int8_t *)malloc((size_t)(N * K));
+    tqo_unpack_format(packed, N, K, format, q);
+    for (int64_t i = 0; i < N * K; ++i) {
+        uint64_t x = tqo_xorshift64(state);
+        float u = (float)(x >> 40) * 0x1p-24f;
+        float a = fabsf(grad[i]) * temperature;
+        float p = a > 1.0f ? 1.0f : a; /* a >= 0 or NaN; NaN stays NaN and u < NaN is false */
+        if (u < p) {
+            int c = q[i] - (grad[i] > 0.0f ? 1 : (grad[i] < 0.0f ? -1 : 0));
+            q[i] = (int8_t)(c > 1 ? 1 : (c < -1 ? -1 : c));
+        }
+    }
+    tqo_pack_format(q, N, K, format, packed);
+    free(q);
 }

@@ -589,3 +589,233 @@ def test_bitlinear_float_gemm_parity_1536():
     q, _ = oracle.unpack(packed, 1536)
     y_float = (xq.astype(np.float32) @ q.T.astype(np.float32)) * (g[0] / (np.float32(127.0) / (sx * np.float32(127.0))))
     assert np.abs(y_float - y).max() < 1e-4
+
+
+# --------------------------------------------------------------------------
+# training: gradient through the layer, STE, stochastic flip
+# --------------------------------------------------------------------------
+
+def _codes_by_table(packed, K):
+    """Foundry's code table applied byte by byte (independent of the oracle's unpack)."""
+    tab = {0b00: -1, 0b01: 0, 0b10: 1}
+    N = packed.shape[0]
+    q = np.empty((N, K), np.int64)
+    for n in range(N):
+        for j in range(K // 4):
+            b = int(packed[n, j])
+            for i in range(4):
+                q[n, 4 * j + i] = tab[(b >> (2 * i)) & 3]
+    return q
+
+
+def test_backward_input_adjoint_identity_exact():
+    # <dX, x_q> = <dY * gamma, x_q W^T> exactly: small integers, a power-of-two
+    # gamma, so every sum is exact.  A transposed operand, a dropped term or a
+    # wrong sign breaks it (N != K).
+    rng = np.random.default_rng(21)
+    M, N, K = 5, 7, 64
+    q = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    packed = oracle.pack(q)
+    xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    dY = rng.integers(-8, 9, (M, N)).astype(np.float32)
+    for per_row, gamma in ((False, np.float32(0.25)), (True, np.float32(2.0) ** rng.integers(-3, 3, N))):
+        gamma = np.atleast_1d(gamma).astype(np.float32)
+        dX = oracle.backward_input(dY, packed, gamma, per_row, K)
+        acc = oracle.matmul_addsub(xq, packed).astype(np.float64)
+        g = gamma.astype(np.float64) if per_row else np.full(N, float(gamma[0]))
+        lhs = float(np.sum(dX.astype(np.float64) * xq.astype(np.float64)))
+        rhs = float(np.sum(dY.astype(np.float64) * g[None, :] * acc))
+        assert lhs == rhs
+
+
+def test_backward_input_closed_forms():
+    M, N, K = 3, 5, 64
+    dY = np.arange(1, M * N + 1, dtype=np.float32).reshape(M, N) / np.float32(8)
+    # all weights +1: every input feature receives the row sum of dY * gamma
+    ones = oracle.pack(np.ones((N, K), np.int8))
+    dX = oracle.backward_input(dY, ones, np.float32(0.5), False, K)
+    assert np.all(dX == (dY.sum(axis=1) * np.float32(0.5))[:, None])
+    # one-hot dY picks one weight row, scaled by its gamma
+    rng = np.random.default_rng(22)
+    q = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    gam = np.array([0.5, 0.25, 2.0, 1.0, 4.0], np.float32)
+    onehot = np.zeros((1, N), np.float32)
+    onehot[0, 3] = 3.0
+    dX = oracle.backward_input(onehot, oracle.pack(q), gam, True, K)
+    assert np.array_equal(dX[0], (3.0 * 1.0 * q[3]).astype(np.float32))
+    # zero gradient gives zero; the accumulate form adds to what is there
+    assert np.all(oracle.backward_input(np.zeros((M, N), np.float32), oracle.pack(q), gam, True, K) == 0)
+    base = np.full((M, K), 1.5, np.float32)
+    acc = oracle.backward_input(dY, ones, np.float32(0.5), False, K, dX_in=base)
+    assert np.all(acc == (dY.sum(axis=1) * np.float32(0.5))[:, None] + np.float32(1.5))
+
+
+def test_backward_input_matches_library_matmul_and_rounds_once():
+    rng = np.random.default_rng(23)
+    M, N, K = 6, 37, 128
+    q = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    packed = oracle.pack(q)
+    dY = rng.standard_normal((M, N)).astype(np.float32)
+    gam = (rng.random(N).astype(np.float32) + np.float32(0.5)).astype(np.float32)
+    rs = (rng.random(M).astype(np.float32) * np.float32(0.01)).astype(np.float32)
+    dX = oracle.backward_input(dY, packed, gam, True, K, row_scale=rs)
+    g = (dY * gam[None, :]).astype(np.float32).astype(np.float64)  # one fp32 product per term
+    ref = (g @ _codes_by_table(packed, K).astype(np.float64)) * rs.astype(np.float64)[:, None]
+    assert np.array_equal(dX, ref.astype(np.float32))
+    # the same codes in Hetman-2b's layouts give the same gradient
+    for enc in (1, 2):
+        assert np.array_equal(oracle.backward_input(dY, oracle.pack_format(q, enc), gam, True, K,
+                                                    row_scale=rs, encoding=enc), dX)
+
+
+def test_ste_backward_closed_forms():
+    one_tenth = np.float32(0.1)
+    cases = [  # w, gamma, tau, grad, sanitize -> expected (exact rational, rounded once to fp32 where noted)
+        (0.25, 0.5, 1.0, 1.0, False, np.float32(2.0)),       # |w/gamma| = 0.5: inside, grad / gamma
+        (0.5, 0.5, 1.0, 1.0, False, np.float32(2.0)),        # |w/gamma| = tau exactly: inside (<=)
+        (-0.5, 0.5, 1.0, -1.0, False, np.float32(-2.0)),
+        (0.75, 0.5, 1.5, 3.0, False, np.float32(6.0)),       # 1.5 <= tau = 1.5
+        (float("nan"), 0.5, 1.0, -1.0, True, np.float32(-2.0)),   # quench nan -> 0: inside
+        (3.0, 3.0, 1.0, 1.0, False, f32_round_rational(Fraction(1, 3))),  # 1/3 rounded once
+    ]
+    for w, gm, tau, gr, san, want in cases:
+        got = oracle.ste_backward(np.array([[gr]], np.float32), np.array([[w]], np.float32), np.float32(gm),
+                                  False, tau, san)[0, 0]
+        assert got == want, (w, gm, tau, gr, san, got, want)
+    # outside the band the gradient is damped by the fp32 constant 0.1:
+    # fp32(fp32(grad / gamma) * fp32(0.1)), checked with exact rationals
+    t = Fraction(float(one_tenth))
+    outside = [(0.75, 0.5, 3.0, Fraction(6)), (-0.75, 0.5, 3.0, Fraction(6)),
+               (float("inf"), 0.5, 1.0, Fraction(2)),    # sanitised +inf -> 1: |1/0.5| = 2 > 1
+               (float("nan"), 0.5, 1.0, Fraction(2))]    # nan kept: |nan| <= tau is false
+    for w, gm, gr, quotient in outside:
+        san = math.isinf(w)
+        got = oracle.ste_backward(np.array([[gr]], np.float32), np.array([[w]], np.float32), np.float32(gm),
+                                  False, 1.0, san)[0, 0]
+        assert got == f32_round_rational(quotient * t), (w, got)
+    # the next float above tau * gamma leaves the band once the quotient rounds above tau
+    w = np.nextafter(np.float32(3.0), np.float32(4.0))
+    got = oracle.ste_backward(np.ones((1, 1), np.float32), np.array([[w]], np.float32), np.float32(3.0),
+                              False, 1.0)[0, 0]
+    assert got == f32_round_rational(Fraction(float(f32_round_rational(Fraction(1, 3)))) * t)
+
+
+def test_ste_backward_per_row_uses_row_gamma():
+    rng = np.random.default_rng(24)
+    w = rng.standard_normal((4, 64)).astype(np.float32)
+    gr = rng.standard_normal((4, 64)).astype(np.float32)
+    gam = np.array([0.5, 1.0, 2.0, 0.25], np.float32)
+    got = oracle.ste_backward(gr, w, gam, True)
+    for n in range(4):
+        assert np.array_equal(got[n], oracle.ste_backward(gr[n:n + 1], w[n:n + 1], gam[n], False)[0])
+
+
+def test_xorshift64_worked_steps():
+    # seed 1 worked by hand from the (13, 7, 17) definition:
+    #   1 ^ 1<<13 = 0x2001;  ^ >>7 -> 0x2041;  ^ <<17 -> 0x40822041
+    #   0x40822041 ^ <<13: 0x81044082000 ^ 0x40822041 = 0x810048A0041
+    #   ^ >>7: 0x810048A0041 ^ 0x1020091400 = 0x80024831441
+    #   ^ <<17: 0x1000490628820000 ^ 0x80024831441 = 0x100041060C011441
+    out, st = oracle.xorshift64(1, 2)
+    assert out == [0x40822041, 0x100041060C011441] and st == out[-1]
+    assert oracle.seed(1) == 1 and oracle.seed(0) != 0
+    assert oracle.xorshift64(0, 3)[0] == [0, 0, 0]  # why seed 0 is mapped away
+
+
+def _gf2_columns(step):
+    return [step(1 << b) for b in range(64)]
+
+
+def _gf2_apply(cols, v):
+    r = 0
+    b = 0
+    while v:
+        if v & 1:
+            r ^= cols[b]
+        v >>= 1
+        b += 1
+    return r
+
+
+def _gf2_mul(a, b):
+    return [_gf2_apply(a, c) for c in b]
+
+
+def _gf2_pow(cols, e):
+    result = [1 << b for b in range(64)]
+    base = cols
+    while e:
+        if e & 1:
+            result = _gf2_mul(result, base)
+        base = _gf2_mul(base, base)
+        e >>= 1
+    return result
+
+
+def test_xorshift64_is_linear_with_maximal_period():
+    # Treat the oracle's step as a black box.  It must be linear over GF(2),
+    # and a generator of maximal period 2^64 - 1 has a transition matrix whose
+    # order is exactly 2^64 - 1 = 3 * 5 * 17 * 257 * 641 * 65537 * 6700417.
+    step = lambda v: oracle.xorshift64(v, 1)[1]
+    rng = np.random.default_rng(25)
+    for _ in range(20):
+        a, b = (int(x) for x in rng.integers(0, 2 ** 63, 2, dtype=np.uint64))
+        assert step(a ^ b) == step(a) ^ step(b)
+    cols = _gf2_columns(step)
+    ident = [1 << b for b in range(64)]
+    order = 2 ** 64 - 1
+    primes = [3, 5, 17, 257, 641, 65537, 6700417]
+    assert math.prod(primes) == order
+    assert _gf2_pow(cols, order) == ident
+    for p in primes:
+        assert _gf2_pow(cols, order // p) != ident, p
+
+
+def test_stochastic_flip_deterministic_limits():
+    rng = np.random.default_rng(26)
+    N, K = 6, 64
+    q = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    grad = rng.standard_normal((N, K)).astype(np.float32)
+    grad[0, :8] = 0.0
+    st0 = oracle.seed(7)
+    for enc in (0, 1, 2):
+        packed = oracle.pack_format(q, enc)
+        # temperature 0: nothing moves, yet one draw per weight was taken
+        out, st = oracle.stochastic_flip(packed, grad, 0.0, st0, enc)
+        assert np.array_equal(out, packed) and st == oracle.xorshift64(st0, N * K)[1]
+        # |grad| * T >= 1: every weight with a nonzero gradient steps toward -grad
+        out, _ = oracle.stochastic_flip(packed, grad, 1e9, st0, enc)
+        want = np.clip(q.astype(np.int64) - np.sign(grad).astype(np.int64), -1, 1)
+        assert np.array_equal(oracle.unpack_format(out, K, enc), want.astype(np.int8)), enc
+    # a NaN gradient never flips, an infinite one always does
+    g2 = np.zeros((1, 64), np.float32)
+    g2[0, 0], g2[0, 1] = np.nan, -np.inf
+    zero = oracle.pack(np.zeros((1, 64), np.int8))
+    out, _ = oracle.stochastic_flip(zero, g2, 0.5, st0)
+    codes = oracle.unpack(out, 64)[0][0]
+    assert codes[0] == 0 and codes[1] == 1 and np.all(codes[2:] == 0)
+
+
+def test_stochastic_flip_rate_and_stream_order():
+    # p = 0.3 everywhere on zero codes: the flipped fraction is binomial(n, 0.3)
+    N, K = 64, 1024
+    grad = np.full((N, K), 0.3, np.float32)
+    grad[::2] *= -1
+    zero = oracle.pack(np.zeros((N, K), np.int8))
+    out, st = oracle.stochastic_flip(zero, grad, 1.0, oracle.seed(11))
+    codes = oracle.unpack(out, K)[0].astype(np.int64)
+    moved = codes != 0
+    n = N * K
+    assert abs(moved.sum() - 0.3 * n) < 5 * math.sqrt(n * 0.3 * 0.7)
+    assert np.all(codes[moved] == -np.sign(grad[moved]))
+    # the draw of weight i is the (i+1)-th output: splitting the rows over two
+    # calls that carry the state gives the same codes
+    a, st_a = oracle.stochastic_flip(zero[:N // 3], grad[:N // 3], 1.0, oracle.seed(11))
+    b, st_b = oracle.stochastic_flip(zero[N // 3:], grad[N // 3:], 1.0, st_a)
+    assert np.array_equal(np.concatenate([a, b]), out) and st_b == st
+    # the comparison uses the top 24 bits of each output as u = (x >> 40) / 2^24
+    xs, _ = oracle.xorshift64(oracle.seed(11), 64)
+    g1 = np.full((1, 64), 0.5, np.float32)
+    out1, _ = oracle.stochastic_flip(oracle.pack(np.zeros((1, 64), np.int8)), g1, 1.0, oracle.seed(11))
+    want = np.array([-1 if (x >> 40) < (1 << 23) else 0 for x in xs], np.int8)
+    assert np.array_equal(oracle.unpack(out1, 64)[0][0], want)
