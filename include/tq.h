@@ -78,6 +78,7 @@ typedef enum tq_status {
 #define TQ_FLAG_SANITIZE_NONFINITE (1u << 4) /* quench NaN / +-Inf inputs first                */
 #define TQ_FLAG_WEIGHTS_STATIC (1u << 5)     /* see "Launch overlap" below                      */
 #define TQ_FLAG_INPUTS_READY (1u << 6)       /* see "Launch overlap" below                      */
+#define TQ_FLAG_ACCUMULATE (1u << 9)         /* tq_ternary_backward_input: dX += result         */
 
 /* Packed-code layout (flag bits 7-8; tq_quantize_ternary_pack[_noalloc],
  * tq_ternary_gemm, tq_bitlinear_fused).  Four codes per byte, LSB first.
@@ -331,6 +332,93 @@ TQ_API tq_status tq_swiglu_mlp(const float *x, int64_t M, int64_t d_model, int64
                                const float *down_gamma, float *y, float *act_out, void *workspace,
                                size_t workspace_bytes, tq_stream_t stream);
 TQ_API size_t tq_swiglu_workspace_bytes(int64_t M, int64_t d_model, int64_t d_ffn, unsigned flags);
+
+/* ------------------------------------------------------------------------
+ * Training
+ * ------------------------------------------------------------------------ */
+
+/*
+ * Gradient with respect to the layer input.  Foundry, docs/quantization.md,
+ * "Ternary Training (Backward Pass + Stochastic Flip) / Backward Pass",
+ * fq_matmul_ternary_backward_input: for the forward Y = scale * X W_ternary,
+ *
+ *   dX[m][k] = (TQ_FLAG_ACCUMULATE ? dX[m][k] : 0)
+ *            + row_scale[m] * sum_n fp32(dY[m][n] * gamma_n) * q[n][k]
+ *
+ * with the codes q of the packed weights [N][K/4] (the layout the flags
+ * name) and gamma_n = gamma[n] (TQ_GAMMA_PER_ROW) or gamma[0].  The page's
+ * "+=" form (caller zeroes d_input) is TQ_FLAG_ACCUMULATE.  row_scale (NULL
+ * = 1) is a per-token factor: Hetman-2b's BitLinear scales the contraction
+ * by gamma * s_x per token (section 5 step 6) and its activation STE passes
+ * the gradient of x_q on unchanged (section 2), so row_scale = s_x gives
+ * that gradient.  Each product g = fp32(dY * gamma) is split exactly into
+ * three bf16 parts and contracted on the tensor cores with fp32
+ * accumulation: every product is exact, the accumulation rounds in fp32
+ * (the result is within 1e-5 of sum_n |g q| of the exact sum).
+ *
+ *   dY         [M][N] fp32.          dX [M][K] fp32 (written, or updated).
+ *   workspace  tq_backward_input_workspace_bytes(M, N) bytes (three bf16
+ *              planes of dY * gamma), 16-byte aligned, owned by the caller.
+ * K % 64 == 0, 64 <= K <= 65536; N >= 1; 1 <= M <= 715827882.
+ * flags: TQ_GAMMA_PER_ROW, TQ_FLAG_ACCUMULATE, TQ_ENC_*.
+ * Errors: TQ_ERR_NULL, TQ_ERR_SHAPE, TQ_ERR_ALIGN (16 bytes), TQ_ERR_ARG
+ * (flags, workspace too small, any overlap between dX or the workspace and
+ * another buffer).
+ */
+TQ_API tq_status tq_ternary_backward_input(const float *dY, const uint8_t *packed, const float *gamma,
+                                           const float *row_scale, unsigned flags, int64_t M, int64_t N,
+                                           int64_t K, float *dX, void *workspace, size_t workspace_bytes,
+                                           tq_stream_t stream);
+TQ_API size_t tq_backward_input_workspace_bytes(int64_t M, int64_t N);
+
+/*
+ * Straight-through estimator of the latent weights.  Hetman-2b,
+ * src/quantization.py, section 2, AbsmeanWeightQuantizer.backward:
+ *
+ *   out[n][k] = (grad[n][k] / gamma_n) * (|w[n][k] / gamma_n| <= tau ? 1 : 0.1)
+ *
+ * in fp32 as written (IEEE division; 0.1 is the fp32 constant).  The page
+ * uses tau = 1 and one gamma per tensor; TQ_GAMMA_PER_ROW takes gamma[n].
+ * TQ_FLAG_SANITIZE_NONFINITE applies the forward's quarantine to w first
+ * (nan -> 0, +-inf -> +-1).
+ *
+ *   grad, w, out  [N][K] fp32; out may be grad or w (in place), no other overlap.
+ * K % 64 == 0, 64 <= K <= 65536; N >= 1; tau >= 0.
+ * Errors: TQ_ERR_NULL, TQ_ERR_SHAPE, TQ_ERR_ALIGN, TQ_ERR_ARG.
+ */
+TQ_API tq_status tq_ste_backward(const float *grad, const float *w, const float *gamma, int64_t N, int64_t K,
+                                 float tau, unsigned flags, float *out, tq_stream_t stream);
+
+/*
+ * Stochastic ternary flip (replaces the optimiser).  Foundry,
+ * docs/quantization.md, "Stochastic Weight Flip", fq_ternary_stochastic_flip:
+ * for every weight i in storage order (row n, then k), one draw each,
+ *
+ *   x = xorshift64(state)      (x ^= x << 13; x ^= x >> 7; x ^= x << 17)
+ *   u = (x >> 40) * 2^-24      (fp32, in [0, 1))
+ *   p = min(|grad_i| * temperature, 1)   (fp32; a NaN gradient never flips)
+ *   if u < p: q_i = clamp(q_i - sign(grad_i), -1, 1)
+ *
+ * packed [N][K/4] is updated in place in the layout the flags name (reserved
+ * fields read as 0).  rng_state is a HOST pointer to the caller's 64-bit
+ * state: the launch takes its value and the call advances it by N*K draws
+ * before returning (the kernel may still be running).  The draws are those
+ * of the sequential loop, bit for bit: each lane of the kernel starts its run
+ * at the right point of the stream by jumping ahead with powers of the
+ * generator's GF(2) matrix.  A CUDA graph that captures this call replays
+ * the draws of the captured state.
+ *
+ *   grad  [N][K] fp32, not overlapping packed.
+ * K % 64 == 0, 64 <= K <= 65536; N >= 1; N * K <= 2^40; 0 <= temperature < inf.
+ * flags: TQ_ENC_*.  Errors: TQ_ERR_NULL, TQ_ERR_SHAPE, TQ_ERR_ALIGN, TQ_ERR_ARG.
+ */
+TQ_API tq_status tq_ternary_stochastic_flip(uint8_t *packed, const float *grad, int64_t N, int64_t K,
+                                            float temperature, uint64_t *rng_state, unsigned flags,
+                                            tq_stream_t stream);
+
+/* fq_seed: state = seed, or 0x9E3779B97F4A7C15 for seed 0 (xorshift's fixed
+ * point).  The page leaves the mapping open.  Host only; NULL is ignored. */
+TQ_API void tq_seed(uint64_t *state, uint64_t seed);
 
 /*
  * Waits for `stream`, then returns and clears the current device's status word:

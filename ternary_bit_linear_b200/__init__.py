@@ -29,6 +29,7 @@ ENC_FOUNDRY = 0 << 7
 ENC_FORMAT0 = 1 << 7
 ENC_FORMAT1 = 2 << 7
 ENC_MASK = 3 << 7
+FLAG_ACCUMULATE = 1 << 9  # tq_ternary_backward_input: dX += result
 
 STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN", 4: "TQ_ERR_ARG",
           5: "TQ_ERR_CUDA", 6: "TQ_ERR_DEVICE", 7: "TQ_ERR_TIMEOUT"}
@@ -51,6 +52,11 @@ SIGNATURES = {
     "tq_fused_workspace_bytes": (_SZ, [_I64, _I64, _U]),
     "tq_swiglu_mlp": (_I, [_P, _I64, _I64, _I64, _U, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tq_swiglu_workspace_bytes": (_SZ, [_I64, _I64, _I64, _U]),
+    "tq_ternary_backward_input": (_I, [_P, _P, _P, _P, _U, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "tq_backward_input_workspace_bytes": (_SZ, [_I64, _I64]),
+    "tq_ste_backward": (_I, [_P, _P, _P, _I64, _I64, _F, _U, _P, _P]),
+    "tq_ternary_stochastic_flip": (_I, [_P, _P, _I64, _I64, _F, ctypes.POINTER(ctypes.c_uint64), _U, _P]),
+    "tq_seed": (None, [ctypes.POINTER(ctypes.c_uint64), ctypes.c_uint64]),
     "tq_get_device_status": (_I, [_P]),
     "tq_status_string": (ctypes.c_char_p, [_I]),
     "tq_version": (_I, []),
@@ -248,6 +254,59 @@ def swiglu_mlp_(x, gate, up, down, flags, y, workspace, clamp_val=10.0, act_out=
            load().tq_swiglu_mlp(_ptr(x), M, D, F, flags, float(clamp_val), _ptr(gate[0]), _ptr(gate[1]),
                                 _ptr(up[0]), _ptr(up[1]), _ptr(down[0]), _ptr(down[1]), _ptr(y), _ptr(act_out),
                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def backward_input_workspace_bytes(M: int, N: int) -> int:
+    return load().tq_backward_input_workspace_bytes(M, N)
+
+
+def ternary_backward_input_(dY, packed, gamma, flags, dX, workspace, row_scale=None, stream=None):
+    import torch
+
+    M, N = dY.shape
+    K = packed.shape[1] * 4
+    _need(dY, torch.float32, (M, N), "dY")
+    _need(packed, torch.uint8, (N, K // 4), "packed")
+    _need(gamma, torch.float32, (N if flags & GAMMA_PER_ROW else 1,), "gamma")
+    _need(row_scale, torch.float32, (M,), "row_scale")
+    _need(dX, torch.float32, (M, K), "dX")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("tq_ternary_backward_input",
+           load().tq_ternary_backward_input(_ptr(dY), _ptr(packed), _ptr(gamma), _ptr(row_scale), flags, M, N, K,
+                                            _ptr(dX), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ste_backward_(grad, w, gamma, flags, out, tau=1.0, stream=None):
+    import torch
+
+    N, K = w.shape
+    _need(grad, torch.float32, (N, K), "grad")
+    _need(w, torch.float32, (N, K), "w")
+    _need(gamma, torch.float32, (N if flags & GAMMA_PER_ROW else 1,), "gamma")
+    _need(out, torch.float32, (N, K), "out")
+    _check("tq_ste_backward", load().tq_ste_backward(_ptr(grad), _ptr(w), _ptr(gamma), N, K, float(tau), flags,
+                                                     _ptr(out), _stream(stream)))
+
+
+def seed(value: int) -> int:
+    """fq_seed: the xorshift64 state for `value`."""
+    st = ctypes.c_uint64(0)
+    load().tq_seed(ctypes.byref(st), ctypes.c_uint64(value))
+    return st.value
+
+
+def ternary_stochastic_flip_(packed, grad, temperature, state: int, flags=0, stream=None) -> int:
+    """Flips `packed` in place; returns the generator state after the N*K draws."""
+    import torch
+
+    N, K = grad.shape
+    _need(grad, torch.float32, (N, K), "grad")
+    _need(packed, torch.uint8, (N, K // 4), "packed")
+    st = ctypes.c_uint64(state)
+    _check("tq_ternary_stochastic_flip",
+           load().tq_ternary_stochastic_flip(_ptr(packed), _ptr(grad), N, K, float(temperature), ctypes.byref(st),
+                                             flags, _stream(stream)))
+    return st.value
 
 
 def device_status(stream=None) -> int:

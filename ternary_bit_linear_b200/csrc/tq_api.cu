@@ -17,6 +17,7 @@
 #include "tq_gemm.cuh"
 #include "tq_gemv.cuh"
 #include "tq_pack.cuh"
+#include "tq_train.cuh"
 
 namespace {
 
@@ -442,6 +443,94 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
     return conv ? contraction<true, false>(a, sms, st) : contraction<false, false>(a, sms, st);
 }
 
+
+// ---------------------------------------------------------------------------
+// Training helpers
+// ---------------------------------------------------------------------------
+// 2-D bf16 tensor [rows][cols] (row stride = 2 cols bytes), box [box_rows][box_cols].
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                    uint32_t box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row length of the bf16 planes of the backward pass: N rounded up to a step.
+inline int64_t bwd_plane_cols(int64_t N) { return (N + kBwdStepN - 1) / kBwdStepN * kBwdStepN; }
+
+// Host copies of the xorshift64 jump tables: the state after a flip call.
+const uint64_t kXsChunkHost[TQ_XS_CHUNK_BITS][64] = TQ_XS_CHUNK_INIT;
+const uint64_t kXsWarpHost[TQ_XS_WARPS][64] = TQ_XS_WARP_INIT;
+const uint64_t kXsLaneHost[64][32] = TQ_XS_LANE_INIT;
+
+inline uint64_t xs_apply(const uint64_t *cols, int stride, uint64_t x) {
+    uint64_t r = 0;
+    for (int b = 0; b < 64; ++b)
+        if ((x >> b) & 1ull) r ^= cols[b * stride];
+    return r;
+}
+
+// A^n x for n % 64 == 0, n < 2^40.
+uint64_t xs_jump(uint64_t x, int64_t n) {
+    const int64_t chunks = n / kFlipChunk;
+    int64_t rem = n % kFlipChunk;
+    for (int j = 0; j < TQ_XS_CHUNK_BITS; ++j)
+        if ((chunks >> j) & 1) x = xs_apply(kXsChunkHost[j], 1, x);
+    x = xs_apply(kXsWarpHost[rem / kFlipWarpRun], 1, x);
+    rem %= kFlipWarpRun;
+    return xs_apply(&kXsLaneHost[0][rem / kFlipRun], 32, x);
+}
+
+template <typename Kern>
+tq_status set_smem_once(Kern kern, int bytes, std::atomic<int> *done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TQ_ERR_CUDA;
+    if (!done[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return TQ_ERR_CUDA;
+        done[dev].store(1);
+    }
+    return TQ_OK;
+}
+
+template <bool CONV>
+tq_status launch_flip(uint8_t *packed, const float *grad, int64_t nw, float temp, uint64_t x0, int mode,
+                      int sms, cudaStream_t st) {
+    static std::atomic<int> done[kMaxDevices];
+    if (tq_status e = set_smem_once(flip_kernel<CONV>, kFlipSmem, done)) return e;
+    const int64_t nchunks = (nw + kFlipChunk - 1) / kFlipChunk;
+    const int64_t target = 2 * (int64_t)sms;  // two CTAs per SM
+    const int64_t per_cta = (nchunks + target - 1) / target;
+    const int64_t grid = (nchunks + per_cta - 1) / per_cta;
+    return launch_pdl(flip_kernel<CONV>, dim3((unsigned)grid), dim3(kFlipThreads), (size_t)kFlipSmem, st, packed,
+                      grad, nw, temp, x0, per_cta, mode);
+}
+
+template <bool CONV>
+tq_status launch_bwd_gemm(const uint16_t *planes, const uint8_t *packed, const float *row_scale, int accumulate,
+                          int64_t M, int64_t N, int64_t K, float *dX, int mode, int sms, cudaStream_t st) {
+    static std::atomic<int> done[kMaxDevices];
+    if (tq_status e = set_smem_once(bwd_gemm_kernel<CONV>, kBwdDynamic, done)) return e;
+    // planes [3 M][Np] bf16 in 64-byte-swizzled [256][32] boxes; packed [N][K/4]
+    // in plain [32][32 B] boxes.
+    CUtensorMap tg, tw;
+    if (!make_tmap_bf16(&tg, planes, (uint64_t)bwd_plane_cols(N), (uint64_t)(3 * M), kBwdStepN, kBwdTileT,
+                        CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_tmap_u8(&tw, packed, (uint64_t)(K / 4), (uint64_t)N, kBwdTileF / 4, kBwdStepN,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+        return TQ_ERR_CUDA;
+    const int64_t tiles = ((M + kBwdTileT - 1) / kBwdTileT) * ((K + kBwdTileF - 1) / kBwdTileF);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    return launch_pdl(bwd_gemm_kernel<CONV>, dim3(grid), dim3(kGemmThreads), (size_t)kBwdDynamic, st, tg, tw,
+                      row_scale, accumulate, (int)M, (int)N, (int)K, dX, mode);
+}
+
 }  // namespace
 
 extern "C" {
@@ -802,6 +891,115 @@ tq_status tq_swiglu_mlp(const float *x, int64_t M, int64_t d_model, int64_t d_ff
                                  st, (const float *)yg, (const float *)yu, clamp_val, p, xq2, sx2, rs2, act_out))
         return e;
     return gemm_dispatch(xq2, sx2, rs2, down_packed, down_gamma, cflags, M, d_model, d_ffn, y, nullptr, sms, st);
+}
+
+// ---------------------------------------------------------------------------
+// Training
+// ---------------------------------------------------------------------------
+size_t tq_backward_input_workspace_bytes(int64_t M, int64_t N) {
+    if (M <= 0 || N <= 0) return 0;
+    return ((size_t)(3 * M * bwd_plane_cols(N)) * 2 + 255) & ~(size_t)255;
+}
+
+tq_status tq_ternary_backward_input(const float *dY, const uint8_t *packed, const float *gamma,
+                                    const float *row_scale, unsigned flags, int64_t M, int64_t N, int64_t K,
+                                    float *dX, void *workspace, size_t workspace_bytes, tq_stream_t stream) {
+    if (!dY || !packed || !gamma || !dX || !workspace) return TQ_ERR_NULL;
+    if (M < 1 || N < 1 || M > INT32_MAX / 3 || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_ACCUMULATE | TQ_ENC_MASK)) return TQ_ERR_ARG;
+    const int enc = flag_encoding(flags);
+    if (enc < 0) return TQ_ERR_ARG;
+    if (!aligned16(dY) || !aligned16(packed) || !aligned16(gamma) || !aligned16(dX) || !aligned16(workspace) ||
+        (row_scale && !aligned16(row_scale)))
+        return TQ_ERR_ALIGN;
+    const size_t need = tq_backward_input_workspace_bytes(M, N);
+    if (workspace_bytes < need) return TQ_ERR_ARG;
+    const size_t xb = (size_t)(M * K) * 4;
+    const void *ins[4] = {dY, packed, gamma, row_scale};
+    const size_t inb[4] = {(size_t)(M * N) * 4, (size_t)(N * K / 4),
+                           ((flags & TQ_GAMMA_PER_ROW) ? (size_t)N : 1) * 4, (size_t)M * 4};
+    for (int i = 0; i < 4; ++i)
+        if (ins[i] && (overlap(ins[i], inb[i], dX, xb) || overlap(ins[i], inb[i], workspace, need)))
+            return TQ_ERR_ARG;
+    if (overlap(dX, xb, workspace, need)) return TQ_ERR_ARG;
+    int sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    cudaStream_t st = cs(stream);
+    uint16_t *planes = reinterpret_cast<uint16_t *>(workspace);
+    const int64_t Np = bwd_plane_cols(N);
+    const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
+    const int64_t groups = M * (Np / 8);
+    const int64_t sgrid64 = (groups + kSplitThreads - 1) / kSplitThreads;
+    const unsigned sgrid = (unsigned)(sgrid64 < 8 * (int64_t)sms ? sgrid64 : 8 * (int64_t)sms);
+    tq_status e = (N % 4 == 0)
+                      ? launch_pdl(bwd_split_kernel<true>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
+                                   per_row, (int)M, (int)N, (int)Np, planes)
+                      : launch_pdl(bwd_split_kernel<false>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
+                                   per_row, (int)M, (int)N, (int)Np, planes);
+    if (e) return e;
+    const int mode = enc << kModeEncShift;
+    const int acc = (flags & TQ_FLAG_ACCUMULATE) ? 1 : 0;
+    return enc != kEncFoundry
+               ? launch_bwd_gemm<true>(planes, packed, row_scale, acc, M, N, K, dX, mode, sms, st)
+               : launch_bwd_gemm<false>(planes, packed, row_scale, acc, M, N, K, dX, mode, sms, st);
+}
+
+tq_status tq_ste_backward(const float *grad, const float *w, const float *gamma, int64_t N, int64_t K,
+                          float tau, unsigned flags, float *out, tq_stream_t stream) {
+    if (!grad || !w || !gamma || !out) return TQ_ERR_NULL;
+    if (N < 1) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE)) return TQ_ERR_ARG;
+    if (!(tau >= 0.0f)) return TQ_ERR_ARG;
+    if (!aligned16(grad) || !aligned16(w) || !aligned16(gamma) || !aligned16(out)) return TQ_ERR_ALIGN;
+    const size_t nb = (size_t)(N * K) * 4, gb = ((flags & TQ_GAMMA_PER_ROW) ? (size_t)N : 1) * 4;
+    // in place on grad or on w is allowed; any other overlap is not
+    if ((out != grad && overlap(out, nb, grad, nb)) || (out != w && overlap(out, nb, w, nb)) ||
+        overlap(out, nb, gamma, gb))
+        return TQ_ERR_ARG;
+    int sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    const int64_t nvec = N * K / 4;
+    const int64_t g64 = (nvec + kSteThreads - 1) / kSteThreads;
+    const unsigned grid = (unsigned)(g64 < 8 * (int64_t)sms ? g64 : 8 * (int64_t)sms);
+    const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
+    const float4 *g4 = reinterpret_cast<const float4 *>(grad), *w4 = reinterpret_cast<const float4 *>(w);
+    float4 *o4 = reinterpret_cast<float4 *>(out);
+    return (flags & TQ_FLAG_SANITIZE_NONFINITE)
+               ? launch_pdl(ste_backward_kernel<true>, dim3(grid), dim3(kSteThreads), 0, cs(stream), g4, w4, gamma,
+                            per_row, nvec, K / 4, tau, o4)
+               : launch_pdl(ste_backward_kernel<false>, dim3(grid), dim3(kSteThreads), 0, cs(stream), g4, w4,
+                            gamma, per_row, nvec, K / 4, tau, o4);
+}
+
+void tq_seed(uint64_t *state, uint64_t seed) {
+    if (state) *state = seed ? seed : 0x9E3779B97F4A7C15ull;
+}
+
+tq_status tq_ternary_stochastic_flip(uint8_t *packed, const float *grad, int64_t N, int64_t K,
+                                     float temperature, uint64_t *rng_state, unsigned flags,
+                                     tq_stream_t stream) {
+    if (!packed || !grad || !rng_state) return TQ_ERR_NULL;
+    if (N < 1) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (N > ((int64_t)1 << 40) / K) return TQ_ERR_SHAPE;
+    if (flags & ~TQ_ENC_MASK) return TQ_ERR_ARG;
+    const int enc = flag_encoding(flags);
+    if (enc < 0) return TQ_ERR_ARG;
+    if (!(temperature >= 0.0f && temperature <= 3.4028235e38f)) return TQ_ERR_ARG;
+    if (!aligned16(packed) || !aligned16(grad)) return TQ_ERR_ALIGN;
+    const int64_t nw = N * K;
+    if (overlap(packed, (size_t)(nw / 4), grad, (size_t)nw * 4)) return TQ_ERR_ARG;
+    int sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    const uint64_t x0 = *rng_state;
+    const int mode = enc << kModeEncShift;
+    tq_status e = enc != kEncFoundry ? launch_flip<true>(packed, grad, nw, temperature, x0, mode, sms, cs(stream))
+                                     : launch_flip<false>(packed, grad, nw, temperature, x0, mode, sms, cs(stream));
+    if (e) return e;
+    *rng_state = xs_jump(x0, nw);
+    return TQ_OK;
 }
 
 tq_status tq_get_device_status(tq_stream_t stream) {

@@ -1,0 +1,587 @@
+// tq_train.cuh -- training kernels of the ternary layer: the gradient with
+// respect to the layer input, the straight-through estimator of the latent
+// weights, and the stochastic ternary flip.
+//
+//   Foundry, docs/quantization.md, "Ternary Training (Backward Pass +
+//   Stochastic Flip)": fq_matmul_ternary_backward_input (dX += dY W_ternary,
+//   same unpacking as the forward, summed over the output features) and
+//   fq_ternary_stochastic_flip (p = clamp(|grad| T, 0, 1), one step toward
+//   -grad, caller-owned xorshift64 state).
+//   Hetman-2b, src/quantization.py, section 2 AbsmeanWeightQuantizer.backward
+//   (grad / gamma, damped by 0.1 outside |w / gamma| <= tau).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "tq_common.cuh"
+#include "tq_gemm.cuh"
+#include "tq_gemv.cuh"
+#include "tq_xorshift_jump.h"
+
+namespace tq {
+
+// ===========================================================================
+// Straight-through estimator (elementwise, HBM-bound: 12 bytes per weight)
+// ===========================================================================
+constexpr int kSteThreads = 256;
+
+__device__ __forceinline__ float ste_one(float g, float w, float gm, float tau, bool san) {
+    if (san) {
+        if (isnan(w)) w = 0.0f;
+        else if (isinf(w)) w = w > 0.0f ? 1.0f : -1.0f;
+    }
+    const float ws = __fdiv_rn(w, gm);
+    const float damp = fabsf(ws) <= tau ? 1.0f : 0.1f;  // NaN compares false: damped
+    return __fmul_rn(__fdiv_rn(g, gm), damp);
+}
+
+// grad, w, out: [N][K] fp32 viewed as float4 (K % 4 == 0, so a vector never
+// crosses a row); gamma [N] (per_row) or [1].  out may be grad or w.
+template <bool SAN>
+__global__ void __launch_bounds__(kSteThreads)
+    ste_backward_kernel(const float4 *grad, const float4 *w, const float *__restrict__ gamma, int per_row,
+                        int64_t nvec, int64_t kvec, float tau, float4 *out) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t stride = (int64_t)gridDim.x * kSteThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kSteThreads + threadIdx.x; i < nvec; i += stride) {
+        const float gm = __ldg(gamma + (per_row ? i / kvec : 0));
+        const float4 g = __ldcs(grad + i), x = __ldcs(w + i);
+        float4 r;
+        r.x = ste_one(g.x, x.x, gm, tau, SAN);
+        r.y = ste_one(g.y, x.y, gm, tau, SAN);
+        r.z = ste_one(g.z, x.z, gm, tau, SAN);
+        r.w = ste_one(g.w, x.w, gm, tau, SAN);
+        __stcs(out + i, r);
+    }
+}
+
+// ===========================================================================
+// Stochastic flip
+// ===========================================================================
+// The stream of draws is Foundry's sequential one: weight i (row-major over
+// [N][K]) compares against the (i+1)-th xorshift64 output after the caller's
+// state.  xorshift64 is linear over GF(2), so the state i steps ahead is
+// A^i x0; the tables of tq_xorshift_jump.h hold the powers of A needed to
+// start every lane's run of kFlipRun weights at its own point of the stream:
+//   CTA    first chunk c: A^(16384 c) from the binary powers TQ_XS_CHUNK
+//          (one warp, 64-column matrix-vector products split over the lanes);
+//          later chunks continue from the end state of the previous one;
+//   warp   w: A^(2048 w) x_chunk (TQ_XS_WARP, same cooperative product);
+//   lane   l: A^(64 l) x_warp (TQ_XS_LANE, copied to shared memory, one
+//          product per lane).
+// Each lane then runs its 64 draws sequentially.  Gradients are staged per
+// warp in shared memory with cp.async (coalesced), packed codes are read and
+// written as one 16-byte vector per lane.
+constexpr int kFlipWarps = TQ_XS_WARPS;
+constexpr int kFlipThreads = 32 * kFlipWarps;
+constexpr int kFlipRun = TQ_XS_RUN;                          // weights per lane
+constexpr int kFlipWarpRun = 32 * kFlipRun;                  // weights per warp
+constexpr int64_t kFlipChunk = (int64_t)kFlipWarps * kFlipWarpRun;  // weights per CTA pass
+constexpr int kFlipTabBytes = 64 * 32 * 8;
+constexpr int kFlipSmem = kFlipTabBytes + kFlipWarps * kFlipWarpRun * 4;
+static_assert(kFlipRun == 64, "one 16-byte packed vector per lane");
+
+__device__ const uint64_t kXsChunk[TQ_XS_CHUNK_BITS][64] = TQ_XS_CHUNK_INIT;
+__device__ const uint64_t kXsWarp[TQ_XS_WARPS][64] = TQ_XS_WARP_INIT;
+__device__ const uint64_t kXsLane[64][32] = TQ_XS_LANE_INIT;
+
+// y = M x for a warp-uniform x: lane l folds columns 2l and 2l+1, then an
+// XOR reduction over the warp gives every lane the product.
+__device__ __forceinline__ uint64_t warp_matvec(const uint64_t *__restrict__ cols, uint64_t x, int lane) {
+    const int b = 2 * lane;
+    uint64_t r = 0;
+    if ((x >> b) & 1ull) r ^= __ldg(cols + b);
+    if ((x >> (b + 1)) & 1ull) r ^= __ldg(cols + b + 1);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) r ^= __shfl_xor_sync(0xffffffffu, r, off);
+    return r;
+}
+
+// y = A^(64 lane) x, each lane its own matrix (column-major table in shared
+// memory: column b of every lane's matrix in 32 consecutive words).
+__device__ __forceinline__ uint64_t lane_matvec(const uint64_t *tab, uint64_t x, int lane) {
+    uint64_t r = 0;
+#pragma unroll 16
+    for (int b = 0; b < 64; ++b) r ^= tab[b * 32 + lane] & (0ull - ((x >> b) & 1ull));
+    return r;
+}
+
+// Four weights (one packed byte in Foundry's layout) against the next four draws.
+__device__ __forceinline__ uint32_t flip_byte(uint32_t byte, const float4 g4, float temp, uint64_t &x) {
+    const float gs[4] = {g4.x, g4.y, g4.z, g4.w};
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x ^= x << 13;
+        x ^= x >> 7;
+        x ^= x << 17;
+        const float u = __fmul_rn(__uint2float_rn((uint32_t)(x >> 40)), 0x1p-24f);  // exact
+        const float a = __fmul_rn(fabsf(gs[i]), temp);
+        const float p = a > 1.0f ? 1.0f : a;  // NaN stays NaN: u < p is false
+        const uint32_t f = (byte >> (2 * i)) & 3u;
+        int q = f == 3u ? 0 : (int)f - 1;     // the unassigned field reads as 0
+        if (u < p) {
+            const int s = gs[i] > 0.0f ? 1 : (gs[i] < 0.0f ? -1 : 0);
+            q = max(-1, min(1, q - s));
+        }
+        out |= (uint32_t)(q + 1) << (2 * i);
+    }
+    return out;
+}
+
+// packed [nw / 4] bytes (in place), grad [nw] fp32, nw % 64 == 0.  CTA b
+// owns chunks [b * per_cta, (b + 1) * per_cta).
+template <bool CONV>
+__global__ void __launch_bounds__(kFlipThreads, 2)
+    flip_kernel(uint8_t *packed, const float *__restrict__ grad, int64_t nw, float temp, uint64_t x0,
+                int64_t per_cta, int mode) {
+    extern __shared__ __align__(16) uint8_t flip_smem[];
+    __shared__ uint64_t chunk_state;
+    uint64_t *tab = reinterpret_cast<uint64_t *>(flip_smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float4 *stage = reinterpret_cast<float4 *>(flip_smem + kFlipTabBytes) + warp * (kFlipWarpRun / 4);
+    const int enc = (mode >> kModeEncShift) & 3;
+    const int64_t nchunks = (nw + kFlipChunk - 1) / kFlipChunk;
+    const int64_t c_begin = (int64_t)blockIdx.x * per_cta;
+    const int64_t c_end = c_begin + per_cta < nchunks ? c_begin + per_cta : nchunks;
+
+    // constant tables only: no dependence on earlier kernels yet
+    for (int i = threadIdx.x; i < 64 * 32; i += kFlipThreads) tab[i] = (&kXsLane[0][0])[i];
+    if (warp == 0) {
+        uint64_t x = x0;
+        for (int j = 0; j < TQ_XS_CHUNK_BITS; ++j)
+            if ((c_begin >> j) & 1) x = warp_matvec(kXsChunk[j], x, lane);
+        if (lane == 0) chunk_state = x;
+    }
+    pdl_wait();  // grad and packed may be written by the previous kernel
+    pdl_trigger();
+    __syncthreads();
+
+    for (int64_t c = c_begin; c < c_end; ++c) {
+        const int64_t wbase = c * kFlipChunk + (int64_t)warp * kFlipWarpRun;  // this warp's first weight
+        const int64_t left = nw - wbase;
+        const int nruns = left <= 0 ? 0 : (left >= kFlipWarpRun ? 32 : (int)(left / kFlipRun));
+        // stage the warp's gradients: float4 g of the warp = run g / 16, vector
+        // g % 16, stored at run * 16 + (vector ^ (run & 7)) (conflict-free reads)
+        for (int i = 0; i < 16; ++i) {
+            const int g = i * 32 + lane, r = g >> 4, j = g & 15;
+            if (r < nruns)
+                cp_async16(smem_u32(stage + r * 16 + (j ^ (r & 7))), grad + wbase + 4 * (int64_t)g);
+        }
+        uint64_t x = warp_matvec(kXsWarp[warp], chunk_state, lane);
+        x = lane_matvec(tab, x, lane);
+        cp_async_wait_all();
+        __syncwarp();
+        if (lane < nruns) {
+            uint8_t *pk = packed + (wbase + (int64_t)lane * kFlipRun) / 4;
+            const uint4 v = *reinterpret_cast<const uint4 *>(pk);
+            uint32_t words[4] = {v.x, v.y, v.z, v.w};
+            if (CONV) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) words[i] = codes_to_foundry(words[i], enc);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float4 g4 = stage[lane * 16 + (j ^ (lane & 7))];
+                const int sh = (j & 3) * 8;
+                const uint32_t b = flip_byte((words[j >> 2] >> sh) & 0xFFu, g4, temp, x);
+                words[j >> 2] = (words[j >> 2] & ~(0xFFu << sh)) | (b << sh);
+            }
+            if (CONV) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) words[i] = codes_from_foundry(words[i], enc);
+            }
+            *reinterpret_cast<uint4 *>(pk) = make_uint4(words[0], words[1], words[2], words[3]);
+        }
+        // A chunk followed by another one is full: its last lane ends where
+        // the next chunk starts.
+        __syncthreads();
+        if (threadIdx.x == kFlipThreads - 1) chunk_state = x;
+        __syncthreads();
+    }
+}
+
+// ===========================================================================
+// Gradient with respect to the input: dX = row_scale * (dY * gamma) W_ternary
+// ===========================================================================
+// The contraction runs over the N output features with fp32 operands on one
+// side and codes in {-1, 0, +1} on the other.  It is a dense GEMM, so it runs
+// on the tensor cores (tcgen05 kind::f16, bf16 operands, fp32 accumulation in
+// tensor memory) with the fp32 side split exactly into three bf16 planes:
+//   g = fp32(dY * gamma_n),  h = bf16(g),  m = bf16(g - h),  l = bf16(g - h - m)
+// (each difference is exact in fp32 and h + m + l = g: 8 + 8 + 8 significant
+// bits hold fp32's 24).  Every product with a code is exact, so the only
+// rounding is the fp32 accumulation of the tensor core.
+
+// --- split pass: planes [3][M][Np] bf16, columns N .. Np - 1 zero ---------
+constexpr int kSplitThreads = 256;
+
+__device__ __forceinline__ void split3(float g, uint16_t &h, uint16_t &m, uint16_t &l) {
+    const __nv_bfloat16 bh = __float2bfloat16_rn(g);
+    const float r1 = __fsub_rn(g, __bfloat162float(bh));
+    const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
+    const float r2 = __fsub_rn(r1, __bfloat162float(bm));
+    const __nv_bfloat16 bl = __float2bfloat16_rn(r2);
+    h = __bfloat16_as_ushort(bh);
+    m = __bfloat16_as_ushort(bm);
+    l = __bfloat16_as_ushort(bl);
+}
+
+// One thread per 8 columns of a row.  VEC: rows are 16-byte aligned (N % 4 == 0).
+template <bool VEC>
+__global__ void __launch_bounds__(kSplitThreads)
+    bwd_split_kernel(const float *__restrict__ dY, const float *__restrict__ gamma, int per_row, int M, int N,
+                     int Np, uint16_t *__restrict__ planes) {
+    pdl_wait();
+    pdl_trigger();
+    const int gpr = Np / 8;  // groups per row
+    const int64_t total = (int64_t)M * gpr, plane = (int64_t)M * Np;
+    const float g0 = __ldg(gamma);
+    for (int64_t i = (int64_t)blockIdx.x * kSplitThreads + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * kSplitThreads) {
+        const int t = (int)(i / gpr), c0 = (int)(i % gpr) * 8;
+        const float *row = dY + (int64_t)t * N;
+        float v[8];
+        if (VEC && c0 + 8 <= N) {
+            const float4 a = __ldcs(reinterpret_cast<const float4 *>(row + c0));
+            const float4 b = __ldcs(reinterpret_cast<const float4 *>(row + c0 + 4));
+            v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = c0 + j < N ? __ldcs(row + c0 + j) : 0.0f;
+        }
+        uint16_t h[8], m[8], l[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float sc = per_row ? (c0 + j < N ? __ldg(gamma + c0 + j) : 0.0f) : g0;
+            split3(c0 + j < N ? __fmul_rn(v[j], sc) : 0.0f, h[j], m[j], l[j]);
+        }
+        auto pack8 = [](const uint16_t (&s)[8]) {
+            return make_uint4(s[0] | (uint32_t)s[1] << 16, s[2] | (uint32_t)s[3] << 16, s[4] | (uint32_t)s[5] << 16,
+                              s[6] | (uint32_t)s[7] << 16);
+        };
+        uint16_t *o = planes + (int64_t)t * Np + c0;
+        *reinterpret_cast<uint4 *>(o) = pack8(h);
+        *reinterpret_cast<uint4 *>(o + plane) = pack8(m);
+        *reinterpret_cast<uint4 *>(o + 2 * plane) = pack8(l);
+    }
+}
+
+// --- the GEMM ---------------------------------------------------------------
+// Persistent, one CTA per SM.  Output tile: 128 input features (the MMA's M,
+// taken by the unpacked codes, A = W^T) x 256 tokens (the MMA's N, taken by
+// the bf16 planes, B = g).  The contraction dimension is the layer's N, in
+// steps of 32.  Per step: the three plane tiles [256 tokens][32 n] (64-byte
+// rows, 64-byte swizzle, K-major, by TMA), the packed tile [32 n][32 B] (by
+// TMA), and the code tile A [32 n][128 features] in bf16, written by the
+// unpackers in the 128-byte-swizzled MN-major layout (features contiguous:
+// the packed rows already are).  Six MMAs of K = 16 per step (two halves of
+// the step times three planes) into one fp32 accumulator.  Feature tiles
+// run fastest, so concurrently running CTAs share the token block's planes
+// in L2.  Warp roles as in the forward GEMM: 0 plane producer, 1 MMA issuer
+// and TMEM owner, 2 packed-weight producer, 4-11 unpackers (two groups
+// taking alternate steps), 12-19 epilogue.
+constexpr int kBwdTileF = 128;   // features per tile (MMA M)
+constexpr int kBwdTileT = 256;   // tokens per tile (MMA N)
+constexpr int kBwdStepN = 32;    // contraction rows per step
+constexpr int kBwdPlanes = 3;
+constexpr int kBwdPlaneBytes = kBwdTileT * kBwdStepN * 2;             // 16 KB
+constexpr int kBwdABytes = kBwdTileF * kBwdStepN * 2;                 // 8 KB
+constexpr int kBwdStage = kBwdPlanes * kBwdPlaneBytes + kBwdABytes;   // 56 KB
+constexpr int kBwdStages = 3;
+constexpr int kBwdWBytes = kBwdStepN * kBwdTileF / 4;                 // 1 KB packed per step
+constexpr int kBwdWStages = 8;
+constexpr int kBwdOffW = kBwdStages * kBwdStage;
+constexpr int kBwdOffBar = kBwdOffW + kBwdWStages * kBwdWBytes;
+constexpr int kBwdBars = 2 * kBwdStages + 2 * kBwdWStages + 5;
+constexpr int kBwdOffTmem = kBwdOffBar + kBwdBars * 8;
+constexpr int kBwdDynamic = kBwdOffTmem + 16 + 1024;
+constexpr uint32_t kBwdTmemCols = 2 * kBwdTileT;  // two accumulators of 256 fp32 columns
+static_assert(kBwdDynamic <= 232448, "shared memory per CTA");
+static_assert(kBwdPlaneBytes % 1024 == 0 && kBwdABytes % 1024 == 0 && kBwdStage % 1024 == 0, "atoms aligned");
+
+// Instruction descriptor, kind::f16: D f32, A and B bf16, A MN-major, B K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_amn(int M, int N) {
+    return (1u << 4)                        // D format: f32
+           | (1u << 7)                      // A: bf16
+           | (1u << 10)                     // B: bf16
+           | (1u << 15)                     // A MN-major
+           | ((uint32_t)(N >> 3) << 17)     // N / 8
+           | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// MN-major bf16 operand, 128-byte swizzle: atoms of 8 contraction rows x 64
+// elements (128 B per row, 16-byte chunk index XOR row % 8); atoms along M
+// are `lbo` bytes apart, atoms along the contraction (8-row groups) `sbo`.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;  // 128-byte swizzle
+    return d;
+}
+
+// K-major operand, 64-byte swizzle: rows of 64 B, 8-row groups 512 B apart.
+__device__ __forceinline__ uint64_t smem_desc_k_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;             // leading byte offset (unused)
+    d |= (uint64_t)(512u >> 4) << 32;    // stride byte offset: 8 rows x 64 B
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)4u << 61;             // 64-byte swizzle
+    return d;
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Four codes (one packed byte, Foundry's layout) -> four bf16 of q = field - 1
+// (0b00 -> -1.0 = 0xBF80, 0b01 -> 0, 0b10 -> +1.0 = 0x3F80; the unassigned
+// 0b11 gives 2.0).  A byte permute picks each half of each bf16 from two
+// four-entry tables (high bytes BF 00 3F 40, low bytes 80 00 80 00).
+__device__ __forceinline__ uint2 codes4_to_bf16(uint32_t byte) {
+    const uint32_t n0 = byte & 0xFu, n1 = (byte >> 4) & 0xFu;
+    const uint32_t s0 = 0x0404u + (n0 & 3u) * 0x11u + (n0 >> 2) * 0x1100u;
+    const uint32_t s1 = 0x0404u + (n1 & 3u) * 0x11u + (n1 >> 2) * 0x1100u;
+    return make_uint2(__byte_perm(0x403F00BFu, 0x00800080u, s0), __byte_perm(0x403F00BFu, 0x00800080u, s1));
+}
+
+// planes: tensor map over [3 M][Np] bf16 (plane p of token t is row p M + t);
+// packed: tensor map over [N][K / 4] bytes.  dX [M][K] fp32.
+template <bool CONV>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_w,
+                    const float *__restrict__ row_scale, int accumulate, int M, int N, int K,
+                    float *__restrict__ dX, int mode) {
+    constexpr int S = kBwdStages, SW = kBwdWStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + kBwdOffBar;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+    auto w_full = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    auto w_empty = [&](int s) { return bar0 + 8u * (2 * S + SW + s); };
+    auto d_full = [&](int b) { return bar0 + 8u * (2 * S + 2 * SW + b); };
+    auto d_empty = [&](int b) { return bar0 + 8u * (2 * S + 2 * SW + 2 + b); };
+    const uint32_t mma_done = bar0 + 8u * (2 * S + 2 * SW + 4);
+    auto g_stage = [&](int s) { return sbase + (uint32_t)(s * kBwdStage); };
+    auto a_stage = [&](int s) { return g_stage(s) + (uint32_t)(kBwdPlanes * kBwdPlaneBytes); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBwdOffTmem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_f = (K + kBwdTileF - 1) / kBwdTileF, num_t = (M + kBwdTileT - 1) / kBwdTileT;
+    const int ntiles = num_f * num_t;
+    const int nkb = (N + kBwdStepN - 1) / kBwdStepN;
+    const int my_tiles =
+        ntiles > (int)blockIdx.x ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+    const int total = my_tiles * nkb;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1 + kUnpackWarps / 2);
+            mbar_init(empty(s), 1);
+        }
+        for (int s = 0; s < SW; ++s) {
+            mbar_init(w_full(s), 1);
+            mbar_init(w_empty(s), kUnpackWarps / 2);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(d_full(b), 1);
+            mbar_init(d_empty(b), kEpiWarps);
+        }
+        mbar_init(mma_done, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tm_g);
+        prefetch_tmap(&tm_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kBwdTmemCols);
+        tmem_relinquish();
+    }
+    pdl_wait();  // the planes come from the split pass just before
+    pdl_trigger();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- plane producer ----------------
+        if (lane == 0) {
+            int g = 0;
+            for (; g < total; ++g) {
+                const int s = g % S, r = g / S;
+                const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
+                const int kb = g % nkb;
+                const int t0 = (t / num_f) * kBwdTileT;
+                if (!mbar_wait_sleep(empty(s), (r & 1) ^ 1)) break;
+                mbar_arrive_expect_tx(full(s), kBwdPlanes * kBwdPlaneBytes);
+#pragma unroll
+                for (int p = 0; p < kBwdPlanes; ++p)
+                    tma_load_2d(g_stage(s) + (uint32_t)(p * kBwdPlaneBytes), &tm_g, kb * kBwdStepN, p * M + t0,
+                                full(s));
+            }
+            for (int j = g - S < 0 ? 0 : g - S; j < g; ++j) mbar_wait(full(j % S), (j / S) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ---------------- packed-weight producer ----------------
+        if (lane == 0) {
+            int g = 0;
+            for (; g < total; ++g) {
+                const int s = g % SW, r = g / SW;
+                const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
+                const int kb = g % nkb;
+                if (!mbar_wait_sleep(w_empty(s), (r & 1) ^ 1)) break;
+                mbar_arrive_expect_tx(w_full(s), kBwdWBytes);
+                tma_load_2d(sbase + (uint32_t)(kBwdOffW + s * kBwdWBytes), &tm_w, (t % num_f) * (kBwdTileF / 4),
+                            kb * kBwdStepN, w_full(s));
+            }
+            for (int j = g - SW < 0 ? 0 : g - SW; j < g; ++j) mbar_wait(w_full(j % SW), (j / SW) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_amn(kBwdTileF, kBwdTileT);
+            int g = 0;
+            bool ok = true;
+            for (int tl = 0; tl < my_tiles && ok; ++tl) {
+                const int b = tl & 1;
+                if (!mbar_wait(d_empty(b), ((tl >> 1) & 1) ^ 1)) break;
+                tc_fence_after();
+                const uint32_t d_col = tmem + (uint32_t)(b * kBwdTileT);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    if (!mbar_wait(full(s), (g / S) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kBwdStepN / 16; ++kk) {
+                        const uint64_t ad = smem_desc_mn_sw128(a_stage(s) + (uint32_t)(kk * 4096), 1024u, 2048u);
+#pragma unroll
+                        for (int p = 0; p < kBwdPlanes; ++p)
+                            mma_bf16(d_col, ad,
+                                     smem_desc_k_sw64(g_stage(s) + (uint32_t)(p * kBwdPlaneBytes + kk * 32)),
+                                     idesc, (kb | kk | p) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(empty(s));
+                }
+                if (ok) mma_commit(d_full(b));
+            }
+            mma_commit(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
+        // ---------------- unpack codes into the MN-major bf16 tile ----------------
+        // Group thread i: contraction row c = 8 (warp % 4) + lane % 8, features
+        // 32 (lane / 8) .. + 32 (8 packed bytes -> four 16-byte chunks).
+        const int par = (warp - 4) >> 2;
+        const int enc = (mode >> kModeEncShift) & 3;
+        const int c = 8 * (warp & 3) + (lane & 7), fq = lane >> 3;
+        const uint32_t r8 = (uint32_t)(c & 7);
+        const uint32_t a_row = (uint32_t)((c >> 3) * 2048) + r8 * 128u;
+        for (int g = par; g < total; g += 2) {
+            const int ws = g % SW, s = g % S;
+            if (!warp_wait_sleep(w_full(ws), (g / SW) & 1, lane)) break;
+            uint32_t w0, w1;
+            asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                         : "=r"(w0), "=r"(w1)
+                         : "r"(sbase + (uint32_t)(kBwdOffW + ws * kBwdWBytes + c * 32 + fq * 8))
+                         : "memory");
+            if (CONV) {
+                w0 = codes_to_foundry(w0, enc);
+                w1 = codes_to_foundry(w1, enc);
+            }
+            uint2 e[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                e[k] = codes4_to_bf16((w0 >> (8 * k)) & 0xFFu);
+                e[4 + k] = codes4_to_bf16((w1 >> (8 * k)) & 0xFFu);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(w_empty(ws));
+            if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
+            const uint32_t base = a_stage(s) + a_row;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int jg = 4 * fq + k;  // chunk of 8 features within the 128
+                const uint32_t addr =
+                    base + (uint32_t)((jg >> 3) * 1024) + ((((uint32_t)(jg & 7)) ^ r8) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(e[2 * k].x),
+                             "r"(e[2 * k].y), "r"(e[2 * k + 1].x), "r"(e[2 * k + 1].y)
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full(s));
+        }
+    } else if (warp >= 12) {
+        // ---------------- epilogue ----------------
+        constexpr int kHalf = kBwdTileT / 2;
+        constexpr int kChunks = kHalf / 32;
+        const int q = warp & 3;
+        const int half = (warp - 12) >> 2;
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+        for (int tl = 0; tl < my_tiles; ++tl) {
+            const int t = (int)blockIdx.x + tl * (int)gridDim.x;
+            const int b = tl & 1;
+            const int f = (t % num_f) * kBwdTileF + 32 * q + lane;
+            const int m0 = (t / num_f) * kBwdTileT + half * kHalf;
+            float rsc[kChunks];
+#pragma unroll
+            for (int cc = 0; cc < kChunks; ++cc) {
+                const int mj = m0 + cc * 32 + lane;
+                rsc[cc] = (row_scale && mj < M) ? __ldg(row_scale + mj) : 1.0f;
+            }
+            if (!warp_wait_sleep(d_full(b), (tl >> 1) & 1, lane)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < kChunks; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + (uint32_t)(b * kBwdTileT + half * kHalf + cc * 32), v);
+                tmem_ld_wait();
+                if (cc == kChunks - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(d_empty(b));
+                }
+                const int mb = m0 + cc * 32;
+                const int jmax = M - mb;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float rs = __shfl_sync(0xffffffffu, rsc[cc], j);
+                    float o = __uint_as_float(v[j]);
+                    if (row_scale) o = __fmul_rn(o, rs);
+                    if (j < jmax && f < K) {
+                        float *p = dX + (int64_t)(mb + j) * K + f;
+                        if (accumulate) o = __fadd_rn(*p, o);
+                        __stcs(p, o);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kBwdTmemCols);
+    }
+}
+
+}  // namespace tq

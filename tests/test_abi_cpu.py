@@ -141,3 +141,74 @@ def test_gemm_and_fused_validation(lib):
     fused[15] = 1 << 20
     fused[5] = tq.FLAG_FWHT | 3 << 7
     assert h(*fused) == 4  # reserved layout
+
+
+def test_training_validation(lib):
+    f = lib.tq_ternary_backward_input
+    ws = lib.tq_backward_input_workspace_bytes(4, 40)
+    assert ws >= 3 * 4 * 64 * 2 and lib.tq_backward_input_workspace_bytes(0, 8) == 0
+    ok = [P(), P(1 << 20), P(2 << 20), None, 0, 4, 40, 128, P(3 << 20), P(4 << 20), ws, None]
+    bad = list(ok); bad[0] = None
+    assert f(*bad) == 1
+    bad = list(ok); bad[7] = 96
+    assert f(*bad) == 2                                   # K % 64
+    bad = list(ok); bad[4] = 1 << 10
+    assert f(*bad) == 4                                   # unknown flag
+    bad = list(ok); bad[4] = 3 << 7
+    assert f(*bad) == 4                                   # reserved layout
+    bad = list(ok); bad[10] = ws - 16
+    assert f(*bad) == 4                                   # workspace too small
+    bad = list(ok); bad[8] = P(16)
+    assert f(*bad) == 4                                   # dX overlaps dY
+    bad = list(ok); bad[3] = P((5 << 20) + 4)
+    assert f(*bad) == 3                                   # misaligned row_scale
+    g = lib.tq_ste_backward
+    ok = [P(), P(1 << 20), P(2 << 20), 4, 64, 1.0, 0, P(3 << 20), None]
+    bad = list(ok); bad[5] = float("nan")
+    assert g(*bad) == 4
+    bad = list(ok); bad[5] = -1.0
+    assert g(*bad) == 4
+    bad = list(ok); bad[6] = tq.FLAG_FWHT
+    assert g(*bad) == 4
+    bad = list(ok); bad[7] = P(64)
+    assert g(*bad) == 4                                   # partial overlap with grad
+    bad = list(ok); bad[4] = 60
+    assert g(*bad) == 2
+    h = lib.tq_ternary_stochastic_flip
+    st = ctypes.c_uint64(5)
+    ok = [P(), P(1 << 20), 4, 64, 0.5, ctypes.byref(st), 0, None]
+    bad = list(ok); bad[5] = None
+    assert h(*bad) == 1
+    for t in (float("nan"), -0.5, float("inf")):
+        bad = list(ok); bad[4] = t
+        assert h(*bad) == 4, t
+    bad = list(ok); bad[1] = P(32)
+    assert h(*bad) == 4                                   # grad overlaps packed
+    bad = list(ok); bad[6] = tq.GAMMA_PER_ROW
+    assert h(*bad) == 4
+    assert st.value == 5                                  # a refused call leaves the state alone
+    s = ctypes.c_uint64(0)
+    lib.tq_seed(ctypes.byref(s), 0)
+    assert s.value == 0x9E3779B97F4A7C15
+    lib.tq_seed(ctypes.byref(s), 12345)
+    assert s.value == 12345
+
+
+def test_xorshift_jump_tables_are_generated_and_jump_the_oracle_stream():
+    import importlib.util
+    import oracle
+    here = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "ternary_bit_linear_b200", "csrc")
+    spec = importlib.util.spec_from_file_location("gen_xorshift_jump", os.path.join(here, "gen_xorshift_jump.py"))
+    gen = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(gen)
+    assert open(os.path.join(here, "tq_xorshift_jump.h")).read() == gen.header()
+    chunk, warp, lane = gen.tables()
+    x = 0x0123456789ABCDEF
+    seq, _ = oracle.xorshift64(x, gen.CHUNK)
+    assert gen.apply(chunk[0], x) == seq[-1]
+    assert gen.apply(warp[3], x) == seq[3 * gen.WARP_RUN - 1]
+    for l in (1, 7, 31):
+        assert gen.apply([lane[b][l] for b in range(64)], x) == seq[gen.RUN * l - 1]
+    # two chunks = chunk[1]
+    seq2, _ = oracle.xorshift64(seq[-1], gen.CHUNK)
+    assert gen.apply(chunk[1], x) == seq2[-1]

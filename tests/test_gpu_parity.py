@@ -872,3 +872,103 @@ def test_swiglu_mlp(cuda_lib, M, D, F, per_row):
     assert torch.equal(y, y_chk)
     check_fused(tq, act_h, Ws[2], per_row)
     assert tq.device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# NEXT row N4: training.  STE and flip bit-exact; the input gradient within
+# 1e-5 of sum_n |fp32(dY gamma) q| * |row_scale| (+ |dX_in|): each product
+# is exact on the GPU (three-way bf16 split), only the fp32 accumulation
+# rounds, and a cancelled sum has no relative accuracy in any fp32 order.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K,per_row,san,tau", [(1, 64, False, False, 1.0), (37, 448, True, True, 1.0),
+                                                  (300, 4096, False, True, 1.5), (1024, 2048, True, False, 0.5)])
+def test_ste_backward_bit_exact(cuda_lib, N, K, per_row, san, tau):
+    tq = cuda_lib
+    W = S.normal((N, K), 0.02, 120, N)
+    G = S.normal((N, K), 1.0, 121, N)
+    if N > 2:
+        W[1, :4] = [np.nan, np.inf, -np.inf, 0.0]
+        G[2, :2] = [np.nan, np.inf]
+    p, gam = oracle.quantize_pack(np.nan_to_num(W, nan=0.0, posinf=1.0, neginf=-1.0), per_row=per_row)
+    fl = (tq.GAMMA_PER_ROW if per_row else 0) | (tq.FLAG_SANITIZE_NONFINITE if san else 0)
+    want = oracle.ste_backward(G, W, gam, per_row, tau, san)
+    out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    gd, wd, gmd = dev(G), dev(W), dev(gam)
+    tq.ste_backward_(gd, wd, gmd, fl, out, tau)
+    got = host(out)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32)) or \
+        np.array_equal(np.nan_to_num(got, nan=7.0), np.nan_to_num(want, nan=7.0))
+    tq.ste_backward_(gd, wd, gmd, fl, gd, tau)  # in place on the gradient
+    assert np.array_equal(np.nan_to_num(host(gd), nan=7.0), np.nan_to_num(want, nan=7.0))
+    assert tq.device_status() == 0
+
+
+@pytest.mark.parametrize("layout", [0, 1, 2])
+@pytest.mark.parametrize("N,K,temp", [(1, 64, 0.5), (37, 448, 0.05), (300, 4096, 0.2), (2048, 4096, 0.05)])
+def test_stochastic_flip_bit_exact(cuda_lib, layout, N, K, temp):
+    tq = cuda_lib
+    q = np.clip(np.rint(S.normal((N, K), 0.7, 130, N)), -1, 1).astype(np.int8)
+    G = S.normal((N, K), 1.0, 131, N)
+    if N > 3:
+        G[3, :3] = [np.nan, np.inf, 0.0]
+    packed = oracle.pack_format(q, layout)
+    st0 = tq.seed(1000 + N)
+    assert st0 == oracle.seed(1000 + N)
+    want, st_want = oracle.stochastic_flip(packed, G, temp, st0, layout)
+    pd, gd = dev(packed), dev(G)
+    st = tq.ternary_stochastic_flip_(pd, gd, temp, st0, layout << 7)
+    assert st == st_want
+    got = host(pd)
+    assert np.array_equal(got, want)
+    # a second call continues the stream where the first one stopped
+    want2, st_want2 = oracle.stochastic_flip(want, G, temp, st_want, layout)
+    assert tq.ternary_stochastic_flip_(pd, gd, temp, st, layout << 7) == st_want2
+    assert np.array_equal(host(pd), want2)
+    assert tq.device_status() == 0
+
+
+def _bwd_check(tq, M, N, K, per_row, use_rs, accumulate, layout, seed, rows=None):
+    dY = S.normal((M, N), 1.0, seed, M)
+    W = S.normal((N, K), 0.02, seed + 1, N)
+    packed, gam = oracle.quantize_pack(W, per_row=per_row, encoding=layout)
+    rs = (S.uniform(seed + 2, 0, 0, M).astype(np.float32) * np.float32(0.02)).astype(np.float32) if use_rs else None
+    dX0 = S.normal((M, K), 1.0, seed + 3, M) if accumulate else None
+    fl = (tq.GAMMA_PER_ROW if per_row else 0) | (tq.FLAG_ACCUMULATE if accumulate else 0) | (layout << 7)
+    dXd = dev(dX0) if accumulate else torch.empty((M, K), dtype=torch.float32, device="cuda")
+    ws = torch.empty((tq.backward_input_workspace_bytes(M, N),), dtype=torch.uint8, device="cuda")
+    tq.ternary_backward_input_(dev(dY), dev(packed), dev(gam), fl, dXd, ws, None if rs is None else dev(rs))
+    got = host(dXd)
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    want = oracle.backward_input(dY[sel], packed, gam, per_row, K, None if rs is None else rs[sel],
+                                 None if dX0 is None else dX0[sel], layout)
+    # magnitude of the terms: |g| @ |q| (+ |dX_in|)
+    q = np.abs(oracle.unpack_format(packed, K, layout).astype(np.float64))
+    g = np.abs((dY[sel] * (gam[None, :] if per_row else gam[0])).astype(np.float32).astype(np.float64))
+    mag = (g @ q) * (np.abs(rs[sel].astype(np.float64))[:, None] if use_rs else 1.0)
+    if accumulate:
+        mag = mag + np.abs(dX0[sel].astype(np.float64))
+    err = np.abs(got[sel].astype(np.float64) - want.astype(np.float64))
+    assert np.all(err <= REL * mag + 1e-30), f"max err/mag {np.max(err / (mag + 1e-30)):.3e}"
+    return err, mag
+
+
+@pytest.mark.parametrize("M,N,K,per_row,use_rs,acc,layout", [
+    (1, 1, 64, False, False, False, 0),        # one token, one output feature
+    (5, 17, 64, True, True, False, 0),         # ragged everything, N % 4 != 0
+    (300, 99, 192, False, False, True, 1),     # two token tiles, ragged; accumulate
+    (257, 1000, 384, True, True, False, 2),    # three feature tiles, ragged token tile
+    (512, 2048, 1024, False, True, True, 0),   # 4 x 8 tiles over 148 SMs
+])
+def test_backward_input_matches_oracle(cuda_lib, M, N, K, per_row, use_rs, acc, layout):
+    err, mag = _bwd_check(cuda_lib, M, N, K, per_row, use_rs, acc, layout, 140 + M)
+    assert cuda_lib.device_status() == 0
+
+
+def test_backward_input_full_size_sampled_rows(cuda_lib):
+    # the training workload: gradient of the prefill layer (2048 tokens,
+    # 11008 -> 4096), rows sampled across token tiles and the ragged corners
+    rows = [0, 1, 255, 256, 1000, 1791, 2046, 2047]
+    err, mag = _bwd_check(cuda_lib, 2048, 11008, 4096, False, False, False, 0, 150, rows)
+    # typical error far below the bound: the accumulation is fp32 over 11008 terms
+    assert np.median(err / (mag + 1e-30)) < 1e-6
+    assert cuda_lib.device_status() == 0
