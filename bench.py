@@ -72,6 +72,7 @@ def peaks():
 KERNEL_FILES = {  # sources that decide a kernel's memory traffic (besides tq_common.cuh, tq_api.cu)
     "pack": ["tq_pack.cuh"], "act_quant": ["tq_act.cuh"], "gemv": ["tq_gemv.cuh"],
     "gemm": ["tq_gemm.cuh"], "fused": ["tq_act.cuh", "tq_gemm.cuh"],
+    "bwd": ["tq_train.cuh", "tq_gemm.cuh"], "ste": ["tq_train.cuh"], "flip": ["tq_train.cuh", "tq_xorshift_jump.h"],
 }
 
 
@@ -225,6 +226,45 @@ class Workload:
                                            fl | tq.FLAG_WEIGHTS_STATIC, self.y[M][l], self.mws[l])
                 for l in range(layers)]))
             return
+        elif name == "train":
+            # one training step of the prefill layer (2048 tokens, 4096 -> 11008 features): the input
+            # gradient dX = (dY * gamma) W, the STE gradient of the latent weights and the
+            # stochastic flip of the packed codes (the weight-gradient GEMM X^T dY is a plain float
+            # GEMM outside this library: its output G is a synthetic input here)
+            M, N, K = 2048, 11008, 4096
+            self.N, self.K, self.Ms, self.L = N, K, [M], layers
+            self.per_row = False
+            self.layout, self.ratio = layout, ratio
+            fl = layout << 7
+            W, _ = S.prefill(M, N, K, seed=0)
+            dY = torch.from_numpy(S.normal((M, N), 1.0, 160, 0))
+            G = torch.from_numpy(S.normal((N, K), 1.0, 161, 0))
+            W = torch.from_numpy(W)
+            self.Wl = [W.to(dev) for _ in range(layers)]
+            self.G = [G.to(dev) for _ in range(layers)]
+            self.gw = [torch.empty((N, K), dtype=f32, device=dev) for _ in range(layers)]
+            self.packed = [torch.empty((N, K // 4), dtype=u8, device=dev) for _ in range(layers)]
+            self.gamma = [torch.empty((1,), dtype=f32, device=dev) for _ in range(layers)]
+            pws = torch.empty((tq.pack_workspace_bytes(N, K, 0),), dtype=u8, device=dev)
+            for l in range(layers):
+                tq.quantize_ternary_pack_(self.Wl[l], fl, self.packed[l], self.gamma[l], pws)
+            self.X = {M: dY}
+            self.Xd = {M: [dY.to(dev) for _ in range(layers)]}
+            self.y = {M: [torch.empty((M, K), dtype=f32, device=dev) for _ in range(layers)]}
+            self.bws = [torch.empty((tq.backward_input_workspace_bytes(M, N),), dtype=u8, device=dev)
+                        for _ in range(layers)]
+            self.rng = tq.seed(42)
+            self.segments.append(("backward dX M=%d" % M, "bwd", layers, layers * 2 * M * N * K, 2 * layers, [
+                lambda l=l: tq.ternary_backward_input_(self.Xd[M][l], self.packed[l], self.gamma[l], fl,
+                                                       self.y[M][l], self.bws[l])
+                for l in range(layers)]))
+            self.segments.append(("ste", "ste", layers, layers * 12 * N * K, layers, [
+                lambda l=l: tq.ste_backward_(self.G[l], self.Wl[l], self.gamma[l], 0, self.gw[l])
+                for l in range(layers)]))
+            self.segments.append(("flip", "flip", layers, layers * (4 * N * K + N * K // 2), layers, [
+                lambda l=l: tq.ternary_stochastic_flip_(self.packed[l], self.G[l], 0.05, self.rng, fl)
+                for l in range(layers)]))
+            return
         elif name == "roundtrip":
             # the FWHT module's int8 round trip on the fused configuration's activations
             M, K = 512, 2048
@@ -320,7 +360,7 @@ class Workload:
         return sum(s[3] for s in self.segments if s[1] in ("pack", "act_quant", "gemv", "roundtrip"))
 
     def step_ops(self):
-        return sum(s[3] for s in self.segments if s[1] in ("gemm", "fused", "mlp"))
+        return sum(s[3] for s in self.segments if s[1] in ("gemm", "fused", "mlp", "bwd"))
 
 
 def run_ours(args, rank, world, local_rank):
@@ -393,9 +433,10 @@ def run_ours(args, rank, world, local_rank):
     kernels = {}
     for (label, kname, launches, work, nlaunch, _), ms in zip(wl.segments, seg_ms):
         per_launch_ms = ms / args.steps / launches
-        if kname in ("gemm", "fused", "mlp"):
+        if kname in ("gemm", "fused", "mlp", "bwd"):
             ach = work / launches / (per_launch_ms * 1e-3) / 1e12
-            peak = pk["bf16"] * INT8_OVER_BF16
+            # the input gradient contracts bf16 operands (the int8 kernels: twice the bf16 rate)
+            peak = pk["bf16"] * (1.0 if kname == "bwd" else INT8_OVER_BF16)
             kernels[label] = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
                               "unit": "TOPS", "frac": round(ach / peak, 4),
                               "us_per_launch": round(per_launch_ms * 1e3, 3)}
@@ -410,6 +451,7 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "GB/s" if dk["unit"] == "GB/s" else "TOPS", "frac": dk["frac"],
                 "traffic": traffic_for(dom[1] + ":" + args.workload), "kernel": dom[0],
                 "peak_source": pk["source"] + (" hbm_gbs (copy, burst)" if dk["bound"] == "hbm"
+                                               else " bf16_tflops (bf16 operands)" if dom[1] == "bwd"
                                                else " bf16_tflops x2 (nominal int8/bf16 ratio)")}
     if wl.name in ("decode", "roundtrip"):
         value = wl.step_bytes() * world / (ms_per_step * 1e-3) / 1e9
@@ -426,7 +468,8 @@ def run_ours(args, rank, world, local_rank):
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.name == "train" else "int8",
         "data": "synthetic", "config": wl_config(wl, world),
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
         "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
@@ -445,6 +488,7 @@ WORKLOAD_SHAPES = {  # name -> (Ms, N, K, default ring of layers, per_row)
     "sweep": ([1, 4, 16, 64, 512, 4096], 8192, 8192, 8, True),
     "roundtrip": ([512], 0, 2048, 64, False),
     "mlp": ([512], 1536, 1536, 8, False),
+    "train": ([2048], 11008, 4096, 4, False),
 }
 
 
@@ -459,13 +503,18 @@ def config_for(name, layers, world, layout="foundry", ratio=0.0, bias=False):
             "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512, ring of %d layers" % L,
             "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L,
             "roundtrip": "FWHT module int8 round trip: 512 x 2048 Student-t(3), ring of %d batches" % L,
-            "mlp": "clamped SwiGLU block of 3 BitLinears: 512 tokens, d_model 1536, d_ffn 6144, ring of %d" % L}[name]
+            "mlp": "clamped SwiGLU block of 3 BitLinears: 512 tokens, d_model 1536, d_ffn 6144, ring of %d" % L,
+            "train": "training step of the prefill layer: dX = (dY gamma) W (M=2048, N=11008, K=4096), STE of "
+                     "the latent weights, stochastic flip (T=0.05), ring of %d layers" % L}[name]
     return {"workload": desc, "M": Ms, "N": N, "K": K, "layers": L,
             "gamma": "per-row" if per_row else "per-tensor", "layout": layout,
             "ternarise": "threshold w > %g * gamma" % ratio if ratio > 0 else "round/clamp",
             "epilogue": "y + bias (tq_ternary_gemm_ex)" if bias else "y",
-            "l2": "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
-                L * N * K * 4 >> 20, L * N * K // 4 >> 20),
+            "l2": ("inputs larger than L2 (no flush): per layer dY %d MiB, latent weights and their gradient "
+                   "2 x %d MiB, packed %d MiB" % (Ms[0] * N * 4 >> 20, N * K * 4 >> 20, N * K // 4 >> 20)
+                   if name == "train" else
+                   "inputs larger than L2 (no flush): fp32 weights %d MiB, packed %d MiB per step" % (
+                       L * N * K * 4 >> 20, L * N * K // 4 >> 20)),
             "parallelism": "replicas x%d" % world if world > 1 else "single GPU"}
 
 
@@ -580,6 +629,16 @@ def oracle_sample(workload):
         def fn():
             oracle.swiglu_mlp(X[:rows], packs[0], packs[1], packs[2], False)
         return fn, 2 * rows * 3 * D * F, "%d tokens through the block (weights pre-packed)" % rows, "TOPS"
+    if workload == "train":
+        M, N, K = 2048, 11008, 4096
+        W, _ = S.prefill(M, N, K, seed=0)
+        dY = S.normal((M, N), 1.0, 160, 0)
+        packed, gamma = oracle.quantize_pack(W, per_row=False)
+        rows = 2
+
+        def fn():
+            oracle.backward_input(dY[:rows], packed, gamma, False, K)
+        return fn, 2 * rows * N * K, "%d tokens of the input gradient (weights pre-packed)" % rows, "TOPS"
     if workload == "roundtrip":
         M, K = 512, 2048
         X = S.fused(M, 16, K, seed=0)[1]
@@ -644,7 +703,7 @@ def run_reference(args, rank, world):
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if args.workload == "train" else "int8",
         "data": "synthetic", "config": dict(config_for(args.workload, args.layers, world, args.layout), sample=what),
         "cpu_baseline": {"value": round(v, 6), "unit": unit, "cores": 1, "kind": "oracle",
                          "sample": what + " per step"},
@@ -677,7 +736,7 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "fused", "sweep", "roundtrip", "mlp"])
+                    choices=["decode", "prefill", "fused", "sweep", "roundtrip", "mlp", "train"])
     ap.add_argument("--bias", action="store_true",
                     help="contractions through tq_ternary_gemm_ex with a bias (the extra epilogue)")
     ap.add_argument("--ratio", type=float, default=0.0,

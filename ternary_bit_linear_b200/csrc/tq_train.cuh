@@ -270,37 +270,41 @@ __global__ void __launch_bounds__(kSplitThreads)
 }
 
 // --- the GEMM ---------------------------------------------------------------
-// Persistent, one CTA per SM.  Output tile: 128 input features (the MMA's M,
-// taken by the unpacked codes, A = W^T) x 256 tokens (the MMA's N, taken by
-// the bf16 planes, B = g).  The contraction dimension is the layer's N, in
-// steps of 32.  Per step: the three plane tiles [256 tokens][32 n] (64-byte
-// rows, 64-byte swizzle, K-major, by TMA), the packed tile [32 n][32 B] (by
-// TMA), and the code tile A [32 n][128 features] in bf16, written by the
-// unpackers in the 128-byte-swizzled MN-major layout (features contiguous:
-// the packed rows already are).  Six MMAs of K = 16 per step (two halves of
-// the step times three planes) into one fp32 accumulator.  Feature tiles
-// run fastest, so concurrently running CTAs share the token block's planes
-// in L2.  Warp roles as in the forward GEMM: 0 plane producer, 1 MMA issuer
-// and TMEM owner, 2 packed-weight producer, 4-11 unpackers (two groups
-// taking alternate steps), 12-19 epilogue.
-constexpr int kBwdTileF = 128;   // features per tile (MMA M)
+// Persistent, one CTA per SM.  Output tile: 256 input features (two MMAs of
+// M = 128, taken by the unpacked codes, A = W^T) x 256 tokens (the MMA's N,
+// taken by the bf16 planes, B = g).  The contraction dimension is the layer's
+// N, in steps of 32.  Per step: the three plane tiles [256 tokens][32 n]
+// (64-byte rows, 64-byte swizzle, K-major, by TMA), the packed tile
+// [32 n][64 B] (by TMA), and the code tiles A [32 n][2 x 128 features] in
+// bf16, written by the unpackers in the 128-byte-swizzled MN-major layout
+// (features contiguous: the packed rows already are).  Twelve MMAs of K = 16
+// per step (two halves of the step x two feature halves x three planes) into
+// two fp32 accumulators of 256 columns (all of tensor memory, so the next
+// tile's MMAs wait for the epilogue).  Both feature halves share each plane
+// tile, which halves the plane bytes each MMA needs from L2 against a
+// 128-feature tile.  Feature tiles run fastest, so concurrently running CTAs
+// share the token block's planes in L2.  Warp roles as in the forward GEMM:
+// 0 plane producer, 1 MMA issuer and TMEM owner, 2 packed-weight producer,
+// 4-11 unpackers (two groups taking alternate steps), 12-19 epilogue.
+constexpr int kBwdTileF = 256;   // features per tile (two MMAs of M = 128)
 constexpr int kBwdTileT = 256;   // tokens per tile (MMA N)
 constexpr int kBwdStepN = 32;    // contraction rows per step
 constexpr int kBwdPlanes = 3;
 constexpr int kBwdPlaneBytes = kBwdTileT * kBwdStepN * 2;             // 16 KB
-constexpr int kBwdABytes = kBwdTileF * kBwdStepN * 2;                 // 8 KB
-constexpr int kBwdStage = kBwdPlanes * kBwdPlaneBytes + kBwdABytes;   // 56 KB
+constexpr int kBwdAHalf = 128 * kBwdStepN * 2;                        // 8 KB per feature half
+constexpr int kBwdABytes = 2 * kBwdAHalf;
+constexpr int kBwdStage = kBwdPlanes * kBwdPlaneBytes + kBwdABytes;   // 64 KB
 constexpr int kBwdStages = 3;
-constexpr int kBwdWBytes = kBwdStepN * kBwdTileF / 4;                 // 1 KB packed per step
+constexpr int kBwdWBytes = kBwdStepN * kBwdTileF / 4;                 // 2 KB packed per step
 constexpr int kBwdWStages = 8;
 constexpr int kBwdOffW = kBwdStages * kBwdStage;
 constexpr int kBwdOffBar = kBwdOffW + kBwdWStages * kBwdWBytes;
-constexpr int kBwdBars = 2 * kBwdStages + 2 * kBwdWStages + 5;
+constexpr int kBwdBars = 2 * kBwdStages + 2 * kBwdWStages + 3;
 constexpr int kBwdOffTmem = kBwdOffBar + kBwdBars * 8;
 constexpr int kBwdDynamic = kBwdOffTmem + 16 + 1024;
-constexpr uint32_t kBwdTmemCols = 2 * kBwdTileT;  // two accumulators of 256 fp32 columns
+constexpr uint32_t kBwdTmemCols = 2 * kBwdTileT;  // two feature halves x 256 fp32 columns
 static_assert(kBwdDynamic <= 232448, "shared memory per CTA");
-static_assert(kBwdPlaneBytes % 1024 == 0 && kBwdABytes % 1024 == 0 && kBwdStage % 1024 == 0, "atoms aligned");
+static_assert(kBwdPlaneBytes % 1024 == 0 && kBwdAHalf % 1024 == 0 && kBwdStage % 1024 == 0, "atoms aligned");
 
 // Instruction descriptor, kind::f16: D f32, A and B bf16, A MN-major, B K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_amn(int M, int N) {
@@ -372,9 +376,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto empty = [&](int s) { return bar0 + 8u * (S + s); };
     auto w_full = [&](int s) { return bar0 + 8u * (2 * S + s); };
     auto w_empty = [&](int s) { return bar0 + 8u * (2 * S + SW + s); };
-    auto d_full = [&](int b) { return bar0 + 8u * (2 * S + 2 * SW + b); };
-    auto d_empty = [&](int b) { return bar0 + 8u * (2 * S + 2 * SW + 2 + b); };
-    const uint32_t mma_done = bar0 + 8u * (2 * S + 2 * SW + 4);
+    const uint32_t d_full = bar0 + 8u * (2 * S + 2 * SW);
+    const uint32_t d_empty = bar0 + 8u * (2 * S + 2 * SW + 1);
+    const uint32_t mma_done = bar0 + 8u * (2 * S + 2 * SW + 2);
     auto g_stage = [&](int s) { return sbase + (uint32_t)(s * kBwdStage); };
     auto a_stage = [&](int s) { return g_stage(s) + (uint32_t)(kBwdPlanes * kBwdPlaneBytes); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBwdOffTmem);
@@ -396,10 +400,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(w_full(s), 1);
             mbar_init(w_empty(s), kUnpackWarps / 2);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(d_full(b), 1);
-            mbar_init(d_empty(b), kEpiWarps);
-        }
+        mbar_init(d_full, 1);
+        mbar_init(d_empty, kEpiWarps);
         mbar_init(mma_done, 1);
         fence_barrier_init();
         prefetch_tmap(&tm_g);
@@ -454,14 +456,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_amn(kBwdTileF, kBwdTileT);
+            constexpr uint32_t idesc = idesc_bf16_amn(128, kBwdTileT);
             int g = 0;
             bool ok = true;
             for (int tl = 0; tl < my_tiles && ok; ++tl) {
-                const int b = tl & 1;
-                if (!mbar_wait(d_empty(b), ((tl >> 1) & 1) ^ 1)) break;
+                if (!mbar_wait(d_empty, (tl & 1) ^ 1)) break;  // the epilogue drained the accumulators
                 tc_fence_after();
-                const uint32_t d_col = tmem + (uint32_t)(b * kBwdTileT);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % S;
                     if (!mbar_wait(full(s), (g / S) & 1)) {
@@ -471,100 +471,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kBwdStepN / 16; ++kk) {
-                        const uint64_t ad = smem_desc_mn_sw128(a_stage(s) + (uint32_t)(kk * 4096), 1024u, 2048u);
 #pragma unroll
-                        for (int p = 0; p < kBwdPlanes; ++p)
-                            mma_bf16(d_col, ad,
-                                     smem_desc_k_sw64(g_stage(s) + (uint32_t)(p * kBwdPlaneBytes + kk * 32)),
-                                     idesc, (kb | kk | p) != 0 ? 1u : 0u);
+                        for (int p = 0; p < kBwdPlanes; ++p) {
+                            const uint64_t bd =
+                                smem_desc_k_sw64(g_stage(s) + (uint32_t)(p * kBwdPlaneBytes + kk * 32));
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                mma_bf16(tmem + (uint32_t)(h * kBwdTileT),
+                                         smem_desc_mn_sw128(a_stage(s) + (uint32_t)(h * kBwdAHalf + kk * 4096),
+                                                            1024u, 2048u),
+                                         bd, idesc, (kb | kk | p) != 0 ? 1u : 0u);
+                        }
                     }
                     mma_commit(empty(s));
                 }
-                if (ok) mma_commit(d_full(b));
+                if (ok) mma_commit(d_full);
             }
             mma_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
-        // ---------------- unpack codes into the MN-major bf16 tile ----------------
-        // Group thread i: contraction row c = 8 (warp % 4) + lane % 8, features
-        // 32 (lane / 8) .. + 32 (8 packed bytes -> four 16-byte chunks).
+        // ---------------- unpack codes into the MN-major bf16 tiles ----------------
+        // Group thread: contraction row c = 8 (warp % 4) + lane % 8, features
+        // 64 (lane / 8) .. + 64 (16 packed bytes -> eight 16-byte chunks).
         const int par = (warp - 4) >> 2;
         const int enc = (mode >> kModeEncShift) & 3;
         const int c = 8 * (warp & 3) + (lane & 7), fq = lane >> 3;
         const uint32_t r8 = (uint32_t)(c & 7);
-        const uint32_t a_row = (uint32_t)((c >> 3) * 2048) + r8 * 128u;
+        const uint32_t a_off = (uint32_t)((fq >> 1) * kBwdAHalf + (c >> 3) * 2048 + (fq & 1) * 1024) + r8 * 128u;
         for (int g = par; g < total; g += 2) {
             const int ws = g % SW, s = g % S;
             if (!warp_wait_sleep(w_full(ws), (g / SW) & 1, lane)) break;
-            uint32_t w0, w1;
-            asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
-                         : "=r"(w0), "=r"(w1)
-                         : "r"(sbase + (uint32_t)(kBwdOffW + ws * kBwdWBytes + c * 32 + fq * 8))
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(sbase + (uint32_t)(kBwdOffW + ws * kBwdWBytes + c * 64 + fq * 16))
                          : "memory");
             if (CONV) {
-                w0 = codes_to_foundry(w0, enc);
-                w1 = codes_to_foundry(w1, enc);
-            }
-            uint2 e[8];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                e[k] = codes4_to_bf16((w0 >> (8 * k)) & 0xFFu);
-                e[4 + k] = codes4_to_bf16((w1 >> (8 * k)) & 0xFFu);
+                for (int i = 0; i < 4; ++i) w[i] = codes_to_foundry(w[i], enc);
             }
+            uint2 e[16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) e[4 * i + k] = codes4_to_bf16((w[i] >> (8 * k)) & 0xFFu);
             __syncwarp();
             if (lane == 0) mbar_arrive(w_empty(ws));
             if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
-            const uint32_t base = a_stage(s) + a_row;
+            const uint32_t base = a_stage(s) + a_off;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int jg = 4 * fq + k;  // chunk of 8 features within the 128
-                const uint32_t addr =
-                    base + (uint32_t)((jg >> 3) * 1024) + ((((uint32_t)(jg & 7)) ^ r8) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(e[2 * k].x),
-                             "r"(e[2 * k].y), "r"(e[2 * k + 1].x), "r"(e[2 * k + 1].y)
+            for (int k = 0; k < 8; ++k)  // chunk k: features 8k .. 8k + 7 of this thread's 64
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base + ((((uint32_t)k) ^ r8) << 4)),
+                             "r"(e[2 * k].x), "r"(e[2 * k].y), "r"(e[2 * k + 1].x), "r"(e[2 * k + 1].y)
                              : "memory");
-            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(full(s));
         }
     } else if (warp >= 12) {
         // ---------------- epilogue ----------------
-        constexpr int kHalf = kBwdTileT / 2;
-        constexpr int kChunks = kHalf / 32;
+        constexpr int kChunks = kBwdTileT / 32;
         const int q = warp & 3;
-        const int half = (warp - 12) >> 2;
-        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+        const int h = (warp - 12) >> 2;  // feature half
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * kBwdTileT);
         for (int tl = 0; tl < my_tiles; ++tl) {
             const int t = (int)blockIdx.x + tl * (int)gridDim.x;
-            const int b = tl & 1;
-            const int f = (t % num_f) * kBwdTileF + 32 * q + lane;
-            const int m0 = (t / num_f) * kBwdTileT + half * kHalf;
-            float rsc[kChunks];
-#pragma unroll
-            for (int cc = 0; cc < kChunks; ++cc) {
-                const int mj = m0 + cc * 32 + lane;
-                rsc[cc] = (row_scale && mj < M) ? __ldg(row_scale + mj) : 1.0f;
-            }
-            if (!warp_wait_sleep(d_full(b), (tl >> 1) & 1, lane)) break;
+            const int f = (t % num_f) * kBwdTileF + 128 * h + 32 * q + lane;
+            const int m0 = (t / num_f) * kBwdTileT;
+            if (!warp_wait_sleep(d_full, tl & 1, lane)) break;
             tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int cc = 0; cc < kChunks; ++cc) {
                 uint32_t v[32];
-                tmem_ld32(lane_addr + (uint32_t)(b * kBwdTileT + half * kHalf + cc * 32), v);
+                tmem_ld32(lane_addr + (uint32_t)(cc * 32), v);
                 tmem_ld_wait();
                 if (cc == kChunks - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(d_empty(b));
+                    if (lane == 0) mbar_arrive(d_empty);
                 }
                 const int mb = m0 + cc * 32;
                 const int jmax = M - mb;
+                const float rsl = (row_scale && mb + lane < M) ? __ldg(row_scale + mb + lane) : 1.0f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float rs = __shfl_sync(0xffffffffu, rsc[cc], j);
+                    const float rs = __shfl_sync(0xffffffffu, rsl, j);
                     float o = __uint_as_float(v[j]);
                     if (row_scale) o = __fmul_rn(o, rs);
                     if (j < jmax && f < K) {

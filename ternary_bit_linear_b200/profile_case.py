@@ -3,6 +3,9 @@ self-contained command that ncu captures are taken on.
 
     python -m ternary_bit_linear_b200.profile_case --kernel gemv --M 8 --N 4096 --K 4096 --reps 3 [--ready]
 
+Training kernels: bwd (input gradient, dY [M][N] against the packed [N][K]),
+ste and flip (latent weights / gradient [N][K]).
+
 Inputs are random device tensors of the workloads' distributions (values do
 not affect timing); every call goes through the C ABI.  Exits non-zero if a
 call fails or the device status word reports a timeout.
@@ -19,7 +22,7 @@ import ternary_bit_linear_b200 as tq
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", required=True,
-                    choices=["pack_row", "pack_tensor", "act", "fwht", "gemv", "gemm", "fused"])
+                    choices=["pack_row", "pack_tensor", "act", "fwht", "gemv", "gemm", "fused", "bwd", "ste", "flip"])
     ap.add_argument("--M", type=int, default=8)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -42,6 +45,13 @@ def main():
                      dtype=torch.uint8, device=dev)
     pws = torch.empty((max(16, tq.pack_workspace_bytes(N, K, flags)),), dtype=torch.uint8, device=dev)
     Xr = torch.empty_like(X)
+    if a.kernel in ("bwd", "ste", "flip"):
+        dY = torch.randn((M, N), generator=g, device=dev)
+        dX = torch.empty((M, K), device=dev)
+        bws = torch.empty((tq.backward_input_workspace_bytes(M, N),), dtype=torch.uint8, device=dev)
+        G = torch.randn((N, K), generator=g, device=dev)
+        GW = torch.empty_like(G)
+        state = tq.seed(42)
     torch.cuda.synchronize()
     for _ in range(a.reps):
         if a.kernel in ("pack_row", "pack_tensor"):
@@ -53,6 +63,12 @@ def main():
         elif a.kernel in ("gemv", "gemm"):
             ready = tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY if a.ready else 0
             tq.ternary_gemm_(xq, sx, rs, packed, gamma, flags | ready, y)
+        elif a.kernel == "bwd":
+            tq.ternary_backward_input_(dY, packed, gamma, flags, dX, bws)
+        elif a.kernel == "ste":
+            tq.ste_backward_(G, W, gamma, flags, GW)
+        elif a.kernel == "flip":
+            state = tq.ternary_stochastic_flip_(packed, G, 0.05, state)
         else:
             tq.bitlinear_fused_(X, packed, gamma, tq.FLAG_FWHT | tq.FLAG_RMSNORM, y, ws)
     torch.cuda.synchronize()
