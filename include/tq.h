@@ -351,15 +351,18 @@ TQ_API size_t tq_swiglu_workspace_bytes(int64_t M, int64_t d_model, int64_t d_ff
  * = 1) is a per-token factor: Hetman-2b's BitLinear scales the contraction
  * by gamma * s_x per token (section 5 step 6) and its activation STE passes
  * the gradient of x_q on unchanged (section 2), so row_scale = s_x gives
- * that gradient.  Each product g = fp32(dY * gamma) is split exactly into
- * three bf16 parts and contracted on the tensor cores with fp32
- * accumulation: every product is exact, the accumulation rounds in fp32
- * (the result is within 1e-5 of sum_n |g q| of the exact sum).
+ * that gradient.  Each row of g = fp32(dY * gamma) is scaled by the power
+ * of two that puts its largest |g| in [2^14, 2^15) and split into two fp16
+ * parts (22 significant bits: error <= 2^-22 of each term, or 2^-39 of the
+ * row's largest term), contracted on the tensor cores with fp32
+ * accumulation and scaled back exactly (the result is within 1e-5 of
+ * sum_n |g q| of the exact sum).
  *
  *   dY         [M][N] fp32.          dX [M][K] fp32 (written, or updated).
- *   workspace  tq_backward_input_workspace_bytes(M, N) bytes (three bf16
- *              planes of dY * gamma), 16-byte aligned, owned by the caller.
- * K % 64 == 0, 64 <= K <= 65536; N >= 1; 1 <= M <= 715827882.
+ *   workspace  tq_backward_input_workspace_bytes(M, N) bytes (two fp16
+ *              planes of the scaled dY * gamma and one scale per token),
+ *              16-byte aligned, owned by the caller.
+ * K % 64 == 0, 64 <= K <= 65536; N >= 1; 1 <= M <= 1073741823.
  * flags: TQ_GAMMA_PER_ROW, TQ_FLAG_ACCUMULATE, TQ_ENC_*.
  * Errors: TQ_ERR_NULL, TQ_ERR_SHAPE, TQ_ERR_ALIGN (16 bytes), TQ_ERR_ARG
  * (flags, workspace too small, any overlap between dX or the workspace and

@@ -447,8 +447,8 @@ tq_status gemm_dispatch(const int8_t *xq, const float *s_x, const int32_t *rowsu
 // ---------------------------------------------------------------------------
 // Training helpers
 // ---------------------------------------------------------------------------
-// 2-D bf16 tensor [rows][cols] (row stride = 2 cols bytes), box [box_rows][box_cols].
-bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+// 2-D fp16 tensor [rows][cols] (row stride = 2 cols bytes), box [box_rows][box_cols].
+bool make_tmap_f16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                     uint32_t box_rows, CUtensorMapSwizzle swz) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
@@ -456,12 +456,12 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t ro
     cuuint64_t strides[1] = {cols * 2};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row length of the bf16 planes of the backward pass: N rounded up to a step.
+// Row length of the fp16 planes of the backward pass: N rounded up to a step.
 inline int64_t bwd_plane_cols(int64_t N) { return (N + kBwdStepN - 1) / kBwdStepN * kBwdStepN; }
 
 // Host copies of the xorshift64 jump tables: the state after a flip call.
@@ -513,14 +513,15 @@ tq_status launch_flip(uint8_t *packed, const float *grad, int64_t nw, float temp
 }
 
 template <bool CONV>
-tq_status launch_bwd_gemm(const uint16_t *planes, const uint8_t *packed, const float *row_scale, int accumulate,
+tq_status launch_bwd_gemm(const __half *planes, const float *inv_scale, const uint8_t *packed,
+                          const float *row_scale, int accumulate,
                           int64_t M, int64_t N, int64_t K, float *dX, int mode, int sms, cudaStream_t st) {
     static std::atomic<int> done[kMaxDevices];
     if (tq_status e = set_smem_once(bwd_gemm_kernel<CONV>, kBwdDynamic, done)) return e;
-    // planes [3 M][Np] bf16 in 64-byte-swizzled [256][32] boxes; packed [N][K/4]
+    // planes [2 M][Np] fp16 in 64-byte-swizzled [256][32] boxes; packed [N][K/4]
     // in plain [32][32 B] boxes.
     CUtensorMap tg, tw;
-    if (!make_tmap_bf16(&tg, planes, (uint64_t)bwd_plane_cols(N), (uint64_t)(3 * M), kBwdStepN, kBwdTileT,
+    if (!make_tmap_f16(&tg, planes, (uint64_t)bwd_plane_cols(N), (uint64_t)(kBwdPlanes * M), kBwdStepN, kBwdTileT,
                         CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_tmap_u8(&tw, packed, (uint64_t)(K / 4), (uint64_t)N, kBwdTileF / 4, kBwdStepN,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -528,7 +529,7 @@ tq_status launch_bwd_gemm(const uint16_t *planes, const uint8_t *packed, const f
     const int64_t tiles = ((M + kBwdTileT - 1) / kBwdTileT) * ((K + kBwdTileF - 1) / kBwdTileF);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
     return launch_pdl(bwd_gemm_kernel<CONV>, dim3(grid), dim3(kGemmThreads), (size_t)kBwdDynamic, st, tg, tw,
-                      row_scale, accumulate, (int)M, (int)N, (int)K, dX, mode);
+                      inv_scale, row_scale, accumulate, (int)M, (int)N, (int)K, dX, mode);
 }
 
 }  // namespace
@@ -898,14 +899,15 @@ tq_status tq_swiglu_mlp(const float *x, int64_t M, int64_t d_model, int64_t d_ff
 // ---------------------------------------------------------------------------
 size_t tq_backward_input_workspace_bytes(int64_t M, int64_t N) {
     if (M <= 0 || N <= 0) return 0;
-    return ((size_t)(3 * M * bwd_plane_cols(N)) * 2 + 255) & ~(size_t)255;
+    const size_t planes = ((size_t)(kBwdPlanes * M * bwd_plane_cols(N)) * 2 + 255) & ~(size_t)255;
+    return planes + (((size_t)M * 4 + 255) & ~(size_t)255);
 }
 
 tq_status tq_ternary_backward_input(const float *dY, const uint8_t *packed, const float *gamma,
                                     const float *row_scale, unsigned flags, int64_t M, int64_t N, int64_t K,
                                     float *dX, void *workspace, size_t workspace_bytes, tq_stream_t stream) {
     if (!dY || !packed || !gamma || !dX || !workspace) return TQ_ERR_NULL;
-    if (M < 1 || N < 1 || M > INT32_MAX / 3 || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (M < 1 || N < 1 || M > INT32_MAX / kBwdPlanes || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
     if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_ACCUMULATE | TQ_ENC_MASK)) return TQ_ERR_ARG;
     const int enc = flag_encoding(flags);
@@ -926,23 +928,23 @@ tq_status tq_ternary_backward_input(const float *dY, const uint8_t *packed, cons
     int sms = 0;
     if (tq_status e = check_device(&sms)) return e;
     cudaStream_t st = cs(stream);
-    uint16_t *planes = reinterpret_cast<uint16_t *>(workspace);
+    __half *planes = reinterpret_cast<__half *>(workspace);
     const int64_t Np = bwd_plane_cols(N);
+    float *inv_scale = reinterpret_cast<float *>(
+        reinterpret_cast<uint8_t *>(workspace) + (((size_t)(kBwdPlanes * M * Np) * 2 + 255) & ~(size_t)255));
     const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
-    const int64_t groups = M * (Np / 8);
-    const int64_t sgrid64 = (groups + kSplitThreads - 1) / kSplitThreads;
-    const unsigned sgrid = (unsigned)(sgrid64 < 8 * (int64_t)sms ? sgrid64 : 8 * (int64_t)sms);
+    const unsigned sgrid = (unsigned)(M < 8 * (int64_t)sms ? M : 8 * (int64_t)sms);  // one CTA per token row
     tq_status e = (N % 4 == 0)
                       ? launch_pdl(bwd_split_kernel<true>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
-                                   per_row, (int)M, (int)N, (int)Np, planes)
+                                   per_row, (int)M, (int)N, (int)Np, planes, inv_scale)
                       : launch_pdl(bwd_split_kernel<false>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
-                                   per_row, (int)M, (int)N, (int)Np, planes);
+                                   per_row, (int)M, (int)N, (int)Np, planes, inv_scale);
     if (e) return e;
     const int mode = enc << kModeEncShift;
     const int acc = (flags & TQ_FLAG_ACCUMULATE) ? 1 : 0;
     return enc != kEncFoundry
-               ? launch_bwd_gemm<true>(planes, packed, row_scale, acc, M, N, K, dX, mode, sms, st)
-               : launch_bwd_gemm<false>(planes, packed, row_scale, acc, M, N, K, dX, mode, sms, st);
+               ? launch_bwd_gemm<true>(planes, inv_scale, packed, row_scale, acc, M, N, K, dX, mode, sms, st)
+               : launch_bwd_gemm<false>(planes, inv_scale, packed, row_scale, acc, M, N, K, dX, mode, sms, st);
 }
 
 tq_status tq_ste_backward(const float *grad, const float *w, const float *gamma, int64_t N, int64_t K,

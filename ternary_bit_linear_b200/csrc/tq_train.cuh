@@ -12,7 +12,7 @@
 #pragma once
 
 #include <cuda.h>
-#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "tq_common.cuh"
 #include "tq_gemm.cuh"
@@ -208,77 +208,103 @@ __global__ void __launch_bounds__(kFlipThreads, 2)
 // ===========================================================================
 // The contraction runs over the N output features with fp32 operands on one
 // side and codes in {-1, 0, +1} on the other.  It is a dense GEMM, so it runs
-// on the tensor cores (tcgen05 kind::f16, bf16 operands, fp32 accumulation in
-// tensor memory) with the fp32 side split exactly into three bf16 planes:
-//   g = fp32(dY * gamma_n),  h = bf16(g),  m = bf16(g - h),  l = bf16(g - h - m)
-// (each difference is exact in fp32 and h + m + l = g: 8 + 8 + 8 significant
-// bits hold fp32's 24).  Every product with a code is exact, so the only
-// rounding is the fp32 accumulation of the tensor core.
+// on the tensor cores (tcgen05 kind::f16, fp16 operands, fp32 accumulation in
+// tensor memory).  The fp32 side is scaled per token by a power of two that
+// puts the row's largest |g| in [2^14, 2^15), then split into two fp16 parts:
+//   g = fp32(dY * gamma_n),  v = g * 2^e_t (exact),
+//   hi = fp16(v),  lo = fp16(v - hi)           (v - hi is exact in fp32)
+// hi + lo keeps 22 of fp32's 24 significant bits (|v - hi - lo| <= 2^-22 |v|,
+// or 2^-25 absolute where lo is subnormal, i.e. 2^-39 of the row's largest
+// term).  Products with a code are exact, the tensor core accumulates in
+// fp32, and the epilogue multiplies by 2^-e_t (exact) and row_scale.
 
-// --- split pass: planes [3][M][Np] bf16, columns N .. Np - 1 zero ---------
+// --- split pass: planes [2][M][Np] fp16 (columns N .. Np - 1 zero), then
+// inv_scale [M] fp32 = 2^-e_t.  One CTA per token row. --------------------
 constexpr int kSplitThreads = 256;
 
-__device__ __forceinline__ void split3(float g, uint16_t &h, uint16_t &m, uint16_t &l) {
-    const __nv_bfloat16 bh = __float2bfloat16_rn(g);
-    const float r1 = __fsub_rn(g, __bfloat162float(bh));
-    const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
-    const float r2 = __fsub_rn(r1, __bfloat162float(bm));
-    const __nv_bfloat16 bl = __float2bfloat16_rn(r2);
-    h = __bfloat16_as_ushort(bh);
-    m = __bfloat16_as_ushort(bm);
-    l = __bfloat16_as_ushort(bl);
+// 8 columns of row `row` starting at c0 (zero beyond N), times the column scale.
+template <bool VEC>
+__device__ __forceinline__ void load_g8(const float *row, const float *gamma, int per_row, float g0, int N, int c0,
+                                        float (&v)[8]) {
+    if (VEC && c0 + 8 <= N) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(row + c0));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(row + c0 + 4));
+        v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = c0 + j < N ? __ldg(row + c0 + j) : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float sc = per_row ? (c0 + j < N ? __ldg(gamma + c0 + j) : 0.0f) : g0;
+        v[j] = c0 + j < N ? __fmul_rn(v[j], sc) : 0.0f;
+    }
 }
 
-// One thread per 8 columns of a row.  VEC: rows are 16-byte aligned (N % 4 == 0).
+// VEC: rows are 16-byte aligned (N % 4 == 0).
 template <bool VEC>
 __global__ void __launch_bounds__(kSplitThreads)
     bwd_split_kernel(const float *__restrict__ dY, const float *__restrict__ gamma, int per_row, int M, int N,
-                     int Np, uint16_t *__restrict__ planes) {
+                     int Np, __half *__restrict__ planes, float *__restrict__ inv_scale) {
+    __shared__ float red[kSplitThreads / 32];
     pdl_wait();
     pdl_trigger();
-    const int gpr = Np / 8;  // groups per row
-    const int64_t total = (int64_t)M * gpr, plane = (int64_t)M * Np;
+    const int64_t plane = (int64_t)M * Np;
     const float g0 = __ldg(gamma);
-    for (int64_t i = (int64_t)blockIdx.x * kSplitThreads + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * kSplitThreads) {
-        const int t = (int)(i / gpr), c0 = (int)(i % gpr) * 8;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int t = blockIdx.x; t < M; t += gridDim.x) {
         const float *row = dY + (int64_t)t * N;
-        float v[8];
-        if (VEC && c0 + 8 <= N) {
-            const float4 a = __ldcs(reinterpret_cast<const float4 *>(row + c0));
-            const float4 b = __ldcs(reinterpret_cast<const float4 *>(row + c0 + 4));
-            v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
-        } else {
+        float mx = 0.0f;
+        for (int c0 = threadIdx.x * 8; c0 < N; c0 += kSplitThreads * 8) {
+            float v[8];
+            load_g8<VEC>(row, gamma, per_row, g0, N, c0, v);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = c0 + j < N ? __ldcs(row + c0 + j) : 0.0f;
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(v[j]));
         }
-        uint16_t h[8], m[8], l[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float sc = per_row ? (c0 + j < N ? __ldg(gamma + c0 + j) : 0.0f) : g0;
-            split3(c0 + j < N ? __fmul_rn(v[j], sc) : 0.0f, h[j], m[j], l[j]);
+        for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red[warp] = mx;
+        __syncthreads();
+        mx = red[0];
+#pragma unroll
+        for (int w = 1; w < kSplitThreads / 32; ++w) mx = fmaxf(mx, red[w]);
+        __syncthreads();  // red is reused by the next row
+        // scale 2^e with mx * 2^e in [2^14, 2^15); 1 for a zero or non-finite row
+        float sc = 1.0f, inv = 1.0f;
+        if (mx > 0.0f && mx <= 3.4028235e38f) {
+            int E;
+            frexpf(mx, &E);  // mx = m 2^E, m in [0.5, 1)
+            sc = ldexpf(1.0f, 15 - E);
+            inv = ldexpf(1.0f, E - 15);
         }
-        auto pack8 = [](const uint16_t (&s)[8]) {
-            return make_uint4(s[0] | (uint32_t)s[1] << 16, s[2] | (uint32_t)s[3] << 16, s[4] | (uint32_t)s[5] << 16,
-                              s[6] | (uint32_t)s[7] << 16);
-        };
-        uint16_t *o = planes + (int64_t)t * Np + c0;
-        *reinterpret_cast<uint4 *>(o) = pack8(h);
-        *reinterpret_cast<uint4 *>(o + plane) = pack8(m);
-        *reinterpret_cast<uint4 *>(o + 2 * plane) = pack8(l);
+        if (threadIdx.x == 0) inv_scale[t] = inv;
+        __half *o = planes + (int64_t)t * Np;
+        for (int c0 = threadIdx.x * 8; c0 < Np; c0 += kSplitThreads * 8) {
+            float v[8];
+            load_g8<VEC>(row, gamma, per_row, g0, N, c0, v);
+            __align__(16) __half hi[8], lo[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float x = __fmul_rn(v[j], sc);
+                hi[j] = __float2half_rn(x);
+                lo[j] = __float2half_rn(__fsub_rn(x, __half2float(hi[j])));
+            }
+            *reinterpret_cast<uint4 *>(o + c0) = *reinterpret_cast<const uint4 *>(hi);
+            *reinterpret_cast<uint4 *>(o + plane + c0) = *reinterpret_cast<const uint4 *>(lo);
+        }
     }
 }
 
 // --- the GEMM ---------------------------------------------------------------
 // Persistent, one CTA per SM.  Output tile: 256 input features (two MMAs of
 // M = 128, taken by the unpacked codes, A = W^T) x 256 tokens (the MMA's N,
-// taken by the bf16 planes, B = g).  The contraction dimension is the layer's
-// N, in steps of 32.  Per step: the three plane tiles [256 tokens][32 n]
+// taken by the fp16 planes, B = g).  The contraction dimension is the layer's
+// N, in steps of 32.  Per step: the two plane tiles [256 tokens][32 n]
 // (64-byte rows, 64-byte swizzle, K-major, by TMA), the packed tile
 // [32 n][64 B] (by TMA), and the code tiles A [32 n][2 x 128 features] in
-// bf16, written by the unpackers in the 128-byte-swizzled MN-major layout
-// (features contiguous: the packed rows already are).  Twelve MMAs of K = 16
-// per step (two halves of the step x two feature halves x three planes) into
+// fp16, written by the unpackers in the 128-byte-swizzled MN-major layout
+// (features contiguous: the packed rows already are).  Eight MMAs of K = 16
+// per step (two halves of the step x two feature halves x two planes) into
 // two fp32 accumulators of 256 columns (all of tensor memory, so the next
 // tile's MMAs wait for the epilogue).  Both feature halves share each plane
 // tile, which halves the plane bytes each MMA needs from L2 against a
@@ -289,12 +315,12 @@ __global__ void __launch_bounds__(kSplitThreads)
 constexpr int kBwdTileF = 256;   // features per tile (two MMAs of M = 128)
 constexpr int kBwdTileT = 256;   // tokens per tile (MMA N)
 constexpr int kBwdStepN = 32;    // contraction rows per step
-constexpr int kBwdPlanes = 3;
+constexpr int kBwdPlanes = 2;
 constexpr int kBwdPlaneBytes = kBwdTileT * kBwdStepN * 2;             // 16 KB
 constexpr int kBwdAHalf = 128 * kBwdStepN * 2;                        // 8 KB per feature half
 constexpr int kBwdABytes = 2 * kBwdAHalf;
-constexpr int kBwdStage = kBwdPlanes * kBwdPlaneBytes + kBwdABytes;   // 64 KB
-constexpr int kBwdStages = 3;
+constexpr int kBwdStage = kBwdPlanes * kBwdPlaneBytes + kBwdABytes;   // 48 KB
+constexpr int kBwdStages = 4;
 constexpr int kBwdWBytes = kBwdStepN * kBwdTileF / 4;                 // 2 KB packed per step
 constexpr int kBwdWStages = 8;
 constexpr int kBwdOffW = kBwdStages * kBwdStage;
@@ -306,17 +332,17 @@ constexpr uint32_t kBwdTmemCols = 2 * kBwdTileT;  // two feature halves x 256 fp
 static_assert(kBwdDynamic <= 232448, "shared memory per CTA");
 static_assert(kBwdPlaneBytes % 1024 == 0 && kBwdAHalf % 1024 == 0 && kBwdStage % 1024 == 0, "atoms aligned");
 
-// Instruction descriptor, kind::f16: D f32, A and B bf16, A MN-major, B K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_amn(int M, int N) {
+// Instruction descriptor, kind::f16: D f32, A and B f16, A MN-major, B K-major.
+__host__ __device__ constexpr uint32_t idesc_f16_amn(int M, int N) {
     return (1u << 4)                        // D format: f32
-           | (1u << 7)                      // A: bf16
-           | (1u << 10)                     // B: bf16
+           | (0u << 7)                      // A: f16
+           | (0u << 10)                     // B: f16
            | (1u << 15)                     // A MN-major
            | ((uint32_t)(N >> 3) << 17)     // N / 8
            | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
-// MN-major bf16 operand, 128-byte swizzle: atoms of 8 contraction rows x 64
+// MN-major 16-bit operand, 128-byte swizzle: atoms of 8 contraction rows x 64
 // elements (128 B per row, 16-byte chunk index XOR row % 8); atoms along M
 // are `lbo` bytes apart, atoms along the contraction (8-row groups) `sbo`.
 __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -340,7 +366,7 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw64(uint32_t saddr) {
     return d;
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -349,24 +375,24 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
-// Four codes (one packed byte, Foundry's layout) -> four bf16 of q = field - 1
-// (0b00 -> -1.0 = 0xBF80, 0b01 -> 0, 0b10 -> +1.0 = 0x3F80; the unassigned
-// 0b11 gives 2.0).  A byte permute picks each half of each bf16 from two
-// four-entry tables (high bytes BF 00 3F 40, low bytes 80 00 80 00).
-__device__ __forceinline__ uint2 codes4_to_bf16(uint32_t byte) {
+// Four codes (one packed byte, Foundry's layout) -> four fp16 of q = field - 1
+// (0b00 -> -1.0 = 0xBC00, 0b01 -> 0, 0b10 -> +1.0 = 0x3C00; the unassigned
+// 0b11 gives 2.0 = 0x4000).  A byte permute picks the high byte of each fp16
+// from the four-entry table BC 00 3C 40 and a zero low byte.
+__device__ __forceinline__ uint2 codes4_to_f16(uint32_t byte) {
     const uint32_t n0 = byte & 0xFu, n1 = (byte >> 4) & 0xFu;
     const uint32_t s0 = 0x0404u + (n0 & 3u) * 0x11u + (n0 >> 2) * 0x1100u;
     const uint32_t s1 = 0x0404u + (n1 & 3u) * 0x11u + (n1 >> 2) * 0x1100u;
-    return make_uint2(__byte_perm(0x403F00BFu, 0x00800080u, s0), __byte_perm(0x403F00BFu, 0x00800080u, s1));
+    return make_uint2(__byte_perm(0x403C00BCu, 0u, s0), __byte_perm(0x403C00BCu, 0u, s1));
 }
 
-// planes: tensor map over [3 M][Np] bf16 (plane p of token t is row p M + t);
-// packed: tensor map over [N][K / 4] bytes.  dX [M][K] fp32.
+// planes: tensor map over [2 M][Np] fp16 (plane p of token t is row p M + t);
+// packed: tensor map over [N][K / 4] bytes; inv_scale [M] = 2^-e_t.  dX [M][K] fp32.
 template <bool CONV>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_w,
-                    const float *__restrict__ row_scale, int accumulate, int M, int N, int K,
-                    float *__restrict__ dX, int mode) {
+                    const float *__restrict__ inv_scale, const float *__restrict__ row_scale, int accumulate, int M,
+                    int N, int K, float *__restrict__ dX, int mode) {
     constexpr int S = kBwdStages, SW = kBwdWStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -456,7 +482,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_amn(128, kBwdTileT);
+            constexpr uint32_t idesc = idesc_f16_amn(128, kBwdTileT);
             int g = 0;
             bool ok = true;
             for (int tl = 0; tl < my_tiles && ok; ++tl) {
@@ -477,7 +503,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 smem_desc_k_sw64(g_stage(s) + (uint32_t)(p * kBwdPlaneBytes + kk * 32));
 #pragma unroll
                             for (int h = 0; h < 2; ++h)
-                                mma_bf16(tmem + (uint32_t)(h * kBwdTileT),
+                                mma_f16(tmem + (uint32_t)(h * kBwdTileT),
                                          smem_desc_mn_sw128(a_stage(s) + (uint32_t)(h * kBwdAHalf + kk * 4096),
                                                             1024u, 2048u),
                                          bd, idesc, (kb | kk | p) != 0 ? 1u : 0u);
@@ -492,7 +518,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
-        // ---------------- unpack codes into the MN-major bf16 tiles ----------------
+        // ---------------- unpack codes into the MN-major fp16 tiles ----------------
         // Group thread: contraction row c = 8 (warp % 4) + lane % 8, features
         // 64 (lane / 8) .. + 64 (16 packed bytes -> eight 16-byte chunks).
         const int par = (warp - 4) >> 2;
@@ -516,7 +542,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int k = 0; k < 4; ++k) e[4 * i + k] = codes4_to_bf16((w[i] >> (8 * k)) & 0xFFu);
+                for (int k = 0; k < 4; ++k) e[4 * i + k] = codes4_to_f16((w[i] >> (8 * k)) & 0xFFu);
             __syncwarp();
             if (lane == 0) mbar_arrive(w_empty(ws));
             if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
@@ -554,11 +580,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 const int mb = m0 + cc * 32;
                 const int jmax = M - mb;
-                const float rsl = (row_scale && mb + lane < M) ? __ldg(row_scale + mb + lane) : 1.0f;
+                const bool in = mb + lane < M;
+                const float isl = in ? __ldg(inv_scale + mb + lane) : 1.0f;
+                const float rsl = (row_scale && in) ? __ldg(row_scale + mb + lane) : 1.0f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const float rs = __shfl_sync(0xffffffffu, rsl, j);
-                    float o = __uint_as_float(v[j]);
+                    float o = __fmul_rn(__uint_as_float(v[j]), __shfl_sync(0xffffffffu, isl, j));  // exact
                     if (row_scale) o = __fmul_rn(o, rs);
                     if (j < jmax && f < K) {
                         float *p = dX + (int64_t)(mb + j) * K + f;
