@@ -69,7 +69,7 @@ def peaks():
                 "source": "fallback"}
 
 
-KERNEL_FILES = {  # sources that decide a kernel's memory traffic (besides tq_common.cuh, tq_api.cu)
+KERNEL_FILES = {  # device sources of each kernel (besides tq_common.cuh)
     "pack": ["tq_pack.cuh"], "act_quant": ["tq_act.cuh"], "gemv": ["tq_gemv.cuh"],
     "gemm": ["tq_gemm.cuh"], "fused": ["tq_act.cuh", "tq_gemm.cuh"],
     "bwd": ["tq_train.cuh", "tq_gemm.cuh"], "ste": ["tq_train.cuh"], "flip": ["tq_train.cuh", "tq_xorshift_jump.h"],
@@ -79,7 +79,7 @@ KERNEL_FILES = {  # sources that decide a kernel's memory traffic (besides tq_co
 def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ternary_bit_linear_b200", "csrc")
-    for name in ["tq_common.cuh", "tq_api.cu"] + KERNEL_FILES[kernel]:
+    for name in ["tq_common.cuh"] + KERNEL_FILES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
