@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int q = warp & 3;                // TMEM lane quarter
         const int half = (warp - 12) >> 2;     // token half of the tile
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+        const bool vec4 = (N & 3) == 0;  // rows of y are 16-byte multiples
         for (int tl = 0; tl < my_tiles; ++tl) {
             const int t = (int)blockIdx.x + tl * (int)gridDim.x;
             const int b = tl & 1;
@@ -333,7 +334,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const float yv = __fmul_rn(__int2float_rn((int)v[j] - rsm), __fmul_rn(gn, sxm));
                         v[j] = __float_as_uint(EPI ? __fadd_rn(yv, bn) : yv);
                     }
-                    if (n < N) {
+                    if (vec4) {
+                        // 4 x 4 transposes inside each lane quad: lane 4g + r then holds
+                        // token 4k + r of features 4g .. 4g + 3 and stores them as one
+                        // 16-byte vector (a quarter of the store instructions).
+                        const int r = lane & 3;
+                        float *yq = y + (int64_t)(mb + r) * N + (n - (lane & 3));
+                        const bool fin = n - r < N;  // the quad's four features are all < N
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            float a0 = __uint_as_float(v[4 * k]), a1 = __uint_as_float(v[4 * k + 1]);
+                            float a2 = __uint_as_float(v[4 * k + 2]), a3 = __uint_as_float(v[4 * k + 3]);
+                            // distance 1: swap the odd/even off-diagonal elements of lane pairs
+                            const bool o1 = r & 1;
+                            const float x1 = __shfl_xor_sync(0xffffffffu, o1 ? a0 : a1, 1);
+                            const float y1 = __shfl_xor_sync(0xffffffffu, o1 ? a2 : a3, 1);
+                            if (o1) { a0 = x1; a2 = y1; } else { a1 = x1; a3 = y1; }
+                            // distance 2: swap the off-diagonal 2 x 2 blocks of lane pairs
+                            const bool o2 = r & 2;
+                            const float x2 = __shfl_xor_sync(0xffffffffu, o2 ? a0 : a2, 2);
+                            const float y2 = __shfl_xor_sync(0xffffffffu, o2 ? a1 : a3, 2);
+                            if (o2) { a0 = x2; a1 = y2; } else { a2 = x2; a3 = y2; }
+                            if (fin && 4 * k + r < jmax)
+                                __stcs(reinterpret_cast<float4 *>(yq + (int64_t)(4 * k) * N), make_float4(a0, a1, a2, a3));
+                        }
+                    } else if (n < N) {
                         float *yp = y + (int64_t)mb * N + n;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
