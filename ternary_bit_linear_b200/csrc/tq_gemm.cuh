@@ -270,8 +270,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint4 e[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) e[c] = expand_word(words[c]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(w_empty(ws));  // packed bytes are in registers
             if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
             // 16-byte chunk c of row r lives at chunk position c ^ (r & 7)
             const uint32_t base = a_stage(s) + a_row;
@@ -282,7 +280,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              : "memory");
             fence_proxy_async_smem();  // generic stores -> visible to the tensor core
             __syncwarp();
-            if (lane == 0) mbar_arrive(full(s));
+            // The packed slot is released only now: the stores above consume the
+            // loaded words, so every lane's read of the slot is complete before
+            // the producer may refill it.
+            if (lane == 0) {
+                mbar_arrive(w_empty(ws));
+                mbar_arrive(full(s));
+            }
         }
     } else if (warp >= 12) {
         // ---------------- epilogue ----------------

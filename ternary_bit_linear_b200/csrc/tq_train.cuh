@@ -108,6 +108,11 @@ __device__ __forceinline__ uint64_t lane_matvec(const uint64_t *tab, uint64_t x,
     return r;
 }
 
+// New field of a weight, two bits per entry at index field + 4 * action, with
+// the field read as q + 1 (the unassigned 0b11 as q = 0) and q clamped to
+// [-1, 1]:  keep 0 1 2 1 | down 0 0 1 0 | up 1 2 2 2.
+constexpr uint32_t kFlipTable = 0x00A91064u;
+
 // Four weights (one packed byte in Foundry's layout) against the next four draws.
 __device__ __forceinline__ uint32_t flip_byte(uint32_t byte, const float4 g4, float temp, uint64_t &x) {
     const float gs[4] = {g4.x, g4.y, g4.z, g4.w};
@@ -120,13 +125,10 @@ __device__ __forceinline__ uint32_t flip_byte(uint32_t byte, const float4 g4, fl
         const float u = __fmul_rn(__uint2float_rn((uint32_t)(x >> 40)), 0x1p-24f);  // exact
         const float a = __fmul_rn(fabsf(gs[i]), temp);
         const float p = a > 1.0f ? 1.0f : a;  // NaN stays NaN: u < p is false
+        // action: 0 keep, 1 one step down (grad > 0), 2 one step up (grad < 0)
+        const uint32_t act = u < p ? (gs[i] > 0.0f ? 1u : (gs[i] < 0.0f ? 2u : 0u)) : 0u;
         const uint32_t f = (byte >> (2 * i)) & 3u;
-        int q = f == 3u ? 0 : (int)f - 1;     // the unassigned field reads as 0
-        if (u < p) {
-            const int s = gs[i] > 0.0f ? 1 : (gs[i] < 0.0f ? -1 : 0);
-            q = max(-1, min(1, q - s));
-        }
-        out |= (uint32_t)(q + 1) << (2 * i);
+        out |= ((kFlipTable >> (2 * (f + 4 * act))) & 3u) << (2 * i);
     }
     return out;
 }
@@ -543,8 +545,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) e[4 * i + k] = codes4_to_f16((w[i] >> (8 * k)) & 0xFFu);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(w_empty(ws));
             if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
             const uint32_t base = a_stage(s) + a_off;
 #pragma unroll
@@ -554,7 +554,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              : "memory");
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(full(s));
+            // The packed slot is released only now: the stores above consume the
+            // loaded words, so every lane's read of the slot is complete before
+            // the producer may refill it (an arrive right after the loads let a
+            // refill overtake a lane's read).
+            if (lane == 0) {
+                mbar_arrive(w_empty(ws));
+                mbar_arrive(full(s));
+            }
         }
     } else if (warp >= 12) {
         // ---------------- epilogue ----------------
@@ -585,13 +592,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const float rsl = (row_scale && in) ? __ldg(row_scale + mb + lane) : 1.0f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float rs = __shfl_sync(0xffffffffu, rsl, j);
                     float o = __fmul_rn(__uint_as_float(v[j]), __shfl_sync(0xffffffffu, isl, j));  // exact
-                    if (row_scale) o = __fmul_rn(o, rs);
-                    if (j < jmax && f < K) {
-                        float *p = dX + (int64_t)(mb + j) * K + f;
-                        if (accumulate) o = __fadd_rn(*p, o);
-                        __stcs(p, o);
+                    if (row_scale) o = __fmul_rn(o, __shfl_sync(0xffffffffu, rsl, j));
+                    v[j] = __float_as_uint(o);
+                }
+                // 4 x 4 transposes inside each lane quad: lane 4g + r then holds token
+                // 4k + r of features 4g .. 4g + 3, stored as one 16-byte vector
+                // (K % 64 == 0 keeps every row 16-byte aligned).
+                const int r = lane & 3;
+                float *xq = dX + (int64_t)(mb + r) * K + (f - r);
+                const bool fin = f - r < K;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    float a0 = __uint_as_float(v[4 * k]), a1 = __uint_as_float(v[4 * k + 1]);
+                    float a2 = __uint_as_float(v[4 * k + 2]), a3 = __uint_as_float(v[4 * k + 3]);
+                    const bool o1 = r & 1;
+                    const float x1 = __shfl_xor_sync(0xffffffffu, o1 ? a0 : a1, 1);
+                    const float y1 = __shfl_xor_sync(0xffffffffu, o1 ? a2 : a3, 1);
+                    if (o1) { a0 = x1; a2 = y1; } else { a1 = x1; a3 = y1; }
+                    const bool o2 = r & 2;
+                    const float x2 = __shfl_xor_sync(0xffffffffu, o2 ? a0 : a2, 2);
+                    const float y2 = __shfl_xor_sync(0xffffffffu, o2 ? a1 : a3, 2);
+                    if (o2) { a0 = x2; a1 = y2; } else { a2 = x2; a3 = y2; }
+                    if (fin && 4 * k + r < jmax) {
+                        float4 *p = reinterpret_cast<float4 *>(xq + (int64_t)(4 * k) * K);
+                        if (accumulate) {
+                            const float4 b = *p;
+                            a0 = __fadd_rn(b.x, a0), a1 = __fadd_rn(b.y, a1);
+                            a2 = __fadd_rn(b.z, a2), a3 = __fadd_rn(b.w, a3);
+                        }
+                        __stcs(p, make_float4(a0, a1, a2, a3));
                     }
                 }
             }

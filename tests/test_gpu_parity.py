@@ -978,3 +978,32 @@ def test_backward_input_full_size_sampled_rows(cuda_lib):
     # typical error far below the bound: the accumulation is fp32 over 11008 terms
     assert np.median(err / (mag + 1e-30)) < 1e-6
     assert cuda_lib.device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# Repeated calls are bit-identical (every result is a fixed function of the
+# inputs).  Full size, where a pipeline hazard shows up: the packed-weight
+# slot of the unpackers was once released before every lane's read of it
+# was complete, and a refill could overtake the read.
+# ---------------------------------------------------------------------------
+def test_gemms_repeat_bit_identical_full_size(cuda_lib):
+    tq = cuda_lib
+    M, N, K = 2048, 11008, 4096
+    W, X = cached("prefill", M, N, K, 0)
+    pk, gm = tq.quantize_ternary_pack(dev(W), per_row=False)
+    xq, sx, rs = tq.quantize_act_int8(dev(X))
+    accs = []
+    for _ in range(4):
+        _, acc = tq.ternary_gemm(xq, sx, rs, pk, gm, per_row=False, with_acc=True)
+        accs.append(host(acc))
+    assert all(np.array_equal(a, accs[0]) for a in accs[1:])
+    dY = dev(S.normal((M, N), 1.0, 160, 0))
+    ws = torch.empty((tq.backward_input_workspace_bytes(M, N),), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(6):
+        dX = torch.full((M, K), float("nan"), dtype=torch.float32, device="cuda")
+        tq.ternary_backward_input_(dY, pk, gm, 0, dX, ws)
+        outs.append(host(dX))
+    assert not np.isnan(outs[0]).any()
+    assert all(np.array_equal(o, outs[0]) for o in outs[1:])
+    assert tq.device_status() == 0
