@@ -1,7 +1,8 @@
 """Benchmark of the ternary linear layer hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|fused|sweep]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload decode|prefill|fused|sweep|roundtrip|mlp|train]
+                    [--layout foundry|format0|format1] [--ratio R] [--bias] [--impl ours|reference]
 
 One JSON line on rank 0.  A *step* is one pass of the whole hot path over one
 batch of synthetic input: quantise + pack the fp32 latent weights (absmean
@@ -29,6 +30,16 @@ Timing: CUDA graphs for each segment (pack, activation quantisation, GEMV
 M=1, GEMV M=8), CUDA events between segments on the launching stream, barrier
 + synchronize around the timed steps, max over ranks.  Per-kernel average
 launch time = segment time / launches in the segment.
+
+Other workloads: "prefill" (2048 x 11008 x 4096 GEMM, per-tensor gamma),
+"fused" (RMSNorm + FWHT + int8 + GEMM, 512 x 5632 x 2048), "sweep" (M from 1
+to 4096 at 8192^2), "roundtrip" (the FWHT module's int8 round trip), "mlp"
+(the clamped SwiGLU block, 512 tokens, 1536 -> 6144 -> 1536) and "train" (the
+input gradient of the prefill layer, the STE of its latent weights and the
+stochastic flip of its codes); --layout, --ratio and --bias select the
+packed-code layout, the threshold ternarisation rule and the bias epilogue.
+Metric: TOPS (TFLOP/s for train) of the step's contractions / step time for
+the GEMM workloads, GB/s for decode and roundtrip.
 
 --impl reference times the CPU oracle (the plain C reference) on a bounded
 sample of the same workload, on this host's cores.
@@ -445,6 +456,8 @@ def run_ours(args, rank, world, local_rank):
             kernels[label] = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"],
                               "unit": "GB/s", "frac": round(ach / pk["hbm"], 4),
                               "us_per_launch": round(per_launch_ms * 1e3, 3)}
+            if kname == "flip":  # the xorshift64 chain keeps the ALU pipe busy before HBM
+                kernels[label]["limiter"] = "alu pipe"
     dom = max(zip(wl.segments, seg_ms), key=lambda t: t[1])[0]
     dk = kernels[dom[0]]
     roofline = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
