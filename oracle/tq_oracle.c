@@ -444,8 +444,8 @@ void tqo_matmul_addsub_format(const int8_t *xq, const uint8_t *packed, int64_t M
 }
 
 /* y[m][n] = acc[m][n] * gamma_n * s_x[m], computed in fp64 and rounded once
- * to fp32 ([H] section 5 step 6 and section 7's single scale fusion; the
- * spec form y = acc * gamma * s_x). */
+ * to fp32 ([H] section 5 step 6 and section 7's single scale fusion,
+ * written as y = acc * gamma * s_x with s_x = eta / 127). */
 void tqo_dequant(const int32_t *acc, const float *gamma, int per_row, const float *s_x,
                  int64_t M, int64_t N, float *y)
 {
