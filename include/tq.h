@@ -79,6 +79,7 @@ typedef enum tq_status {
 #define TQ_FLAG_WEIGHTS_STATIC (1u << 5)     /* see "Launch overlap" below                      */
 #define TQ_FLAG_INPUTS_READY (1u << 6)       /* see "Launch overlap" below                      */
 #define TQ_FLAG_ACCUMULATE (1u << 9)         /* tq_ternary_backward_input: dX += result         */
+#define TQ_FLAG_SHARED_INPUT (1u << 10)      /* tq_bitlinear_grouped: one x for all G layers    */
 
 /* Packed-code layout (flag bits 7-8; tq_quantize_ternary_pack[_noalloc],
  * tq_ternary_gemm, tq_bitlinear_fused).  Four codes per byte, LSB first.
@@ -172,11 +173,15 @@ TQ_API tq_status tq_quantize_ternary_pack_threshold(const float *w, int64_t N, i
  * device memory (a runtime whose allocator owns all of HBM and refuses new
  * reservations, a host that only receives device pointers, or a path where a
  * cudaMalloc and the synchronisation it may cause are not allowed).  It takes
- * no workspace: the per-tensor partial sums live in a fixed ~32 KB array inside
+ * no workspace: the per-tensor partial sums live in a fixed 16 KB array inside
  * the library, held on every GPU that loads it until the process exits.  The
  * pages have no counterpart of this entry point; it only moves scratch memory.
  *
- *   w, N, K, flags, packed, gamma, stream: as for tq_quantize_ternary_pack.
+ *   w, N, K, packed, gamma, stream: as for tq_quantize_ternary_pack.
+ *   flags: TQ_GAMMA_PER_ROW, TQ_FLAG_SANITIZE_NONFINITE and the layout bits
+ *   TQ_ENC_*, as for tq_quantize_ternary_pack.  TQ_FLAG_INPUTS_READY is
+ *   rejected (TQ_ERR_ARG): a call must not overlap the one before it, which
+ *   may still be using the shared array.
  *   Limit: with per-tensor gamma, N * K <= 134,217,728 weights (2048 partial
  *   sums of 65,536 weights); larger calls return TQ_ERR_SHAPE and launch
  *   nothing.  Per-row gamma uses no scratch and has no extra limit.
@@ -322,6 +327,12 @@ TQ_API tq_status tq_fwht_roundtrip(const float *x, float *y, int64_t rows, int64
  *   y          [M][d_model] fp32, written.
  *   act_out    [M][d_ffn] fp32 or NULL: the clamped activation.
  *   workspace  tq_swiglu_workspace_bytes(M, d_model, d_ffn, flags) bytes.
+ *              After the call it holds the block's intermediates, eight
+ *              parts in this order, each starting on a 256-byte boundary:
+ *              the gate/up input codes x_q [M][d_model] int8, their s_x [M]
+ *              fp32 and rowsum [M] int32; the gate and up projections
+ *              [M][d_ffn] fp32 each; the down projection's input codes
+ *              [M][d_ffn] int8, s_x [M] fp32 and rowsum [M] int32.
  * flags: TQ_FLAG_FWHT (required), TQ_FLAG_RMSNORM, TQ_GAMMA_PER_ROW,
  * TQ_FLAG_SANITIZE_NONFINITE, TQ_FLAG_WEIGHTS_STATIC, TQ_ENC_*.  SiLU is
  * computed in fp32 (v / (1 + e^-v)), within a few ulp of its exact value.
@@ -332,6 +343,47 @@ TQ_API tq_status tq_swiglu_mlp(const float *x, int64_t M, int64_t d_model, int64
                                const float *down_gamma, float *y, float *act_out, void *workspace,
                                size_t workspace_bytes, tq_stream_t stream);
 TQ_API size_t tq_swiglu_workspace_bytes(int64_t M, int64_t d_model, int64_t d_ffn, unsigned flags);
+
+/*
+ * Grouped small-M layer: G independent layers of one shape (N x K, packed
+ * weights and gamma of their own) applied to their activation batches in two
+ * launches -- one activation pass (per-token int8, Hetman-2b section 2
+ * SymmetricActivationQuantizer) over all batches, then one persistent GEMV
+ * that streams every layer's packed weights back to back (Hetman-2b section 7
+ * simulate_hardware_bitnet_gemv; Foundry "Native Matmul Kernel"):
+ *
+ *   y[g][m][n] = (sum_k x_q[g][m][k] * q_g[n][k]) * gamma_g[n or 0] * s_x[g][m]
+ *
+ * with x_q, s_x the per-token quantisation of x[g] (no RMSNorm, no FWHT, eta
+ * floor 1e-6, no clamp).  For the independent projections of a decode step
+ * (q/k/v or gate/up over one input: TQ_FLAG_SHARED_INPUT), the experts of a
+ * mixture-of-experts layer, or any set of same-shape layers whose inputs are
+ * ready together.  Each y[g] equals what tq_quantize_act_int8 followed by
+ * tq_ternary_gemm computes for that layer.
+ *
+ *   x          [G][M][K] fp32, or [M][K] with TQ_FLAG_SHARED_INPUT.
+ *   packed     HOST array of G device pointers, each [N][K/4] bytes in the
+ *              layout the flags name; gamma: HOST array of G device
+ *              pointers, each [N] (TQ_GAMMA_PER_ROW) or [1] fp32.  The arrays
+ *              are read during the call only.
+ *   y          [G][M][N] fp32, written.
+ *   workspace  tq_grouped_workspace_bytes(G, M, K, flags) bytes, 16-byte
+ *              aligned.  After the call it holds x_q [Gx][M][K] int8 (Gx = 1
+ *              with TQ_FLAG_SHARED_INPUT, else G) with each 16-byte chunk c of a
+ *              row stored 4x4-byte transposed (word j = elements 16c + j,
+ *              16c + 4 + j, 16c + 8 + j, 16c + 12 + j) at chunk position
+ *              c ^ (2 * ((c >> 3) & 1)), then s_x [Gx][M] fp32 and rowsum
+ *              [Gx][M] int32, each part starting on a 256-byte boundary.
+ *   Shapes: 1 <= G <= 64, 1 <= M <= 16, 64 <= K <= 8192 (K % 64 == 0);
+ *   otherwise TQ_ERR_SHAPE.
+ *   flags: TQ_GAMMA_PER_ROW, TQ_FLAG_SHARED_INPUT, TQ_FLAG_WEIGHTS_STATIC,
+ *   TQ_FLAG_INPUTS_READY (see "Launch overlap"), TQ_ENC_*.
+ */
+TQ_API tq_status tq_bitlinear_grouped(const float *x, int64_t G, const uint8_t *const *packed,
+                                      const float *const *gamma, unsigned flags, int64_t M, int64_t N,
+                                      int64_t K, float *y, void *workspace, size_t workspace_bytes,
+                                      tq_stream_t stream);
+TQ_API size_t tq_grouped_workspace_bytes(int64_t G, int64_t M, int64_t K, unsigned flags);
 
 /* ------------------------------------------------------------------------
  * Training

@@ -30,6 +30,7 @@ ENC_FORMAT0 = 1 << 7
 ENC_FORMAT1 = 2 << 7
 ENC_MASK = 3 << 7
 FLAG_ACCUMULATE = 1 << 9  # tq_ternary_backward_input: dX += result
+FLAG_SHARED_INPUT = 1 << 10  # tq_bitlinear_grouped: one activation batch for all layers
 
 STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN", 4: "TQ_ERR_ARG",
           5: "TQ_ERR_CUDA", 6: "TQ_ERR_DEVICE", 7: "TQ_ERR_TIMEOUT"}
@@ -52,6 +53,8 @@ SIGNATURES = {
     "tq_fused_workspace_bytes": (_SZ, [_I64, _I64, _U]),
     "tq_swiglu_mlp": (_I, [_P, _I64, _I64, _I64, _U, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tq_swiglu_workspace_bytes": (_SZ, [_I64, _I64, _I64, _U]),
+    "tq_bitlinear_grouped": (_I, [_P, _I64, _P, _P, _U, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "tq_grouped_workspace_bytes": (_SZ, [_I64, _I64, _I64, _U]),
     "tq_ternary_backward_input": (_I, [_P, _P, _P, _P, _U, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "tq_backward_input_workspace_bytes": (_SZ, [_I64, _I64]),
     "tq_ste_backward": (_I, [_P, _P, _P, _I64, _I64, _F, _U, _P, _P]),
@@ -236,6 +239,70 @@ def fwht_roundtrip_(x, y, eta_min=0.05, eta_max=40.0, eta_out=None, stream=None)
 
 def swiglu_workspace_bytes(M: int, d_model: int, d_ffn: int, flags: int) -> int:
     return int(load().tq_swiglu_workspace_bytes(M, d_model, d_ffn, flags))
+
+
+def grouped_workspace_bytes(G: int, M: int, K: int, flags: int) -> int:
+    return int(load().tq_grouped_workspace_bytes(G, M, K, flags))
+
+
+def bitlinear_grouped_(x, packed, gamma, flags, y, workspace, stream=None):
+    """G same-shape layers: x [G, M, K] (or [M, K] with FLAG_SHARED_INPUT),
+    packed / gamma: sequences of G device tensors, y [G, M, N]."""
+    import torch
+
+    G = len(packed)
+    if len(gamma) != G:
+        raise ValueError("packed and gamma must have one entry per layer")
+    M, K = x.shape[-2], x.shape[-1]
+    N = packed[0].shape[0]
+    _need(x, torch.float32, (M, K) if flags & FLAG_SHARED_INPUT else (G, M, K), "x")
+    _need(y, torch.float32, (G, M, N), "y")
+    for p in packed:
+        _need(p, torch.uint8, (N, K // 4), "packed")
+    arr = ctypes.c_void_p * G
+    pp = arr(*[p.data_ptr() for p in packed])
+    gp = arr(*[g.data_ptr() for g in gamma])
+    _check("tq_bitlinear_grouped",
+           load().tq_bitlinear_grouped(_ptr(x), G, ctypes.cast(pp, ctypes.c_void_p), ctypes.cast(gp, ctypes.c_void_p),
+                                       flags, M, N, K, _ptr(y), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def grouped_intermediates(workspace, G: int, M: int, K: int, flags: int) -> dict:
+    """x_q (back in plain [Gx, M, K] order), s_x and rowsum from the
+    workspace of tq_bitlinear_grouped (the layout the header states)."""
+    import torch
+
+    Gx = 1 if flags & FLAG_SHARED_INPUT else G
+    al = lambda b: (b + 255) & ~255
+    o1 = al(Gx * M * K)
+    o2 = o1 + al(Gx * M * 4)
+    raw = workspace[:Gx * M * K].view(Gx * M, K // 16, 4, 4)
+    c = torch.arange(K // 16, device=workspace.device)
+    pos = c ^ (2 * ((c >> 3) & 1))
+    xq = raw[:, pos].transpose(2, 3).reshape(Gx, M, K).view(torch.int8)
+    sx = workspace[o1:o1 + Gx * M * 4].view(torch.float32).view(Gx, M)
+    rs = workspace[o2:o2 + Gx * M * 4].view(torch.int32).view(Gx, M)
+    return {"xq": xq, "s_x": sx, "rowsum": rs}
+
+
+def swiglu_intermediates(workspace, M: int, d_model: int, d_ffn: int) -> dict:
+    """Views of what tq_swiglu_mlp leaves in its workspace (the layout the
+    header states: eight parts, each starting on a 256-byte boundary)."""
+    import torch
+
+    sizes = [(M * d_model, torch.int8, (M, d_model), "xq1"), (M, torch.float32, (M,), "s_x1"),
+             (M, torch.int32, (M,), "rowsum1"), (M * d_ffn, torch.float32, (M, d_ffn), "y_gate"),
+             (M * d_ffn, torch.float32, (M, d_ffn), "y_up"), (M * d_ffn, torch.int8, (M, d_ffn), "xq2"),
+             (M, torch.float32, (M,), "s_x2"), (M, torch.int32, (M,), "rowsum2")]
+    out, off = {}, 0
+    for n, dt, shape, name in sizes:
+        nb = n * torch.tensor([], dtype=dt).element_size()
+        out[name] = workspace[off:off + nb].view(dt).view(shape)
+        off += (nb + 255) & ~255
+    if off > workspace.numel():
+        raise ValueError("workspace smaller than tq_swiglu_workspace_bytes")
+    return out
 
 
 def swiglu_mlp_(x, gate, up, down, flags, y, workspace, clamp_val=10.0, act_out=None, stream=None):

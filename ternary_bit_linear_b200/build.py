@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtq.so")
 SOURCES = ["tq_api.cu"]
-DEPS = ["tq_api.cu", "tq_common.cuh", "tq_pack.cuh", "tq_act.cuh", "tq_gemv.cuh", "tq_gemm.cuh",
+DEPS = ["tq_api.cu", "tq_common.cuh", "tq_pack.cuh", "tq_act.cuh", "tq_gemv.cuh", "tq_gemv_group.cuh", "tq_gemm.cuh",
         "tq_train.cuh", "tq_xorshift_jump.h"]
 
 

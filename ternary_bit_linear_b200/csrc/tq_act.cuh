@@ -122,8 +122,14 @@ __device__ __forceinline__ float rms_apply(float x, double r, const float *gain,
 // Per-token quantisation (optionally after RMSNorm) of one row that a CTA of
 // kActThreads holds in registers: thread tid has float4 tid + i * kActThreads
 // (i < VEC; zeros past the row).  Writes x_q, s_x[m] and rowsum[m].
+//
+// XT: x_q in the layout the grouped small-M GEMV copies straight into shared
+// memory -- each 16-byte chunk 4x4-byte transposed (word j holds elements
+// 16c + j, 16c + 4 + j, 16c + 8 + j, 16c + 12 + j) and stored at chunk position
+// gemv_chunk_pos(c).  The four words of a chunk sit in four consecutive lanes
+// (kActThreads is a multiple of 4), which exchange them by shuffles.
 // ---------------------------------------------------------------------------
-template <int VEC>
+template <int VEC, bool XT = false>
 __device__ __forceinline__ void act_row_regs(float4 (&v)[VEC], int K, const ActParams &p, int64_t m,
                                              int8_t *__restrict__ xq, float *__restrict__ s_x,
                                              int32_t *__restrict__ rowsum, float *redf, int *redi,
@@ -160,10 +166,23 @@ __device__ __forceinline__ void act_row_regs(float4 (&v)[VEC], int K, const ActP
 #pragma unroll
     for (int i = 0; i < VEC; ++i) {
         const int idx = tid + i * kActThreads;
+        // past the row (K % 64 == 0: whole chunks, whole lane quads) the codes are 0
+        const int a = quant_code(v[i].x, scale), b = quant_code(v[i].y, scale),
+                  c = quant_code(v[i].z, scale), d = quant_code(v[i].w, scale);
+        uint32_t word = pack_codes4(a, b, c, d);
+        if (XT) {
+            const int q0 = (threadIdx.x & 31) & ~3;
+            uint4 q;
+            q.x = __shfl_sync(0xffffffffu, word, q0);
+            q.y = __shfl_sync(0xffffffffu, word, q0 + 1);
+            q.z = __shfl_sync(0xffffffffu, word, q0 + 2);
+            q.w = __shfl_sync(0xffffffffu, word, q0 + 3);
+            const uint4 t = transpose_bytes4x4(q);
+            const int j = idx & 3;
+            word = j == 0 ? t.x : j == 1 ? t.y : j == 2 ? t.z : t.w;
+        }
         if (idx < nv) {
-            const int a = quant_code(v[i].x, scale), b = quant_code(v[i].y, scale),
-                      c = quant_code(v[i].z, scale), d = quant_code(v[i].w, scale);
-            dst[idx] = pack_codes4(a, b, c, d);
+            dst[XT ? 4 * gemv_chunk_pos(idx >> 2) + (idx & 3) : idx] = word;
             sum += a + b + c + d;
         }
     }
@@ -181,10 +200,12 @@ __device__ __forceinline__ float4 quench4(float4 v, const ActParams &p) {
 
 // One CTA per token.  VEC > 0: the row lives in registers (K <= 1024*VEC);
 // VEC == 0: streamed (two passes over the row, the second from cache).
-template <int VEC>
+// XT: x_q in the grouped GEMV's layout (see act_row_regs; VEC > 0 only).
+template <int VEC, bool XT = false>
 __global__ void __launch_bounds__(kActThreads)
-    act_quant_kernel(const float *__restrict__ x, int K, ActParams p, int8_t *__restrict__ xq,
+    tq_act_quant_kernel(const float *__restrict__ x, int K, ActParams p, int8_t *__restrict__ xq,
                      float *__restrict__ s_x, int32_t *__restrict__ rowsum) {
+    static_assert(!XT || VEC > 0, "the GEMV layout is written from registers");
     __shared__ float redf[32];
     __shared__ int redi[32];
     __shared__ double redd[32];
@@ -206,7 +227,7 @@ __global__ void __launch_bounds__(kActThreads)
             const int idx = tid + i * kActThreads;
             v[i] = idx < nv ? load(idx) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        act_row_regs<V>(v, K, p, m, xq, s_x, rowsum, redf, redi, redd);
+        act_row_regs<V, XT>(v, K, p, m, xq, s_x, rowsum, redf, redi, redd);
         if (p.ready) pdl_wait();  // complete no earlier than the previous kernel
         return;
     }
@@ -265,7 +286,7 @@ constexpr int kActRing = 4;
 
 template <int VEC>
 __global__ void __launch_bounds__(kActThreads)
-    act_ring_kernel(const float *__restrict__ x, int64_t M, int K, ActParams p,
+    tq_act_ring_kernel(const float *__restrict__ x, int64_t M, int K, ActParams p,
                     int8_t *__restrict__ xq, float *__restrict__ s_x, int32_t *__restrict__ rowsum) {
     extern __shared__ __align__(16) float4 rowbuf[];  // [kActRing][nv]
     __shared__ uint64_t rbar[kActRing];
@@ -365,7 +386,7 @@ __device__ __forceinline__ void fwht512_regs(float (&f)[16], bool normalize) {
 
 // Standalone transform: one warp per 512-block, 8 warps per CTA.
 __global__ void __launch_bounds__(256)
-    fwht512_kernel(const float *x, float *y, int64_t nblocks, int normalize) {
+    tq_fwht512_kernel(const float *x, float *y, int64_t nblocks, int normalize) {
     pdl_wait();
     pdl_trigger();
     const int64_t blk = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -399,7 +420,7 @@ __global__ void __launch_bounds__(256)
 // it writes it).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
-    fwht_roundtrip_kernel(const float *x, float *y, float eta_min, float eta_max,
+    tq_fwht_roundtrip_kernel(const float *x, float *y, float eta_min, float eta_max,
                           float *__restrict__ eta_out) {
     __shared__ float redf[32];
     pdl_wait();
@@ -443,7 +464,7 @@ __global__ void __launch_bounds__(1024)
 // SwiGLUClamped.forward), fused with the down projection's activation pass:
 // a = clamp(SiLU(gate) * up, +-clamp_val) (SiLU(v) = v / (1 + e^-v), fp32),
 // then [quench] -> [RMSNorm] -> FWHT-512 -> per-token int8, as
-// prologue_fwht_kernel.  One CTA per token, one warp per 512-block
+// tq_prologue_fwht_kernel.  One CTA per token, one warp per 512-block
 // (K = 512 * blockDim.x / 32).  act_out (or NULL) receives a.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float swiglu_one(float g, float u, float c) {
@@ -452,7 +473,7 @@ __device__ __forceinline__ float swiglu_one(float g, float u, float c) {
 }
 
 __global__ void __launch_bounds__(1024)
-    swiglu_prologue_kernel(const float *__restrict__ gate, const float *__restrict__ up, float clamp_val,
+    tq_swiglu_prologue_kernel(const float *__restrict__ gate, const float *__restrict__ up, float clamp_val,
                            ActParams p, int8_t *__restrict__ xq, float *__restrict__ s_x,
                            int32_t *__restrict__ rowsum, float *__restrict__ act_out) {
     __shared__ float redf[32];
@@ -535,7 +556,7 @@ __global__ void __launch_bounds__(1024)
 // ---------------------------------------------------------------------------
 template <int NW>
 __global__ void __launch_bounds__(NW * 32)
-    prologue_fwht_kernel(const float *__restrict__ x, ActParams p, int8_t *__restrict__ xq,
+    tq_prologue_fwht_kernel(const float *__restrict__ x, ActParams p, int8_t *__restrict__ xq,
                          float *__restrict__ s_x, int32_t *__restrict__ rowsum) {
     __shared__ float redf[32];
     __shared__ int redi[32];

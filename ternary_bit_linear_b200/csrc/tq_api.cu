@@ -16,6 +16,7 @@
 #include "tq_common.cuh"
 #include "tq_gemm.cuh"
 #include "tq_gemv.cuh"
+#include "tq_gemv_group.cuh"
 #include "tq_pack.cuh"
 #include "tq_train.cuh"
 
@@ -164,7 +165,7 @@ tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemm_kernel<BT, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tq_gemm_kernel<BT, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  L::kDynamic) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
@@ -178,7 +179,7 @@ tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
         return TQ_ERR_CUDA;
     const int64_t tiles = ((a.M + BT - 1) / BT) * ((a.N + kTileN - 1) / kTileN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
-    return launch_pdl(gemm_kernel<BT, CONV, EPI>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
+    return launch_pdl(tq_gemm_kernel<BT, CONV, EPI>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
                       a.s_x, a.rowsum, a.gamma, a.per_row, (int)a.M, (int)a.N, (int)a.K, a.y, a.acc, a.mode,
                       a.ep);
 }
@@ -191,14 +192,14 @@ tq_status launch_gemv(const GemmArgs &a, cudaStream_t st) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemv_kernel<NB, W, SPW, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tq_gemv_kernel<NB, W, SPW, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemv_x_bytes(8 * NB, kGemvMaxK)) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
     }
     const int64_t grid = (a.N + 15) / 16;
     const size_t smem = (size_t)gemv_x_bytes((int)a.M, (int)a.K);
-    return launch_pdl(gemv_kernel<NB, W, SPW, CONV, EPI>, dim3((unsigned)grid), dim3(W * 32), smem, st, a.xq,
+    return launch_pdl(tq_gemv_kernel<NB, W, SPW, CONV, EPI>, dim3((unsigned)grid), dim3(W * 32), smem, st, a.xq,
                       a.s_x, a.rowsum, a.packed, a.gamma, a.per_row, (int)a.M, a.N, (int)a.K, a.y, a.acc,
                       a.mode, a.ep);
 }
@@ -213,7 +214,7 @@ tq_status launch_gemv_stream_t(const int8_t *xq, const float *s_x, const int32_t
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(gemv_stream_kernel<ENC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tq_gemv_stream_kernel<ENC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemv_x_bytes(8, kStreamMaxK)) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
@@ -223,7 +224,7 @@ tq_status launch_gemv_stream_t(const int8_t *xq, const float *s_x, const int32_t
     if (per_cta < kStreamGroups) per_cta = kStreamGroups;
     const int64_t grid = (nstrips + per_cta - 1) / per_cta;
     const size_t smem = (size_t)gemv_x_bytes((int)M, (int)K);
-    return launch_pdl(gemv_stream_kernel<ENC>, dim3((unsigned)grid), dim3(kStreamThreads), smem, st, xq,
+    return launch_pdl(tq_gemv_stream_kernel<ENC>, dim3((unsigned)grid), dim3(kStreamThreads), smem, st, xq,
                       s_x, rowsum, packed, gamma, per_row, (int)M, N, (int)K, y, acc, (int)per_cta);
 }
 
@@ -252,7 +253,7 @@ tq_status gemv_shape(const GemmArgs &a, cudaStream_t st) {
 template <int NW>
 void launch_prologue(const float *x, const ActParams &p, int64_t M, int8_t *xq, float *sx,
                      int32_t *rs, cudaStream_t st) {
-    launch_pdl(prologue_fwht_kernel<NW>, dim3((unsigned)M), dim3(NW * 32), 0, st, x, p, xq, sx, rs);
+    launch_pdl(tq_prologue_fwht_kernel<NW>, dim3((unsigned)M), dim3(NW * 32), 0, st, x, p, xq, sx, rs);
 }
 
 typedef void (*PrologueFn)(const float *, const ActParams &, int64_t, int8_t *, float *, int32_t *,
@@ -282,9 +283,9 @@ void launch_act_ring(const float *x, const ActParams &p, int64_t M, int64_t K, i
     if ((key >> 8) == smem + 1) {
         per_sm = key & 0xff;
     } else {
-        if (cudaFuncSetAttribute(act_ring_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        if (cudaFuncSetAttribute(tq_act_ring_kernel<VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
                 cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, act_ring_kernel<VEC>, kActThreads,
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tq_act_ring_kernel<VEC>, kActThreads,
                                                           (size_t)smem) != cudaSuccess)
             per_sm = 1;
         if (per_sm < 1) per_sm = 1;
@@ -292,7 +293,7 @@ void launch_act_ring(const float *x, const ActParams &p, int64_t M, int64_t K, i
     }
     const int64_t cap = (int64_t)per_sm * sms;
     const unsigned grid = (unsigned)(M < cap ? M : cap);
-    launch_pdl(act_ring_kernel<VEC>, dim3(grid), dim3(kActThreads), (size_t)smem, st, x, M, (int)K, p, xq,
+    launch_pdl(tq_act_ring_kernel<VEC>, dim3(grid), dim3(kActThreads), (size_t)smem, st, x, M, (int)K, p, xq,
                sx, rs);
 }
 
@@ -309,18 +310,18 @@ void launch_act(const float *x, const ActParams &p, int64_t M, int64_t K, int8_t
     }
     const dim3 grid((unsigned)M), block(kActThreads);
     if (nv <= 256)
-        launch_pdl(act_quant_kernel<1>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+        launch_pdl(tq_act_quant_kernel<1>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else if (nv <= 512)
-        launch_pdl(act_quant_kernel<2>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+        launch_pdl(tq_act_quant_kernel<2>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else if (nv <= 1024)
-        launch_pdl(act_quant_kernel<4>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+        launch_pdl(tq_act_quant_kernel<4>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else if (nv <= 2048)
-        launch_pdl(act_quant_kernel<8>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+        launch_pdl(tq_act_quant_kernel<8>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
     else
-        launch_pdl(act_quant_kernel<0>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+        launch_pdl(tq_act_quant_kernel<0>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
 }
 
-// Per-tensor mode of the pack pass: the partial sums of absum_partial_kernel
+// Per-tensor mode of the pack pass: the partial sums of tq_absum_partial_kernel
 // and the height of the whole summation tree (partial == nullptr: per row).
 struct PerTensor {
     const double *partial = nullptr;
@@ -365,14 +366,14 @@ tq_status launch_pack_rows_s(const float *w, int64_t N, int64_t K, uint8_t *pack
     const int64_t nv = K / 4;
     const int k = (int)K;
     if (nv <= 32 * kTeamVec * 1)
-        return launch_pack_grid(pack_team_kernel<1, SAN, CONV>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
+        return launch_pack_grid(tq_pack_team_kernel<1, SAN, CONV>, occ[0], kPackWarps / 1, pack_team_smem(1, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
     if (nv <= 32 * kTeamVec * 2)
-        return launch_pack_grid(pack_team_kernel<2, SAN, CONV>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
+        return launch_pack_grid(tq_pack_team_kernel<2, SAN, CONV>, occ[1], kPackWarps / 2, pack_team_smem(2, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
     if (nv <= 32 * kTeamVec * 4)
-        return launch_pack_grid(pack_team_kernel<4, SAN, CONV>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
+        return launch_pack_grid(tq_pack_team_kernel<4, SAN, CONV>, occ[2], kPackWarps / 4, pack_team_smem(4, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
     if (nv <= 32 * kTeamVec * 8)
-        return launch_pack_grid(pack_team_kernel<8, SAN, CONV>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
-    return launch_pack_grid(pack_rows_kernel<SAN, CONV>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
+        return launch_pack_grid(tq_pack_team_kernel<8, SAN, CONV>, occ[3], kPackWarps / 8, pack_team_smem(8, k), w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
+    return launch_pack_grid(tq_pack_rows_kernel<SAN, CONV>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
 }
 
 // Options word of the pack kernels: bit 0 inputs ready, bits 1-2 layout.
@@ -503,12 +504,12 @@ template <bool CONV>
 tq_status launch_flip(uint8_t *packed, const float *grad, int64_t nw, float temp, uint64_t x0, int mode,
                       int sms, cudaStream_t st) {
     static std::atomic<int> done[kMaxDevices];
-    if (tq_status e = set_smem_once(flip_kernel<CONV>, kFlipSmem, done)) return e;
+    if (tq_status e = set_smem_once(tq_flip_kernel<CONV>, kFlipSmem, done)) return e;
     const int64_t nchunks = (nw + kFlipChunk - 1) / kFlipChunk;
     const int64_t target = 2 * (int64_t)sms;  // two CTAs per SM
     const int64_t per_cta = (nchunks + target - 1) / target;
     const int64_t grid = (nchunks + per_cta - 1) / per_cta;
-    return launch_pdl(flip_kernel<CONV>, dim3((unsigned)grid), dim3(kFlipThreads), (size_t)kFlipSmem, st, packed,
+    return launch_pdl(tq_flip_kernel<CONV>, dim3((unsigned)grid), dim3(kFlipThreads), (size_t)kFlipSmem, st, packed,
                       grad, nw, temp, x0, per_cta, mode);
 }
 
@@ -517,7 +518,7 @@ tq_status launch_bwd_gemm(const __half *planes, const float *inv_scale, const ui
                           const float *row_scale, int accumulate,
                           int64_t M, int64_t N, int64_t K, float *dX, int mode, int sms, cudaStream_t st) {
     static std::atomic<int> done[kMaxDevices];
-    if (tq_status e = set_smem_once(bwd_gemm_kernel<CONV>, kBwdDynamic, done)) return e;
+    if (tq_status e = set_smem_once(tq_bwd_gemm_kernel<CONV>, kBwdDynamic, done)) return e;
     // planes [2 M][Np] fp16 in 64-byte-swizzled [256][32] boxes; packed [N][K/4]
     // in plain [32][32 B] boxes.
     CUtensorMap tg, tw;
@@ -528,8 +529,53 @@ tq_status launch_bwd_gemm(const __half *planes, const float *inv_scale, const ui
         return TQ_ERR_CUDA;
     const int64_t tiles = ((M + kBwdTileT - 1) / kBwdTileT) * ((K + kBwdTileF - 1) / kBwdTileF);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    return launch_pdl(bwd_gemm_kernel<CONV>, dim3(grid), dim3(kGemmThreads), (size_t)kBwdDynamic, st, tg, tw,
+    return launch_pdl(tq_bwd_gemm_kernel<CONV>, dim3(grid), dim3(kGemmThreads), (size_t)kBwdDynamic, st, tg, tw,
                       inv_scale, row_scale, accumulate, (int)M, (int)N, (int)K, dX, mode);
+}
+
+// ---------------------------------------------------------------------------
+// Grouped small-M contraction
+// ---------------------------------------------------------------------------
+constexpr int kGroupSmemBudget = 226 * 1024;  // dynamic; the opt-in limit is 227 KiB including static
+
+// Workspace of tq_bitlinear_grouped: x_q [Gx][M][K] (in the grouped GEMV's
+// layout), s_x [Gx][M], rowsum [Gx][M], each part 256-byte aligned.
+inline size_t grouped_parts(int64_t Gx, int64_t M, int64_t K, size_t off[3]) {
+    auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
+    off[0] = 0;
+    off[1] = al((size_t)(Gx * M * K));
+    off[2] = off[1] + al((size_t)(Gx * M) * 4);
+    return off[2] + al((size_t)(Gx * M) * 4);
+}
+
+template <int NB, int ENC>
+tq_status launch_group_gemv(const GroupTable &tab, const GroupPlan &pl, const int8_t *xq, const float *sx,
+                            const int32_t *rs, float *y, int sms, cudaStream_t st) {
+    static std::atomic<int> done[kMaxDevices];
+    if (tq_status e = set_smem_once(tq_gemv_group_kernel<NB, ENC>, kGroupSmemBudget, done)) return e;
+    const int64_t grid = pl.nstrips < sms ? pl.nstrips : sms;
+    return launch_pdl(tq_gemv_group_kernel<NB, ENC>, dim3((unsigned)grid), dim3(kGrpThreads), (size_t)pl.smem,
+                      st, tab, pl, xq, sx, rs, y);
+}
+
+template <int NB>
+tq_status launch_group_gemv_enc(const GroupTable &tab, const GroupPlan &pl, const int8_t *xq, const float *sx,
+                                const int32_t *rs, float *y, int sms, cudaStream_t st) {
+    if (pl.enc == kEncFormat0) return launch_group_gemv<NB, kEncFormat0>(tab, pl, xq, sx, rs, y, sms, st);
+    if (pl.enc == kEncFormat1) return launch_group_gemv<NB, kEncFormat1>(tab, pl, xq, sx, rs, y, sms, st);
+    return launch_group_gemv<NB, kEncFoundry>(tab, pl, xq, sx, rs, y, sms, st);
+}
+
+// Activation pass of the grouped call: rows of x quantised per token, x_q
+// written in the grouped GEMV's layout.
+inline tq_status launch_act_group(const float *x, const ActParams &p, int64_t rows, int64_t K, int8_t *xq,
+                                  float *sx, int32_t *rs, cudaStream_t st) {
+    const int nv = (int)(K / 4);
+    const dim3 grid((unsigned)rows), block(kActThreads);
+    if (nv <= 256) return launch_pdl(tq_act_quant_kernel<1, true>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+    if (nv <= 512) return launch_pdl(tq_act_quant_kernel<2, true>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+    if (nv <= 1024) return launch_pdl(tq_act_quant_kernel<4, true>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
+    return launch_pdl(tq_act_quant_kernel<8, true>, grid, block, 0, st, x, (int)K, p, xq, sx, rs);
 }
 
 }  // namespace
@@ -599,7 +645,7 @@ static tq_status pack_impl(const float *w, int64_t N, int64_t K, unsigned flags,
     const size_t nparts = pack_parts(total_v);
     const int64_t chunk = (total_v + (int64_t)nparts - 1) / (int64_t)nparts;
     double *partial = reinterpret_cast<double *>(workspace);
-    if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
+    if (tq_status e = launch_pdl(tq_absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
                                  st, w, total_v, chunk, sanitize, partial, ready))
         return e;
     PerTensor pt;
@@ -659,7 +705,7 @@ tq_status tq_fwht512(const float *x, float *y, int64_t rows, int64_t K, int norm
     if (x != y && overlap(x, b, y, b)) return TQ_ERR_ARG;
     if (tq_status e = check_device(nullptr)) return e;
     const int64_t nblocks = rows * (K / 512);
-    return launch_pdl(fwht512_kernel, dim3((unsigned)((nblocks + 7) / 8)), dim3(256), 0, cs(stream),
+    return launch_pdl(tq_fwht512_kernel, dim3((unsigned)((nblocks + 7) / 8)), dim3(256), 0, cs(stream),
                       x, y, nblocks, normalize);
 }
 
@@ -674,7 +720,7 @@ tq_status tq_fwht_roundtrip(const float *x, float *y, int64_t rows, int64_t K, f
     if (eta_out && (overlap(eta_out, (size_t)rows * 4, x, b) || overlap(eta_out, (size_t)rows * 4, y, b)))
         return TQ_ERR_ARG;
     if (tq_status e = check_device(nullptr)) return e;
-    return launch_pdl(fwht_roundtrip_kernel, dim3((unsigned)rows), dim3((unsigned)(K / 512 * 32)), 0, cs(stream),
+    return launch_pdl(tq_fwht_roundtrip_kernel, dim3((unsigned)rows), dim3((unsigned)(K / 512 * 32)), 0, cs(stream),
                       x, y, eta_min, eta_max, eta_out);
 }
 
@@ -888,7 +934,7 @@ tq_status tq_swiglu_mlp(const float *x, int64_t M, int64_t d_model, int64_t d_ff
     if (tq_status e = gemm_dispatch(xq1, sx1, rs1, up_packed, up_gamma, cflags, M, d_ffn, d_model, yu, nullptr,
                                     sms, st))
         return e;
-    if (tq_status e = launch_pdl(swiglu_prologue_kernel, dim3((unsigned)M), dim3((unsigned)(d_ffn / 512 * 32)), 0,
+    if (tq_status e = launch_pdl(tq_swiglu_prologue_kernel, dim3((unsigned)M), dim3((unsigned)(d_ffn / 512 * 32)), 0,
                                  st, (const float *)yg, (const float *)yu, clamp_val, p, xq2, sx2, rs2, act_out))
         return e;
     return gemm_dispatch(xq2, sx2, rs2, down_packed, down_gamma, cflags, M, d_model, d_ffn, y, nullptr, sms, st);
@@ -935,9 +981,9 @@ tq_status tq_ternary_backward_input(const float *dY, const uint8_t *packed, cons
     const int per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
     const unsigned sgrid = (unsigned)(M < 8 * (int64_t)sms ? M : 8 * (int64_t)sms);  // one CTA per token row
     tq_status e = (N % 4 == 0)
-                      ? launch_pdl(bwd_split_kernel<true>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
+                      ? launch_pdl(tq_bwd_split_kernel<true>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
                                    per_row, (int)M, (int)N, (int)Np, planes, inv_scale)
-                      : launch_pdl(bwd_split_kernel<false>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
+                      : launch_pdl(tq_bwd_split_kernel<false>, dim3(sgrid), dim3(kSplitThreads), 0, st, dY, gamma,
                                    per_row, (int)M, (int)N, (int)Np, planes, inv_scale);
     if (e) return e;
     const int mode = enc << kModeEncShift;
@@ -969,9 +1015,9 @@ tq_status tq_ste_backward(const float *grad, const float *w, const float *gamma,
     const float4 *g4 = reinterpret_cast<const float4 *>(grad), *w4 = reinterpret_cast<const float4 *>(w);
     float4 *o4 = reinterpret_cast<float4 *>(out);
     return (flags & TQ_FLAG_SANITIZE_NONFINITE)
-               ? launch_pdl(ste_backward_kernel<true>, dim3(grid), dim3(kSteThreads), 0, cs(stream), g4, w4, gamma,
+               ? launch_pdl(tq_ste_backward_kernel<true>, dim3(grid), dim3(kSteThreads), 0, cs(stream), g4, w4, gamma,
                             per_row, nvec, K / 4, tau, o4)
-               : launch_pdl(ste_backward_kernel<false>, dim3(grid), dim3(kSteThreads), 0, cs(stream), g4, w4,
+               : launch_pdl(tq_ste_backward_kernel<false>, dim3(grid), dim3(kSteThreads), 0, cs(stream), g4, w4,
                             gamma, per_row, nvec, K / 4, tau, o4);
 }
 
@@ -1004,6 +1050,75 @@ tq_status tq_ternary_stochastic_flip(uint8_t *packed, const float *grad, int64_t
     return TQ_OK;
 }
 
+size_t tq_grouped_workspace_bytes(int64_t G, int64_t M, int64_t K, unsigned flags) {
+    if (G <= 0 || M <= 0 || K <= 0) return 0;
+    size_t off[3];
+    return grouped_parts((flags & TQ_FLAG_SHARED_INPUT) ? 1 : G, M, K, off);
+}
+
+tq_status tq_bitlinear_grouped(const float *x, int64_t G, const uint8_t *const *packed, const float *const *gamma,
+                               unsigned flags, int64_t M, int64_t N, int64_t K, float *y, void *workspace,
+                               size_t workspace_bytes, tq_stream_t stream) {
+    if (!x || !packed || !gamma || !y || !workspace) return TQ_ERR_NULL;
+    if (G < 1 || G > kGroupMax || M < 1 || M > 16 || N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (K > kGemvMaxK) return TQ_ERR_SHAPE;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SHARED_INPUT | TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY |
+                  TQ_ENC_MASK))
+        return TQ_ERR_ARG;
+    const int enc = flag_encoding(flags);
+    if (enc < 0) return TQ_ERR_ARG;
+    const bool shared = flags & TQ_FLAG_SHARED_INPUT;
+    const int64_t Gx = shared ? 1 : G;
+    for (int64_t g = 0; g < G; ++g)
+        if (!packed[g] || !gamma[g]) return TQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return TQ_ERR_ALIGN;
+    for (int64_t g = 0; g < G; ++g)
+        if (!aligned16(packed[g]) || !aligned16(gamma[g])) return TQ_ERR_ALIGN;
+    size_t off[3];
+    const size_t need = grouped_parts(Gx, M, K, off);
+    if (workspace_bytes < need) return TQ_ERR_ARG;
+    const size_t xb = (size_t)(Gx * M * K) * 4, yb = (size_t)(G * M * N) * 4, pb = (size_t)(N * K / 4),
+                 gb = ((flags & TQ_GAMMA_PER_ROW) ? (size_t)N : 1) * 4;
+    if (overlap(x, xb, y, yb) || overlap(x, xb, workspace, need) || overlap(y, yb, workspace, need)) return TQ_ERR_ARG;
+    for (int64_t g = 0; g < G; ++g)
+        if (overlap(packed[g], pb, y, yb) || overlap(packed[g], pb, workspace, need) ||
+            overlap(gamma[g], gb, y, yb) || overlap(gamma[g], gb, workspace, need))
+            return TQ_ERR_ARG;
+    int sms = 0;
+    if (tq_status e = check_device(&sms)) return e;
+    cudaStream_t st = cs(stream);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    int8_t *xq = reinterpret_cast<int8_t *>(ws + off[0]);
+    float *sx = reinterpret_cast<float *>(ws + off[1]);
+    int32_t *rs = reinterpret_cast<int32_t *>(ws + off[2]);
+
+    GroupPlan pl{};
+    pl.M = (int)M;
+    pl.K = (int)K;
+    pl.N = N;
+    pl.spp = (N + 15) / 16;
+    pl.nstrips = G * pl.spp;
+    pl.x_shared = shared ? 1 : 0;
+    pl.per_row = (flags & TQ_GAMMA_PER_ROW) ? 1 : 0;
+    pl.weights_static = (flags & (TQ_FLAG_WEIGHTS_STATIC | TQ_FLAG_INPUTS_READY)) ? 1 : 0;
+    pl.enc = enc;
+    const int NB = M <= 8 ? 1 : 2;
+    if (!grp_plan(pl, NB, kGroupSmemBudget)) return TQ_ERR_SHAPE;
+    GroupTable tab{};
+    for (int64_t g = 0; g < G; ++g) {
+        tab.packed[g] = packed[g];
+        tab.gamma[g] = gamma[g];
+    }
+    ActParams p{};
+    p.ready = (flags & TQ_FLAG_INPUTS_READY) ? 1 : 0;
+    if (tq_status e = launch_act_group(x, p, Gx * M, K, xq, sx, rs, st)) return e;
+    if (tq_status e = NB == 1 ? launch_group_gemv_enc<1>(tab, pl, xq, sx, rs, y, sms, st)
+                              : launch_group_gemv_enc<2>(tab, pl, xq, sx, rs, y, sms, st))
+        return e;
+    return launch_status();
+}
+
 tq_status tq_get_device_status(tq_stream_t stream) {
     if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return TQ_ERR_CUDA;
     unsigned v = 0, zero = 0;
@@ -1031,8 +1146,8 @@ tq_status tq_get_device_status(tq_stream_t stream) {
 //     (134,217,728, e.g. 8192 x 16384); larger calls return TQ_ERR_SHAPE
 //     before launching anything.  Per-row gamma needs no scratch and has no
 //     extra limit.
-//   * every GPU that loads the library holds the array (about 32 KB) until the
-//     process exits.
+//   * every GPU that loads the library holds the array (16 KB: one fp64
+//     partial sum per slot) until the process exits.
 //   * all calls share the one array: calls whose work overlaps on the GPU (for
 //     example on two streams at once) race and give wrong results.  Each call
 //     writes every slot it reads before reading it, so nothing needs clearing
@@ -1046,8 +1161,7 @@ namespace {
 constexpr int kNoAllocSlots = 2048;
 constexpr int64_t kNoAllocChunk = 16384;  // float4 per partial sum (65,536 weights)
 constexpr int64_t kNoAllocMaxElems = (int64_t)kNoAllocSlots * kNoAllocChunk * 4;
-constexpr size_t kNoAllocThreshOff = (size_t)kNoAllocSlots * sizeof(tq::DD);
-constexpr size_t kNoAllocBytes = kNoAllocThreshOff + 256;
+constexpr size_t kNoAllocBytes = (size_t)kNoAllocSlots * sizeof(double);  // tq_absum_partial_kernel's output
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
@@ -1078,7 +1192,9 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     if (!w || !packed || !gamma) return TQ_ERR_NULL;
     if (N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
     if (tq_status e = check_k(K)) return e;
-    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE)) return TQ_ERR_ARG;
+    if (flags & ~(TQ_GAMMA_PER_ROW | TQ_FLAG_SANITIZE_NONFINITE | TQ_ENC_MASK)) return TQ_ERR_ARG;
+    const int enc = flag_encoding(flags);
+    if (enc < 0) return TQ_ERR_ARG;
     const bool per_row = flags & TQ_GAMMA_PER_ROW;
     if (!per_row && N * K > kNoAllocMaxElems) return TQ_ERR_SHAPE;
     if (!aligned16(w) || !aligned16(packed) || !aligned16(gamma)) return TQ_ERR_ALIGN;
@@ -1091,7 +1207,9 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
     cudaStream_t st = cs(stream);
     if (per_row) {
-        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, 0, 0.0f, st)) return e;
+        if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, pack_opts(0, enc),
+                                           0.0f, st))
+            return e;
         return launch_status();
     }
     void *scratch = nullptr;
@@ -1099,13 +1217,14 @@ extern "C" tq_status tq_quantize_ternary_pack_noalloc(const float *w, int64_t N,
     const int64_t total_v = N * K / 4;
     const int64_t nparts = (total_v + kNoAllocChunk - 1) / kNoAllocChunk;  // <= kNoAllocSlots
     double *partial = reinterpret_cast<double *>(scratch);
-    if (tq_status e = launch_pdl(absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
+    if (tq_status e = launch_pdl(tq_absum_partial_kernel, dim3((unsigned)nparts), dim3(kPackThreads), 0,
                                  st, w, total_v, kNoAllocChunk, sanitize, partial, 0))
         return e;
     PerTensor pt;
     pt.partial = partial;
     pt.nparts = (int)nparts;
     pt.height = absum_tree_height(kNoAllocChunk, (int)nparts);
-    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, 0, 0.0f, st)) return e;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, pt, 1, pack_opts(0, enc), 0.0f, st))
+        return e;
     return launch_status();
 }

@@ -310,6 +310,19 @@ __device__ __forceinline__ void mma_16x8x32_u8s8(int (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// 4x4 byte transpose: out word j = (in0.byte j, in1.byte j, in2.byte j, in3.byte j).
+__device__ __forceinline__ uint4 transpose_bytes4x4(uint4 q) {
+    const uint32_t t0 = __byte_perm(q.x, q.y, 0x5140), t1 = __byte_perm(q.x, q.y, 0x7362);
+    const uint32_t t2 = __byte_perm(q.z, q.w, 0x5140), t3 = __byte_perm(q.z, q.w, 0x7362);
+    return make_uint4(__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
+                      __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632));
+}
+
+// Position of 16-byte chunk c inside an x_q row as the small-M GEMV keeps it
+// in shared memory: chunks 8..15 of every 16 swap in pairs, so the chunk reads
+// of a quarter warp (two rows, four column offsets) hit distinct banks.
+__host__ __device__ __forceinline__ int gemv_chunk_pos(int c) { return c ^ (((c >> 3) & 1) << 1); }
+
 // ---------------------------------------------------------------------------
 // Double-double accumulation of non-negative terms, and the correctly
 // rounded fp32 mean derived from it.

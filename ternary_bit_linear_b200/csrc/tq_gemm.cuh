@@ -104,7 +104,7 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
 // (bias, integer bias and shift) is applied.
 template <int BT, bool CONV, bool EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+    tq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
                 const float *__restrict__ gamma, int per_row, int M, int N, int K,
                 float *__restrict__ y, int32_t *__restrict__ acc_out, int mode, Epilogue ep) {

@@ -9,11 +9,11 @@
 // 4096 x 4096 layer is 4 MiB, about 0.65 us of HBM time -- less than the
 // latency of one launch.  Two kernels share the per-strip arithmetic:
 //
-//   gemv_kernel (a layer that waits for its predecessor): one CTA per 16-row
+//   tq_gemv_kernel (a layer that waits for its predecessor): one CTA per 16-row
 //     strip over the whole GPU, so the time from "inputs ready" to "y stored"
 //     -- the critical path of a chain of dependent layers -- is as short as
 //     possible.
-//   gemv_stream_kernel (independent calls, TQ_FLAG_INPUTS_READY): a narrow
+//   tq_gemv_stream_kernel (independent calls, TQ_FLAG_INPUTS_READY): a narrow
 //     grid of 32-odd CTAs that stream runs of strips.  Under programmatic
 //     dependent launch the next kernel starts only once every CTA of this one
 //     is resident; a narrow grid is resident at once, so several layers'
@@ -51,16 +51,8 @@ constexpr int kGemvMaxK = 8192;
 // Shared-memory row stride of x_q (16 bytes past a multiple of 128) and the
 // swizzled position of 16-byte chunk c inside a row.
 __host__ __device__ inline int gemv_x_stride(int K) { return K + ((16 - K % 128) + 128) % 128; }
-__device__ __forceinline__ uint32_t x_chunk(int c) { return (uint32_t)(c ^ (((c >> 3) & 1) << 1)) << 4; }
+__device__ __forceinline__ uint32_t x_chunk(int c) { return (uint32_t)gemv_chunk_pos(c) << 4; }
 __host__ __device__ inline int gemv_x_bytes(int M, int K) { return M * gemv_x_stride(K); }
-
-// 4x4 byte transpose: out word j = (in0.byte j, in1.byte j, in2.byte j, in3.byte j).
-__device__ __forceinline__ uint4 transpose_bytes4x4(uint4 q) {
-    const uint32_t t0 = __byte_perm(q.x, q.y, 0x5140), t1 = __byte_perm(q.x, q.y, 0x7362);
-    const uint32_t t2 = __byte_perm(q.z, q.w, 0x5140), t3 = __byte_perm(q.z, q.w, 0x7362);
-    return make_uint4(__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
-                      __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632));
-}
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 r;
@@ -211,7 +203,7 @@ __device__ __forceinline__ void transpose_x(uint32_t x_s, int M, int K, int XS, 
 // stream's results in order; the other CTAs leave as soon as they are done.
 template <int NB, int W, int SPW, bool CONV, bool EPI>
 __global__ void __launch_bounds__(W * 32, gemv_min_blocks(NB, W))
-    gemv_kernel(const int8_t *__restrict__ xq, const float *__restrict__ s_x,
+    tq_gemv_kernel(const int8_t *__restrict__ xq, const float *__restrict__ s_x,
                 const int32_t *__restrict__ rowsum, const uint8_t *__restrict__ packed,
                 const float *__restrict__ gamma, int per_row, int M, int64_t N, int K,
                 float *__restrict__ y, int32_t *__restrict__ acc_out, int mode, Epilogue ep) {
@@ -328,7 +320,7 @@ __device__ __forceinline__ void group_sync(int group) {
 // the two-CTAs-per-SM limit.
 template <int ENC>
 __global__ void __launch_bounds__(kStreamThreads, 2)
-    gemv_stream_kernel(const int8_t *__restrict__ xq, const float *__restrict__ s_x,
+    tq_gemv_stream_kernel(const int8_t *__restrict__ xq, const float *__restrict__ s_x,
                        const int32_t *__restrict__ rowsum, const uint8_t *__restrict__ packed,
                        const float *__restrict__ gamma, int per_row, int M, int64_t N, int K,
                        float *__restrict__ y, int32_t *__restrict__ acc_out, int per_cta) {

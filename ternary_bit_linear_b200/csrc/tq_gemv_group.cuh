@@ -1,0 +1,345 @@
+// tq_gemv_group.cuh -- grouped small-M (decode) ternary GEMV: G independent
+// layers of one shape, y_g = (x_q,g . q_g) * gamma_g * s_x,g, in one launch.
+//
+// The per-strip arithmetic is the small-M GEMV's (tq_gemv.cuh; Hetman-2b,
+// src/quantization.py, section 7 simulate_hardware_bitnet_gemv: decode the
+// packed codes branch-free and accumulate in int32, then one fp32 rescale).
+// What changes is how the bytes move: a 4096 x 4096 layer is 4 MiB, less HBM
+// time than one launch takes, so G layers share one persistent launch that
+// streams all of their packed weights back to back.
+//
+//   * Work unit: a strip of 16 consecutive weight rows of one problem (16 x
+//     K/4 contiguous bytes).  The G * ceil(N/16) strips are split into
+//     contiguous runs, one per CTA (one CTA per SM).
+//   * Warp 8 (lane 0) is the producer: 1-D bulk copies (TMA engine) bring each
+//     strip into a ring of `stages` shared-memory slots, one copy per row so
+//     that rows land kRowPad bytes past a multiple of 128 apart (conflict-free
+//     fragment reads); the copies of the first slots are issued before the
+//     wait for the previous kernel when the weights are static.  The same
+//     thread copies each problem's x_q rows (written by the activation pass in
+//     the GEMV's transposed, chunk-swizzled layout) into one of two x buffers.
+//   * Warps 0-7 form teams of `ksplit` warps; team q takes strips q, q + T,
+//     ... of the run; warp j of a team takes the strip's 64-byte column steps
+//     j, j + ksplit, ...; the team's partial sums meet in shared memory
+//     (double-buffered by strip) and its first warp finishes the outputs.
+//   * Synchronisation: full/empty mbarriers per ring slot; xfull/xempty per x
+//     buffer (every consumer warp passes every problem of the run in order,
+//     so a buffer is refilled only after all warps are done with it).  All
+//     waits are bounded; a wait that gives up records TQ_ERR_TIMEOUT, and the
+//     CTA skips the rest of its work but keeps the barrier protocol, and the
+//     producer lets its copies land before it exits.
+#pragma once
+
+#include "tq_common.cuh"
+#include "tq_gemv.cuh"
+
+namespace tq {
+
+constexpr int kGroupMax = 64;  // problems per launch
+constexpr int kGrpConsumerWarps = 8;
+constexpr int kGrpThreads = (kGrpConsumerWarps + 1) * 32;
+constexpr int kGrpStagesMax = 8;
+constexpr int kRowPad = 64;  // a strip row's shared-memory stride is K/4 + kRowPad
+
+// Per-problem pointers (device), read by dynamic index from parameter space.
+struct GroupTable {
+    const uint8_t *packed[kGroupMax];
+    const float *gamma[kGroupMax];
+};
+
+// Host-computed shape and shared-memory plan of one launch.
+struct GroupPlan {
+    int M, K, KB;           // tokens, contraction length, packed bytes per row
+    int64_t N;              // rows per problem
+    int64_t spp;            // strips per problem
+    int64_t nstrips;        // G * spp
+    int x_shared;           // one x_q batch serves every problem
+    int per_row;            // gamma per row (else one per problem)
+    int weights_static;     // weight copies may start before the wait
+    int enc;                // packed-code layout (kEnc*)
+    int ksplit;             // warps per strip (1, 2, 4, 8)
+    int stages, xbufs;      // ring slots, x buffers (1 or 2)
+    int RS, XS;             // shared-memory row strides: strip rows, x_q rows
+    int off_x, off_red, off_bar;  // byte offsets of the x buffers, partial sums, barriers
+    int smem;               // dynamic shared memory bytes
+};
+
+__host__ __device__ inline int grp_red_bytes(int NB) { return 2 * kGrpConsumerWarps * 4 * NB * 32 * 4; }
+
+// Shared-memory plan; returns false if even one x buffer and two slots do not fit.
+inline bool grp_plan(GroupPlan &p, int NB, int budget) {
+    p.KB = p.K / 4;
+    p.RS = p.KB + kRowPad;
+    p.XS = gemv_x_stride(p.K);
+    const int stage = 16 * p.RS, xbytes = p.M * p.XS, red = grp_red_bytes(NB);
+    const int bars = (2 * kGrpStagesMax + 4) * 8 + 16;
+    for (int xb = 2; xb >= 1; --xb) {
+        const int avail = budget - xb * xbytes - red - bars;
+        int st = avail / stage;
+        if (st > kGrpStagesMax) st = kGrpStagesMax;
+        if (st >= (xb == 2 ? 3 : 2)) {
+            p.stages = st;
+            p.xbufs = xb;
+            p.off_x = st * stage;
+            p.off_red = p.off_x + xb * xbytes;
+            p.off_bar = p.off_red + red;
+            p.smem = p.off_bar + bars;
+            // warps per strip: keep about half of the slots in flight
+            const int nsteps = p.KB / 64;
+            int teams = st / 2 < 1 ? 1 : st / 2;
+            if (teams > kGrpConsumerWarps) teams = kGrpConsumerWarps;
+            int ks = (kGrpConsumerWarps + teams - 1) / teams;
+            int k2 = 1;
+            while (k2 < ks) k2 <<= 1;  // a power of two dividing 8
+            if (k2 > kGrpConsumerWarps) k2 = kGrpConsumerWarps;
+            while (k2 > 1 && k2 > nsteps) k2 >>= 1;
+            p.ksplit = k2;
+            return true;
+        }
+    }
+    return false;
+}
+
+// Partial sums of one warp over the column steps j, j + ks, ... of a strip in
+// shared memory (rows at stride RS; x_q chunks transposed and swizzled).
+template <int NB, int CH, bool CONV>
+__device__ __forceinline__ void strip_mma_smem(int (&d)[CH][NB][4], uint32_t w_s, int RS, uint32_t x_s, int XS,
+                                               int M, int KB, int j0, int ks, int lane, int enc) {
+    const int g = lane >> 2, t = lane & 3;
+    const int nsteps = KB >> 6;
+    const uint32_t xsw = (uint32_t)(t & 2) << 4;
+#pragma unroll
+    for (int i = 0; i < CH; ++i)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) d[i][nb][0] = d[i][nb][1] = d[i][nb][2] = d[i][nb][3] = 0;
+    const uint32_t ra = w_s + (uint32_t)(g * RS + t * 16), rb = ra + (uint32_t)(8 * RS);
+    for (int step = j0; step < nsteps; step += ks) {
+        const int bo = step * 64 + t * 16;
+        const uint4 wa = lds128(ra + (uint32_t)(step * 64)), wb = lds128(rb + (uint32_t)(step * 64));
+        const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w};
+        const uint32_t b4[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t ar = CONV ? codes_to_foundry(a4[i], enc) : a4[i];
+            const uint32_t br = CONV ? codes_to_foundry(b4[i], enc) : b4[i];
+            uint32_t ua[4], ub[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                ua[jj] = (ar >> (2 * jj)) & 0x03030303u;
+                ub[jj] = (br >> (2 * jj)) & 0x03030303u;
+            }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int m = g + 8 * nb;
+                uint4 xt = make_uint4(0u, 0u, 0u, 0u);
+                if (m < M) xt = lds128(x_s + (uint32_t)(m * XS + 4 * bo) + ((uint32_t)(i << 4) ^ xsw));
+                mma_16x8x32_u8s8(d[i % CH][nb], ua[0], ub[0], ua[1], ub[1], xt.x, xt.y);
+                mma_16x8x32_u8s8(d[i % CH][nb], ua[2], ub[2], ua[3], ub[3], xt.z, xt.w);
+            }
+        }
+    }
+}
+
+// NB: token blocks of 8 (M <= 8 NB).  ENC: packed-code layout.
+template <int NB, int ENC>
+__global__ void __launch_bounds__(kGrpThreads, 1)
+    tq_gemv_group_kernel(const __grid_constant__ GroupTable tab, const __grid_constant__ GroupPlan pl,
+                         const int8_t *__restrict__ xq, const float *__restrict__ s_x,
+                         const int32_t *__restrict__ rowsum, float *__restrict__ y) {
+    constexpr bool CONV = ENC != kEncFoundry;
+    constexpr int CH = 2;
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(dsm);
+    const int S = pl.stages, M = pl.M, KB = pl.KB, RS = pl.RS, XS = pl.XS;
+    const uint32_t bar0 = sbase + (uint32_t)pl.off_bar;
+    auto full = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+    auto empty = [&](int s) { return bar0 + 8u * (uint32_t)(kGrpStagesMax + s); };
+    auto xfull = [&](int b) { return bar0 + 8u * (uint32_t)(2 * kGrpStagesMax + b); };
+    auto xempty = [&](int b) { return bar0 + 8u * (uint32_t)(2 * kGrpStagesMax + 2 + b); };
+    const uint32_t stage_bytes = 16u * (uint32_t)RS;
+    auto stage_addr = [&](int s) { return sbase + (uint32_t)s * stage_bytes; };
+    auto xbuf_addr = [&](int b) { return sbase + (uint32_t)pl.off_x + (uint32_t)(b * M * XS); };
+
+    // contiguous run of strips of this CTA
+    const int64_t s0 = (int64_t)blockIdx.x * pl.nstrips / gridDim.x;
+    const int64_t s1 = (int64_t)(blockIdx.x + 1) * pl.nstrips / gridDim.x;
+    const int nloc = (int)(s1 - s0);
+    const int64_t p_first = s0 / pl.spp;
+    const int np = nloc > 0 ? (int)((s1 - 1) / pl.spp - p_first + 1) : 0;
+    const int ks = pl.ksplit, T = kGrpConsumerWarps / ks;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGrpStagesMax; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), (uint32_t)ks);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(xfull(b), 1);
+            mbar_init(xempty(b), kGrpConsumerWarps);
+        }
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_trigger();
+
+    volatile int *abrt = &abort_flag;
+    auto wait_spin = [&](uint32_t bar, uint32_t par) {
+        if (*abrt) return false;
+        if (mbar_wait(bar, par)) return true;
+        *abrt = 1;
+        return false;
+    };
+    auto wait_sleep = [&](uint32_t bar, uint32_t par) {
+        if (*abrt) return false;
+        if (mbar_wait_sleep(bar, par)) return true;
+        *abrt = 1;
+        return false;
+    };
+
+    if (warp == kGrpConsumerWarps) {
+        // ---------------- producer ----------------
+        if (lane == 0 && nloc > 0) {
+            const int8_t *xq0 = xq;
+            auto issue_x = [&](int pi) {
+                const int b = pi & 1;
+                if (pl.xbufs == 1 || pi >= 2) {  // buffer b last held problem pi - xbufs
+                    const int prev = pi - pl.xbufs;
+                    if (prev >= 0 && !wait_sleep(xempty(pl.xbufs == 1 ? 0 : b), (uint32_t)((prev / pl.xbufs) & 1)))
+                        return false;
+                }
+                const int bb = pl.xbufs == 1 ? 0 : b;
+                const int64_t p = p_first + pi;
+                const int8_t *src = xq0 + (pl.x_shared ? 0 : p) * (int64_t)M * pl.K;
+                mbar_arrive_expect_tx(xfull(bb), (uint32_t)(M * pl.K));
+                for (int m = 0; m < M; ++m)
+                    bulk_g2s(xbuf_addr(bb) + (uint32_t)(m * XS), src + (int64_t)m * pl.K, (uint32_t)pl.K, xfull(bb));
+                return true;
+            };
+            auto issue_w = [&](int i) {
+                const int s = i % S;
+                if (i >= S && !wait_sleep(empty(s), (uint32_t)(((i / S) - 1) & 1))) return false;
+                const int64_t t = s0 + i, p = t / pl.spp, ls = t - p * pl.spp;
+                const int64_t r0 = ls * 16;
+                const int rows = (int)(pl.N - r0 < 16 ? pl.N - r0 : 16);
+                const uint8_t *src = tab.packed[p] + r0 * KB;
+                mbar_arrive_expect_tx(full(s), (uint32_t)(rows * KB));
+                for (int r = 0; r < rows; ++r)
+                    bulk_g2s(stage_addr(s) + (uint32_t)(r * RS), src + (int64_t)r * KB, (uint32_t)KB, full(s));
+                return true;
+            };
+            int issued = 0;
+            const int pre = pl.weights_static ? (nloc < S ? nloc : S) : 0;
+            for (; issued < pre; ++issued) issue_w(issued);
+            pdl_wait();
+            int next_x = 0, x_issued = 0;
+            bool ok = true;
+            for (int i = 0; i < nloc && ok; ++i) {
+                const int pi = (int)((s0 + i) / pl.spp - p_first);
+                while (ok && next_x <= pi) {
+                    ok = issue_x(next_x++);
+                    if (ok) x_issued = next_x;
+                }
+                if (ok && i >= issued) {
+                    ok = issue_w(i);
+                    if (ok) issued = i + 1;
+                }
+            }
+            // Every copy lands before this thread exits.  In normal operation
+            // the consumers have waited for (or will wait for) each one; after
+            // a timeout they may have skipped theirs, and then only the last
+            // copy issued into each slot and buffer can still be in flight (no
+            // copy is issued once a wait has given up).
+            for (int s = 0; s < S && s < issued; ++s) {
+                const int last = s + ((issued - 1 - s) / S) * S;
+                mbar_wait_sleep(full(s), (uint32_t)((last / S) & 1));
+            }
+            for (int b = 0; b < pl.xbufs && b < x_issued; ++b) {
+                const int last = b + ((x_issued - 1 - b) / pl.xbufs) * pl.xbufs;
+                mbar_wait_sleep(xfull(b), (uint32_t)((last / pl.xbufs) & 1));
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers ----------------
+    pdl_wait();  // s_x, rowsum (and y) belong to work before this kernel
+    const int team = warp / ks, kw = warp % ks;
+    int *red = reinterpret_cast<int *>(dsm + pl.off_red);  // [2][8 warps][4 NB][32]
+    int par = 0;
+    int i = team;
+    for (int pi = 0; pi < np; ++pi) {
+        const int bb = pl.xbufs == 1 ? 0 : (pi & 1);
+        const int64_t p = p_first + pi;
+        const bool xok = !*abrt && warp_wait(xfull(bb), (uint32_t)((pi / pl.xbufs) & 1), lane);
+        if (!xok && lane == 0) *abrt = 1;
+        const uint32_t x_s = xbuf_addr(bb);
+        const float *sx_p = s_x + (pl.x_shared ? 0 : p) * (int64_t)M;
+        const int32_t *rs_p = rowsum + (pl.x_shared ? 0 : p) * (int64_t)M;
+        const float *gam = tab.gamma[p];
+        for (; i < nloc && (s0 + i) / pl.spp == p; i += T) {
+            const int s = i % S;
+            const bool ok = !*abrt && warp_wait(full(s), (uint32_t)((i / S) & 1), lane);
+            if (!ok && lane == 0) *abrt = 1;
+            int d[CH][NB][4];
+            if (ok && !*abrt)
+                strip_mma_smem<NB, CH, CONV>(d, stage_addr(s), RS, x_s, XS, M, KB, kw, ks, lane, ENC);
+            else
+#pragma unroll
+                for (int c = 0; c < CH; ++c)
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) d[c][nb][0] = d[c][nb][1] = d[c][nb][2] = d[c][nb][3] = 0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(s));  // the slot's words are in registers (consumed)
+            int acc[NB][4];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[nb][c] = d[0][nb][c] + d[1][nb][c];
+            if (ks > 1) {
+                int *rb = red + par * (kGrpConsumerWarps * 4 * NB * 32);
+                if (kw != 0) {
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) rb[(warp * 4 * NB + nb * 4 + c) * 32 + lane] = acc[nb][c];
+                }
+                asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(ks * 32) : "memory");
+                if (kw == 0) {
+                    for (int w2 = warp + 1; w2 < warp + ks; ++w2)
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) acc[nb][c] += rb[(w2 * 4 * NB + nb * 4 + c) * 32 + lane];
+                }
+                par ^= 1;
+            }
+            if (kw == 0 && !*abrt) {
+                // fragment c of lane (g, t): row g (+8 for c >= 2), token 8 nb + 2 t + (c & 1)
+                const int64_t t = s0 + i, ls = t - p * pl.spp;
+                const int g = lane >> 2, tt = lane & 3;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int64_t n = ls * 16 + g + ((c & 2) ? 8 : 0);
+                    if (n >= pl.N) continue;
+                    const float gv = __ldg(gam + (pl.per_row ? n : 0));
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        const int m = 8 * nb + 2 * tt + (c & 1);
+                        if (m < M) {
+                            const int a = acc[nb][c] - __ldcg(rs_p + m);
+                            y[(p * M + m) * pl.N + n] =
+                                __fmul_rn(__int2float_rn(a), __fmul_rn(gv, __ldcg(sx_p + m)));
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xempty(bb));
+    }
+}
+
+}  // namespace tq

@@ -136,7 +136,7 @@ __device__ __forceinline__ double sum_error_bound(int h) { return (double)(h + 3
 //   pass 2: re-read the row (L2 hit: pass 1 left it there) and write one byte
 //           per float4; a warp stores 32 consecutive bytes per instruction.
 // ---------------------------------------------------------------------------
-// Per-tensor gamma from the partial sums of absum_partial_kernel, computed by
+// Per-tensor gamma from the partial sums of tq_absum_partial_kernel, computed by
 // every CTA of the pack pass (all kPackThreads threads take part): a fixed
 // thread-strided chain over the partials and a fixed block tree, then the
 // rounding-margin check of mean_fast_or_fail with the error bound of the
@@ -186,7 +186,7 @@ constexpr int kPackUnroll = 8;
 
 template <bool SAN, bool CONV>
 __global__ void __launch_bounds__(kPackThreads)
-    pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
+    tq_pack_rows_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
                      int opts, float ratio) {
@@ -290,7 +290,7 @@ __host__ __device__ constexpr int pack_team_smem(int T, int K) {
 
 template <int T, bool SAN, bool CONV>
 __global__ void __launch_bounds__(kPackThreads, 2)
-    pack_team_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
+    tq_pack_team_kernel(const float *__restrict__ w, int64_t N, int K, double inv_k,
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
                      int opts, float ratio) {
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kPackThreads, 2)
 // Per-tensor gamma, pass 1: CTA b sums |w| over float4 range [b*chunk, ...) in
 // plain fp64 (each thread sequentially, then a fixed block tree).
 __global__ void __launch_bounds__(kPackThreads)
-    absum_partial_kernel(const float *__restrict__ w, int64_t nv, int64_t chunk, int sanitize,
+    tq_absum_partial_kernel(const float *__restrict__ w, int64_t nv, int64_t chunk, int sanitize,
                          double *__restrict__ partial, int ready) {
     __shared__ double red[kPackWarps];
     if (!ready) pdl_wait();

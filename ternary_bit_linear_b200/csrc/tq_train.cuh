@@ -40,7 +40,7 @@ __device__ __forceinline__ float ste_one(float g, float w, float gm, float tau, 
 // crosses a row); gamma [N] (per_row) or [1].  out may be grad or w.
 template <bool SAN>
 __global__ void __launch_bounds__(kSteThreads)
-    ste_backward_kernel(const float4 *grad, const float4 *w, const float *__restrict__ gamma, int per_row,
+    tq_ste_backward_kernel(const float4 *grad, const float4 *w, const float *__restrict__ gamma, int per_row,
                         int64_t nvec, int64_t kvec, float tau, float4 *out) {
     pdl_wait();
     pdl_trigger();
@@ -137,7 +137,7 @@ __device__ __forceinline__ uint32_t flip_byte(uint32_t byte, const float4 g4, fl
 // owns chunks [b * per_cta, (b + 1) * per_cta).
 template <bool CONV>
 __global__ void __launch_bounds__(kFlipThreads, 2)
-    flip_kernel(uint8_t *packed, const float *__restrict__ grad, int64_t nw, float temp, uint64_t x0,
+    tq_flip_kernel(uint8_t *packed, const float *__restrict__ grad, int64_t nw, float temp, uint64_t x0,
                 int64_t per_cta, int mode) {
     extern __shared__ __align__(16) uint8_t flip_smem[];
     __shared__ uint64_t chunk_state;
@@ -246,7 +246,7 @@ __device__ __forceinline__ void load_g8(const float *row, const float *gamma, in
 // VEC: rows are 16-byte aligned (N % 4 == 0).
 template <bool VEC>
 __global__ void __launch_bounds__(kSplitThreads)
-    bwd_split_kernel(const float *__restrict__ dY, const float *__restrict__ gamma, int per_row, int M, int N,
+    tq_bwd_split_kernel(const float *__restrict__ dY, const float *__restrict__ gamma, int per_row, int M, int N,
                      int Np, __half *__restrict__ planes, float *__restrict__ inv_scale) {
     __shared__ float red[kSplitThreads / 32];
     pdl_wait();
@@ -392,7 +392,7 @@ __device__ __forceinline__ uint2 codes4_to_f16(uint32_t byte) {
 // packed: tensor map over [N][K / 4] bytes; inv_scale [M] = 2^-e_t.  dX [M][K] fp32.
 template <bool CONV>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_w,
+    tq_bwd_gemm_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_w,
                     const float *__restrict__ inv_scale, const float *__restrict__ row_scale, int accumulate, int M,
                     int N, int K, float *__restrict__ dX, int mode) {
     constexpr int S = kBwdStages, SW = kBwdWStages;

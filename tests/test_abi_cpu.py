@@ -38,7 +38,8 @@ def test_header_flag_values_match_binding():
     flags = dict((k, int(v)) for k, v in re.findall(r"#define\s+TQ_(\w+)\s+\(1u\s*<<\s*(\d+)\)", src))
     py = {"GAMMA_PER_ROW": tq.GAMMA_PER_ROW, "FLAG_FWHT": tq.FLAG_FWHT, "FLAG_RMSNORM": tq.FLAG_RMSNORM,
           "FLAG_ETA_CLAMP": tq.FLAG_ETA_CLAMP, "FLAG_SANITIZE_NONFINITE": tq.FLAG_SANITIZE_NONFINITE,
-          "FLAG_WEIGHTS_STATIC": tq.FLAG_WEIGHTS_STATIC, "FLAG_INPUTS_READY": tq.FLAG_INPUTS_READY}
+          "FLAG_WEIGHTS_STATIC": tq.FLAG_WEIGHTS_STATIC, "FLAG_INPUTS_READY": tq.FLAG_INPUTS_READY,
+          "FLAG_ACCUMULATE": tq.FLAG_ACCUMULATE, "FLAG_SHARED_INPUT": tq.FLAG_SHARED_INPUT}
     for name, value in py.items():
         assert name in flags, name
         assert value == 1 << flags[name], name
@@ -86,6 +87,58 @@ def test_pack_validation(lib):
     assert f(P(), 4, 64, 1, P(16), P(2 << 20), None, 0, None) == 4           # overlap w/packed
     assert f(P(), 4, 64, 0, P(1 << 20), P(2 << 20), None, 0, None) == 1      # needs workspace
     assert f(P(), 4, 64, 0, P(1 << 20), P(2 << 20), P(3 << 20), 8, None) == 4  # too small
+
+
+def test_noalloc_validation(lib):
+    """tq_quantize_ternary_pack_noalloc: its own limits, checked before any
+    device work (the pointers are fake and never touched)."""
+    f = lib.tq_quantize_ternary_pack_noalloc
+    limit = 2048 * 65536  # per-tensor weights the fixed scratch array covers
+    N, K = limit // 65536 + 1, 65536  # one row past the limit
+    big = ctypes.c_void_p(1 << 40)
+    assert f(big, N, K, 0, ctypes.c_void_p((1 << 40) + (1 << 36)), ctypes.c_void_p((1 << 40) + (1 << 37)),
+             None) == 2                                                       # over the limit
+    assert f(None, 4, 64, 0, P(1 << 20), P(2 << 20), None) == 1                # NULL
+    assert f(P(4), 4, 64, 0, P(1 << 20), P(2 << 20), None) == 3                # misaligned
+    assert f(P(), 4, 64, tq.FLAG_INPUTS_READY, P(1 << 20), P(2 << 20), None) == 4  # shared scratch: no overlap
+    assert f(P(), 4, 64, 3 << 7, P(1 << 20), P(2 << 20), None) == 4            # reserved layout
+    assert f(P(), 4, 60, 0, P(1 << 20), P(2 << 20), None) == 2                 # K % 64
+
+
+def test_grouped_validation(lib):
+    """tq_bitlinear_grouped: shape, flag, pointer-table and workspace checks
+    before any device work (fake device pointers, never touched)."""
+    f = lib.tq_bitlinear_grouped
+    G, M, N, K = 3, 4, 64, 256
+    arr = ctypes.c_void_p * G
+    pk = arr(*[FAKE + (8 << 20) + i * (1 << 20) for i in range(G)])
+    gm = arr(*[FAKE + (16 << 20) + i * 4096 for i in range(G)])
+    ws_need = lib.tq_grouped_workspace_bytes(G, M, K, 0)
+    assert ws_need >= G * M * K + 2 * G * M * 4
+    assert lib.tq_grouped_workspace_bytes(G, M, K, tq.FLAG_SHARED_INPUT) < ws_need
+    x, y, ws = P(), P(1 << 20), P(2 << 20)
+    ok = [x, G, ctypes.cast(pk, ctypes.c_void_p), ctypes.cast(gm, ctypes.c_void_p), 0, M, N, K, y, ws, ws_need, None]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["x", "G", "packed", "gamma", "flags", "M", "N", "K", "y", "ws", "wsb", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return f(*a)
+    assert call(x=None) == 1
+    assert call(packed=None) == 1
+    assert call(G=0) == 2 and call(G=65) == 2           # 1 <= G <= 64
+    assert call(M=17) == 2 and call(M=0) == 2           # the small-M range
+    assert call(K=8256) == 2 and call(K=100) == 2       # K <= 8192, K % 64 == 0
+    assert call(flags=1 << 11) == 4                     # unknown flag
+    assert call(flags=3 << 7) == 4                      # reserved layout
+    assert call(wsb=ws_need - 1) == 4                   # workspace too small
+    assert call(x=P(4)) == 3                            # misaligned
+    assert call(y=P(64)) == 4                           # y overlaps x
+    bad = arr(*([FAKE + (8 << 20)] * (G - 1) + [0]))
+    assert call(packed=ctypes.cast(bad, ctypes.c_void_p)) == 1  # a NULL entry
+    odd = arr(*([FAKE + (8 << 20)] * (G - 1) + [FAKE + (9 << 20) + 4]))
+    assert call(packed=ctypes.cast(odd, ctypes.c_void_p)) == 3  # a misaligned entry
 
 
 def test_pack_threshold_validation(lib):

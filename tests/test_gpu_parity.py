@@ -842,35 +842,77 @@ def test_gemm_ex_bias_and_integer_epilogue(cuda_lib, M, N, K, layout):
 
 
 # ---------------------------------------------------------------------------
-# NEXT row N3: Hetman-2b's clamped SwiGLU block of three BitLinear layers.
-# gate/up projections within 1e-5 (through the clamped activation, compared
-# to the oracle's within a few ulp of SiLU's fp32 evaluation); the block's
-# output equals the fused layer run on its own activation, which in turn is
-# checked against the oracle with the fused path's rule.
+# NEXT row N3: Hetman-2b's clamped SwiGLU block of three BitLinear layers,
+# every stage against the oracle's own chain (nothing the GPU produced is fed
+# to the oracle):
+#   * the gate/up projections' input codes and the projections themselves,
+#     with the fused layer's rule (codes within 1 LSB on <= 1e-4 of the
+#     elements; y within 1e-5, or bounded by the flipped codes);
+#   * the clamped activation within the error its fp32 evaluation can carry:
+#     SiLU(g) * u as g / (1 + expf(-g)) * u is within 4 ulp of the exact value
+#     for the GPU's own g, u (expf <= 2 ulp, three IEEE operations), and the
+#     differences of g and u from the oracle's propagate with the condition
+#     numbers |1 + g (1 - sigmoid(g))| and 1 (the clamp is 1-Lipschitz);
+#   * the down projection's input codes and the block output, again with the
+#     fused layer's rule.
 # ---------------------------------------------------------------------------
+def check_codes_and_y(xq, sx, y, xq_ref, sx_ref, y_ref, gamma_n):
+    """The fused layer's bar: codes within 1 LSB on <= 1e-4 of the elements,
+    s_x within 1e-5; y within 1e-5 where no code of its token moved, else
+    within the flips' bound (each flip moves acc by one)."""
+    d = np.abs(xq.astype(np.int32) - xq_ref.astype(np.int32))
+    assert d.max() <= 1
+    assert (d != 0).sum() <= 1e-4 * d.size, f"{(d != 0).sum()} codes differ"
+    rel_sx = np.abs(sx.astype(np.float64) - sx_ref) / sx_ref
+    assert rel_sx.max() <= REL
+    flips = (d != 0).sum(axis=1)
+    if flips.sum() == 0 and np.array_equal(sx, sx_ref):
+        assert_y_close(y, y_ref)
+    else:
+        bound = flips[:, None] * gamma_n[None, :].astype(np.float64) * sx_ref[:, None] * (1 + 1e-5) \
+            + REL * np.abs(y_ref) + np.abs(y_ref) * rel_sx[:, None]
+        assert np.all(np.abs(y.astype(np.float64) - y_ref) <= bound)
+    return int(flips.sum())
+
+
 @pytest.mark.parametrize("M,D,F,per_row", [(5, 512, 1024, False), (64, 1536, 6144, False), (33, 1024, 2048, True)])
 def test_swiglu_mlp(cuda_lib, M, D, F, per_row):
     tq = cuda_lib
     X = S.student_t3((M, D), 110, M)
     Ws = [S.normal(shape, 0.02, 111 + i, shape[0]) for i, shape in enumerate([(F, D), (F, D), (D, F)])]
     packs = [oracle.quantize_pack(W, per_row=per_row) for W in Ws]
-    y_ref, act_ref, _, yg_ref, yu_ref = oracle.swiglu_mlp(X, packs[0], packs[1], packs[2], per_row)
+    y_ref, act_ref, xq2_ref, yg_ref, yu_ref = oracle.swiglu_mlp(X, packs[0], packs[1], packs[2], per_row)
+    _, xq1_ref, sx1_ref, _ = oracle.bitlinear(X, packs[0][0], packs[0][1], per_row)
+    sx2_ref = oracle.bitlinear(act_ref, packs[2][0], packs[2][1], per_row)[2]
     fl = tq.FLAG_FWHT | tq.FLAG_RMSNORM | (tq.GAMMA_PER_ROW if per_row else 0)
     dp = [(dev(p), dev(g)) for p, g in packs]
     y = torch.empty((M, D), dtype=torch.float32, device="cuda")
     act = torch.empty((M, F), dtype=torch.float32, device="cuda")
-    ws = torch.empty((tq.swiglu_workspace_bytes(M, D, F, fl),), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros((tq.swiglu_workspace_bytes(M, D, F, fl),), dtype=torch.uint8, device="cuda")
     tq.swiglu_mlp_(dev(X), dp[0], dp[1], dp[2], fl, y, ws, 10.0, act)
-    act_h = host(act)
+    mid = {k: host(v) for k, v in tq.swiglu_intermediates(ws, M, D, F).items()}
+
+    def gam(i, n):
+        g = packs[i][1]
+        return g if per_row else np.full(n, g[0], np.float32)
+
+    # gate and up projections (one activation pass feeds both)
+    for yk, yr, i in (("y_gate", yg_ref, 0), ("y_up", yu_ref, 1)):
+        check_codes_and_y(mid["xq1"], mid["s_x1"], mid[yk], xq1_ref, sx1_ref, yr.astype(np.float64), gam(i, F))
+    # the clamped activation, from the GPU's own projections and against the oracle's
+    act_h = host(act).astype(np.float64)
     assert np.abs(act_h).max() <= 10.0
-    err = np.abs(act_h.astype(np.float64) - act_ref.astype(np.float64))
-    assert np.all(err <= 2e-5 * np.abs(act_ref.astype(np.float64)) + 1e-6)
-    # the down projection: the fused layer on the block's own activation, bit for bit
-    y_chk = torch.empty_like(y)
-    fws = torch.empty((tq.fused_workspace_bytes(M, F, fl),), dtype=torch.uint8, device="cuda")
-    tq.bitlinear_fused_(act, dp[2][0], dp[2][1], fl, y_chk, fws)
-    assert torch.equal(y, y_chk)
-    check_fused(tq, act_h, Ws[2], per_row)
+    g64, u64 = mid["y_gate"].astype(np.float64), mid["y_up"].astype(np.float64)
+    gr, ur = yg_ref.astype(np.float64), yu_ref.astype(np.float64)
+    sig = 1.0 / (1.0 + np.exp(-gr))
+    unclamped = gr * sig * ur
+    eps_g = np.abs(g64 - gr) / np.maximum(np.abs(gr), 1e-300)
+    eps_u = np.abs(u64 - ur) / np.maximum(np.abs(ur), 1e-300)
+    kappa = np.abs(1.0 + gr * (1.0 - sig))
+    bound = 2.0 * np.abs(unclamped) * (kappa * eps_g + eps_u + 4 * 2.0 ** -24) + 1e-30
+    assert np.all(np.abs(act_h - act_ref.astype(np.float64)) <= bound)
+    # the down projection and the block output
+    check_codes_and_y(mid["xq2"], mid["s_x2"], host(y), xq2_ref, sx2_ref, y_ref.astype(np.float64), gam(2, D))
     assert tq.device_status() == 0
 
 
