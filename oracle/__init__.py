@@ -58,6 +58,7 @@ def _load():
         _lib.tqo_quantize_pack.argtypes = [P, I64, I64, I, I, P, P]
         _lib.tqo_quantize_pack_format.argtypes = [P, I64, I64, I, I, I, P, P]
         _lib.tqo_quantize_pack_threshold.argtypes = [P, I64, I64, I, I, I, F, P, P]
+        _lib.tqo_quantize_pack_abs_threshold.argtypes = [P, I64, I64, I, I, F, P, P]
         _lib.tqo_dequant_bias.argtypes = [P, P, I, P, P, I64, I64, P]
         _lib.tqo_int_epilogue.argtypes = [P, P, I, I64, I64, P]
         _lib.tqo_fwht_roundtrip.argtypes = [P, I64, I64, F, F, P, P]
@@ -168,6 +169,20 @@ def quantize_pack_threshold(w, per_row: bool, ratio: float, sanitize: bool = Fal
     _load().tqo_quantize_pack_threshold(pw, N, K, int(per_row), int(sanitize), int(encoding), float(ratio),
                                         packed.ctypes.data_as(ctypes.c_void_p),
                                         gamma.ctypes.data_as(ctypes.c_void_p))
+    return packed, gamma
+
+
+def quantize_pack_abs_threshold(w, threshold: float, sanitize: bool = False, encoding: int = 0):
+    """Foundry's manual threshold (fq_quantize_ternary_threshold): code =
+    sign(w) where |w| > threshold, scale gamma[0] = threshold; returns
+    (packed, gamma) like quantize_pack."""
+    w, pw = _c(w, np.float32)
+    N, K = w.shape
+    packed = np.empty((N, K // 4), np.uint8)
+    gamma = np.empty((1,), np.float32)
+    _load().tqo_quantize_pack_abs_threshold(pw, N, K, int(sanitize), int(encoding), float(threshold),
+                                            packed.ctypes.data_as(ctypes.c_void_p),
+                                            gamma.ctypes.data_as(ctypes.c_void_p))
     return packed, gamma
 
 

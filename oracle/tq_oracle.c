@@ -319,6 +319,35 @@ void tqo_quantize_pack_threshold(const float *w_in, int64_t N, int64_t K, int pe
     free(tmp);
 }
 
+/* [F] "Ternary Quantization": the manual-threshold variant
+ * fq_quantize_ternary_threshold(weights, shape, ndim, threshold).  The page
+ * gives the absmean rule as "threshold = mean |w|; w > threshold -> +1,
+ * w < -threshold -> -1, otherwise 0; scale = threshold" and says a manual
+ * threshold replaces the automatic absmean one, so here the caller's threshold
+ * takes mean |w|'s place in all three lines: codes by strict comparison with
+ * +-thr, and the stored scale (gamma[0]) is thr itself.  One scale for the
+ * tensor, as the page's call takes one threshold.  thr >= 0, finite. */
+void tqo_quantize_pack_abs_threshold(const float *w_in, int64_t N, int64_t K, int sanitize, int format,
+                                     float thr, uint8_t *packed, float *gamma)
+{
+    const float *w = w_in;
+    float *tmp = NULL;
+    if (sanitize) {
+        tmp = (float *)malloc((size_t)(N * K) * sizeof(float));
+        tqo_sanitize_weights(w_in, N * K, tmp);
+        w = tmp;
+    }
+    int8_t *q = (int8_t *)malloc((size_t)(N * K));
+    for (int64_t i = 0; i < N * K; ++i) {
+        float v = w[i];
+        q[i] = (int8_t)(v > thr ? 1 : (v < -thr ? -1 : 0));
+    }
+    gamma[0] = thr;
+    tqo_pack_format(q, N, K, format, packed);
+    free(q);
+    free(tmp);
+}
+
 /* ratio 0: the round/clamp rule of tqo_ternary_codes. */
 void tqo_quantize_pack_format(const float *w_in, int64_t N, int64_t K, int per_row,
                               int sanitize, int format, uint8_t *packed, float *gamma)

@@ -149,6 +149,43 @@ def test_threshold_rule_hand_worked_rows():
         assert q[0].tolist() == [int(c) for c in codes.split()], ln
 
 
+def test_manual_threshold_hand_worked_rows():
+    """Foundry's manual threshold: codes and packed bytes worked by hand, the
+    stored scale equal to the threshold itself, every layout decoding to the
+    same codes."""
+    for ln in golden_lines("abs_threshold_codes.txt"):
+        t, ws, codes, bytes_ = [f.strip() for f in ln.split("|")]
+        w = np.array([[float(v) for v in ws.split()]], np.float32)
+        p, g = oracle.quantize_pack_abs_threshold(w, float(t))
+        assert g.tolist() == [np.float32(float(t))], ln
+        assert p[0].tolist() == [int(b, 16) for b in bytes_.split()], ln
+        want = [int(c) for c in codes.split()]
+        for enc in (1, 2):
+            pe, _ = oracle.quantize_pack_abs_threshold(w, float(t), encoding=enc)
+            assert oracle.unpack_format(pe, 8, enc)[0].tolist() == want, (ln, enc)
+
+
+def test_manual_threshold_limits_and_sanitising():
+    """t = 0 is the sign (zeros stay 0); t above every |w| gives all zeros; with
+    t = the row's mean |w| it is the absmean threshold rule (ratio 1); NaN -> 0
+    and +-inf -> +-1 under sanitising."""
+    W = S.laplace((16, 256), 0.02, 22, 16)
+    p, g = oracle.quantize_pack_abs_threshold(W, 0.0)
+    q, _ = oracle.unpack(p, 256)
+    assert np.array_equal(q, np.sign(W).astype(np.int8))
+    p, _ = oracle.quantize_pack_abs_threshold(W, float(np.abs(W).max()))
+    assert np.all(oracle.unpack(p, 256)[0] == 0)
+    for n in range(3):
+        row = W[n:n + 1]
+        gamma = oracle.absmean_gamma(row)
+        p_abs, _ = oracle.quantize_pack_abs_threshold(row, float(gamma))
+        p_thr, _ = oracle.quantize_pack_threshold(row, per_row=True, ratio=1.0)
+        assert np.array_equal(p_abs, p_thr)
+    bad = np.array([[np.nan, np.inf, -np.inf, 0.5]], np.float32)
+    p, _ = oracle.quantize_pack_abs_threshold(bad, 0.75, sanitize=True)
+    assert oracle.unpack(p, 4)[0][0].tolist() == [0, 1, -1, 0]
+
+
 def test_threshold_rule_one_half_matches_round_rule_off_ties():
     # ratio 0.5: w > gamma/2 is the round rule's |w/gamma| > 0.5 except where the
     # fp32 quotient lands exactly on 0.5 (the round rule then gives 0, as strict > does,
