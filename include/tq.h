@@ -169,6 +169,25 @@ TQ_API tq_status tq_quantize_ternary_pack_threshold(const float *w, int64_t N, i
                                              size_t workspace_bytes, tq_stream_t stream);
 
 /*
+ * Ternarisation with a manual (absolute) threshold, and 2-bit packing.
+ * Foundry, docs/quantization.md, "Ternary Quantization":
+ * fq_quantize_ternary_threshold(weights, shape, 2, 0.05f) ("Or with manual
+ * threshold"), read with the page's "Absmean Thresholding (BitNet b1.58)"
+ * rule with the caller's threshold t in place of mean |w|:
+ *
+ *   q = +1 if w > t, -1 if w < -t, else 0 (strict);  gamma[0] = t (the scale).
+ *
+ *   w, N, K, packed, stream: as for tq_quantize_ternary_pack.
+ *   gamma      [1] fp32, written: t.
+ *   threshold  t >= 0 and finite (else TQ_ERR_ARG); t = 0 gives sign(w).
+ *   flags      TQ_FLAG_SANITIZE_NONFINITE, TQ_FLAG_INPUTS_READY, TQ_ENC_*.
+ * One pass over W (no reduction, no workspace).
+ */
+TQ_API tq_status tq_quantize_ternary_pack_abs_threshold(const float *w, int64_t N, int64_t K, unsigned flags,
+                                                        float threshold, uint8_t *packed, float *gamma,
+                                                        tq_stream_t stream);
+
+/*
  * Same result as tq_quantize_ternary_pack, for callers that cannot allocate
  * device memory (a runtime whose allocator owns all of HBM and refuses new
  * reservations, a host that only receives device pointers, or a path where a

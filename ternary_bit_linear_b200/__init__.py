@@ -43,6 +43,7 @@ SIGNATURES = {
     "tq_pack_workspace_bytes": (_SZ, [_I64, _I64, _U]),
     "tq_quantize_ternary_pack_threshold": (_I, [_P, _I64, _I64, _U, _F, _P, _P, _P, _SZ, _P]),
     "tq_quantize_ternary_pack_noalloc": (_I, [_P, _I64, _I64, _U, _P, _P, _P]),
+    "tq_quantize_ternary_pack_abs_threshold": (_I, [_P, _I64, _I64, _U, _F, _P, _P, _P]),
     "tq_quantize_act_int8": (_I, [_P, _I64, _I64, _U, _F, _F, _P, _P, _P, _P]),
     "tq_fwht512": (_I, [_P, _P, _I64, _I64, _I, _P]),
     "tq_fwht_roundtrip": (_I, [_P, _P, _I64, _I64, _F, _F, _P, _P]),
@@ -152,6 +153,18 @@ def quantize_ternary_pack_threshold_(w, flags, ratio, packed, gamma, workspace=N
            load().tq_quantize_ternary_pack_threshold(_ptr(w), N, K, flags, float(ratio), _ptr(packed),
                                                      _ptr(gamma), _ptr(workspace), ws_bytes,
                                                      _stream(stream)))
+
+
+def quantize_ternary_pack_abs_threshold_(w, flags, threshold, packed, gamma, stream=None):
+    import torch
+
+    N, K = w.shape
+    _need(w, torch.float32, (N, K), "w")
+    _need(packed, torch.uint8, (N, K // 4), "packed")
+    _need(gamma, torch.float32, (1,), "gamma")
+    _check("tq_quantize_ternary_pack_abs_threshold",
+           load().tq_quantize_ternary_pack_abs_threshold(_ptr(w), N, K, flags, float(threshold), _ptr(packed),
+                                                         _ptr(gamma), _stream(stream)))
 
 
 def quantize_act_int8_(x, flags, eta_min, eta_max, xq, s_x, rowsum, stream=None):

@@ -376,12 +376,13 @@ tq_status launch_pack_rows_s(const float *w, int64_t N, int64_t K, uint8_t *pack
     return launch_pack_grid(tq_pack_rows_kernel<SAN, CONV>, occ[4], kPackWarps, 0, w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
 }
 
-// Options word of the pack kernels: bit 0 inputs ready, bits 1-2 layout.
+// Options word of the pack kernels: bit 0 inputs ready, bits 1-2 layout (bit 3:
+// kPackOptFixed).
 inline int pack_opts(int ready, int enc) { return (ready ? 1 : 0) | (enc << 1); }
 
 tq_status launch_pack_rows(const float *w, int64_t N, int64_t K, int sanitize, uint8_t *packed,
                            float *gamma, const PerTensor &pt, int reverse, int opts, float ratio, cudaStream_t st) {
-    if (opts >> 1)  // a layout other than Foundry's
+    if ((opts >> 1) & 3)  // a layout other than Foundry's
         return sanitize ? launch_pack_rows_s<true, true>(w, N, K, packed, gamma, pt, reverse, opts, ratio, st)
                         : launch_pack_rows_s<false, true>(w, N, K, packed, gamma, pt, reverse, opts, ratio, st);
     return sanitize ? launch_pack_rows_s<true, false>(w, N, K, packed, gamma, pt, reverse, opts, ratio, st)
@@ -669,6 +670,28 @@ tq_status tq_quantize_ternary_pack_threshold(const float *w, int64_t N, int64_t 
                                              tq_stream_t stream) {
     if (!(ratio > 0.0f && ratio <= 64.0f)) return TQ_ERR_ARG;  // NaN fails too
     return pack_impl(w, N, K, flags, ratio, packed, gamma, workspace, workspace_bytes, stream);
+}
+
+tq_status tq_quantize_ternary_pack_abs_threshold(const float *w, int64_t N, int64_t K, unsigned flags,
+                                                 float threshold, uint8_t *packed, float *gamma,
+                                                 tq_stream_t stream) {
+    if (!w || !packed || !gamma) return TQ_ERR_NULL;
+    if (N < 1 || N > INT32_MAX) return TQ_ERR_SHAPE;
+    if (tq_status e = check_k(K)) return e;
+    if (flags & ~(TQ_FLAG_SANITIZE_NONFINITE | TQ_FLAG_INPUTS_READY | TQ_ENC_MASK)) return TQ_ERR_ARG;
+    const int enc = flag_encoding(flags);
+    if (enc < 0) return TQ_ERR_ARG;
+    if (!(threshold >= 0.0f && threshold <= 3.4028235e38f)) return TQ_ERR_ARG;  // NaN fails too
+    if (!aligned16(w) || !aligned16(packed) || !aligned16(gamma)) return TQ_ERR_ALIGN;
+    const size_t wbytes = (size_t)(N * K) * 4, pbytes = (size_t)(N * K / 4);
+    if (overlap(w, wbytes, packed, pbytes) || overlap(w, wbytes, gamma, 4) || overlap(packed, pbytes, gamma, 4))
+        return TQ_ERR_ARG;
+    if (tq_status e = check_device(nullptr)) return e;
+    const int sanitize = (flags & TQ_FLAG_SANITIZE_NONFINITE) ? 1 : 0;
+    const int opts = pack_opts((flags & TQ_FLAG_INPUTS_READY) ? 1 : 0, enc) | kPackOptFixed;
+    if (tq_status e = launch_pack_rows(w, N, K, sanitize, packed, gamma, PerTensor{}, 0, opts, threshold, cs(stream)))
+        return e;
+    return launch_status();
 }
 
 tq_status tq_quantize_act_int8(const float *x, int64_t M, int64_t K, unsigned flags, float eta_min,

@@ -11,14 +11,14 @@
 //   * Work unit: a strip of 16 consecutive weight rows of one problem (16 x
 //     K/4 contiguous bytes).  The G * ceil(N/16) strips are split into
 //     contiguous runs, one per CTA (one CTA per SM).
-//   * Warp 8 (lane 0) is the producer: 1-D bulk copies (TMA engine) bring each
-//     strip into a ring of `stages` shared-memory slots, one copy per row so
-//     that rows land kRowPad bytes past a multiple of 128 apart (conflict-free
-//     fragment reads); the copies of the first slots are issued before the
-//     wait for the previous kernel when the weights are static.  The same
+//   * Warp 16 (lane 0) is the producer: one 1-D bulk copy (TMA engine) brings
+//     each strip (and, with per-row gamma, the strip's 16 gammas) into a ring
+//     of `stages` shared-memory slots; the copies of the first slots are
+//     issued before the wait for the previous kernel when the weights are
+//     static.  The same
 //     thread copies each problem's x_q rows (written by the activation pass in
 //     the GEMV's transposed, chunk-swizzled layout) into one of two x buffers.
-//   * Warps 0-7 form teams of `ksplit` warps; team q takes strips q, q + T,
+//   * Warps 0-15 form teams of `ksplit` warps; team q takes strips q, q + T,
 //     ... of the run; warp j of a team takes the strip's 64-byte column steps
 //     j, j + ksplit, ...; the team's partial sums meet in shared memory
 //     (double-buffered by strip) and its first warp finishes the outputs.
@@ -36,10 +36,10 @@
 namespace tq {
 
 constexpr int kGroupMax = 64;  // problems per launch
-constexpr int kGrpConsumerWarps = 8;
+constexpr int kGrpConsumerWarps = 16;
 constexpr int kGrpThreads = (kGrpConsumerWarps + 1) * 32;
 constexpr int kGrpStagesMax = 8;
-constexpr int kRowPad = 64;  // a strip row's shared-memory stride is K/4 + kRowPad
+constexpr int kGammaSlot = 64;  // bytes after a slot's 16 rows: the strip's per-row gammas
 
 // Per-problem pointers (device), read by dynamic index from parameter space.
 struct GroupTable {
@@ -69,9 +69,9 @@ __host__ __device__ inline int grp_red_bytes(int NB) { return 2 * kGrpConsumerWa
 // Shared-memory plan; returns false if even one x buffer and two slots do not fit.
 inline bool grp_plan(GroupPlan &p, int NB, int budget) {
     p.KB = p.K / 4;
-    p.RS = p.KB + kRowPad;
+    p.RS = p.KB;
     p.XS = gemv_x_stride(p.K);
-    const int stage = 16 * p.RS, xbytes = p.M * p.XS, red = grp_red_bytes(NB);
+    const int stage = 16 * p.RS + kGammaSlot, xbytes = p.M * p.XS, red = grp_red_bytes(NB);
     const int bars = (2 * kGrpStagesMax + 4) * 8 + 16;
     for (int xb = 2; xb >= 1; --xb) {
         const int avail = budget - xb * xbytes - red - bars;
@@ -85,7 +85,7 @@ inline bool grp_plan(GroupPlan &p, int NB, int budget) {
             p.off_bar = p.off_red + red;
             p.smem = p.off_bar + bars;
             // warps per strip: keep about half of the slots in flight
-            const int nsteps = p.KB / 64;
+            const int nsteps = (p.KB + 63) / 64;
             int teams = st / 2 < 1 ? 1 : st / 2;
             if (teams > kGrpConsumerWarps) teams = kGrpConsumerWarps;
             int ks = (kGrpConsumerWarps + teams - 1) / teams;
@@ -101,21 +101,41 @@ inline bool grp_plan(GroupPlan &p, int NB, int budget) {
 }
 
 // Partial sums of one warp over the column steps j, j + ks, ... of a strip in
-// shared memory (rows at stride RS; x_q chunks transposed and swizzled).
+// shared memory (rows at stride RS; x_q chunks transposed and swizzled).  The
+// next step's weight words and the current step's x chunks are loaded before
+// the current step's MMAs, so the loads' latency overlaps the arithmetic.
 template <int NB, int CH, bool CONV>
 __device__ __forceinline__ void strip_mma_smem(int (&d)[CH][NB][4], uint32_t w_s, int RS, uint32_t x_s, int XS,
                                                int M, int KB, int j0, int ks, int lane, int enc) {
     const int g = lane >> 2, t = lane & 3;
-    const int nsteps = KB >> 6;
+    // the last 64-byte step may be partial (K % 256 != 0): past the row the
+    // weight words are padding and the x chunks are taken as 0, so they add nothing
+    const int nsteps = (KB + 63) >> 6;
     const uint32_t xsw = (uint32_t)(t & 2) << 4;
 #pragma unroll
     for (int i = 0; i < CH; ++i)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) d[i][nb][0] = d[i][nb][1] = d[i][nb][2] = d[i][nb][3] = 0;
+    if (j0 >= nsteps) return;
     const uint32_t ra = w_s + (uint32_t)(g * RS + t * 16), rb = ra + (uint32_t)(8 * RS);
+    uint4 wa = lds128(ra + (uint32_t)(j0 * 64)), wb = lds128(rb + (uint32_t)(j0 * 64));
     for (int step = j0; step < nsteps; step += ks) {
         const int bo = step * 64 + t * 16;
-        const uint4 wa = lds128(ra + (uint32_t)(step * 64)), wb = lds128(rb + (uint32_t)(step * 64));
+        uint4 xt[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            const int m = g + 8 * nb;
+            const bool ok = m < M && bo < KB;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                xt[nb][i] = ok ? lds128(x_s + (uint32_t)(m * XS + 4 * bo) + ((uint32_t)(i << 4) ^ xsw))
+                               : make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint4 na = wa, nbw = wb;
+        if (step + ks < nsteps) {
+            na = lds128(ra + (uint32_t)((step + ks) * 64));
+            nbw = lds128(rb + (uint32_t)((step + ks) * 64));
+        }
         const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w};
         const uint32_t b4[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
@@ -130,13 +150,12 @@ __device__ __forceinline__ void strip_mma_smem(int (&d)[CH][NB][4], uint32_t w_s
             }
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                const int m = g + 8 * nb;
-                uint4 xt = make_uint4(0u, 0u, 0u, 0u);
-                if (m < M) xt = lds128(x_s + (uint32_t)(m * XS + 4 * bo) + ((uint32_t)(i << 4) ^ xsw));
-                mma_16x8x32_u8s8(d[i % CH][nb], ua[0], ub[0], ua[1], ub[1], xt.x, xt.y);
-                mma_16x8x32_u8s8(d[i % CH][nb], ua[2], ub[2], ua[3], ub[3], xt.z, xt.w);
+                mma_16x8x32_u8s8(d[i % CH][nb], ua[0], ub[0], ua[1], ub[1], xt[nb][i].x, xt[nb][i].y);
+                mma_16x8x32_u8s8(d[i % CH][nb], ua[2], ub[2], ua[3], ub[3], xt[nb][i].z, xt[nb][i].w);
             }
         }
+        wa = na;
+        wb = nbw;
     }
 }
 
@@ -158,7 +177,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
     auto empty = [&](int s) { return bar0 + 8u * (uint32_t)(kGrpStagesMax + s); };
     auto xfull = [&](int b) { return bar0 + 8u * (uint32_t)(2 * kGrpStagesMax + b); };
     auto xempty = [&](int b) { return bar0 + 8u * (uint32_t)(2 * kGrpStagesMax + 2 + b); };
-    const uint32_t stage_bytes = 16u * (uint32_t)RS;
+    const uint32_t stage_bytes = 16u * (uint32_t)RS + kGammaSlot;
     auto stage_addr = [&](int s) { return sbase + (uint32_t)s * stage_bytes; };
     auto xbuf_addr = [&](int b) { return sbase + (uint32_t)pl.off_x + (uint32_t)(b * M * XS); };
 
@@ -192,12 +211,6 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         *abrt = 1;
         return false;
     };
-    auto wait_sleep = [&](uint32_t bar, uint32_t par) {
-        if (*abrt) return false;
-        if (mbar_wait_sleep(bar, par)) return true;
-        *abrt = 1;
-        return false;
-    };
 
     if (warp == kGrpConsumerWarps) {
         // ---------------- producer ----------------
@@ -207,7 +220,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
                 const int b = pi & 1;
                 if (pl.xbufs == 1 || pi >= 2) {  // buffer b last held problem pi - xbufs
                     const int prev = pi - pl.xbufs;
-                    if (prev >= 0 && !wait_sleep(xempty(pl.xbufs == 1 ? 0 : b), (uint32_t)((prev / pl.xbufs) & 1)))
+                    if (prev >= 0 && !wait_spin(xempty(pl.xbufs == 1 ? 0 : b), (uint32_t)((prev / pl.xbufs) & 1)))
                         return false;
                 }
                 const int bb = pl.xbufs == 1 ? 0 : b;
@@ -220,14 +233,14 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
             };
             auto issue_w = [&](int i) {
                 const int s = i % S;
-                if (i >= S && !wait_sleep(empty(s), (uint32_t)(((i / S) - 1) & 1))) return false;
+                if (i >= S && !wait_spin(empty(s), (uint32_t)(((i / S) - 1) & 1))) return false;
                 const int64_t t = s0 + i, p = t / pl.spp, ls = t - p * pl.spp;
                 const int64_t r0 = ls * 16;
                 const int rows = (int)(pl.N - r0 < 16 ? pl.N - r0 : 16);
-                const uint8_t *src = tab.packed[p] + r0 * KB;
-                mbar_arrive_expect_tx(full(s), (uint32_t)(rows * KB));
-                for (int r = 0; r < rows; ++r)
-                    bulk_g2s(stage_addr(s) + (uint32_t)(r * RS), src + (int64_t)r * KB, (uint32_t)KB, full(s));
+                const bool gslot = pl.per_row && rows == 16;  // 64 gamma bytes, 16-byte aligned
+                mbar_arrive_expect_tx(full(s), (uint32_t)(rows * KB) + (gslot ? kGammaSlot : 0u));
+                bulk_g2s(stage_addr(s), tab.packed[p] + r0 * KB, (uint32_t)(rows * KB), full(s));
+                if (gslot) bulk_g2s(stage_addr(s) + 16u * (uint32_t)RS, tab.gamma[p] + r0, kGammaSlot, full(s));
                 return true;
             };
             int issued = 0;
@@ -267,21 +280,51 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
     // ---------------- consumers ----------------
     pdl_wait();  // s_x, rowsum (and y) belong to work before this kernel
     const int team = warp / ks, kw = warp % ks;
-    int *red = reinterpret_cast<int *>(dsm + pl.off_red);  // [2][8 warps][4 NB][32]
+    int *red = reinterpret_cast<int *>(dsm + pl.off_red);  // [2][consumer warps][4 NB][32]
     int par = 0;
     int i = team;
     for (int pi = 0; pi < np; ++pi) {
         const int bb = pl.xbufs == 1 ? 0 : (pi & 1);
         const int64_t p = p_first + pi;
-        const bool xok = !*abrt && warp_wait(xfull(bb), (uint32_t)((pi / pl.xbufs) & 1), lane);
+        const bool xok = !*abrt && warp_wait_sleep(xfull(bb), (uint32_t)((pi / pl.xbufs) & 1), lane);
         if (!xok && lane == 0) *abrt = 1;
         const uint32_t x_s = xbuf_addr(bb);
         const float *sx_p = s_x + (pl.x_shared ? 0 : p) * (int64_t)M;
         const int32_t *rs_p = rowsum + (pl.x_shared ? 0 : p) * (int64_t)M;
         const float *gam = tab.gamma[p];
+        const int g = lane >> 2, tt = lane & 3;
+        const float g_tensor = pl.per_row ? 0.0f : __ldg(gam);
+        // the finishing lanes' token scales and offsets: tokens 8 nb + 2 tt + e
+        float sxv[NB][2];
+        int rsv[NB][2];
+        if (kw == 0)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int m = 8 * nb + 2 * tt + e;
+                    sxv[nb][e] = m < M ? __ldcg(sx_p + m) : 0.0f;
+                    rsv[nb][e] = m < M ? __ldcg(rs_p + m) : 0;
+                }
         for (; i < nloc && (s0 + i) / pl.spp == p; i += T) {
             const int s = i % S;
-            const bool ok = !*abrt && warp_wait(full(s), (uint32_t)((i / S) & 1), lane);
+            const int64_t ls = s0 + i - p * pl.spp;
+            const bool ok = !*abrt && warp_wait_sleep(full(s), (uint32_t)((i / S) & 1), lane);
+            // gamma of rows g and g + 8: from the slot (full strips, per row), else from memory
+            float gv[2] = {g_tensor, g_tensor};
+            if (kw == 0 && pl.per_row) {
+                if (ls * 16 + 16 <= pl.N) {
+                    const float *gs = reinterpret_cast<const float *>(dsm + (size_t)s * stage_bytes + 16 * RS);
+                    gv[0] = gs[g];
+                    gv[1] = gs[g + 8];
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int64_t n = ls * 16 + g + 8 * h;
+                        gv[h] = n < pl.N ? __ldg(gam + n) : 0.0f;
+                    }
+                }
+            }
             if (!ok && lane == 0) *abrt = 1;
             int d[CH][NB][4];
             if (ok && !*abrt)
@@ -317,21 +360,18 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
                 par ^= 1;
             }
             if (kw == 0 && !*abrt) {
-                // fragment c of lane (g, t): row g (+8 for c >= 2), token 8 nb + 2 t + (c & 1)
-                const int64_t t = s0 + i, ls = t - p * pl.spp;
-                const int g = lane >> 2, tt = lane & 3;
+                // fragment c of lane (g, tt): row g (+8 for c >= 2), token 8 nb + 2 tt + (c & 1)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int64_t n = ls * 16 + g + ((c & 2) ? 8 : 0);
                     if (n >= pl.N) continue;
-                    const float gv = __ldg(gam + (pl.per_row ? n : 0));
 #pragma unroll
                     for (int nb = 0; nb < NB; ++nb) {
                         const int m = 8 * nb + 2 * tt + (c & 1);
                         if (m < M) {
-                            const int a = acc[nb][c] - __ldcg(rs_p + m);
+                            const int a = acc[nb][c] - rsv[nb][c & 1];
                             y[(p * M + m) * pl.N + n] =
-                                __fmul_rn(__int2float_rn(a), __fmul_rn(gv, __ldcg(sx_p + m)));
+                                __fmul_rn(__int2float_rn(a), __fmul_rn(gv[c >> 1], sxv[nb][c & 1]));
                         }
                     }
                 }

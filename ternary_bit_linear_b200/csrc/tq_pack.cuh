@@ -16,7 +16,8 @@
 // Codes come from one fp32 threshold per gamma (code_threshold), equivalent to
 // rounding the fp32 quotient w / gamma and clamping, without a divide; or, for
 // the threshold rule (Foundry "Absmean Thresholding", BitRASP ternarize_weight),
-// from w > fp32(ratio * gamma) (pack_threshold).
+// from w > fp32(ratio * gamma) (pack_threshold); or, for Foundry's manual
+// threshold (fq_quantize_ternary_threshold), from w > t with gamma = t.
 //
 // HBM traffic: read 4 B and write 0.25 B per weight.  Per-row gamma is one
 // pass; per-tensor gamma reads W twice (reduction, then packing walking the
@@ -180,6 +181,17 @@ __device__ __noinline__ float per_tensor_threshold(const double *__restrict__ pa
     return pack_threshold(g, ratio);
 }
 
+// Foundry's manual threshold: gamma is the caller's threshold t (CTA 0 writes
+// it), and a weight is +1 iff w > t, i.e. w >= the next float above t.
+__device__ __forceinline__ float fixed_threshold(float t, float *__restrict__ gamma) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) gamma[0] = t;
+    return nextafterf(t, __int_as_float(0x7f800000));
+}
+
+// Options word of the pack kernels: bit 0 inputs ready, bits 1-2 the packed-code
+// layout, bit 3 a fixed scale (the manual threshold, passed in `ratio`).
+constexpr int kPackOptFixed = 8;
+
 // No block-level synchronisation: warps are independent.
 // ---------------------------------------------------------------------------
 constexpr int kPackUnroll = 8;
@@ -190,15 +202,18 @@ __global__ void __launch_bounds__(kPackThreads)
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
                      int opts, float ratio) {
-    const int ready = opts & 1, enc = opts >> 1;  // inputs ready; packed-code layout
+    const int ready = opts & 1, enc = (opts >> 1) & 3;  // inputs ready; packed-code layout
+    const bool fixed = (opts & kPackOptFixed) != 0;
     if (!ready) pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * kPackWarps;
     const int nv = K >> 2;
-    const bool per_tensor = partial != nullptr;
+    const bool per_tensor = partial != nullptr || fixed;
     const float t_tensor =
-        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma, ratio) : 0.0f;
+        fixed ? fixed_threshold(ratio, gamma)
+              : per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma, ratio)
+                           : 0.0f;
     // per-lane chain length (float4) of pass 1, for the error bound
     const int chain = (nv + 31) / 32;
     const double eps = sum_error_bound(4 * chain + 5);
@@ -294,7 +309,8 @@ __global__ void __launch_bounds__(kPackThreads, 2)
                      uint8_t *__restrict__ packed, float *__restrict__ gamma,
                      const double *__restrict__ partial, int nparts, int height, int reverse,
                      int opts, float ratio) {
-    const int ready = opts & 1, enc = opts >> 1;  // inputs ready; packed-code layout
+    const int ready = opts & 1, enc = (opts >> 1) & 3;  // inputs ready; packed-code layout
+    const bool fixed = (opts & kPackOptFixed) != 0;
     constexpr int TEAMS = kPackWarps / T;
     extern __shared__ __align__(16) float4 rowbuf[];  // [TEAMS][kPackRing][nv]
     __shared__ uint64_t rbar[TEAMS][kPackRing];
@@ -330,9 +346,11 @@ __global__ void __launch_bounds__(kPackThreads, 2)
     if (leader)
         for (int64_t k = 0; k < issued; ++k) issue(k);
     // the first rows are in flight: now the per-tensor threshold (if any)
-    const bool per_tensor = partial != nullptr;
+    const bool per_tensor = partial != nullptr || fixed;
     const float t_tensor =
-        per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma, ratio) : 0.0f;
+        fixed ? fixed_threshold(ratio, gamma)
+              : per_tensor ? per_tensor_threshold(partial, nparts, height, w, (int64_t)nv * N, SAN, gamma, ratio)
+                           : 0.0f;
     const double eps = sum_error_bound(4 * kTeamVec + 5 + T);
     int parity = 0;
     int64_t k = 0;

@@ -2,6 +2,7 @@
 self-contained command that ncu captures are taken on.
 
     python -m ternary_bit_linear_b200.profile_case --kernel gemv --M 8 --N 4096 --K 4096 --reps 3 [--ready]
+    python -m ternary_bit_linear_b200.profile_case --kernel grouped --G 64 --M 8 --N 4096 --K 4096 --reps 3
 
 Training kernels: bwd (input gradient, dY [M][N] against the packed [N][K]),
 ste and flip (latent weights / gradient [N][K]).
@@ -22,7 +23,9 @@ import ternary_bit_linear_b200 as tq
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", required=True,
-                    choices=["pack_row", "pack_tensor", "act", "fwht", "gemv", "gemm", "fused", "bwd", "ste", "flip"])
+                    choices=["pack_row", "pack_tensor", "act", "fwht", "gemv", "gemm", "grouped", "fused", "bwd", "ste",
+                             "flip"])
+    ap.add_argument("--G", type=int, default=8, help="layers per grouped call")
     ap.add_argument("--M", type=int, default=8)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -45,6 +48,13 @@ def main():
                      dtype=torch.uint8, device=dev)
     pws = torch.empty((max(16, tq.pack_workspace_bytes(N, K, flags)),), dtype=torch.uint8, device=dev)
     Xr = torch.empty_like(X)
+    if a.kernel == "grouped":  # G distinct packed copies of the layer, one activation batch per layer
+        Pg = [packed.clone() for _ in range(a.G)]
+        Gg = [gamma.clone() for _ in range(a.G)]
+        Xg = X.unsqueeze(0).expand(a.G, M, K).contiguous()
+        Yg = torch.empty((a.G, M, N), device=dev)
+        gfl = flags | tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY
+        gws = torch.empty((tq.grouped_workspace_bytes(a.G, M, K, gfl),), dtype=torch.uint8, device=dev)
     if a.kernel in ("bwd", "ste", "flip"):
         dY = torch.randn((M, N), generator=g, device=dev)
         dX = torch.empty((M, K), device=dev)
@@ -63,6 +73,8 @@ def main():
         elif a.kernel in ("gemv", "gemm"):
             ready = tq.FLAG_WEIGHTS_STATIC | tq.FLAG_INPUTS_READY if a.ready else 0
             tq.ternary_gemm_(xq, sx, rs, packed, gamma, flags | ready, y)
+        elif a.kernel == "grouped":
+            tq.bitlinear_grouped_(Xg, Pg, Gg, gfl, Yg, gws)
         elif a.kernel == "bwd":
             tq.ternary_backward_input_(dY, packed, gamma, flags, dX, bws)
         elif a.kernel == "ste":

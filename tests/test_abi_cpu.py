@@ -141,6 +141,31 @@ def test_grouped_validation(lib):
     assert call(packed=ctypes.cast(odd, ctypes.c_void_p)) == 3  # a misaligned entry
 
 
+def test_pack_abs_threshold_validation(lib):
+    f = lib.tq_quantize_ternary_pack_abs_threshold
+    ok = [P(), 4, 64, 0, 0.05, P(1 << 20), P(2 << 20), None]
+    for bad_t in (-0.01, float("nan"), float("inf")):
+        a = list(ok)
+        a[4] = bad_t
+        assert f(*a) == 4, bad_t
+    for flags, code in ((tq.GAMMA_PER_ROW, 4), (1 << 9, 4), (3 << 7, 4)):
+        a = list(ok)
+        a[3] = flags
+        assert f(*a) == code, flags
+    a = list(ok)
+    a[0] = None
+    assert f(*a) == 1
+    a = list(ok)
+    a[2] = 100
+    assert f(*a) == 2
+    a = list(ok)
+    a[6] = P(4)
+    assert f(*a) == 3
+    a = list(ok)
+    a[5] = P(16)  # packed overlaps w
+    assert f(*a) == 4
+
+
 def test_pack_threshold_validation(lib):
     f = lib.tq_quantize_ternary_pack_threshold
     ok = [P(), 4, 64, 1, 0.55, P(1 << 20), P(2 << 20), None, 0, None]

@@ -100,6 +100,36 @@ def test_pack_exact_ties():
     assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
 
 
+@pytest.mark.parametrize("N,K", [(1, 64), (17, 512), (129, 4160), (64, 8192), (5, 8256), (2, 65536)])
+@pytest.mark.parametrize("t", [0.05, 0.0, 0.02])
+def test_pack_abs_threshold_matches_oracle(cuda_lib, N, K, t):
+    """Foundry's manual threshold: bytes and the stored scale bit-exact, in both
+    pack kernels (K <= 8192 team kernel, larger K the row kernel)."""
+    tq = cuda_lib
+    W = S.laplace((N, K), 0.03, 8, 300 + N)
+    if N > 2:  # weights exactly at +-t and one float beyond
+        W[1, :4] = [t, -t, np.nextafter(np.float32(t), np.float32(1)), -np.nextafter(np.float32(t), np.float32(1))]
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty((1,), dtype=torch.float32, device="cuda")
+    tq.quantize_ternary_pack_abs_threshold_(dev(W), 0, t, packed, gamma)
+    p_ref, g_ref = oracle.quantize_pack_abs_threshold(W, t)
+    assert np.array_equal(host(gamma), g_ref)
+    assert np.array_equal(host(packed), p_ref)
+
+
+@pytest.mark.parametrize("enc", [1, 2])
+def test_pack_abs_threshold_layouts_and_sanitize(cuda_lib, enc):
+    tq = cuda_lib
+    W = S.normal((40, 1024), 0.02, 9, 41)
+    W[0, 0], W[3, 5], W[7, 9] = np.nan, np.inf, -np.inf
+    packed = torch.empty((40, 256), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty((1,), dtype=torch.float32, device="cuda")
+    tq.quantize_ternary_pack_abs_threshold_(dev(W), tq.FLAG_SANITIZE_NONFINITE | (enc << 7), 0.01, packed, gamma)
+    p_ref, g_ref = oracle.quantize_pack_abs_threshold(W, 0.01, sanitize=True, encoding=enc)
+    assert np.array_equal(host(gamma), g_ref) and np.array_equal(host(packed), p_ref)
+    assert tq.device_status() == 0
+
+
 def test_pack_dense_threshold_sweep(cuda_lib):
     # Row r: one probe value w_r followed by 63 entries of +-1.  Its gamma is
     # (|w_r| + 63) / 64, and w_r / gamma crosses 0.5 at w_r = 63/127.  4096
