@@ -495,6 +495,19 @@ TQ_API tq_status tq_ternary_stochastic_flip(uint8_t *packed, const float *grad, 
 TQ_API void tq_seed(uint64_t *state, uint64_t seed);
 
 /*
+ * Self-test of the failure-detection path (no counterpart on the pages).  One
+ * warp of a one-CTA kernel waits on a shared-memory mbarrier that nothing ever
+ * completes, through the same bounded wait every kernel of the library uses
+ * (spinning, or with sleeping = 1 the suspending form), gives up after
+ * limit_ns nanoseconds of %globaltimer, records TQ_ERR_TIMEOUT in the
+ * per-device status word and exits normally -- the context stays usable.  The
+ * next tq_get_device_status() returns TQ_ERR_TIMEOUT and clears the word.
+ *   limit_ns  in [1000, 1e9] (1 us .. 1 s), else TQ_ERR_ARG.
+ *   sleeping  0 or 1, else TQ_ERR_ARG.
+ */
+TQ_API tq_status tq_selftest_wait_timeout(uint64_t limit_ns, int sleeping, tq_stream_t stream);
+
+/*
  * Waits for `stream`, then returns and clears the current device's status word:
  * TQ_OK, or TQ_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the
  * last call.  TQ_ERR_CUDA if the synchronisation itself failed.

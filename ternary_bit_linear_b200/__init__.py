@@ -62,6 +62,7 @@ SIGNATURES = {
     "tq_ternary_stochastic_flip": (_I, [_P, _P, _I64, _I64, _F, ctypes.POINTER(ctypes.c_uint64), _U, _P]),
     "tq_seed": (None, [ctypes.POINTER(ctypes.c_uint64), ctypes.c_uint64]),
     "tq_get_device_status": (_I, [_P]),
+    "tq_selftest_wait_timeout": (_I, [ctypes.c_uint64, _I, _P]),
     "tq_status_string": (ctypes.c_char_p, [_I]),
     "tq_version": (_I, []),
 }
@@ -392,6 +393,13 @@ def ternary_stochastic_flip_(packed, grad, temperature, state: int, flags=0, str
 def device_status(stream=None) -> int:
     """Synchronises the stream; returns and clears the device status word."""
     return load().tq_get_device_status(_stream(stream))
+
+
+def selftest_wait_timeout(limit_ns: int, sleeping: bool = False, stream=None):
+    """Launch the bounded-wait self-test (a wait that nothing completes, given
+    up after limit_ns); the next device_status() reports TQ_ERR_TIMEOUT."""
+    _check("tq_selftest_wait_timeout",
+           load().tq_selftest_wait_timeout(int(limit_ns), int(bool(sleeping)), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

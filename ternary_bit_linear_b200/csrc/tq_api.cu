@@ -549,14 +549,21 @@ inline size_t grouped_parts(int64_t Gx, int64_t M, int64_t K, size_t off[3]) {
     return off[2] + al((size_t)(Gx * M) * 4);
 }
 
+template <int NB, int ENC, bool FULL>
+tq_status launch_group_gemv_k(const GroupTable &tab, const GroupPlan &pl, const int8_t *xq, const float *sx,
+                              const int32_t *rs, float *y, int sms, cudaStream_t st) {
+    static std::atomic<int> done[kMaxDevices];
+    if (tq_status e = set_smem_once(tq_gemv_group_kernel<NB, ENC, FULL>, kGroupSmemBudget, done)) return e;
+    const int64_t grid = pl.nstrips < sms ? pl.nstrips : sms;
+    return launch_pdl(tq_gemv_group_kernel<NB, ENC, FULL>, dim3((unsigned)grid), dim3(kGrpThreads), (size_t)pl.smem,
+                      st, tab, pl, xq, sx, rs, y);
+}
+
 template <int NB, int ENC>
 tq_status launch_group_gemv(const GroupTable &tab, const GroupPlan &pl, const int8_t *xq, const float *sx,
                             const int32_t *rs, float *y, int sms, cudaStream_t st) {
-    static std::atomic<int> done[kMaxDevices];
-    if (tq_status e = set_smem_once(tq_gemv_group_kernel<NB, ENC>, kGroupSmemBudget, done)) return e;
-    const int64_t grid = pl.nstrips < sms ? pl.nstrips : sms;
-    return launch_pdl(tq_gemv_group_kernel<NB, ENC>, dim3((unsigned)grid), dim3(kGrpThreads), (size_t)pl.smem,
-                      st, tab, pl, xq, sx, rs, y);
+    return pl.K % 256 == 0 ? launch_group_gemv_k<NB, ENC, true>(tab, pl, xq, sx, rs, y, sms, st)
+                           : launch_group_gemv_k<NB, ENC, false>(tab, pl, xq, sx, rs, y, sms, st);
 }
 
 template <int NB>
@@ -1140,6 +1147,14 @@ tq_status tq_bitlinear_grouped(const float *x, int64_t G, const uint8_t *const *
                               : launch_group_gemv_enc<2>(tab, pl, xq, sx, rs, y, sms, st))
         return e;
     return launch_status();
+}
+
+tq_status tq_selftest_wait_timeout(uint64_t limit_ns, int sleeping, tq_stream_t stream) {
+    if (limit_ns < 1000 || limit_ns > 1000000000ull) return TQ_ERR_ARG;
+    if (sleeping != 0 && sleeping != 1) return TQ_ERR_ARG;
+    if (tq_status e = check_device(nullptr)) return e;
+    return launch_pdl(tq_selftest_wait_kernel, dim3(1), dim3(32), 0, cs(stream), (unsigned long long)limit_ns,
+                      sleeping);
 }
 
 tq_status tq_get_device_status(tq_stream_t stream) {

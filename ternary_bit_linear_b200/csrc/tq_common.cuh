@@ -113,13 +113,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // form is for waits on a kernel's critical path; the sleeping form for warps
 // that wait long while others on the SM do the work.
 template <bool SLEEP>
-__device__ __forceinline__ bool mbar_wait_t(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_t(uint32_t bar, uint32_t parity,
+                                            unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < (SLEEP ? 8 : 64); ++i)
             if (SLEEP ? mbar_try_wait_sleep(bar, parity) : mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             flag_timeout();
             return false;
         }
@@ -143,6 +144,22 @@ __device__ __forceinline__ bool warp_wait_sleep(uint32_t bar, uint32_t parity, i
     int ok = 0;
     if (lane == 0) ok = mbar_wait_sleep(bar, parity) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Self-test of the bounded wait: one warp waits (as the kernels' waits do, with
+// the given limit) on an mbarrier that nothing ever completes, gives up, and
+// records the timeout in the status word.  Touches no memory but its own
+// shared mbarrier; exits normally.
+__global__ void __launch_bounds__(32) tq_selftest_wait_kernel(unsigned long long limit_ns, int sleeping) {
+    __shared__ uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncwarp();
+    int ok = 1;
+    if (threadIdx.x == 0) ok = (sleeping ? mbar_wait_t<true>(b, 0, limit_ns) : mbar_wait_t<false>(b, 0, limit_ns)) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    (void)ok;
 }
 
 // Generic-proxy writes to shared memory become visible to the async proxy

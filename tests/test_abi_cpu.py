@@ -166,6 +166,13 @@ def test_pack_abs_threshold_validation(lib):
     assert f(*a) == 4
 
 
+def test_selftest_wait_validation(lib):
+    f = lib.tq_selftest_wait_timeout
+    assert f(999, 0, None) == 4            # below 1 us
+    assert f(10 ** 9 + 1, 0, None) == 4    # above 1 s
+    assert f(10 ** 6, 2, None) == 4       # sleeping must be 0 or 1
+
+
 def test_pack_threshold_validation(lib):
     f = lib.tq_quantize_ternary_pack_threshold
     ok = [P(), 4, 64, 1, 0.55, P(1 << 20), P(2 << 20), None, 0, None]
