@@ -263,11 +263,15 @@ class Workload:
         self.gamma = [torch.empty((N if self.per_row else 1,), dtype=f32, device=dev) for _ in range(L)]
         nws = tq.pack_workspace_bytes(N, K, self.flags)
         self.pack_ws = [torch.empty((max(nws, 16),), dtype=u8, device=dev) for _ in range(L)]
-        self.Xd = {M: [x.to(dev) for _ in range(L)] for M, x in self.X.items()}
+        # every layer's activations and outputs in one contiguous [L][M][.] buffer per batch size
+        # (each layer uses its own slice): the end-to-end run copies them in and out in one piece
+        self.Xall = {M: x.unsqueeze(0).expand(L, *x.shape).contiguous().to(dev) for M, x in self.X.items()}
+        self.Yall = {M: torch.empty((L, M, N), dtype=f32, device=dev) for M in self.Ms}
+        self.Xd = {M: [self.Xall[M][l] for l in range(L)] for M in self.Ms}
+        self.y = {M: [self.Yall[M][l] for l in range(L)] for M in self.Ms}
         self.xq = {M: [torch.empty((M, K), dtype=i8, device=dev) for _ in range(L)] for M in self.Ms}
         self.sx = {M: [torch.empty((M,), dtype=f32, device=dev) for _ in range(L)] for M in self.Ms}
         self.rs = {M: [torch.empty((M,), dtype=i32, device=dev) for _ in range(L)] for M in self.Ms}
-        self.y = {M: [torch.empty((M, N), dtype=f32, device=dev) for _ in range(L)] for M in self.Ms}
 
         # packing: once per weight (aux, outside the step)
         pack_bytes = 4 * N * K + N * K // 4 + 4 * (N if self.per_row else 1)
@@ -300,7 +304,9 @@ class Workload:
             work = (N * K // 4 + 4 * N * (1 if self.per_row else 0) + M * K + 8 * M + 4 * M * N) if gemv \
                 else 2 * M * N * K
             if gemv and group > 1:
-                self._grouped_gemv(M, act_bytes, work)
+                self._grouped_gemv(M, act_bytes, work, group, True)
+                if group < L and L <= 64:  # the whole ring in one call, for comparison
+                    self._grouped_gemv(M, act_bytes, work, L, False)
             else:
                 self.segs.append(Seg("act M=%d" % M, "act_quant", L, L * act_bytes, L, [
                     lambda M=M, l=l: tq.quantize_act_int8_(self.Xd[M][l], tq.FLAG_INPUTS_READY, 0.05, 40.0,
@@ -324,26 +330,27 @@ class Workload:
                                               self.gamma[l], flags, self.y[M][l])
                 for l in range(self.L)]
 
-    def _grouped_gemv(self, M, act_bytes, work):
+    def _grouped_gemv(self, M, act_bytes, work, G, in_step):
         """Groups of G consecutive ring layers, each with its own activation
-        batch: one call (activation pass + GEMV launch) per group."""
-        tq, torch, G, L, K, N = self.tq, self.torch, self.group, self.L, self.K, self.N
+        batch: one call (activation pass + GEMV launch) per group.  Work per
+        layer: the packed weights, gamma, the fp32 activations read and the
+        outputs written, plus the x_q, s_x and rowsum the activation pass
+        writes and the GEMV reads."""
+        tq, torch, L, K, N = self.tq, self.torch, self.L, self.K, self.N
         assert L % G == 0
         ng = L // G
-        # per group: x [G][M][K] contiguous, y [G][M][N], workspace for the G x_q batches
-        self.gx = self.__dict__.setdefault("gx", {})
-        self.gy = self.__dict__.setdefault("gy", {})
-        self.gws = self.__dict__.setdefault("gws", {})
-        x1 = self.X[M]
-        self.gx[M] = [x1.unsqueeze(0).expand(G, M, K).contiguous().to(self.dev) for _ in range(ng)]
-        self.gy[M] = [torch.empty((G, M, N), dtype=torch.float32, device=self.dev) for _ in range(ng)]
+        # per group: contiguous slices x [G][M][K] and y [G][M][N] of the ring's buffers
+        gx = [self.Xall[M][g * G:(g + 1) * G] for g in range(ng)]
+        gy = [self.Yall[M][g * G:(g + 1) * G] for g in range(ng)]
         wsz = tq.grouped_workspace_bytes(G, M, K, 0)
-        self.gws[M] = [torch.empty((max(wsz, 16),), dtype=torch.uint8, device=self.dev) for _ in range(ng)]
+        gws = [torch.empty((max(wsz, 16),), dtype=torch.uint8, device=self.dev) for _ in range(ng)]
+        self.__dict__.setdefault("keep", []).append((gx, gy, gws))
         fl = self.ready_flags
-        fns = [lambda g=g: tq.bitlinear_grouped_(self.gx[M][g], self.packed[g * G:(g + 1) * G],
-                                                 self.gamma[g * G:(g + 1) * G], fl, self.gy[M][g], self.gws[M][g])
+        fns = [lambda g=g: tq.bitlinear_grouped_(gx[g], self.packed[g * G:(g + 1) * G], self.gamma[g * G:(g + 1) * G],
+                                                 fl, gy[g], gws[g])
                for g in range(ng)]
-        self.segs.append(Seg("gemv M=%d grouped x%d" % (M, G), "gemv", L, L * (work + act_bytes), 2 * ng, fns))
+        self.segs.append(Seg("gemv M=%d grouped x%d" % (M, G), "gemv", L, L * (work + act_bytes), 2 * ng, fns,
+                             in_step=in_step))
 
     def _build_pack(self, S, layers):
         """Quantise + pack as the step: the 8192^2 sweep weight per row and the
@@ -548,9 +555,11 @@ def roofline_of(wl, seg, kernels, pk):
     if k["bound"] == "hbm":
         r["peak_source"] = pk["source"] + " hbm_gbs (copy, burst)"
         if seg.kname == "gemv":
-            r["algorithmic_bytes"] = ("per layer: packed N*K/4 + gamma 4N + x_q M*K + s_x, rowsum 8M + y 4MN"
-                                      + (" + the fp32 activations 4MK and the x_q written by the activation pass"
-                                         if "grouped" in seg.label else ""))
+            r["algorithmic_bytes"] = (
+                "per layer of the grouped call (activation pass + GEMV): packed N*K/4 + gamma 4N + fp32 "
+                "activations 4MK + x_q written and read 2MK + s_x, rowsum written and read 16M + y 4MN"
+                if "grouped" in seg.label else
+                "per layer: packed N*K/4 + gamma 4N + x_q M*K + s_x, rowsum 8M + y 4MN")
     elif seg.kname == "bwd":
         r["peak_source"] = pk["source"] + " bf16_tflops (fp16 operands)"
     else:
@@ -688,9 +697,9 @@ def run_e2e(args, wl, torch, stream, graphs, world):
     the step's outputs copied back inside the timed region."""
     ins, outs = [], []
     for M in wl.Ms:
-        if getattr(wl, "gx", {}).get(M) is not None:
-            ins += wl.gx[M]
-            outs += wl.gy[M]
+        if getattr(wl, "Xall", None) is not None:
+            ins.append(wl.Xall[M])
+            outs.append(wl.Yall[M])
         else:
             ins += wl.Xd[M]
             outs += wl.y[M]
@@ -974,7 +983,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="metric", choices=["metric"] + list(WORKLOAD_SHAPES))
-    ap.add_argument("--decode-group", type=int, default=1,
+    ap.add_argument("--decode-group", type=int, default=8,
                     help="decode GEMVs as grouped calls of G same-shape layers (1: one call per layer)")
     ap.add_argument("--bias", action="store_true",
                     help="contractions through tq_ternary_gemm_ex with a bias (the extra epilogue)")

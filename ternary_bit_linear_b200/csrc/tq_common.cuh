@@ -340,6 +340,17 @@ __device__ __forceinline__ uint4 transpose_bytes4x4(uint4 q) {
 // of a quarter warp (two rows, four column offsets) hit distinct banks.
 __host__ __device__ __forceinline__ int gemv_chunk_pos(int c) { return c ^ (((c >> 3) & 1) << 1); }
 
+// The same MMA as a plain (non-volatile) asm: a pure function of its register
+// operands, so the compiler may schedule it among independent work (used where
+// the operands come from registers only).
+__device__ __forceinline__ void mma_16x8x32_u8s8_pure(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                       uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // ---------------------------------------------------------------------------
 // Double-double accumulation of non-negative terms, and the correctly
 // rounded fp32 mean derived from it.

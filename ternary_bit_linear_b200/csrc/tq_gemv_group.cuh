@@ -188,7 +188,7 @@ __device__ __forceinline__ void strip_mma_fields(int (&d)[4][NB][4], uint32_t w_
                     const uint4 &u = xt[nb][2 * pr], &v = xt[nb][2 * pr + 1];
                     const uint32_t x0 = j == 0 ? u.x : j == 1 ? u.y : j == 2 ? u.z : u.w;
                     const uint32_t x1 = j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
-                    mma_16x8x32_u8s8(d[j][nb], a0, a1, a2, a3, x0, x1);
+                    mma_16x8x32_u8s8_pure(d[j][nb], a0, a1, a2, a3, x0, x1);
                 }
             }
         wa = na;
