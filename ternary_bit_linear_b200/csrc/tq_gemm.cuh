@@ -254,14 +254,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!warp_wait_sleep(w_full(ws), (g / SW) & 1, lane)) break;
             uint4 p0, p1;
             const uint32_t src = w_row + (uint32_t)(ws * kWStageBytes);
+            // Rows are 32 bytes apart, so rows r and r + 4 share banks: threads
+            // with (r >> 2) odd read their second half first, which makes each
+            // quarter warp's 16-byte loads hit eight distinct bank groups.
+            const uint32_t h = (uint32_t)((r >> 2) & 1) << 4;
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                          : "=r"(p0.x), "=r"(p0.y), "=r"(p0.z), "=r"(p0.w)
-                         : "r"(src)
+                         : "r"(src + h)
                          : "memory");
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                          : "=r"(p1.x), "=r"(p1.y), "=r"(p1.z), "=r"(p1.w)
-                         : "r"(src + 16u)
+                         : "r"(src + (h ^ 16u))
                          : "memory");
+            if (h) {  // back to natural order
+                const uint4 tmp = p0;
+                p0 = p1;
+                p1 = tmp;
+            }
             uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
             if (CONV) {
 #pragma unroll
