@@ -89,7 +89,7 @@ def peaks():
 
 
 KERNEL_FILES = {  # device sources of each kernel (besides tq_common.cuh)
-    "pack": ["tq_pack.cuh"], "act_quant": ["tq_act.cuh"], "gemv": ["tq_gemv.cuh"],
+    "pack": ["tq_pack.cuh"], "act_quant": ["tq_act.cuh"], "gemv": ["tq_gemv.cuh", "tq_gemv_group.cuh", "tq_act.cuh"],
     "gemm": ["tq_gemm.cuh"], "fused": ["tq_act.cuh", "tq_gemm.cuh"],
     "bwd": ["tq_train.cuh", "tq_gemm.cuh"], "ste": ["tq_train.cuh"], "flip": ["tq_train.cuh", "tq_xorshift_jump.h"],
 }
