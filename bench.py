@@ -474,7 +474,7 @@ def config_for(name, layers, world, layout="foundry", ratio=0.0, bias=False, gro
     desc = {"decode": "decode GEMV: K=N=4096, per-row gamma, M in {1, 8}, ring of %d layers%s" % (L, grp),
             "prefill": "prefill GEMM: M=2048, N=11008, K=4096, per-tensor gamma, ring of %d layers" % L,
             "fused": "fused BitLinear: M=512, N=5632, K=2048, RMSNorm+FWHT-512, ring of %d layers" % L,
-            "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers" % L,
+            "sweep": "M sweep over K=N=8192, per-row gamma, ring of %d layers%s" % (L, grp),
             "pack": "quantise+pack: 8192x8192 per-row (Laplace) and 11008x4096 per-tensor, ring of %d each" % L,
             "roundtrip": "FWHT module int8 round trip: 512 x 2048 Student-t(3), ring of %d batches" % L,
             "mlp": "clamped SwiGLU block of 3 BitLinears: 512 tokens, d_model 1536, d_ffn 6144, ring of %d" % L,
@@ -498,7 +498,7 @@ def config_for(name, layers, world, layout="foundry", ratio=0.0, bias=False, gro
 def line_config(args, world):
     """`config` of the JSON line (both arms print the same one)."""
     main = "decode" if args.workload == "metric" else args.workload
-    group = args.decode_group if main == "decode" else 1
+    group = min(args.decode_group, args.layers or WORKLOAD_SHAPES[main][3]) if main in ("decode", "sweep") else 1
     cfg = config_for(main, args.layers, world, args.layout, args.ratio, args.bias, group)
     if args.workload == "metric":
         cfg["workload"] = "metric: " + cfg["workload"] + "; prefill GEMM record: M=2048, N=11008, K=4096"
@@ -754,7 +754,7 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
     layout = LAYOUTS.index(args.layout)
     main = "decode" if args.workload == "metric" else args.workload
-    group = args.decode_group if main == "decode" else 1
+    group = min(args.decode_group, args.layers or WORKLOAD_SHAPES[main][3]) if main in ("decode", "sweep") else 1
     layers = args.layers or WORKLOAD_SHAPES[main][3]
     wl = Workload(main, tq, S, torch, dev, layers, layout, args.ratio, args.bias, group)
     rec = measure(args, wl, torch, tq, stream, world, local_rank)
@@ -984,7 +984,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="metric", choices=["metric"] + list(WORKLOAD_SHAPES))
     ap.add_argument("--decode-group", type=int, default=8,
-                    help="decode GEMVs as grouped calls of G same-shape layers (1: one call per layer)")
+                    help="small-M GEMVs (decode, sweep) as grouped calls of G same-shape layers (1: one call per layer)")
     ap.add_argument("--bias", action="store_true",
                     help="contractions through tq_ternary_gemm_ex with a bias (the extra epilogue)")
     ap.add_argument("--ratio", type=float, default=0.0,
