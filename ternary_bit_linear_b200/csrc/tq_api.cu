@@ -158,14 +158,14 @@ struct GemmArgs {
     Epilogue ep;
 };
 
-template <int BT, bool CONV, bool EPI>
+template <int BT, bool CONV, bool EPI, bool ATMEM = false>
 tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
-    using L = GemmLayout<BT>;
+    using L = GemmLayout<BT, ATMEM>;
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(tq_gemm_kernel<BT, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tq_gemm_kernel<BT, CONV, EPI, ATMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  L::kDynamic) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
@@ -179,7 +179,7 @@ tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
         return TQ_ERR_CUDA;
     const int64_t tiles = ((a.M + BT - 1) / BT) * ((a.N + kTileN - 1) / kTileN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
-    return launch_pdl(tq_gemm_kernel<BT, CONV, EPI>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
+    return launch_pdl(tq_gemm_kernel<BT, CONV, EPI, ATMEM>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
                       a.s_x, a.rowsum, a.gamma, a.per_row, (int)a.M, (int)a.N, (int)a.K, a.y, a.acc, a.mode,
                       a.ep);
 }
@@ -399,7 +399,11 @@ size_t pack_parts(int64_t nv) {
 // Tokens per GEMM tile.  Cost model: rounds of tiles over the SMs times the
 // time of one K-step, 4 MMAs of BT/2 cycles each but no faster than the
 // single-thread issue rate (about 72 cycles per MMA); ties go to the smaller
-// tile (less padding and x_q traffic).
+// tile (less padding and x_q traffic).  Tiles of up to 128 tokens keep their
+// codes in tensor memory (measured faster there: M = 64 at 8192^2 15.5 ->
+// 14.1 us); the larger ones stage them in shared memory (at 2048 x 11008 x
+// 4096, 128-token tiles with codes in TMEM took 117 us, 256-token tiles in
+// shared memory 82 us).
 int gemm_tile_tokens(int64_t M, int64_t N, int sms) {
     int best = 64;
     int64_t best_cost = -1;
@@ -420,8 +424,8 @@ tq_status contraction(const GemmArgs &a, int sms, cudaStream_t st) {
     if (a.M <= 16 && a.K <= kGemvMaxK)
         return a.M <= 8 ? gemv_shape<1, CONV, EPI>(a, st) : gemv_shape<2, CONV, EPI>(a, st);
     switch (gemm_tile_tokens(a.M, a.N, sms)) {
-    case 64: return launch_gemm<64, CONV, EPI>(a, sms, st);
-    case 128: return launch_gemm<128, CONV, EPI>(a, sms, st);
+    case 64: return launch_gemm<64, CONV, EPI, true>(a, sms, st);
+    case 128: return launch_gemm<128, CONV, EPI, true>(a, sms, st);
     case 192: return launch_gemm<192, CONV, EPI>(a, sms, st);
     default: return launch_gemm<256, CONV, EPI>(a, sms, st);
     }

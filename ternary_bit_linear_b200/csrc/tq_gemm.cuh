@@ -61,15 +61,22 @@ __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t v) {
     return p;
 }
 
-template <int BT>
+// ATMEM: the unpacked codes (the A operand) live in tensor memory instead of
+// shared memory -- written by the unpackers with tcgen05.st, read by the MMA
+// from TMEM -- which takes their stores and the MMA's A reads off the SM's
+// shared-memory bandwidth.  TMEM then holds two accumulators of BT columns and
+// one 32-column code tile (128 lanes x 128 codes) per stage: BT <= 128.
+template <int BT, bool ATMEM = false>
 struct GemmLayout {
+    static_assert(!ATMEM || BT <= 128, "tensor memory holds two accumulators and the code stages");
     static constexpr int kWStages = 8;      // packed-weight ring
     static constexpr int kB = BT * kTileK;  // x_q bytes per stage
-    static constexpr int kStage = kB + kAStageBytes;
-    // x_q + code ring: as many stages as fit beside the weight ring
-    // (4 for BT = 256, 6 for 128, 8 for 64)
+    static constexpr int kStage = kB + (ATMEM ? 0 : kAStageBytes);
+    // x_q (+ code) ring: as many stages as fit beside the weight ring
+    // (4 for BT = 256, 6 for 128, 8 for 64; with the codes in TMEM, at most 8)
     static constexpr int kStagesFit = (232448 - 1024 - 512 - kWStages * kWStageBytes) / kStage;
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    static constexpr int kACols = kTileK / 4;  // TMEM columns of one stage's code tile
     static constexpr int offStage = 0;  // stage s: x_q tile, then code tile (both 1024-aligned)
     static constexpr int offW = kStages * kStage;
     static constexpr int offBar = offW + kWStages * kWStageBytes;
@@ -78,9 +85,13 @@ struct GemmLayout {
     static constexpr int offTmem = offBar + kBars * 8;
     static constexpr int kBytes = offTmem + 16;
     static constexpr int kDynamic = kBytes + 1024;  // slack for 1024-byte alignment
-    // accumulator buffers start at multiples of kDStride TMEM columns
+    // accumulator buffers start at multiples of kDStride TMEM columns; with
+    // ATMEM the code stages follow them
     static constexpr int kDStride = BT <= 128 ? BT : 256;
-    static constexpr uint32_t kTmemCols = pow2_at_least(BT + kDStride);
+    static constexpr int kAColBase = 2 * kDStride;
+    static constexpr uint32_t kTmemCols =
+        pow2_at_least(ATMEM ? kAColBase + kStages * kACols : BT + kDStride);
+    static_assert(kTmemCols <= 512, "tensor memory columns");
     static_assert(kDynamic <= 232448, "shared memory per CTA");
     static_assert(kB % 1024 == 0 && kAStageBytes % 1024 == 0, "swizzle atoms stay aligned");
 };
@@ -102,13 +113,14 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
 // 2-3) and every word is rewritten in Foundry's layout before the unpack; the
 // default layout compiles without that step.  EPI: the extra epilogue `ep`
 // (bias, integer bias and shift) is applied.
-template <int BT, bool CONV, bool EPI>
+// ATMEM: the code tiles in tensor memory (GemmLayout).
+template <int BT, bool CONV, bool EPI, bool ATMEM = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
                 const float *__restrict__ gamma, int per_row, int M, int N, int K,
                 float *__restrict__ y, int32_t *__restrict__ acc_out, int mode, Epilogue ep) {
-    using L = GemmLayout<BT>;
+    using L = GemmLayout<BT, ATMEM>;
     constexpr int S = L::kStages, SW = L::kWStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -226,10 +238,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t a_addr = a_stage(s), b_addr = x_stage(s);
+                    if (ATMEM) {
+                        // codes of stage s: TMEM columns kAColBase + 32 s ..., 8 columns per K = 32
+                        const uint32_t a_col = tmem + (uint32_t)(L::kAColBase + s * L::kACols);
 #pragma unroll
-                    for (int kk = 0; kk < kTileK / 32; ++kk)
-                        mma_i8(d_col, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
-                               idesc, (kb | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kTileK / 32; ++kk)
+                            mma_i8_ts(d_col, a_col + (uint32_t)(kk * 8), smem_desc_sw128(b_addr + kk * 32), idesc,
+                                      (kb | kk) != 0 ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kTileK / 32; ++kk)
+                            mma_i8(d_col, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
+                                   idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
                     mma_commit(empty(s));
                 }
                 if (ok) mma_commit(d_full(b));  // accumulator b complete
@@ -280,14 +301,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int c = 0; c < 8; ++c) e[c] = expand_word(words[c]);
             if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
-            // 16-byte chunk c of row r lives at chunk position c ^ (r & 7)
-            const uint32_t base = a_stage(s) + a_row;
+            if (ATMEM) {
+                // row r's 128 codes -> TMEM lane r (this warp's lane quarter is
+                // 32 (warp % 4) .. + 31), 32 consecutive columns of 4 codes each
+                uint32_t cw[32];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base + (((uint32_t)c ^ sw) << 4)),
-                             "r"(e[c].x), "r"(e[c].y), "r"(e[c].z), "r"(e[c].w)
-                             : "memory");
-            fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+                for (int c = 0; c < 8; ++c) {
+                    cw[4 * c] = e[c].x;
+                    cw[4 * c + 1] = e[c].y;
+                    cw[4 * c + 2] = e[c].z;
+                    cw[4 * c + 3] = e[c].w;
+                }
+                tmem_st32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(L::kAColBase + s * L::kACols), cw);
+                tmem_st_wait();
+                tc_fence_before();  // the stores are complete before the MMA warp is told
+            } else {
+                // 16-byte chunk c of row r lives at chunk position c ^ (r & 7)
+                const uint32_t base = a_stage(s) + a_row;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base + (((uint32_t)c ^ sw) << 4)),
+                                 "r"(e[c].x), "r"(e[c].y), "r"(e[c].z), "r"(e[c].w)
+                                 : "memory");
+                fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+            }
             __syncwarp();
             // The packed slot is released only now: the stores above consume the
             // loaded words, so every lane's read of the slot is complete before
