@@ -64,11 +64,13 @@ __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t v) {
 // ATMEM: the unpacked codes (the A operand) live in tensor memory instead of
 // shared memory -- written by the unpackers with tcgen05.st, read by the MMA
 // from TMEM -- which takes their stores and the MMA's A reads off the SM's
-// shared-memory bandwidth.  TMEM then holds two accumulators of BT columns and
-// one 32-column code tile (128 lanes x 128 codes) per stage: BT <= 128.
+// shared-memory bandwidth.  TMEM then holds the accumulators and one 32-column
+// code tile (128 lanes x 128 codes) per stage: two accumulators up to BT = 128,
+// one for larger tiles (the MMAs of a tile then start once the epilogue has
+// read the previous tile's accumulator).
 template <int BT, bool ATMEM = false>
 struct GemmLayout {
-    static_assert(!ATMEM || BT <= 128, "tensor memory holds two accumulators and the code stages");
+    static constexpr int kAccBufs = (ATMEM && BT > 128) ? 1 : 2;
     static constexpr int kWStages = 8;      // packed-weight ring
     static constexpr int kB = BT * kTileK;  // x_q bytes per stage
     static constexpr int kStage = kB + (ATMEM ? 0 : kAStageBytes);
@@ -88,7 +90,7 @@ struct GemmLayout {
     // accumulator buffers start at multiples of kDStride TMEM columns; with
     // ATMEM the code stages follow them
     static constexpr int kDStride = BT <= 128 ? BT : 256;
-    static constexpr int kAColBase = 2 * kDStride;
+    static constexpr int kAColBase = kAccBufs * kDStride;
     static constexpr uint32_t kTmemCols =
         pow2_at_least(ATMEM ? kAColBase + kStages * kACols : BT + kDStride);
     static_assert(kTmemCols <= 512, "tensor memory columns");
@@ -226,8 +228,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int g = 0;
             bool ok = true;
             for (int tl = 0; tl < my_tiles && ok; ++tl) {
-                const int b = tl & 1;
-                if (!mbar_wait(d_empty(b), ((tl >> 1) & 1) ^ 1)) break;
+                const int b = tl % L::kAccBufs;
+                if (!mbar_wait(d_empty(b), ((tl / L::kAccBufs) & 1) ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_col = tmem + (uint32_t)(b * L::kDStride);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool vec4 = (N & 3) == 0;  // rows of y are 16-byte multiples
         for (int tl = 0; tl < my_tiles; ++tl) {
             const int t = (int)blockIdx.x + tl * (int)gridDim.x;
-            const int b = tl & 1;
+            const int b = tl % L::kAccBufs;
             const int m0 = (t % num_m) * BT + half * kHalf, n0 = (t / num_m) * kTileN;
             const int n = n0 + 32 * q + lane;
             // per-tile scalars, loaded while the accumulator is still being computed
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 sxc[cc] = mj < M ? __ldg(s_x + mj) : 0.0f;
                 rsc[cc] = mj < M ? __ldg(rowsum + mj) : 0;
             }
-            if (!warp_wait_sleep(d_full(b), (tl >> 1) & 1, lane)) break;
+            if (!warp_wait_sleep(d_full(b), (tl / L::kAccBufs) & 1, lane)) break;
             tc_fence_after();
 #pragma unroll
             for (int cc = 0; cc < kChunks; ++cc) {
