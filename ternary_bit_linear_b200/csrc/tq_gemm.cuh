@@ -345,76 +345,105 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int half = (warp - 12) >> 2;     // token half of the tile
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
         const bool vec4 = (N & 3) == 0;  // rows of y are 16-byte multiples
+        // vec4 layout: after a 4 x 4 transpose inside each lane quad, lane 4g + r
+        // holds token 4k + r of the quad's features 4g .. 4g + 3 (one 16-byte store)
+        const int r = lane & 3;
         for (int tl = 0; tl < my_tiles; ++tl) {
             const int t = (int)blockIdx.x + tl * (int)gridDim.x;
             const int b = tl % L::kAccBufs;
             const int m0 = (t % num_m) * BT + half * kHalf, n0 = (t / num_m) * kTileN;
             const int n = n0 + 32 * q + lane;
+            const int nq = n - r;  // first feature of the lane's quad
             // per-tile scalars, loaded while the accumulator is still being computed
-            const float gn = n < N ? __ldg(gamma + (per_row ? n : 0)) : 0.0f;
-            const float bn = (EPI && n < N && ep.bias) ? __ldg(ep.bias + n) : 0.0f;
-            const int abn = (EPI && n < N && ep.acc_bias) ? __ldg(ep.acc_bias + n) : 0;
+            float gn = 0.0f, bn = 0.0f;
+            int abn = 0;
+            float g4[4] = {0.0f, 0.0f, 0.0f, 0.0f}, b4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             float sxc[kChunks];
             int rsc[kChunks];
+            const bool quads = vec4 && !acc_out;
+            if (quads) {
+                if (nq < N) {  // N % 4 == 0: the quad's four features are all < N
 #pragma unroll
-            for (int cc = 0; cc < kChunks; ++cc) {
-                const int mj = m0 + cc * 32 + lane;  // lane j holds token m0 + 32 cc + j
-                sxc[cc] = mj < M ? __ldg(s_x + mj) : 0.0f;
-                rsc[cc] = mj < M ? __ldg(rowsum + mj) : 0;
+                    for (int i = 0; i < 4; ++i) {
+                        g4[i] = __ldg(gamma + (per_row ? nq + i : 0));
+                        if (EPI && ep.bias) b4[i] = __ldg(ep.bias + nq + i);
+                    }
+                }
+            } else {
+                gn = n < N ? __ldg(gamma + (per_row ? n : 0)) : 0.0f;
+                bn = (EPI && n < N && ep.bias) ? __ldg(ep.bias + n) : 0.0f;
+                abn = (EPI && n < N && ep.acc_bias) ? __ldg(ep.acc_bias + n) : 0;
+#pragma unroll
+                for (int cc = 0; cc < kChunks; ++cc) {
+                    const int mj = m0 + cc * 32 + lane;  // lane j holds token m0 + 32 cc + j
+                    sxc[cc] = mj < M ? __ldg(s_x + mj) : 0.0f;
+                    rsc[cc] = mj < M ? __ldg(rowsum + mj) : 0;
+                }
             }
             if (!warp_wait_sleep(d_full(b), (tl / L::kAccBufs) & 1, lane)) break;
             tc_fence_after();
 #pragma unroll
             for (int cc = 0; cc < kChunks; ++cc) {
+                const int mb = m0 + cc * 32;
+                const int jmax = M - mb;  // tokens of this chunk inside [0, M)
                 uint32_t v[32];
                 tmem_ld32(lane_addr + (uint32_t)(b * L::kDStride + half * kHalf + cc * 32), v);
+                // the lane's own tokens of the transposed layout (quads), fetched
+                // while the accumulator load is in flight
+                float sxk[8];
+                int rsk[8];
+                if (quads) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int mk = mb + 4 * k + r;
+                        sxk[k] = mk < M ? __ldg(s_x + mk) : 0.0f;
+                        rsk[k] = mk < M ? __ldg(rowsum + mk) : 0;
+                    }
+                }
                 tmem_ld_wait();
                 if (cc == kChunks - 1) {  // accumulator fully read: hand it back to the MMA warp
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(d_empty(b));
                 }
-                // Branch-free pass first (the shuffles of all 32 tokens can then
-                // overlap), then a pure store pass.
-                const int mb = m0 + cc * 32;
-                const int jmax = M - mb;  // tokens of this chunk inside [0, M)
-                if (!acc_out) {
+                if (quads) {
+                    float *yq = y + (int64_t)(mb + r) * N + nq;
+                    const bool fin = nq < N;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
+                    for (int k = 0; k < 8; ++k) {
+                        // lane 4g + r holds feature 4g + r of tokens 4k .. 4k + 3;
+                        // transpose the raw accumulators inside the quad
+                        uint32_t a0 = v[4 * k], a1 = v[4 * k + 1], a2 = v[4 * k + 2], a3 = v[4 * k + 3];
+                        // distance 1: swap the odd/even off-diagonal elements of lane pairs
+                        const bool o1 = r & 1;
+                        const uint32_t x1 = __shfl_xor_sync(0xffffffffu, o1 ? a0 : a1, 1);
+                        const uint32_t y1 = __shfl_xor_sync(0xffffffffu, o1 ? a2 : a3, 1);
+                        if (o1) { a0 = x1; a2 = y1; } else { a1 = x1; a3 = y1; }
+                        // distance 2: swap the off-diagonal 2 x 2 blocks of lane pairs
+                        const bool o2 = r & 2;
+                        const uint32_t x2 = __shfl_xor_sync(0xffffffffu, o2 ? a0 : a2, 2);
+                        const uint32_t y2 = __shfl_xor_sync(0xffffffffu, o2 ? a1 : a3, 2);
+                        if (o2) { a0 = x2; a1 = y2; } else { a2 = x2; a3 = y2; }
+                        // now token 4k + r of features 4g + i: y = fp32(acc - rowsum) * (gamma * s_x)
+                        const uint32_t ai[4] = {a0, a1, a2, a3};
+                        float yv[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            yv[i] = __fmul_rn(__int2float_rn((int)ai[i] - rsk[k]), __fmul_rn(g4[i], sxk[k]));
+                            if (EPI) yv[i] = __fadd_rn(yv[i], b4[i]);
+                        }
+                        if (fin && 4 * k + r < jmax)
+                            __stcs(reinterpret_cast<float4 *>(yq + (int64_t)(4 * k) * N),
+                                   make_float4(yv[0], yv[1], yv[2], yv[3]));
+                    }
+                } else if (!acc_out) {
+                    float *yp = y + (int64_t)mb * N + n;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {  // every lane takes part in the shuffles
                         const float sxm = __shfl_sync(0xffffffffu, sxc[cc], j);
                         const int rsm = __shfl_sync(0xffffffffu, rsc[cc], j);
                         const float yv = __fmul_rn(__int2float_rn((int)v[j] - rsm), __fmul_rn(gn, sxm));
-                        v[j] = __float_as_uint(EPI ? __fadd_rn(yv, bn) : yv);
-                    }
-                    if (vec4) {
-                        // 4 x 4 transposes inside each lane quad: lane 4g + r then holds
-                        // token 4k + r of features 4g .. 4g + 3 and stores them as one
-                        // 16-byte vector (a quarter of the store instructions).
-                        const int r = lane & 3;
-                        float *yq = y + (int64_t)(mb + r) * N + (n - (lane & 3));
-                        const bool fin = n - r < N;  // the quad's four features are all < N
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            float a0 = __uint_as_float(v[4 * k]), a1 = __uint_as_float(v[4 * k + 1]);
-                            float a2 = __uint_as_float(v[4 * k + 2]), a3 = __uint_as_float(v[4 * k + 3]);
-                            // distance 1: swap the odd/even off-diagonal elements of lane pairs
-                            const bool o1 = r & 1;
-                            const float x1 = __shfl_xor_sync(0xffffffffu, o1 ? a0 : a1, 1);
-                            const float y1 = __shfl_xor_sync(0xffffffffu, o1 ? a2 : a3, 1);
-                            if (o1) { a0 = x1; a2 = y1; } else { a1 = x1; a3 = y1; }
-                            // distance 2: swap the off-diagonal 2 x 2 blocks of lane pairs
-                            const bool o2 = r & 2;
-                            const float x2 = __shfl_xor_sync(0xffffffffu, o2 ? a0 : a2, 2);
-                            const float y2 = __shfl_xor_sync(0xffffffffu, o2 ? a1 : a3, 2);
-                            if (o2) { a0 = x2; a1 = y2; } else { a2 = x2; a3 = y2; }
-                            if (fin && 4 * k + r < jmax)
-                                __stcs(reinterpret_cast<float4 *>(yq + (int64_t)(4 * k) * N), make_float4(a0, a1, a2, a3));
-                        }
-                    } else if (n < N) {
-                        float *yp = y + (int64_t)mb * N + n;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (j < jmax) __stcs(yp + (int64_t)j * N, __uint_as_float(v[j]));
+                        if (j < jmax && n < N) __stcs(yp + (int64_t)j * N, EPI ? __fadd_rn(yv, bn) : yv);
                     }
                 } else {
 #pragma unroll
