@@ -626,8 +626,11 @@ def test_pack_inputs_ready_layers_then_dependent_reader(cuda_lib, per_row):
 
 
 # Shapes whose tile choice (tokens per tile, from the launcher's cost model on
-# 148 SMs) is 128, 192 and 256 respectively, all ragged in M, N and K.
-@pytest.mark.parametrize("M,N,K", [(383, 11000, 192), (500, 5600, 320), (1000, 4000, 192)])
+# 148 SMs) is 128, 192 and 256 respectively, all ragged in M, N and K; 256-token
+# tiles run on CTA pairs (256 features per tile), and in the last shape the
+# second CTA's half of the last token tile and of the last feature tile lies
+# wholly outside the matrices.
+@pytest.mark.parametrize("M,N,K", [(383, 11000, 192), (500, 5600, 320), (1000, 4000, 192), (580, 4956, 192)])
 def test_gemm_tile_sizes_sampled(cuda_lib, M, N, K):
     W = S.normal((N, K), 0.02, 70, N)
     X = S.decode_acts(M, K, seed=71)
