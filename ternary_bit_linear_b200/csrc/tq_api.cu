@@ -6,7 +6,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -75,31 +74,21 @@ inline tq_status launch_status() {
 // kernel waits (griddepcontrol.wait) before touching memory an earlier kernel
 // may have produced, so the attribute only lets launches overlap.
 template <typename... KArgs, typename... Args>
-tq_status launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                             cudaStream_t st, unsigned cluster_x, Args... args) {
+tq_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = cluster_x;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = cluster_x > 1 ? 2 : 1;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess
                ? TQ_OK
                : TQ_ERR_CUDA;
-}
-
-template <typename... KArgs, typename... Args>
-tq_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                     cudaStream_t st, Args... args) {
-    return launch_pdl_cluster(kernel, grid, block, smem, st, 1u, args...);
 }
 
 // Packed-code layout from the flags (kEnc*), or -1 for the reserved value.
@@ -169,53 +158,30 @@ struct GemmArgs {
     Epilogue ep;
 };
 
-template <int BT, bool CONV, bool EPI, bool ATMEM = false, bool PAIR = false>
+template <int BT, bool CONV, bool EPI, bool ATMEM = false>
 tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
-    using L = GemmLayout<BT, ATMEM, PAIR>;
+    using L = GemmLayout<BT, ATMEM>;
     static std::atomic<int> attr_done[kMaxDevices];
-    static std::atomic<int> max_pairs[kMaxDevices];  // pairs resident at once (cluster occupancy)
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(tq_gemm_kernel<BT, CONV, EPI, ATMEM, PAIR>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynamic) != cudaSuccess)
+        if (cudaFuncSetAttribute(tq_gemm_kernel<BT, CONV, EPI, ATMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::kDynamic) != cudaSuccess)
             return TQ_ERR_CUDA;
-        if (PAIR) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3((unsigned)(sms & ~1));
-            cfg.blockDim = dim3(kGemmThreads);
-            cfg.dynamicSmemBytes = L::kDynamic;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = 2;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, tq_gemm_kernel<BT, CONV, EPI, ATMEM, PAIR>, &cfg) != cudaSuccess ||
-                n < 1)
-                return TQ_ERR_CUDA;
-            max_pairs[dev].store(n);
-        }
         attr_done[dev].store(1);
     }
-    // x_q [M][K] in 128-byte-swizzled [rows][128] boxes (a pair's CTAs load
-    // half of the tile's tokens each); packed weights [N][K/4] in plain
-    // [128][32] boxes (K % 64 == 0 keeps both row strides 16-byte multiples).
+    // x_q [M][K] in 128-byte-swizzled [BT][128] boxes; packed weights [N][K/4]
+    // in plain [128][32] boxes (K % 64 == 0 keeps both row strides 16-byte multiples).
     CUtensorMap tx, tw;
-    if (!make_tmap_u8(&tx, a.xq, (uint64_t)a.K, (uint64_t)a.M, kTileK, L::kXRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_tmap_u8(&tx, a.xq, (uint64_t)a.K, (uint64_t)a.M, kTileK, BT, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_u8(&tw, a.packed, (uint64_t)(a.K / 4), (uint64_t)a.N, kTileK / 4, kTileN,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return TQ_ERR_CUDA;
-    constexpr int kFeat = PAIR ? 2 * kTileN : kTileN;
-    const int64_t tiles = ((a.M + BT - 1) / BT) * ((a.N + kFeat - 1) / kFeat);
-    // persistent, one CTA per SM (one pair per two SMs)
-    const int64_t units = PAIR ? std::min<int64_t>(sms / 2, max_pairs[dev].load()) : sms;
-    const unsigned grid = (unsigned)((tiles < units ? tiles : units) * (PAIR ? 2 : 1));
-    return launch_pdl_cluster(tq_gemm_kernel<BT, CONV, EPI, ATMEM, PAIR>, dim3(grid), dim3(kGemmThreads),
-                              L::kDynamic, st, PAIR ? 2u : 1u, tx, tw, a.s_x, a.rowsum, a.gamma, a.per_row, (int)a.M,
-                              (int)a.N, (int)a.K, a.y, a.acc, a.mode, a.ep);
+    const int64_t tiles = ((a.M + BT - 1) / BT) * ((a.N + kTileN - 1) / kTileN);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
+    return launch_pdl(tq_gemm_kernel<BT, CONV, EPI, ATMEM>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
+                      a.s_x, a.rowsum, a.gamma, a.per_row, (int)a.M, (int)a.N, (int)a.K, a.y, a.acc, a.mode,
+                      a.ep);
 }
 
 // Grid: one CTA per 16-row strip.  Dynamic shared memory holds x_q only.
@@ -461,7 +427,7 @@ tq_status contraction(const GemmArgs &a, int sms, cudaStream_t st) {
     case 64: return launch_gemm<64, CONV, EPI, true>(a, sms, st);
     case 128: return launch_gemm<128, CONV, EPI, true>(a, sms, st);
     case 192: return launch_gemm<192, CONV, EPI>(a, sms, st);
-    default: return launch_gemm<256, CONV, EPI, true, true>(a, sms, st);
+    default: return launch_gemm<256, CONV, EPI, true>(a, sms, st);
     }
 }
 

@@ -68,19 +68,11 @@ __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t v) {
 // code tile (128 lanes x 128 codes) per stage: two accumulators up to BT = 128,
 // one for larger tiles (the MMAs of a tile then start once the epilogue has
 // read the previous tile's accumulator).
-//
-// PAIR: a cluster of two CTAs computes a 256-feature x BT-token tile with pair
-// MMAs (cta_group::2): each CTA unpacks the codes of its 128 features into its
-// own TMEM and loads half of the tile's tokens (BT / 2 rows of x_q); the pair
-// MMA feeds both halves of B to both tensor cores, so each SM moves half the
-// x_q bytes per MMA of the single-CTA tile.
-template <int BT, bool ATMEM = false, bool PAIR = false>
+template <int BT, bool ATMEM = false>
 struct GemmLayout {
-    static_assert(!PAIR || (ATMEM && BT == 256), "the pair tile is 256 x 256 with the codes in TMEM");
     static constexpr int kAccBufs = (ATMEM && BT > 128) ? 1 : 2;
     static constexpr int kWStages = 8;      // packed-weight ring
-    static constexpr int kXRows = PAIR ? BT / 2 : BT;  // x_q rows this CTA loads per stage
-    static constexpr int kB = kXRows * kTileK;  // x_q bytes per stage
+    static constexpr int kB = BT * kTileK;  // x_q bytes per stage
     static constexpr int kStage = kB + (ATMEM ? 0 : kAStageBytes);
     // x_q (+ code) ring: as many stages as fit beside the weight ring
     // (4 for BT = 256, 6 for 128, 8 for 64; with the codes in TMEM, at most 8)
@@ -123,17 +115,15 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
 // 2-3) and every word is rewritten in Foundry's layout before the unpack; the
 // default layout compiles without that step.  EPI: the extra epilogue `ep`
 // (bias, integer bias and shift) is applied.
-// ATMEM: the code tiles in tensor memory; PAIR: two-CTA tiles (GemmLayout).
-// A PAIR kernel is launched in clusters of two CTAs.
-template <int BT, bool CONV, bool EPI, bool ATMEM = false, bool PAIR = false>
+// ATMEM: the code tiles in tensor memory (GemmLayout).
+template <int BT, bool CONV, bool EPI, bool ATMEM = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
                 const float *__restrict__ gamma, int per_row, int M, int N, int K,
                 float *__restrict__ y, int32_t *__restrict__ acc_out, int mode, Epilogue ep) {
-    using L = GemmLayout<BT, ATMEM, PAIR>;
+    using L = GemmLayout<BT, ATMEM>;
     constexpr int S = L::kStages, SW = L::kWStages;
-    constexpr int kFeat = PAIR ? 2 * kTileN : kTileN;  // features per tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -149,28 +139,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto x_stage = [&](int s) { return sbase + (uint32_t)(L::offStage + s * L::kStage); };
     auto a_stage = [&](int s) { return x_stage(s) + (uint32_t)L::kB; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::offTmem);
-    // In a pair, the first CTA's full and d_empty barriers gate the pair MMAs:
-    // both CTAs' copies, unpackers and epilogues signal those.
-    const uint32_t rank = PAIR ? cluster_rank() : 0u;
-    auto lead = [&](uint32_t bar) { return PAIR ? mapa_shared(bar, 0) : bar; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_m = (M + BT - 1) / BT, num_n = (N + kFeat - 1) / kFeat;
+    const int num_m = (M + BT - 1) / BT, num_n = (N + kTileN - 1) / kTileN;
     const int ntiles = num_m * num_n;
     const int nkb = (K + kTileK - 1) / kTileK;
-    // tiles are dealt to schedule units: CTAs, or CTA pairs
-    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     // steps this CTA runs: its tiles times the steps per tile
-    const int my_tiles = ntiles > unit ? (ntiles - unit + units - 1) / units : 0;
+    const int my_tiles = ntiles > (int)blockIdx.x
+                             ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                             : 0;
     const int total = my_tiles * nkb;
-    // this CTA's feature rows and x_q rows within a tile
-    const int feat_off = (int)rank * kTileN, xrow_off = (int)rank * L::kXRows;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            // TMA bytes + the step's four unpacker warps (of each CTA of a pair)
-            mbar_init(full(s), 1 + (PAIR ? kUnpackWarps : kUnpackWarps / 2));
+            mbar_init(full(s), 1 + kUnpackWarps / 2);  // TMA bytes + the step's four unpacker warps
             mbar_init(empty(s), 1);
         }
         for (int s = 0; s < SW; ++s) {
@@ -179,7 +161,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(d_full(b), 1);
-            mbar_init(d_empty(b), PAIR ? 2 * kEpiWarps : kEpiWarps);
+            mbar_init(d_empty(b), kEpiWarps);
         }
         mbar_init(mma_done, 1);
         fence_barrier_init();
@@ -187,13 +169,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         prefetch_tmap(&tm_w);
     }
     if (warp == 1) {
-        if (PAIR) {
-            tmem_alloc_pair(smem_u32(tmem_slot), L::kTmemCols);
-            tmem_relinquish_pair();
-        } else {
-            tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
-            tmem_relinquish();
-        }
+        tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+        tmem_relinquish();
     }
     // Everything above touched no global memory; inputs of the previous kernel
     // on the stream are visible after this wait.  With static weights only the
@@ -206,10 +183,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (!w_early) pdl_wait();
     pdl_trigger();
     tc_fence_before();
-    if (PAIR)
-        cluster_sync_all();  // both CTAs' barriers are initialised before either signals the other
-    else
-        __syncthreads();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -220,23 +194,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int g = 0;
             for (; g < total; ++g) {
                 const int s = g % S, r = g / S;
-                const int t = unit + (g / nkb) * units;
+                const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
                 const int kb = g % nkb;
                 if (!mbar_wait_sleep(empty(s), (r & 1) ^ 1)) break;
-                if (PAIR) {  // the first CTA expects both halves' bytes
-                    if (rank == 0) mbar_arrive_expect_tx(full(s), 2 * L::kB);
-                    tma_load_2d_pair(x_stage(s), &tm_x, kb * kTileK, (t % num_m) * BT + xrow_off, lead(full(s)));
-                } else {
-                    mbar_arrive_expect_tx(full(s), L::kB);
-                    tma_load_2d(x_stage(s), &tm_x, kb * kTileK, (t % num_m) * BT, full(s));
-                }
+                mbar_arrive_expect_tx(full(s), L::kB);
+                tma_load_2d(x_stage(s), &tm_x, kb * kTileK, (t % num_m) * BT, full(s));
             }
             // Own copies must have landed before the CTA may exit (already
-            // true unless a wait gave up).  A pair's copies complete on the
-            // first CTA's barriers: that CTA waits for both halves, and the
-            // cluster barrier before exit holds the second CTA until then.
-            if (rank == 0)
-                for (int j = g - S < 0 ? 0 : g - S; j < g; ++j) mbar_wait(full(j % S), (j / S) & 1);
+            // true unless a wait gave up).
+            for (int j = g - S < 0 ? 0 : g - S; j < g; ++j) mbar_wait(full(j % S), (j / S) & 1);
         }
         __syncwarp();
     } else if (warp == 2) {
@@ -245,22 +211,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int g = 0;
             for (; g < total; ++g) {
                 const int s = g % SW, r = g / SW;
-                const int t = unit + (g / nkb) * units;
+                const int t = (int)blockIdx.x + (g / nkb) * (int)gridDim.x;
                 const int kb = g % nkb;
                 if (!mbar_wait_sleep(w_empty(s), (r & 1) ^ 1)) break;
                 mbar_arrive_expect_tx(w_full(s), kWStageBytes);
                 tma_load_2d(sbase + (uint32_t)(L::offW + s * kWStageBytes), &tm_w, kb * (kTileK / 4),
-                            (t / num_m) * kFeat + feat_off, w_full(s));
+                            (t / num_m) * kTileN, w_full(s));
             }
             for (int j = g - SW < 0 ? 0 : g - SW; j < g; ++j) mbar_wait(w_full(j % SW), (j / SW) & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        // (in a pair, the first CTA's thread issues the pair MMAs; the second
-        // CTA's waits until they are done, as they read its TMEM and shared memory)
-        if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_i8_u8s8(kFeat, BT);
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8_u8s8(kTileN, BT);
             int g = 0;
             bool ok = true;
             for (int tl = 0; tl < my_tiles && ok; ++tl) {
@@ -280,40 +244,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         // codes of stage s: TMEM columns kAColBase + 32 s ..., 8 columns per K = 32
                         const uint32_t a_col = tmem + (uint32_t)(L::kAColBase + s * L::kACols);
 #pragma unroll
-                        for (int kk = 0; kk < kTileK / 32; ++kk) {
-                            if (PAIR)
-                                mma_i8_ts_pair(d_col, a_col + (uint32_t)(kk * 8), smem_desc_sw128(b_addr + kk * 32),
-                                               idesc, (kb | kk) != 0 ? 1u : 0u);
-                            else
-                                mma_i8_ts(d_col, a_col + (uint32_t)(kk * 8), smem_desc_sw128(b_addr + kk * 32),
-                                          idesc, (kb | kk) != 0 ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < kTileK / 32; ++kk)
+                            mma_i8_ts(d_col, a_col + (uint32_t)(kk * 8), smem_desc_sw128(b_addr + kk * 32), idesc,
+                                      (kb | kk) != 0 ? 1u : 0u);
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < kTileK / 32; ++kk)
                             mma_i8(d_col, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
                                    idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    if (PAIR)
-                        mma_commit_pair_both(empty(s));
-                    else
-                        mma_commit(empty(s));
+                    mma_commit(empty(s));
                 }
-                if (ok) {  // accumulator b complete
-                    if (PAIR)
-                        mma_commit_pair_both(d_full(b));
-                    else
-                        mma_commit(d_full(b));
-                }
+                if (ok) mma_commit(d_full(b));  // accumulator b complete
             }
             // No MMA may still use TMEM when it is freed: this commit fires
             // once every MMA issued above has completed.
-            if (PAIR)
-                mma_commit_pair_both(mma_done);
-            else
-                mma_commit(mma_done);
-            mbar_wait(mma_done, 0);
-        } else if (PAIR && lane == 0) {
+            mma_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
         __syncwarp();
@@ -387,10 +333,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // the producer may refill it.
             if (lane == 0) {
                 mbar_arrive(w_empty(ws));
-                if (PAIR)
-                    mbar_arrive_cluster(lead(full(s)));
-                else
-                    mbar_arrive(full(s));
+                mbar_arrive(full(s));
             }
         }
     } else if (warp >= 12) {
@@ -406,9 +349,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // holds token 4k + r of the quad's features 4g .. 4g + 3 (one 16-byte store)
         const int r = lane & 3;
         for (int tl = 0; tl < my_tiles; ++tl) {
-            const int t = unit + tl * units;
+            const int t = (int)blockIdx.x + tl * (int)gridDim.x;
             const int b = tl % L::kAccBufs;
-            const int m0 = (t % num_m) * BT + half * kHalf, n0 = (t / num_m) * kFeat + feat_off;
+            const int m0 = (t % num_m) * BT + half * kHalf, n0 = (t / num_m) * kTileN;
             const int n = n0 + 32 * q + lane;
             const int nq = n - r;  // first feature of the lane's quad
             // per-tile scalars, loaded while the accumulator is still being computed
@@ -461,12 +404,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (cc == kChunks - 1) {  // accumulator fully read: hand it back to the MMA warp
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) {
-                        if (PAIR)
-                            mbar_arrive_cluster(lead(d_empty(b)));
-                        else
-                            mbar_arrive(d_empty(b));
-                    }
+                    if (lane == 0) mbar_arrive(d_empty(b));
                 }
                 if (quads) {
                     float *yq = y + (int64_t)(mb + r) * N + nq;
@@ -525,19 +463,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     if (ready || w_early) pdl_wait();  // no-op for roles that already waited
     tc_fence_before();
-    if (PAIR) {
-        // neither CTA of a pair leaves while the other may still signal its
-        // barriers or the pair MMAs may still read its memory
-        cluster_sync_all();
-    } else {
-        __syncthreads();
-    }
+    __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        if (PAIR)
-            tmem_dealloc_pair(tmem, L::kTmemCols);
-        else
-            tmem_dealloc(tmem, L::kTmemCols);
+        tmem_dealloc(tmem, L::kTmemCols);
     }
 }
 
