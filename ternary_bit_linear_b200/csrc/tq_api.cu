@@ -426,7 +426,7 @@ tq_status contraction(const GemmArgs &a, int sms, cudaStream_t st) {
     switch (gemm_tile_tokens(a.M, a.N, sms)) {
     case 64: return launch_gemm<64, CONV, EPI, true>(a, sms, st);
     case 128: return launch_gemm<128, CONV, EPI, true>(a, sms, st);
-    case 192: return launch_gemm<192, CONV, EPI>(a, sms, st);
+    case 192: return launch_gemm<192, CONV, EPI, true>(a, sms, st);
     default: return launch_gemm<256, CONV, EPI, true>(a, sms, st);
     }
 }
