@@ -158,14 +158,14 @@ struct GemmArgs {
     Epilogue ep;
 };
 
-template <int BT, bool CONV, bool EPI, bool ATMEM = false>
+template <int BT, bool CONV, bool EPI>
 tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
-    using L = GemmLayout<BT, ATMEM>;
+    using L = GemmLayout<BT>;
     static std::atomic<int> attr_done[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(tq_gemm_kernel<BT, CONV, EPI, ATMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tq_gemm_kernel<BT, CONV, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  L::kDynamic) != cudaSuccess)
             return TQ_ERR_CUDA;
         attr_done[dev].store(1);
@@ -179,7 +179,7 @@ tq_status launch_gemm(const GemmArgs &a, int sms, cudaStream_t st) {
         return TQ_ERR_CUDA;
     const int64_t tiles = ((a.M + BT - 1) / BT) * ((a.N + kTileN - 1) / kTileN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // persistent, one CTA per SM
-    return launch_pdl(tq_gemm_kernel<BT, CONV, EPI, ATMEM>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
+    return launch_pdl(tq_gemm_kernel<BT, CONV, EPI>, dim3(grid), dim3(kGemmThreads), L::kDynamic, st, tx, tw,
                       a.s_x, a.rowsum, a.gamma, a.per_row, (int)a.M, (int)a.N, (int)a.K, a.y, a.acc, a.mode,
                       a.ep);
 }
@@ -424,10 +424,10 @@ tq_status contraction(const GemmArgs &a, int sms, cudaStream_t st) {
     if (a.M <= 16 && a.K <= kGemvMaxK)
         return a.M <= 8 ? gemv_shape<1, CONV, EPI>(a, st) : gemv_shape<2, CONV, EPI>(a, st);
     switch (gemm_tile_tokens(a.M, a.N, sms)) {
-    case 64: return launch_gemm<64, CONV, EPI, true>(a, sms, st);
-    case 128: return launch_gemm<128, CONV, EPI, true>(a, sms, st);
-    case 192: return launch_gemm<192, CONV, EPI, true>(a, sms, st);
-    default: return launch_gemm<256, CONV, EPI, true>(a, sms, st);
+    case 64: return launch_gemm<64, CONV, EPI>(a, sms, st);
+    case 128: return launch_gemm<128, CONV, EPI>(a, sms, st);
+    case 192: return launch_gemm<192, CONV, EPI>(a, sms, st);
+    default: return launch_gemm<256, CONV, EPI>(a, sms, st);
     }
 }
 

@@ -9,25 +9,28 @@
 // taken by the weights) x BT tokens (the MMA's N: 64, 128, 192 or 256, chosen
 // per problem by the launcher to fill the SMs), token blocks
 // fastest so that concurrently running CTAs share weight tiles in L2.  K is
-// consumed in steps of 128 codes; one step is four MMAs of K = 32 with both
-// operands in shared memory (128-byte swizzled, K-major).  Twenty warps:
+// consumed in steps of 128 codes; one step is four MMAs of K = 32, the codes
+// (A) read from tensor memory and x_q (B) from shared memory (128-byte
+// swizzled, K-major).  Twenty warps:
 //
 //   warp 0      x_q producer (lane 0): TMA of the x_q tile [BT][128 B] into
 //               stage s of the operand ring.
 //   warp 1      TMEM owner; lane 0 issues the MMAs.  Per step: one wait on
 //               full(s), four MMAs, one commit that frees stage s.  The
-//               accumulator alternates between two TMEM buffers per tile.
+//               accumulator alternates between two TMEM buffers per tile
+//               (BT <= 128) or is a single buffer (BT = 192, 256).
 //   warp 2      weight producer (lane 0): TMA of the packed tile [128][32 B]
 //               into a deeper ring of its own, so that weights coming from
 //               HBM are requested well before they are needed.
 //   warps 4-11  unpackers, two groups of four taking alternate steps: thread
 //               r of a group expands row r's 32 packed bytes to 128 unsigned
-//               codes c = q + 1 in {0, 1, 2} and stores them into the code
-//               tile of stage s in the swizzled layout the MMA reads.
+//               codes c = q + 1 in {0, 1, 2} and stores them into TMEM lane r
+//               of stage s's code tile (tcgen05.st).
 //   warps 12-19 epilogue: wait for a finished accumulator, read it with
 //               tcgen05.ld (lane = feature, column = token), release it, and
 //               write y = (acc - rowsum) * gamma * s_x with evict-first
-//               stores -- overlapping the next tile's MMAs.
+//               stores -- overlapping the next tile's MMAs where there are
+//               two accumulator buffers.
 //
 // The single-thread issue loops matter: an MMA-issuing warp that waits with
 // warp-wide votes or commits twice per step leaves the tensor pipe idle for
@@ -53,7 +56,6 @@ constexpr int kEpiWarps = 8;     // warps 12 .. 19
 constexpr int kTileN = 128;      // features per tile (MMA M)
 constexpr int kTileK = 128;      // codes (bytes of x_q) per step
 constexpr int kWStageBytes = kTileN * kTileK / 4;  // packed bytes of one step's weight tile
-constexpr int kAStageBytes = kTileN * kTileK;      // unpacked codes of one step
 
 __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t v) {
     uint32_t p = 32;
@@ -61,25 +63,25 @@ __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t v) {
     return p;
 }
 
-// ATMEM: the unpacked codes (the A operand) live in tensor memory instead of
-// shared memory -- written by the unpackers with tcgen05.st, read by the MMA
-// from TMEM -- which takes their stores and the MMA's A reads off the SM's
-// shared-memory bandwidth.  TMEM then holds the accumulators and one 32-column
-// code tile (128 lanes x 128 codes) per stage: two accumulators up to BT = 128,
-// one for larger tiles (the MMAs of a tile then start once the epilogue has
-// read the previous tile's accumulator).
-template <int BT, bool ATMEM = false>
+// The unpacked codes (the A operand) live in tensor memory -- written by the
+// unpackers with tcgen05.st, read by the MMA from TMEM -- so neither their
+// stores nor the MMA's A reads take shared-memory bandwidth.  TMEM holds the
+// accumulators and one 32-column code tile (128 lanes x 128 codes) per stage:
+// two accumulators up to BT = 128, one for larger tiles (the MMAs of a tile
+// then start once the epilogue has read the previous tile's accumulator).
+// Shared memory holds the x_q ring (the B operand) and the packed-weight ring.
+template <int BT>
 struct GemmLayout {
-    static constexpr int kAccBufs = (ATMEM && BT > 128) ? 1 : 2;
+    static constexpr int kAccBufs = BT > 128 ? 1 : 2;
     static constexpr int kWStages = 8;      // packed-weight ring
     static constexpr int kB = BT * kTileK;  // x_q bytes per stage
-    static constexpr int kStage = kB + (ATMEM ? 0 : kAStageBytes);
-    // x_q (+ code) ring: as many stages as fit beside the weight ring
-    // (4 for BT = 256, 6 for 128, 8 for 64; with the codes in TMEM, at most 8)
+    static constexpr int kStage = kB;
+    // x_q ring: as many stages as fit beside the weight ring, at most 8
+    // (6 for BT = 256, 8 for the smaller tiles)
     static constexpr int kStagesFit = (232448 - 1024 - 512 - kWStages * kWStageBytes) / kStage;
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
     static constexpr int kACols = kTileK / 4;  // TMEM columns of one stage's code tile
-    static constexpr int offStage = 0;  // stage s: x_q tile, then code tile (both 1024-aligned)
+    static constexpr int offStage = 0;  // stage s: x_q tile (1024-aligned)
     static constexpr int offW = kStages * kStage;
     static constexpr int offBar = offW + kWStages * kWStageBytes;
     // barriers: full[S], empty[S], w_full[SW], w_empty[SW], d_full[2], d_empty[2], mma_done
@@ -87,15 +89,14 @@ struct GemmLayout {
     static constexpr int offTmem = offBar + kBars * 8;
     static constexpr int kBytes = offTmem + 16;
     static constexpr int kDynamic = kBytes + 1024;  // slack for 1024-byte alignment
-    // accumulator buffers start at multiples of kDStride TMEM columns; with
-    // ATMEM the code stages follow them
+    // accumulator buffers start at multiples of kDStride TMEM columns; the
+    // code stages follow them
     static constexpr int kDStride = BT <= 128 ? BT : 256;
     static constexpr int kAColBase = kAccBufs * kDStride;
-    static constexpr uint32_t kTmemCols =
-        pow2_at_least(ATMEM ? kAColBase + kStages * kACols : BT + kDStride);
+    static constexpr uint32_t kTmemCols = pow2_at_least(kAColBase + kStages * kACols);
     static_assert(kTmemCols <= 512, "tensor memory columns");
     static_assert(kDynamic <= 232448, "shared memory per CTA");
-    static_assert(kB % 1024 == 0 && kAStageBytes % 1024 == 0, "swizzle atoms stay aligned");
+    static_assert(kB % 1024 == 0, "swizzle atoms stay aligned");
 };
 
 // Natural-order expansion of one 32-bit packed word (16 codes) into 16
@@ -115,14 +116,13 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
 // 2-3) and every word is rewritten in Foundry's layout before the unpack; the
 // default layout compiles without that step.  EPI: the extra epilogue `ep`
 // (bias, integer bias and shift) is applied.
-// ATMEM: the code tiles in tensor memory (GemmLayout).
-template <int BT, bool CONV, bool EPI, bool ATMEM = false>
+template <int BT, bool CONV, bool EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const float *__restrict__ s_x, const int32_t *__restrict__ rowsum,
                 const float *__restrict__ gamma, int per_row, int M, int N, int K,
                 float *__restrict__ y, int32_t *__restrict__ acc_out, int mode, Epilogue ep) {
-    using L = GemmLayout<BT, ATMEM>;
+    using L = GemmLayout<BT>;
     constexpr int S = L::kStages, SW = L::kWStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -137,7 +137,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto d_empty = [&](int b) { return bar0 + 8u * (2 * S + 2 * SW + 2 + b); };
     const uint32_t mma_done = bar0 + 8u * (2 * S + 2 * SW + 4);
     auto x_stage = [&](int s) { return sbase + (uint32_t)(L::offStage + s * L::kStage); };
-    auto a_stage = [&](int s) { return x_stage(s) + (uint32_t)L::kB; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::offTmem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -239,20 +238,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_addr = a_stage(s), b_addr = x_stage(s);
-                    if (ATMEM) {
-                        // codes of stage s: TMEM columns kAColBase + 32 s ..., 8 columns per K = 32
-                        const uint32_t a_col = tmem + (uint32_t)(L::kAColBase + s * L::kACols);
+                    const uint32_t b_addr = x_stage(s);
+                    // codes of stage s: TMEM columns kAColBase + 32 s ..., 8 columns per K = 32
+                    const uint32_t a_col = tmem + (uint32_t)(L::kAColBase + s * L::kACols);
 #pragma unroll
-                        for (int kk = 0; kk < kTileK / 32; ++kk)
-                            mma_i8_ts(d_col, a_col + (uint32_t)(kk * 8), smem_desc_sw128(b_addr + kk * 32), idesc,
-                                      (kb | kk) != 0 ? 1u : 0u);
-                    } else {
-#pragma unroll
-                        for (int kk = 0; kk < kTileK / 32; ++kk)
-                            mma_i8(d_col, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
-                                   idesc, (kb | kk) != 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < kTileK / 32; ++kk)
+                        mma_i8_ts(d_col, a_col + (uint32_t)(kk * 8), smem_desc_sw128(b_addr + kk * 32), idesc,
+                                  (kb | kk) != 0 ? 1u : 0u);
                     mma_commit(empty(s));
                 }
                 if (ok) mma_commit(d_full(b));  // accumulator b complete
@@ -264,14 +256,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 4 + kUnpackWarps) {
-        // ---------------- unpack codes into the swizzled operand tile ----------------
+        // ---------------- unpack codes into the TMEM operand tile ----------------
         // Two groups of four warps take alternate steps, so each has two steps'
         // time for its waits, loads and stores; thread r of a group owns row r.
         const int par = (warp - 4) >> 2;
         const int enc = (mode >> kModeEncShift) & 3;  // packed-code layout
         const int r = 32 * (warp & 3) + lane;  // weight row of the tile
         const uint32_t w_row = sbase + (uint32_t)(L::offW + r * (kTileK / 4));
-        const uint32_t a_row = (uint32_t)(r * kTileK), sw = (uint32_t)(r & 7);
         for (int g = par; g < total; g += 2) {
             const int ws = g % SW, s = g % S;
             if (!warp_wait_sleep(w_full(ws), (g / SW) & 1, lane)) break;
@@ -303,30 +294,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int c = 0; c < 8; ++c) e[c] = expand_word(words[c]);
             if (!warp_wait_sleep(empty(s), ((g / S) & 1) ^ 1, lane)) break;
-            if (ATMEM) {
-                // row r's 128 codes -> TMEM lane r (this warp's lane quarter is
-                // 32 (warp % 4) .. + 31), 32 consecutive columns of 4 codes each
-                uint32_t cw[32];
+            // row r's 128 codes -> TMEM lane r (this warp's lane quarter is
+            // 32 (warp % 4) .. + 31), 32 consecutive columns of 4 codes each
+            uint32_t cw[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    cw[4 * c] = e[c].x;
-                    cw[4 * c + 1] = e[c].y;
-                    cw[4 * c + 2] = e[c].z;
-                    cw[4 * c + 3] = e[c].w;
-                }
-                tmem_st32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(L::kAColBase + s * L::kACols), cw);
-                tmem_st_wait();
-                tc_fence_before();  // the stores are complete before the MMA warp is told
-            } else {
-                // 16-byte chunk c of row r lives at chunk position c ^ (r & 7)
-                const uint32_t base = a_stage(s) + a_row;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base + (((uint32_t)c ^ sw) << 4)),
-                                 "r"(e[c].x), "r"(e[c].y), "r"(e[c].z), "r"(e[c].w)
-                                 : "memory");
-                fence_proxy_async_smem();  // generic stores -> visible to the tensor core
+            for (int c = 0; c < 8; ++c) {
+                cw[4 * c] = e[c].x;
+                cw[4 * c + 1] = e[c].y;
+                cw[4 * c + 2] = e[c].z;
+                cw[4 * c + 3] = e[c].w;
             }
+            tmem_st32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(L::kAColBase + s * L::kACols), cw);
+            tmem_st_wait();
+            tc_fence_before();  // the stores are complete before the MMA warp is told
             __syncwarp();
             // The packed slot is released only now: the stores above consume the
             // loaded words, so every lane's read of the slot is complete before
