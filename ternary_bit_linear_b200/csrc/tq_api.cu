@@ -399,15 +399,14 @@ size_t pack_parts(int64_t nv) {
 // Tokens per GEMM tile.  Cost model: rounds of tiles over the SMs times the
 // time of one K-step, 4 MMAs of BT/2 cycles each but no faster than the
 // single-thread issue rate (about 72 cycles per MMA); ties go to the smaller
-// tile (less padding and x_q traffic).  Tiles of up to 128 tokens keep their
-// codes in tensor memory (measured faster there: M = 64 at 8192^2 15.5 ->
-// 14.1 us); the larger ones stage them in shared memory (at 2048 x 11008 x
-// 4096, 128-token tiles with codes in TMEM took 117 us, 256-token tiles in
-// shared memory 82 us).
+// tile (less padding and x_q traffic).  No 192-token tiles: where the model
+// preferred them (one round of tiles either way) the 256-token tile measured
+// faster or close (fused 512 x 5632 x 2048 layer 19.8 -> 15.8 us; SwiGLU
+// block 67.7 -> 70.3 us), and with more rounds 256 wins the model anyway.
 int gemm_tile_tokens(int64_t M, int64_t N, int sms) {
     int best = 64;
     int64_t best_cost = -1;
-    for (int bt : {64, 128, 192, 256}) {
+    for (int bt : {64, 128, 256}) {
         const int64_t tiles = ((M + bt - 1) / bt) * ((N + kTileN - 1) / kTileN);
         const int64_t rounds = (tiles + sms - 1) / sms;
         const int64_t cost = rounds * (bt / 2 > 72 ? bt / 2 : 72);
@@ -426,7 +425,6 @@ tq_status contraction(const GemmArgs &a, int sms, cudaStream_t st) {
     switch (gemm_tile_tokens(a.M, a.N, sms)) {
     case 64: return launch_gemm<64, CONV, EPI>(a, sms, st);
     case 128: return launch_gemm<128, CONV, EPI>(a, sms, st);
-    case 192: return launch_gemm<192, CONV, EPI>(a, sms, st);
     default: return launch_gemm<256, CONV, EPI>(a, sms, st);
     }
 }

@@ -6,7 +6,7 @@
 // as tcgen05.mma kind::i8 with int32 accumulators in tensor memory.
 //
 // Persistent: one CTA per SM walks output tiles of 128 features (the MMA's M,
-// taken by the weights) x BT tokens (the MMA's N: 64, 128, 192 or 256, chosen
+// taken by the weights) x BT tokens (the MMA's N: 64, 128 or 256, chosen
 // per problem by the launcher to fill the SMs), token blocks
 // fastest so that concurrently running CTAs share weight tiles in L2.  K is
 // consumed in steps of 128 codes; one step is four MMAs of K = 32, the codes
@@ -18,7 +18,7 @@
 //   warp 1      TMEM owner; lane 0 issues the MMAs.  Per step: one wait on
 //               full(s), four MMAs, one commit that frees stage s.  The
 //               accumulator alternates between two TMEM buffers per tile
-//               (BT <= 128) or is a single buffer (BT = 192, 256).
+//               (BT <= 128) or is a single buffer (BT = 256).
 //   warp 2      weight producer (lane 0): TMA of the packed tile [128][32 B]
 //               into a deeper ring of its own, so that weights coming from
 //               HBM are requested well before they are needed.

@@ -626,7 +626,7 @@ def test_pack_inputs_ready_layers_then_dependent_reader(cuda_lib, per_row):
 
 
 # Shapes whose tile choice (tokens per tile, from the launcher's cost model on
-# 148 SMs) is 128, 192, 256 and 256, all ragged in M, N and K; in the last one the
+# 148 SMs) is 128, 256, 256 and 256, all ragged in M, N and K; in the last one the
 # last token tile holds 68 tokens and the last feature tile 92 features.
 @pytest.mark.parametrize("M,N,K", [(383, 11000, 192), (500, 5600, 320), (1000, 4000, 192), (580, 4956, 192)])
 def test_gemm_tile_sizes_sampled(cuda_lib, M, N, K):
